@@ -1,0 +1,170 @@
+"""KDA oracle: the fp64 token-by-token recurrence, for tests only.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference leg of ``bench.py`` may import this package.  The
+product library never does, and this package imports nothing from it.
+
+The arithmetic lives in ``kda_oracle.c`` (plain C, fp64, one head per host
+thread); this module only builds that file with gcc, loads it and marshals
+arrays.  The recurrence it evaluates is
+
+    S_t = (I - beta_t k_t k_t^T) Diag(exp g_t) S_{t-1} + beta_t k_t v_t^T,
+    o_t = S_t^T q_t,
+
+the delta-rule recurrence with a channel-wise forget gate of Kimi Delta
+Attention ("Kimi K3 goes trillion-scale with sparse MoE efficiency"
+subtitles, cue 14; "T11E1: K3 tech report" transcript, the KDA turn).
+
+Layouts follow the library: q, k, g are [B, T, H, dk]; v and o are
+[B, T, H, dv]; beta is [B, T, H]; states are [B, H, dk, dv].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "kda_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libkda_oracle.so")
+_default = None
+
+
+def compile_c(src: str, out: str) -> str:
+    """gcc -O2 a C file of the oracle into a shared library at `out`."""
+    tmp = out + ".tmp.%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+           "-o", tmp, src, "-lm", "-lpthread"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile kda_oracle.c into libkda_oracle.so beside it (if stale)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(SOURCE)):
+        return _LIB_PATH
+    return compile_c(SOURCE, _LIB_PATH)
+
+
+def _f64(x):
+    """Any array-like (numpy, torch of any float dtype) -> contiguous float64."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor, possibly bf16 and/or on a device
+        import torch
+        x = x.detach().to("cpu", torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+class Oracle:
+    """A loaded build of the oracle's C file (the default one, or a test's
+    deliberately altered copy)."""
+
+    def __init__(self, lib_path: str):
+        lib = ctypes.CDLL(lib_path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.kda_oracle_heads.argtypes = [
+            ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+            dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+        lib.kda_oracle_heads.restype = ctypes.c_int
+        lib.kda_oracle_num_cores.argtypes = []
+        lib.kda_oracle_num_cores.restype = ctypes.c_int
+        self.lib = lib
+
+    def num_cores(self) -> int:
+        return int(self.lib.kda_oracle_num_cores())
+
+    def heads(self, q, k, v, g, beta, h0=None, want_o=True, n_threads=0):
+        """n independent heads stacked on axis 0.
+
+        q, k, g: [n, T, dk]; v: [n, T, dv]; beta: [n, T]; h0: [n, dk, dv]
+        or None.  Returns (o [n, T, dv] or None, hT [n, dk, dv]) in float64.
+        """
+        q, k, v, g, beta, h0 = map(_f64, (q, k, v, g, beta, h0))
+        n, T, dk = q.shape
+        dv = v.shape[2]
+        assert k.shape == (n, T, dk) and g.shape == (n, T, dk)
+        assert v.shape == (n, T, dv) and beta.shape == (n, T)
+        if h0 is not None:
+            assert h0.shape == (n, dk, dv)
+        o = np.empty((n, T, dv), np.float64) if want_o else None
+        hT = np.empty((n, dk, dv), np.float64)
+        rc = self.lib.kda_oracle_heads(n, T, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(g), _ptr(beta), _ptr(h0), _ptr(o),
+                                       _ptr(hT), int(n_threads))
+        if rc != 0:
+            raise RuntimeError("kda oracle failed with code %d" % rc)
+        return o, hT
+
+    def fwd(self, q, k, v, g, beta, h0=None, want_o=True, n_threads=0):
+        """Whole-batch prefill in the library layout.
+
+        q, k, g: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H];
+        h0: [B, H, dk, dv] or None (zero state).
+        Returns (o [B, T, H, dv] or None, hT [B, H, dk, dv]) in float64.
+        """
+        q, k, v, g, beta, h0 = map(_f64, (q, k, v, g, beta, h0))
+        B, T, H, dk = q.shape
+        dv = v.shape[3]
+
+        def per_head(x):
+            return np.ascontiguousarray(
+                x.transpose(0, 2, 1, 3).reshape(B * H, T, x.shape[3]))
+
+        o, hT = self.heads(
+            per_head(q), per_head(k), per_head(v), per_head(g),
+            np.ascontiguousarray(beta.transpose(0, 2, 1).reshape(B * H, T)),
+            None if h0 is None else h0.reshape(B * H, dk, dv),
+            want_o=want_o, n_threads=n_threads)
+        if o is not None:
+            o = o.reshape(B, H, T, dv).transpose(0, 2, 1, 3)
+        return o, hT.reshape(B, H, dk, dv)
+
+    def decode_step(self, q, k, v, g, beta, state, n_threads=0):
+        """One token per request: the same recurrence applied once.
+
+        q, k, g: [N, H, dk]; v: [N, H, dv]; beta: [N, H];
+        state: [N, H, dk, dv].  Returns (o [N, H, dv], new state) in float64.
+        """
+        q, k, v, g, beta, state = map(_f64, (q, k, v, g, beta, state))
+        N, H, dk = q.shape
+        dv = v.shape[2]
+        o, hT = self.heads(q.reshape(N * H, 1, dk), k.reshape(N * H, 1, dk),
+                           v.reshape(N * H, 1, dv), g.reshape(N * H, 1, dk),
+                           beta.reshape(N * H, 1), state.reshape(N * H, dk, dv),
+                           n_threads=n_threads)
+        return o.reshape(N, H, dv), hT.reshape(N, H, dk, dv)
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle(build())
+    return _default
+
+
+def num_cores() -> int:
+    """Host cores the oracle's thread pool uses by default."""
+    return default().num_cores()
+
+
+def heads(*a, **kw):
+    return default().heads(*a, **kw)
+
+
+def fwd(*a, **kw):
+    return default().fwd(*a, **kw)
+
+
+def decode_step(*a, **kw):
+    return default().decode_step(*a, **kw)
