@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""KDA prefill/decode benchmark on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
+                    [--workload prefill_8k] [--no-decode] [--no-cpu-baseline]
+
+A step is one kda_chunk_fwd over one batch of the prefill workload (B=1,
+H=32, T=8192, d=128, bf16 inputs, fp32 state).  Two independent input sets
+of 269 MB each (together > 4x the 126 MB L2) alternate between steps, so no
+step starts with its inputs in L2.  The decode workload (256 requests x 32
+heads, 1000 successive kda_decode_step calls) is timed in the same run and
+reported under "decode".  Multi-GPU: one process per GPU (torchrun), every
+rank runs the same per-GPU workload on its own seed with no collective on
+the data path (weak scaling); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on
+this host's cores over a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+BYTES_BF16 = 2
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ------------------------------------------------------------ accounting --
+
+def prefill_alg_bytes(B, T, H, dk, dv, with_h0=True, with_hT=True):
+    """Algorithmic HBM bytes of one prefill: q, k, g, v, beta read once, o
+    written once, h0 read and hT written once (fp32)."""
+    per_token_head = (3 * dk + dv + 1) * BYTES_BF16 + dv * BYTES_BF16
+    state = dk * dv * 4
+    return B * T * H * per_token_head + B * H * state * (int(with_h0) + int(with_hT))
+
+
+def prefill_alg_flops(B, T, H, dk, dv, C=16):
+    """Algorithmic flops of the chunked form (per token-head: W S, Q S and
+    K^T U state products 6 dk dv; intra-tile products ~ C (4 dk + 2 dv);
+    the triangular solve ~ C^2/3)."""
+    per = 6 * dk * dv + C * (4 * dk + 2 * dv) + C * C / 3.0
+    return B * T * H * per
+
+
+def decode_alg_bytes(N, H, dk, dv):
+    """Per decode step: state read + written (fp32), q, k, g, v, beta read,
+    o written (bf16)."""
+    return N * H * (2 * dk * dv * 4 + (3 * dk + dv + 1 + dv) * BYTES_BF16)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ---------------------------------------------------------------- ranks ---
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Every rank draws its own independent batch of the same shape."""
+    return int(base) + 7919 * int(rank)
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# --------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            if self._t is not None:
+                self._t.join(timeout=2)
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- kda arm ----
+
+def bench_kda(args, rank, world, local):
+    import torch
+    import linear_attention_07_b200 as kda
+    from linear_attention_07_b200.inputs import WORKLOADS, prefill_inputs, decode_inputs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    kda.load_library()
+    w = WORKLOADS[args.workload]
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+
+    # two independent input sets, alternated between steps
+    sets = [prefill_inputs(B, T, H, dk, dv, seed=rank_seed(w.seed + 17 * i, rank),
+                           device=dev, h0_std=w.h0_std, pin_frac=w.pin_frac)
+            for i in range(2)]
+    outs = [(torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev),
+             torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)) for _ in range(2)]
+
+    def step(i):
+        x = sets[i % 2]
+        o, hT = outs[i % 2]
+        kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"], o=o, hT=hT)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    n0 = kda.launch_count()
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        barrier(dev)
+        torch.cuda.synchronize()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step(i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        barrier(dev)
+    launches = kda.launch_count() - n0
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    total_ms = max_over_ranks(total_ms, dev)
+    ms_per_step = total_ms / args.steps
+    tokens = B * T * world * args.steps
+    value = tokens / (total_ms / 1e3)
+
+    # roofline of the prefill kernel (one launch per step)
+    hbm_gbs, bf16_tf, peak_src = load_peaks()
+    alg_b = prefill_alg_bytes(B, T, H, dk, dv, with_h0=w.h0_std > 0)
+    alg_f = prefill_alg_flops(B, T, H, dk, dv)
+    launch_ms = statistics.mean(per_step)
+    achieved_gbs = alg_b / (launch_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1),
+                "peak": hbm_gbs, "unit": "GB/s",
+                "frac": round(achieved_gbs / hbm_gbs, 4),
+                "traffic": None, "peak_source": peak_src + " hbm_gbs (burst copy)",
+                "alg_bytes_per_launch": alg_b,
+                "kernel": "kda_chunk_fwd",
+                "tensor_alg_tflops": round(alg_f / (launch_ms / 1e3) / 1e12, 2),
+                "tensor_frac_alg": round(alg_f / (launch_ms / 1e3) / 1e12 / bf16_tf, 4)}
+
+    result = {
+        "metric": "KDA prefill tokens/s on 1 B200 (B1 H32 T8192 d128 bf16); decode steps/s under 'decode'",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
+                   "global_batch": B * world, "seq_len": T,
+                   "parallelism": "dp%d" % world,
+                   "l2": "two 269 MB input sets alternate (inputs > L2)"},
+        "roofline": roofline,
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+
+    # end to end through the public API: pinned host inputs -> device ->
+    # kda_chunk_fwd -> o and hT back to pinned host memory, every step
+    result["e2e"] = bench_e2e(args, kda, sets, dev, B, T, world)
+
+    if args.decode:
+        result["decode"] = bench_decode(args, kda, dev, rank, world, hbm_gbs, peak_src)
+    del sets, outs
+    torch.cuda.empty_cache()
+    return result
+
+
+def bench_e2e(args, kda, sets, dev, B, T, world):
+    import torch
+    host = []
+    for x in sets:
+        host.append({k: (None if t is None else t.cpu().pin_memory()) for k, t in x.items()})
+    dbuf = {k: (None if t is None else torch.empty_like(t)) for k, t in sets[0].items()}
+    o_h = torch.empty(tuple(sets[0]["v"].shape), dtype=torch.bfloat16).pin_memory()
+    s_h = torch.empty(tuple(dbuf["h0"].shape) if dbuf["h0"] is not None else
+                      (B, sets[0]["q"].shape[2], sets[0]["q"].shape[3], sets[0]["v"].shape[3]),
+                      dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host[0].values() if t is not None)
+    d2h = o_h.numel() * 2 + s_h.numel() * 4
+
+    def step(i):
+        hx = host[i % 2]
+        for k2, t in hx.items():
+            if t is not None:
+                dbuf[k2].copy_(t, non_blocking=True)
+        o, hT = kda.chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], dbuf["h0"])
+        o_h.copy_(o, non_blocking=True)
+        s_h.copy_(hT, non_blocking=True)
+
+    for i in range(max(1, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    return {"value": round(B * T * world * args.steps / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(ms / args.steps, 4)}
+
+
+def bench_decode(args, kda, dev, rank, world, hbm_gbs, peak_src):
+    import torch
+    from linear_attention_07_b200.inputs import WORKLOADS, decode_inputs
+    w = WORKLOADS["decode_256"]
+    N, H, dk, dv, steps = w.B, w.H, w.dk, w.dv, w.T
+    d = decode_inputs(N, H, dk, dv, steps, seed=rank_seed(w.seed, rank), device=dev,
+                      state_std=w.h0_std)
+    S = d["state"]
+    o = torch.empty((N, H, dv), dtype=torch.bfloat16, device=dev)
+    for t in range(3):
+        kda.decode_step(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t], S, o=o)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    barrier(dev)
+    ev[0].record(stream)
+    for t in range(steps):
+        kda.decode_step(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t], S, o=o)
+        ev[t + 1].record(stream)
+    torch.cuda.synchronize()
+    per = sorted(ev[t].elapsed_time(ev[t + 1]) for t in range(steps))
+    total = max_over_ranks(ev[0].elapsed_time(ev[-1]), dev)
+    alg = decode_alg_bytes(N, H, dk, dv)
+    mean_ms = statistics.mean(per)
+    ach = alg / (mean_ms / 1e3) / 1e9
+    out = {"metric": "KDA decode steps/s (256 requests x H32 d128, fp32 state)",
+           "value": round(steps * world / (total / 1e3) / world, 1), "unit": "steps/s per GPU",
+           "aggregate_steps_per_s": round(steps * world / (total / 1e3), 1),
+           "steps": steps, "ms_per_step_p50": round(per[len(per) // 2], 5),
+           "ms_per_step_p99": round(per[int(len(per) * 0.99) - 1], 5),
+           "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_gbs,
+                        "unit": "GB/s", "frac": round(ach / hbm_gbs, 4), "traffic": None,
+                        "peak_source": peak_src + " hbm_gbs (burst copy)",
+                        "alg_bytes_per_launch": alg, "kernel": "kda_decode_step"}}
+    del d
+    return out
+
+
+# -------------------------------------------------------- oracle on CPU ---
+
+def oracle_sample(workload_name, heads, seed, budget_s=None):
+    """Time the fp64 oracle on `heads` whole (b, h) sequences of a prefill
+    workload on all host cores.  Returns (tokens_per_s, seconds, cores,
+    sample_description); tokens/s counts full tokens (all H heads), i.e.
+    sampled token-heads / H / seconds."""
+    import torch
+    import oracle
+    from linear_attention_07_b200.inputs import WORKLOADS, prefill_inputs
+    w = WORKLOADS[workload_name]
+    x = prefill_inputs(1, w.T, heads, w.dk, w.dv, seed=seed, dtype=w.dtype,
+                       h0_std=w.h0_std, pin_frac=w.pin_frac)
+    t0 = time.perf_counter()
+    oracle.fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"])
+    dt = time.perf_counter() - t0
+    tok_s = heads * w.T / w.H / dt
+    desc = "%d of %d heads x %d tokens of %s, fp64 token-by-token, all cores" % (
+        heads, w.H, w.T, w.name)
+    return tok_s, dt, oracle.num_cores(), desc
+
+
+def cpu_baseline(args):
+    tok_s, dt, cores, desc = oracle_sample(args.workload, args.cpu_heads, 4242)
+    return {"value": round(tok_s, 2), "unit": "tokens/s", "cores": cores,
+            "kind": "oracle", "sample": desc, "seconds": round(dt, 2)}
+
+
+def bench_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    from linear_attention_07_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    for i in range(args.warmup):
+        oracle_sample(args.workload, args.ref_heads, 99 + i)
+    times, toks = [], 0
+    for i in range(args.steps):
+        tok_s, dt, cores, desc = oracle_sample(args.workload, args.ref_heads, 199 + i)
+        times.append(dt)
+        toks += args.ref_heads * w.T / w.H
+    total = sum(times)
+    value = toks / total
+    return {"metric": "KDA prefill tokens/s on 1 B200 (B1 H32 T8192 d128 bf16); decode steps/s under 'decode'",
+            "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total / args.steps * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk,
+                       "dv": w.dv, "global_batch": w.B, "seq_len": w.T,
+                       "parallelism": "host threads"},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": "each step: " + desc},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s",
+                    "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------- main ---
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kda", choices=["kda", "reference"])
+    ap.add_argument("--workload", default="prefill_8k")
+    ap.add_argument("--no-decode", dest="decode", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_base", action="store_false")
+    ap.add_argument("--cpu-heads", type=int, default=8)
+    ap.add_argument("--ref-heads", type=int, default=4)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_env()
+
+    if args.impl == "reference":
+        res = bench_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        res = bench_kda(args, rank, world, local)
+        if rank == 0 and args.cpu_base:
+            res["cpu_baseline"] = cpu_baseline(args)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,119 @@
+/*
+ * kda.h -- C ABI of libkda.so: Kimi Delta Attention (KDA) on NVIDIA B200.
+ *
+ * The operation.  Per head, a fixed-size d_k x d_v fp32 state S is carried
+ * through the sequence by the gated delta rule
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp g_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * with a scalar write strength beta_t in (0, 1) and a channel-wise log-decay
+ * g_t (one value per key channel) bounded to [-5, 0].  Sources:
+ *   - "T11E1: K3 tech report" podcast transcript (williamliu.ai): the KDA
+ *     turn (recurrent state, learned write strength, channel-wise
+ *     forgetting; decay bounded so chunk work stays in bf16 range on dense
+ *     tensor cores) and the next turn (log-decay floor of -5 keeps the
+ *     reciprocal scaling over a 16-token tile below the bf16 limit);
+ *   - "Kimi K3 goes trillion-scale with sparse MoE efficiency" subtitles
+ *     (podcast.do-not-panic.com), cue 14: delta-rule recurrence with a
+ *     channel-wise forget gate, one fixed-size state, lower-bounded sigmoid
+ *     decay, dense diagonal and off-diagonal tiles;
+ *   - "177: Kimi K3 in Detail" episode notes (zjai.club), Deep dive 17 and 10:
+ *     decoding reads a fixed per-request state that is rewritten in place
+ *     for every token.
+ * No output scale is applied (no 1/sqrt(d_k)); q and k are expected to be
+ * L2-normalised by the caller.  Preconditions on values (g in [-5, 0],
+ * beta in (0, 1), unit-norm keys) are documented, not checked or clamped.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers, owned by the caller, 16-byte
+ *     aligned, densely packed in the row-major layouts given per function.
+ *     No entry point allocates, frees or keeps a pointer after it returns.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream) and do
+ *     no host synchronisation.  Asynchronous device errors surface at the
+ *     caller's next synchronisation, as for any CUDA launch.
+ *   - Return value: KDA_OK, or a negative kda_status.  Argument errors are
+ *     detected on the host and return before anything is launched.
+ *   - Inputs and outputs must not overlap, except that hT may equal h0.
+ *   - Thread-safe: no global mutable state besides a launch counter.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* kda_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, negative size   */
+    KDA_ERR_UNSUPPORTED = -2,  /* valid but unsupported shape (dk, dv)      */
+    KDA_ERR_CUDA = -3,         /* a CUDA launch or runtime call failed      */
+    KDA_ERR_TIMEOUT = -4,      /* reserved: a bounded device wait expired   */
+    KDA_ERR_NO_MEMORY = -5     /* reserved                                  */
+} kda_status;
+
+/*
+ * kda_chunk_fwd -- chunked prefill, bf16 inputs and output, fp32 state.
+ *
+ *   q, k, g : bf16 [B][T][H][dk]        v, o : bf16 [B][T][H][dv]
+ *   beta    : bf16 [B][T][H]
+ *   h0      : fp32 [B][H][dk][dv], or NULL for a zero initial state
+ *   hT      : fp32 [B][H][dk][dv], or NULL to skip; may equal h0
+ *   B, T, H >= 0 (any of them 0: nothing to compute; with T == 0 and hT
+ *   given, hT receives h0, or zeros).  Supported: dk == dv == 128.
+ * o_t is written for every token; hT is S after the last token.  The work is
+ * done in 16-token tiles on the tensor cores with an fp32 master state (the
+ * "T11E1" transcript's log-decay-bound turn is what makes the diagonal tiles
+ * dense).  Returns KDA_ERR_UNSUPPORTED for other dk/dv.
+ */
+int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
+                  const void* beta, const float* h0, void* o, float* hT,
+                  int B, int T, int H, int dk, int dv, kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_f32 -- the same recurrence with fp32 inputs and fp32 output,
+ * evaluated in fp32 arithmetic (for tolerance-critical callers).
+ * Layouts as kda_chunk_fwd with every tensor fp32.
+ * Supported: dk, dv in {32, 64, 128}.
+ */
+int kda_chunk_fwd_f32(const float* q, const float* k, const float* v,
+                      const float* g, const float* beta, const float* h0,
+                      float* o, float* hT,
+                      int B, int T, int H, int dk, int dv, kda_stream_t stream);
+
+/*
+ * kda_decode_step -- one token for each of N requests, state updated IN PLACE
+ * ("177: Kimi K3 in Detail", Deep dive 10: the state is a whiteboard that is
+ * rewritten for every token).
+ *
+ *   q, k, g : bf16 [N][H][dk]     v, o : bf16 [N][H][dv]     beta : bf16 [N][H]
+ *   state   : fp32 [N][H][dk][dv], read and overwritten with S_t
+ *   N, H >= 0.  Supported: dk, dv in {32, 64, 128}.
+ * The state layout is the one kda_chunk_fwd writes to hT, so a prefill's hT
+ * is directly a decode state.
+ */
+int kda_decode_step(const void* q, const void* k, const void* v, const void* g,
+                    const void* beta, float* state, void* o,
+                    int N, int H, int dk, int dv, kda_stream_t stream);
+
+/* Human-readable name of a kda_status value (static storage). */
+const char* kda_status_string(int status);
+
+/* Number of kernels this library has launched in this process (all entry
+ * points, all devices); lets callers count launches in a timed region. */
+uint64_t kda_launch_count(void);
+
+/* ABI version: (major << 16) | minor. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

@@ -1,0 +1,185 @@
+"""Kimi Delta Attention (KDA) prefill and decode on NVIDIA B200 (sm_100a).
+
+Thin ctypes binding over ``libkda.so`` (the C ABI declared in
+``include/kda.h``).  Every step of the computation runs in the library's
+CUDA kernels; this module only checks tensors and passes pointers, sizes
+and the current CUDA stream.  PyTorch is used for device memory and streams.
+
+Raw C functions are exposed under their C names (``kda_chunk_fwd``,
+``kda_chunk_fwd_f32``, ``kda_decode_step``, ``kda_status_string``,
+``kda_launch_count``, ``kda_version``); the tensor-level helpers
+``chunk_fwd``, ``chunk_fwd_f32`` and ``decode_step`` wrap them.
+
+If the library is missing or cannot be loaded, every call raises
+``KdaLibraryError``: there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_OK = 0
+KDA_ERR_INVALID_ARG = -1
+KDA_ERR_UNSUPPORTED = -2
+KDA_ERR_CUDA = -3
+KDA_ERR_TIMEOUT = -4
+KDA_ERR_NO_MEMORY = -5
+
+EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_f32", "kda_decode_step",
+            "kda_status_string", "kda_launch_count", "kda_version")
+
+
+class KdaLibraryError(RuntimeError):
+    pass
+
+
+class KdaError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (fn, status_string(status), status))
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libkda.so (once) and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise KdaLibraryError(
+            "libkda.so not found at %s; build it with "
+            "`python -m linear_attention_07_b200.build`" % path)
+    try:
+        lib = ctypes.CDLL(path)
+    except OSError as e:  # pragma: no cover - depends on the machine
+        raise KdaLibraryError("cannot load %s: %s" % (path, e)) from e
+    vp, fp, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+    lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, vp]
+    lib.kda_chunk_fwd.restype = i
+    lib.kda_chunk_fwd_f32.argtypes = [fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, i, vp]
+    lib.kda_chunk_fwd_f32.restype = i
+    lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, fp, vp, i, i, i, i, vp]
+    lib.kda_decode_step.restype = i
+    lib.kda_status_string.argtypes = [i]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_launch_count.argtypes = []
+    lib.kda_launch_count.restype = ctypes.c_uint64
+    lib.kda_version.argtypes = []
+    lib.kda_version.restype = i
+    _lib = lib
+    return lib
+
+
+def __getattr__(name):
+    # raw C entry points under their C names, resolved on first use
+    if name in EXPORTED:
+        return getattr(load_library(), name)
+    raise AttributeError(name)
+
+
+def status_string(status: int) -> str:
+    return load_library().kda_status_string(int(status)).decode()
+
+
+def launch_count() -> int:
+    """Kernels launched by libkda.so so far in this process."""
+    return int(load_library().kda_launch_count())
+
+
+# ---------------------------------------------------------------- tensors --
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(t, name, dtype, shape, device):
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if t.device != device:
+        raise ValueError("%s must be on %s, got %s" % (name, device, t.device))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def _prefill(fn_name, dtype, q, k, v, g, beta, h0, o, hT, output_final_state):
+    import torch
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)),
+                         ("g", g, (B, T, H, dk)), ("v", v, (B, T, H, dv)),
+                         ("beta", beta, (B, T, H))):
+        _check(t, name, dtype, shp, dev)
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (B, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dtype, device=dev)
+    _check(o, "o", dtype, (B, T, H, dv), dev)
+    if hT is None and output_final_state:
+        hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    if hT is not None:
+        _check(hT, "hT", torch.float32, (B, H, dk, dv), dev)
+    fn = getattr(load_library(), fn_name)
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o),
+            _ptr(hT), B, T, H, dk, dv, _stream(dev))
+    if st != KDA_OK:
+        raise KdaError(fn_name, st)
+    return o, hT
+
+
+def chunk_fwd(q, k, v, g, beta, h0=None, *, o=None, hT=None, output_final_state=True):
+    """KDA prefill, bf16 in/out, fp32 state (kda_chunk_fwd).
+
+    q, k, g: [B, T, H, dk]; v: [B, T, H, dv]; beta: [B, T, H] (bf16, CUDA,
+    contiguous); h0: [B, H, dk, dv] fp32 or None.  Returns (o, hT).
+    hT may be passed as h0 to update a state in place.
+    """
+    import torch
+    return _prefill("kda_chunk_fwd", torch.bfloat16, q, k, v, g, beta, h0, o,
+                    hT, output_final_state)
+
+
+def chunk_fwd_f32(q, k, v, g, beta, h0=None, *, o=None, hT=None, output_final_state=True):
+    """KDA prefill with fp32 inputs/outputs and fp32 arithmetic."""
+    import torch
+    return _prefill("kda_chunk_fwd_f32", torch.float32, q, k, v, g, beta, h0, o,
+                    hT, output_final_state)
+
+
+def decode_step(q, k, v, g, beta, state, *, o=None):
+    """One decode token per request; `state` [N, H, dk, dv] fp32 is updated
+    in place.  q, k, g: [N, H, dk]; v: [N, H, dv]; beta: [N, H] (bf16).
+    Returns o [N, H, dv] bf16."""
+    import torch
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("inputs must be CUDA tensors")
+    for name, t, shp in (("q", q, (N, H, dk)), ("k", k, (N, H, dk)),
+                         ("g", g, (N, H, dk)), ("v", v, (N, H, dv)),
+                         ("beta", beta, (N, H))):
+        _check(t, name, torch.bfloat16, shp, dev)
+    _check(state, "state", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=torch.bfloat16, device=dev)
+    _check(o, "o", torch.bfloat16, (N, H, dv), dev)
+    st = load_library().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                        _ptr(state), _ptr(o), N, H, dk, dv, _stream(dev))
+    if st != KDA_OK:
+        raise KdaError("kda_decode_step", st)
+    return o

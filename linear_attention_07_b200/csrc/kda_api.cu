@@ -1,0 +1,124 @@
+// C ABI of libkda.so: host-side argument checks and kernel dispatch.
+// Every argument error is detected here, before any launch.
+#include <atomic>
+
+#include "kda_common.cuh"
+
+namespace kda {
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+cudaError_t decode_step_launch(const void* q, const void* k, const void* v,
+                               const void* g, const void* beta, float* state,
+                               void* o, int64_t NH, int dk, int dv,
+                               cudaStream_t stream);
+
+template <typename Tin, typename Tout>
+cudaError_t prefill_serial_launch(const void* q, const void* k, const void* v,
+                                  const void* g, const void* beta, const float* h0,
+                                  void* o, float* hT, int B, int T, int H,
+                                  int dk, int dv, cudaStream_t stream);
+
+static bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+static bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
+static bool opt_ptr_ok(const void* p) { return p == nullptr || aligned16(p); }
+
+// Largest element count of any tensor must stay far below 2^62 bytes.
+static bool sizes_ok(int64_t a, int64_t b, int64_t c, int64_t d)
+{
+    const int64_t lim = (int64_t)1 << 40;
+    return a < lim && b < lim && c < lim && d < lim && a * b < lim && a * b * c < lim &&
+           (double)a * (double)b * (double)c * (double)d < 4.0e18;
+}
+
+static int status_of(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+// Common checks of the two prefill entry points.
+static int check_prefill(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const void* h0, const void* o,
+                         const void* hT, int B, int T, int H, int dk, int dv)
+{
+    if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, H, dk > dv ? dk : dv)) return KDA_ERR_INVALID_ARG;
+    if (H > 65535 || B > 65535) return KDA_ERR_UNSUPPORTED;
+    if (!opt_ptr_ok(h0) || !opt_ptr_ok(hT)) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * T * H > 0) {
+        if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) || !ptr_ok(o))
+            return KDA_ERR_INVALID_ARG;
+        // beta rows are [B][T][H] scalars: only element alignment is needed
+        if (beta == nullptr) return KDA_ERR_INVALID_ARG;
+    }
+    return KDA_OK;
+}
+
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
+                  const void* beta, const float* h0, void* o, float* hT,
+                  int B, int T, int H, int dk, int dv, kda_stream_t stream)
+{
+    int st = check_prefill(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv);
+    if (st != KDA_OK) return st;
+    if (!(dk == 128 && dv == 128)) return KDA_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(beta) & 1u) != 0) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * H == 0) return KDA_OK;
+    if (T == 0 && hT == nullptr) return KDA_OK;
+    return status_of(prefill_serial_launch<__nv_bfloat16, __nv_bfloat16>(
+        q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, (cudaStream_t)stream));
+}
+
+int kda_chunk_fwd_f32(const float* q, const float* k, const float* v,
+                      const float* g, const float* beta, const float* h0,
+                      float* o, float* hT,
+                      int B, int T, int H, int dk, int dv, kda_stream_t stream)
+{
+    int st = check_prefill(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv);
+    if (st != KDA_OK) return st;
+    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(beta) & 3u) != 0) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * H == 0) return KDA_OK;
+    if (T == 0 && hT == nullptr) return KDA_OK;
+    return status_of(prefill_serial_launch<float, float>(
+        q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, (cudaStream_t)stream));
+}
+
+int kda_decode_step(const void* q, const void* k, const void* v, const void* g,
+                    const void* beta, float* state, void* o,
+                    int N, int H, int dk, int dv, kda_stream_t stream)
+{
+    if (N < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    const int64_t NH = (int64_t)N * H;
+    if (NH == 0) return KDA_OK;
+    if (NH > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) || !ptr_ok(state) || !ptr_ok(o))
+        return KDA_ERR_INVALID_ARG;
+    if (beta == nullptr || (reinterpret_cast<uintptr_t>(beta) & 1u) != 0) return KDA_ERR_INVALID_ARG;
+    return status_of(decode_step_launch(q, k, v, g, beta, state, o, NH, dk, dv,
+                                        (cudaStream_t)stream));
+}
+
+const char* kda_status_string(int status)
+{
+    switch (status) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+        case KDA_ERR_NO_MEMORY: return "KDA_ERR_NO_MEMORY";
+        default: return "KDA_ERR_UNKNOWN";
+    }
+}
+
+uint64_t kda_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int kda_version(void) { return (1 << 16) | 0; }
+
+}  // extern "C"

@@ -1,0 +1,126 @@
+"""The C ABI: library loads, exports what include/kda.h declares, and rejects
+bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_07_b200 as kda
+from linear_attention_07_b200 import build as kbuild
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "kda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.load_library()
+
+
+def declared_functions():
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("kda_chunk_fwd", "kda_chunk_fwd_f32", "kda_decode_step", "kda_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(kda.EXPORTED) >= set(declared_functions())
+
+
+def test_status_strings(lib):
+    assert kda.status_string(0) == "KDA_OK"
+    assert kda.status_string(-1) == "KDA_ERR_INVALID_ARG"
+    assert kda.status_string(-2) == "KDA_ERR_UNSUPPORTED"
+    assert kda.status_string(-3) == "KDA_ERR_CUDA"
+    assert kda.status_string(12345) == "KDA_ERR_UNKNOWN"
+    assert lib.kda_version() >> 16 == 1
+
+
+# Fake, never-dereferenced addresses: every call below fails a host check
+# first, so nothing is launched and no address is touched.
+A = ctypes.c_void_p(0x10000)
+A2 = ctypes.c_void_p(0x20000)
+MIS = ctypes.c_void_p(0x10008)   # 8-byte aligned only
+NUL = None
+
+
+def prefill(lib, fn, q=A, k=A, v=A, g=A, beta=A2, h0=NUL, o=A, hT=NUL,
+            B=1, T=16, H=2, dk=128, dv=128):
+    return getattr(lib, fn)(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, None)
+
+
+@pytest.mark.parametrize("fn", ["kda_chunk_fwd", "kda_chunk_fwd_f32"])
+def test_prefill_argument_errors(lib, fn):
+    n0 = lib.kda_launch_count()
+    assert prefill(lib, fn, q=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert prefill(lib, fn, o=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert prefill(lib, fn, beta=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert prefill(lib, fn, k=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert prefill(lib, fn, h0=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert prefill(lib, fn, hT=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert prefill(lib, fn, B=-1) == kda.KDA_ERR_INVALID_ARG
+    assert prefill(lib, fn, T=-5) == kda.KDA_ERR_INVALID_ARG
+    assert prefill(lib, fn, dk=0) == kda.KDA_ERR_INVALID_ARG
+    assert prefill(lib, fn, dk=96) == kda.KDA_ERR_UNSUPPORTED
+    assert prefill(lib, fn, dv=256) == kda.KDA_ERR_UNSUPPORTED
+    assert prefill(lib, fn, H=70000) == kda.KDA_ERR_UNSUPPORTED
+    assert prefill(lib, fn, B=1 << 30, T=1 << 30, H=1 << 10) == kda.KDA_ERR_INVALID_ARG
+    # nothing to do: returns OK without a launch
+    assert prefill(lib, fn, B=0) == kda.KDA_OK
+    assert prefill(lib, fn, H=0) == kda.KDA_OK
+    assert prefill(lib, fn, T=0, q=NUL, k=NUL, v=NUL, g=NUL, beta=NUL, o=NUL) == kda.KDA_OK
+    assert lib.kda_launch_count() == n0
+
+
+def test_bf16_prefill_shape_support(lib):
+    # the tensor-core path is specialised to d_k = d_v = 128
+    assert prefill(lib, "kda_chunk_fwd", dk=64, dv=64) == kda.KDA_ERR_UNSUPPORTED
+    assert prefill(lib, "kda_chunk_fwd", dk=128, dv=64) == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_decode_argument_errors(lib):
+    n0 = lib.kda_launch_count()
+
+    def dec(q=A, k=A, v=A, g=A, beta=A2, state=A, o=A, N=4, H=2, dk=128, dv=128):
+        return lib.kda_decode_step(q, k, v, g, beta, state, o, N, H, dk, dv, None)
+
+    assert dec(state=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert dec(state=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert dec(o=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert dec(beta=ctypes.c_void_p(0x20001)) == kda.KDA_ERR_INVALID_ARG
+    assert dec(N=-1) == kda.KDA_ERR_INVALID_ARG
+    assert dec(dk=48) == kda.KDA_ERR_UNSUPPORTED
+    assert dec(N=0) == kda.KDA_OK
+    assert dec(H=0, q=NUL) == kda.KDA_OK
+    assert lib.kda_launch_count() == n0
+
+
+def test_binding_requires_cuda_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 128, dtype=torch.bfloat16)
+    b = torch.zeros(1, 4, 1, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        kda.chunk_fwd(x, x, x, x, b)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(kda.KdaLibraryError):
+        import importlib
+        mod = importlib.import_module("linear_attention_07_b200")
+        saved = mod._lib
+        mod._lib = None
+        try:
+            mod.load_library(str(tmp_path / "nope.so"))
+        finally:
+            mod._lib = saved
