@@ -54,7 +54,7 @@ typedef enum {
     KDA_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, negative size   */
     KDA_ERR_UNSUPPORTED = -2,  /* valid but unsupported shape (dk, dv)      */
     KDA_ERR_CUDA = -3,         /* a CUDA launch or runtime call failed      */
-    KDA_ERR_TIMEOUT = -4,      /* reserved: a bounded device wait expired   */
+    KDA_ERR_TIMEOUT = -4,      /* a bounded device wait expired (see below) */
     KDA_ERR_NO_MEMORY = -5     /* reserved                                  */
 } kda_status;
 
@@ -101,6 +101,14 @@ int kda_chunk_fwd_f32(const float* q, const float* k, const float* v,
 int kda_decode_step(const void* q, const void* k, const void* v, const void* g,
                     const void* beta, float* state, void* o,
                     int N, int H, int dk, int dv, kda_stream_t stream);
+
+/*
+ * kda_device_status -- KDA_OK, or KDA_ERR_TIMEOUT if a kernel of this
+ * library gave up on a bounded device-side wait since the last call (the
+ * kernel then returned early and its outputs are incomplete).  Reads and
+ * clears the flag; synchronises `stream`.  KDA_ERR_CUDA if a CUDA call fails.
+ */
+int kda_device_status(kda_stream_t stream);
 
 /* Human-readable name of a kda_status value (static storage). */
 const char* kda_status_string(int status);

@@ -29,7 +29,8 @@ KDA_ERR_TIMEOUT = -4
 KDA_ERR_NO_MEMORY = -5
 
 EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_f32", "kda_decode_step",
-            "kda_status_string", "kda_launch_count", "kda_version")
+            "kda_device_status", "kda_status_string", "kda_launch_count",
+            "kda_version")
 
 
 class KdaLibraryError(RuntimeError):
@@ -65,6 +66,8 @@ def load_library(path: str = LIB_PATH):
     lib.kda_chunk_fwd_f32.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, fp, vp, i, i, i, i, vp]
     lib.kda_decode_step.restype = i
+    lib.kda_device_status.argtypes = [vp]
+    lib.kda_device_status.restype = i
     lib.kda_status_string.argtypes = [i]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_launch_count.argtypes = []
@@ -84,6 +87,14 @@ def __getattr__(name):
 
 def status_string(status: int) -> str:
     return load_library().kda_status_string(int(status)).decode()
+
+
+def device_status(device=None) -> int:
+    """KDA_OK or KDA_ERR_TIMEOUT (a bounded device wait expired since the
+    last call); synchronises the current stream and clears the flag."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    return int(load_library().kda_device_status(_stream(dev)))
 
 
 def launch_count() -> int:

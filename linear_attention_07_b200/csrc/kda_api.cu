@@ -14,6 +14,11 @@ cudaError_t decode_step_launch(const void* q, const void* k, const void* v,
                                void* o, int64_t NH, int dk, int dv,
                                cudaStream_t stream);
 
+cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
+                              const void* beta, const float* h0, void* o, float* hT,
+                              int B, int T, int H, cudaStream_t stream);
+int prefill_device_status(cudaStream_t stream);
+
 template <typename Tin, typename Tout>
 cudaError_t prefill_serial_launch(const void* q, const void* k, const void* v,
                                   const void* g, const void* beta, const float* h0,
@@ -69,8 +74,8 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
     if ((reinterpret_cast<uintptr_t>(beta) & 1u) != 0) return KDA_ERR_INVALID_ARG;
     if ((int64_t)B * H == 0) return KDA_OK;
     if (T == 0 && hT == nullptr) return KDA_OK;
-    return status_of(prefill_serial_launch<__nv_bfloat16, __nv_bfloat16>(
-        q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, (cudaStream_t)stream));
+    return status_of(prefill_tc_launch(q, k, v, g, beta, h0, o, hT, B, T, H,
+                                       (cudaStream_t)stream));
 }
 
 int kda_chunk_fwd_f32(const float* q, const float* k, const float* v,
@@ -115,6 +120,11 @@ const char* kda_status_string(int status)
         case KDA_ERR_NO_MEMORY: return "KDA_ERR_NO_MEMORY";
         default: return "KDA_ERR_UNKNOWN";
     }
+}
+
+int kda_device_status(kda_stream_t stream)
+{
+    return prefill_device_status((cudaStream_t)stream);
 }
 
 uint64_t kda_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -1,0 +1,456 @@
+// KDA chunked prefill on the sm_100a tensor cores (tcgen05, kind::tf32,
+// fp32 accumulation in tensor memory).
+//
+// The recurrence ("T11E1: K3 tech report" transcript, KDA turn; "Kimi K3 goes
+// trillion-scale ..." subtitles, cue 14)
+//     S_t = (I - b_t k_t k_t^T) Diag(exp g_t) S_{t-1} + b_t k_t v_t^T,  o_t = S_t^T q_t
+// is evaluated exactly (up to rounding) in 16-token tiles.  Inside a tile,
+// with Gam_r = sum_{s<=r} g_s (per key channel, from the tile start) and
+// gamma_r = exp(Gam_r):
+//     Kt = K * gamma,  Qt = Q * gamma           (<= 1)
+//     Kh = K / gamma                             (reciprocal scaling, <= e^80)
+//     Kb = K * gamma_16 / gamma                  (<= 1)
+//     A  = diag(b) strict_lower(Kt Kh^T),  P = lower_incl(Qt Kh^T)
+//     T  = (I + A)^-1 diag(b),   W = T Kt,   U' = T V
+//     U  = U' - W S,   O = Qt S + P U,   S <- Diag(gamma_16) S + Kb^T U
+// The log-decay floor g >= -5 bounds the reciprocal scaling over a 16-token
+// tile by e^80, inside the fp32/tf32 range, so the diagonal tiles are dense
+// MMAs with no position-by-position path (the "T11E1" transcript's
+// log-decay-bound turn; cue 14 of the subtitles).
+//
+// Mapping (one CTA of 128 threads per (batch, head); d_k = d_v = 128):
+//   * Everything is "transposed" so that the 128-wide dimension is the MMA M:
+//     tensor-memory lane j holds column j of S (thread j owns it).
+//   * The fp32 master state lives in registers (thread j: S[:, j]); a tf32
+//     copy of S^T is written to tensor memory each tile and used as the A
+//     operand of  X = S^T [W | Qt]^T  (M 128, N 32, K 128).
+//   * U^T goes to tensor memory as the A operand of  S^T += U^T Kb  (N 128,
+//     K 16) and  O^T += U^T P^T  (N 16, K 16).
+//   * Two tiles form a group: the Gram products Kh [Kt | Qt]^T of both tiles
+//     are one M=64 MMA, W^T = Kt^T T^T and U'^T = V^T T^T are M=128 MMAs
+//     with a block-diagonal T.
+//   * All MMAs are tf32 with operands rounded to nearest (cvt.rna): bf16
+//     operands would leave errors of a few percent of rms(o) on these
+//     products (the q.k diagonal times large u), tf32 leaves ~0.3%.
+// Shared-memory operands use the no-swizzle K-major layout; when the thread
+// that produces a value owns the K index, the K-direction core-matrix stride
+// is padded to 144 B so that a warp's scalar stores hit 32 distinct banks.
+#include "kda_common.cuh"
+#include "kda_tc.cuh"
+
+namespace kda {
+
+namespace pf {
+
+constexpr int D = 128;         // d_k = d_v
+constexpr int TILE = 16;
+constexpr int GRP = 32;        // tokens per group (two tiles)
+constexpr int NT = 128;        // threads per CTA
+
+constexpr uint32_t PAD_LBO = 144;            // padded K-direction core-matrix stride
+constexpr uint32_t LBO = 128;                // dense K-direction core-matrix stride
+
+// shared memory map (bytes)
+constexpr uint32_t RAW_Q = 0;
+constexpr uint32_t RAW_K = RAW_Q + GRP * D * 2;
+constexpr uint32_t RAW_V = RAW_K + GRP * D * 2;
+constexpr uint32_t RAW_G = RAW_V + GRP * D * 2;
+constexpr uint32_t BETA = RAW_G + GRP * D * 2;                 // GRP fp32
+constexpr uint32_t GA = BETA + 128;                            // Kh, 32 rows x K 128 (padded)
+constexpr uint32_t GA_SBO = (D / 4) * PAD_LBO;                 // 4608
+constexpr uint32_t GB = GA + (GRP / 8) * GA_SBO;               // [Kt | Qt], 64 rows x K 128
+constexpr uint32_t WA = GB + (2 * GRP / 8) * GA_SBO;           // Kt^T: M 128 x K 32
+constexpr uint32_t WA_SBO = (GRP / 4) * LBO;                   // 1024
+constexpr uint32_t VA = WA + (D / 8) * WA_SBO;                 // V^T:  M 128 x K 32
+constexpr uint32_t TB = VA + (D / 8) * WA_SBO;                 // T (block diag): N 32 x K 32 (padded)
+constexpr uint32_t TB_SBO = (GRP / 4) * PAD_LBO;               // 1152
+constexpr uint32_t B1 = TB + (GRP / 8) * TB_SBO;               // per tile [W | Qt]: N 32 x K 128 (padded)
+constexpr uint32_t B1_SZ = (2 * TILE / 8) * GA_SBO;            // 18432
+constexpr uint32_t B2 = B1 + 2 * B1_SZ;                        // per tile Kb: N 128 x K 16
+constexpr uint32_t B2_SBO = (TILE / 4) * LBO;                  // 512
+constexpr uint32_t B2_SZ = (D / 8) * B2_SBO;                   // 8192
+constexpr uint32_t B3 = B2 + 2 * B2_SZ;                        // per tile P: N 16 x K 16 (padded)
+constexpr uint32_t B3_SBO = (TILE / 4) * PAD_LBO;              // 576
+constexpr uint32_t B3_SZ = (TILE / 8) * B3_SBO;                // 1152
+constexpr uint32_t GAM = B3 + 2 * B3_SZ;                       // per tile gamma_16, 2 x 128 fp32
+constexpr uint32_t AM = GAM + 2 * D * 4;                       // per tile A scratch 16 x 17 fp32
+constexpr uint32_t SMEM_BYTES = AM + 2 * TILE * 17 * 4;
+
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(GA % 16 == 0 && GB % 16 == 0 && WA % 16 == 0 && VA % 16 == 0 && TB % 16 == 0 &&
+              B1 % 16 == 0 && B2 % 16 == 0 && B3 % 16 == 0, "descriptor alignment");
+
+// tensor memory columns
+constexpr uint32_t T_AS = 0;     // S^T (tf32), 128 cols
+constexpr uint32_t T_AU = 128;   // U^T (tf32), 16 cols
+constexpr uint32_t T_DX = 160;   // [ (W S)^T | (Qt S + P U)^T ], 32 cols
+constexpr uint32_t T_DKU = 192;  // (Kb^T U)^T, 128 cols
+constexpr uint32_t T_DG = 320;   // Gram (M = 64), 64 cols
+constexpr uint32_t T_DW = 384;   // W^T, 32 cols
+constexpr uint32_t T_DU = 416;   // U'^T, 32 cols
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr uint64_t WAIT_NS = 2000000000ull;   // bounded waits: 2 s
+
+}  // namespace pf
+
+__device__ int g_prefill_status;   // set to KDA_ERR_TIMEOUT by a wait that expired
+
+__device__ __forceinline__ void st_f32(unsigned char* base, uint32_t off, float v) {
+    *reinterpret_cast<float*>(base + off) = v;
+}
+
+__global__ void __launch_bounds__(pf::NT, 1)
+prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                  const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ g,
+                  const __nv_bfloat16* __restrict__ beta, const float* h0,
+                  __nv_bfloat16* __restrict__ o, float* hT, int T, int H)
+{
+    using namespace pf;
+    using namespace tc;
+    extern __shared__ __align__(1024) unsigned char sm[];
+    __shared__ uint32_t s_taddr;
+    __shared__ __align__(8) uint64_t s_bar;
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int64_t head_off = (int64_t)b * H + h;          // (b, h) index
+    const int64_t row_stride = (int64_t)H * D;            // elements between tokens
+    const __nv_bfloat16* qh = q + ((int64_t)b * T * H + h) * D;
+    const __nv_bfloat16* kh = k + ((int64_t)b * T * H + h) * D;
+    const __nv_bfloat16* vh = v + ((int64_t)b * T * H + h) * D;
+    const __nv_bfloat16* gh = g + ((int64_t)b * T * H + h) * D;
+    const __nv_bfloat16* bh = beta + (int64_t)b * T * H + h;
+    __nv_bfloat16* oh = o + ((int64_t)b * T * H + h) * D;
+
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&s_taddr), TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(smem_u32(&s_bar), 1);
+        fence_mbar_init();
+        s_abort = 0;
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = s_taddr;
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;   // this warp's TMEM lanes
+    const uint32_t bar = smem_u32(&s_bar);
+    uint32_t phase = 0;
+
+    // master state: thread j holds column j of S
+    const int j = tid;
+    float S[D];
+    {
+        const float* h0h = h0 ? h0 + head_off * D * D : nullptr;
+#pragma unroll
+        for (int c = 0; c < D; ++c) S[c] = h0h ? h0h[(int64_t)c * D + j] : 0.f;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            float t32[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) t32[i] = to_tf32(S[c0 + i]);
+            tmem_st32(tm + lane_base + T_AS + c0, t32);
+        }
+        wait_st();
+    }
+
+    auto wait_mma = [&]() {
+        const bool ok = mbar_wait(bar, phase & 1u, WAIT_NS);
+        ++phase;
+        if (!ok) {
+            s_abort = 1;
+            atomicExch(&g_prefill_status, (int)KDA_ERR_TIMEOUT);
+        }
+        fence_after_sync();
+    };
+    auto cta_sync_tc = [&]() {      // order tcgen05 work around a CTA barrier
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+    };
+
+    const int n_groups = (T + GRP - 1) / GRP;
+    for (int grp = 0; grp < n_groups; ++grp) {
+        const int t0 = grp * GRP;
+
+        // ---- phase 0: raw tile inputs (bf16) into shared memory, zero past T
+        for (int idx = tid; idx < 4 * GRP * (D / 8); idx += NT) {
+            const int tensor = idx / (GRP * (D / 8));
+            const int rem = idx % (GRP * (D / 8));
+            const int r = rem / (D / 8), vec = rem % (D / 8);
+            const __nv_bfloat16* src = tensor == 0 ? qh : tensor == 1 ? kh : tensor == 2 ? vh : gh;
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (t0 + r < T) val = *reinterpret_cast<const uint4*>(src + (int64_t)(t0 + r) * row_stride + vec * 8);
+            *reinterpret_cast<uint4*>(sm + RAW_Q + tensor * (GRP * D * 2) + (r * D + vec * 8) * 2) = val;
+        }
+        if (tid < GRP)
+            reinterpret_cast<float*>(sm + BETA)[tid] =
+                (t0 + tid < T) ? to_f32(bh[(int64_t)(t0 + tid) * H]) : 0.f;
+        __syncthreads();
+
+        // ---- phase 1: decay scaling; thread c = key channel -----------------
+        {
+            const int c = tid;
+            const __nv_bfloat16* rq = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_Q);
+            const __nv_bfloat16* rk = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_K);
+            const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_V);
+            const __nv_bfloat16* rg = reinterpret_cast<const __nv_bfloat16*>(sm + RAW_G);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                float a[TILE];
+                float gam = 1.f;
+                float ktv[4];
+#pragma unroll
+                for (int rr = 0; rr < TILE; ++rr) {
+                    const int r = t * TILE + rr;
+                    a[rr] = __expf(to_f32(rg[r * D + c]));
+                    gam *= a[rr];
+                    const float kv = to_f32(rk[r * D + c]);
+                    const float qv = to_f32(rq[r * D + c]);
+                    const float kt = to_tf32(kv * gam);
+                    const float qt = to_tf32(qv * gam);
+                    st_f32(sm, GB + off_kmajor(r, c, PAD_LBO, GA_SBO), kt);              // Kt rows
+                    st_f32(sm, GB + off_kmajor(GRP + r, c, PAD_LBO, GA_SBO), qt);        // Qt rows
+                    st_f32(sm, B1 + t * B1_SZ + off_kmajor(TILE + rr, c, PAD_LBO, GA_SBO), qt);
+                    ktv[rr & 3] = kt;
+                    if ((rr & 3) == 3)
+                        *reinterpret_cast<float4*>(sm + WA + off_kmajor(c, r - 3, LBO, WA_SBO)) =
+                            make_float4(ktv[0], ktv[1], ktv[2], ktv[3]);
+                }
+                reinterpret_cast<float*>(sm + GAM)[t * D + c] = gam;
+                const float inv = 1.f / gam;
+                float sig = 1.f;
+                float kbv[4];
+#pragma unroll
+                for (int rr = TILE - 1; rr >= 0; --rr) {
+                    const int r = t * TILE + rr;
+                    const float kv = to_f32(rk[r * D + c]);
+                    const float kb = kv * sig;
+                    st_f32(sm, GA + off_kmajor(r, c, PAD_LBO, GA_SBO), to_tf32(kb * inv));
+                    kbv[rr & 3] = to_tf32(kb);
+                    if ((rr & 3) == 0)
+                        *reinterpret_cast<float4*>(sm + B2 + t * B2_SZ + off_kmajor(c, rr, LBO, B2_SBO)) =
+                            make_float4(kbv[0], kbv[1], kbv[2], kbv[3]);
+                    sig *= a[rr];
+                }
+            }
+            // V^T (thread c acts as value column j)
+#pragma unroll
+            for (int r = 0; r < GRP; r += 4) {
+                float4 vv;
+                vv.x = to_tf32(to_f32(rv[(r + 0) * D + c]));
+                vv.y = to_tf32(to_f32(rv[(r + 1) * D + c]));
+                vv.z = to_tf32(to_f32(rv[(r + 2) * D + c]));
+                vv.w = to_tf32(to_f32(rv[(r + 3) * D + c]));
+                *reinterpret_cast<float4*>(sm + VA + off_kmajor(c, r, LBO, WA_SBO)) = vv;
+            }
+        }
+        fence_smem_to_async();
+        cta_sync_tc();
+
+        // ---- phase 2: Gram  D_G = Kh [Kt | Qt]^T  (M 64, N 64, K 128) -------
+        if (tid == 0) {
+            const uint32_t id = idesc_tf32(64, 64, false, false);
+#pragma unroll 1
+            for (int ks = 0; ks < D / 8; ++ks) {
+                const uint64_t ad = sdesc(smem_u32(sm + GA) + ks * 2 * PAD_LBO, PAD_LBO, GA_SBO);
+                const uint64_t bd = sdesc(smem_u32(sm + GB) + ks * 2 * PAD_LBO, PAD_LBO, GA_SBO);
+                mma_tf32_ss(tm + T_DG, ad, bd, id, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(bar);
+        }
+        __syncwarp();
+        wait_mma();
+
+        // ---- phase 3: A, P and the triangular solve (warps 0, 1: tile = warp)
+        if (warp < 2) {
+            float gk[TILE], gq[TILE];
+            tmem_ld16(tm + lane_base + T_DG + warp * TILE, gk);          // Kh_i . Kt_r
+            tmem_ld16(tm + lane_base + T_DG + GRP + warp * TILE, gq);    // Kh_i . Qt_r
+            wait_ld();
+            const int t = warp;
+            float* am = reinterpret_cast<float*>(sm + AM) + t * TILE * 17;
+            const float* bt = reinterpret_cast<const float*>(sm + BETA) + t * TILE;
+            if (lane < TILE) {
+                const int i = lane;
+                // column i of A: A[r][i] = b_r Kt_r . Kh_i for r > i
+#pragma unroll
+                for (int r = 0; r < TILE; ++r) am[r * 17 + i] = (r > i) ? bt[r] * gk[r] : 0.f;
+                // column i of P (lower incl.) into B3: element (n = r, k = i)
+#pragma unroll
+                for (int r = 0; r < TILE; ++r)
+                    st_f32(sm, B3 + t * B3_SZ + off_kmajor(r, i, PAD_LBO, B3_SBO), to_tf32(r >= i ? gq[r] : 0.f));
+            }
+            __syncwarp();
+            if (lane < TILE) {
+                const int i = lane;
+                // x = (I + A)^-1 e_i by forward substitution
+                float x[TILE];
+#pragma unroll
+                for (int r = 0; r < TILE; ++r) {
+                    float acc = (r == i) ? 1.f : 0.f;
+#pragma unroll
+                    for (int s = 0; s < r; ++s) acc = fmaf(-am[r * 17 + s], x[s], acc);
+                    x[r] = (r < i) ? 0.f : acc;
+                }
+                const float bi = bt[i];
+                const int ig = t * TILE + i;
+#pragma unroll
+                for (int r = 0; r < GRP; ++r) {
+                    const float val = (r / TILE == t) ? to_tf32(x[r % TILE] * bi) : 0.f;
+                    st_f32(sm, TB + off_kmajor(r, ig, PAD_LBO, TB_SBO), val);
+                }
+            }
+        }
+        fence_smem_to_async();
+        cta_sync_tc();
+
+        // ---- phase 4: W^T = Kt^T T^T, U'^T = V^T T^T  (M 128, N 32, K 32) -----
+        if (tid == 0) {
+            const uint32_t id = idesc_tf32(128, 32, false, false);
+#pragma unroll 1
+            for (int ks = 0; ks < GRP / 8; ++ks) {
+                const uint64_t bd = sdesc(smem_u32(sm + TB) + ks * 2 * PAD_LBO, PAD_LBO, TB_SBO);
+                const uint64_t aw = sdesc(smem_u32(sm + WA) + ks * 2 * LBO, LBO, WA_SBO);
+                const uint64_t av = sdesc(smem_u32(sm + VA) + ks * 2 * LBO, LBO, WA_SBO);
+                mma_tf32_ss(tm + T_DW, aw, bd, id, ks > 0 ? 1u : 0u);
+                mma_tf32_ss(tm + T_DU, av, bd, id, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(bar);
+        }
+        __syncwarp();
+        wait_mma();
+
+        // ---- phase 5: W into the B operand of the state product -------------
+        {
+            const int c = tid;
+            float w[16];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                tmem_ld16(tm + lane_base + T_DW + t * TILE, w);
+                wait_ld();
+#pragma unroll
+                for (int rr = 0; rr < TILE; ++rr)
+                    st_f32(sm, B1 + t * B1_SZ + off_kmajor(rr, c, PAD_LBO, GA_SBO), to_tf32(w[rr]));
+            }
+        }
+        fence_smem_to_async();
+        cta_sync_tc();
+        if (s_abort) break;
+
+        // ---- phase 6: the sequential state chain over the two tiles ----------
+#pragma unroll 1
+        for (int t = 0; t < 2; ++t) {
+            if (tid == 0) {
+                const uint32_t id = idesc_tf32(128, 32, false, false);
+#pragma unroll 1
+                for (int ks = 0; ks < D / 8; ++ks) {
+                    const uint64_t bd = sdesc(smem_u32(sm + B1 + t * B1_SZ) + ks * 2 * PAD_LBO, PAD_LBO, GA_SBO);
+                    mma_tf32_ts(tm + T_DX, tm + T_AS + ks * 8, bd, id, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(bar);
+            }
+            __syncwarp();
+            wait_mma();
+            {   // U = U' - W S  (thread j, 16 tokens)
+                float x[16], up[16];
+                tmem_ld16(tm + lane_base + T_DX, x);
+                tmem_ld16(tm + lane_base + T_DU + t * TILE, up);
+                wait_ld();
+#pragma unroll
+                for (int r = 0; r < TILE; ++r) x[r] = to_tf32(up[r] - x[r]);
+                tmem_st16(tm + lane_base + T_AU, x);
+                wait_st();
+            }
+            cta_sync_tc();
+            if (tid == 0) {
+                const uint32_t id2 = idesc_tf32(128, 128, false, false);
+                const uint32_t id3 = idesc_tf32(128, 16, false, false);
+#pragma unroll 1
+                for (int ks = 0; ks < TILE / 8; ++ks) {
+                    const uint64_t b2 = sdesc(smem_u32(sm + B2 + t * B2_SZ) + ks * 2 * LBO, LBO, B2_SBO);
+                    const uint64_t b3 = sdesc(smem_u32(sm + B3 + t * B3_SZ) + ks * 2 * PAD_LBO, PAD_LBO, B3_SBO);
+                    mma_tf32_ts(tm + T_DKU, tm + T_AU + ks * 8, b2, id2, ks > 0 ? 1u : 0u);
+                    mma_tf32_ts(tm + T_DX + TILE, tm + T_AU + ks * 8, b3, id3, 1u);
+                }
+                mma_commit(bar);
+            }
+            __syncwarp();
+            wait_mma();
+            {   // S <- Diag(gamma_16) S + Kb^T U ; refresh the tf32 copy; emit o
+                const float* gam = reinterpret_cast<const float*>(sm + GAM) + t * D;
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    float d[32];
+                    tmem_ld32(tm + lane_base + T_DKU + c0, d);
+                    wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        S[c0 + i] = fmaf(gam[c0 + i], S[c0 + i], d[i]);
+                        d[i] = to_tf32(S[c0 + i]);
+                    }
+                    tmem_st32(tm + lane_base + T_AS + c0, d);
+                }
+                float ov[16];
+                tmem_ld16(tm + lane_base + T_DX + TILE, ov);
+                wait_ld();
+                wait_st();
+                const int tb = t0 + t * TILE;
+#pragma unroll
+                for (int r = 0; r < TILE; ++r)
+                    if (tb + r < T) oh[(int64_t)(tb + r) * row_stride + j] = __float2bfloat16_rn(ov[r]);
+            }
+            cta_sync_tc();
+            if (s_abort) break;
+        }
+        if (s_abort) break;
+    }
+
+    if (hT && !s_abort) {
+        float* hTh = hT + head_off * D * D;
+#pragma unroll
+        for (int c = 0; c < D; ++c) hTh[(int64_t)c * D + j] = S[c];
+    }
+    cta_sync_tc();
+    if (warp == 0) tmem_dealloc(tm, TMEM_COLS);
+}
+
+cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
+                              const void* beta, const float* h0, void* o, float* hT,
+                              int B, int T, int H, cudaStream_t stream)
+{
+    static bool attr_set = false;   // idempotent; races only repeat the same call
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)pf::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    dim3 grid(H, B);
+    prefill_tc_kernel<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(
+        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+        (const __nv_bfloat16*)g, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
+// Reads and clears the timeout flag of the prefill kernels (blocking).
+int prefill_device_status(cudaStream_t stream)
+{
+    int st = 0, zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&st, g_prefill_status, sizeof(int), 0,
+                                  cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (cudaMemcpyToSymbolAsync(g_prefill_status, &zero, sizeof(int), 0,
+                                cudaMemcpyHostToDevice, stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
+    return st;
+}
+
+}  // namespace kda

@@ -158,6 +158,7 @@ def test_workload_prefill_8k_full():
     x = prefill_inputs(w.B, w.T, w.H, w.dk, w.dv, seed=w.seed, h0_std=w.h0_std)
     o, hT = run_prefill(x)
     check_prefill(x, o, hT, TOL_BF16)
+    assert kda.device_status() == kda.KDA_OK
 
 
 def test_workload_pretrain_64k_sampled():
