@@ -51,11 +51,9 @@ constexpr uint32_t PAD_LBO = 144;            // padded K-direction core-matrix s
 constexpr uint32_t LBO = 128;                // dense K-direction core-matrix stride
 
 // shared memory map (bytes)
-constexpr uint32_t RAW_Q = 0;
-constexpr uint32_t RAW_K = RAW_Q + GRP * D * 2;
-constexpr uint32_t RAW_V = RAW_K + GRP * D * 2;
-constexpr uint32_t RAW_G = RAW_V + GRP * D * 2;
-constexpr uint32_t BETA = RAW_G + GRP * D * 2;                 // GRP fp32
+constexpr uint32_t RAW_SZ = 4 * GRP * D * 2;                 // q, k, v, g of one group (bf16)
+constexpr uint32_t RAW = 0;                                    // two buffers (prefetch)
+constexpr uint32_t BETA = RAW + 2 * RAW_SZ;                    // GRP fp32
 constexpr uint32_t GA = BETA + 128;                            // Kh, 32 rows x K 128 (padded)
 constexpr uint32_t GA_SBO = (D / 4) * PAD_LBO;                 // 4608
 constexpr uint32_t GB = GA + (GRP / 8) * GA_SBO;               // [Kt | Qt], 64 rows x K 128
@@ -99,6 +97,14 @@ __device__ int g_prefill_status;   // set to KDA_ERR_TIMEOUT by a wait that expi
 __device__ __forceinline__ void st_f32(unsigned char* base, uint32_t off, float v) {
     *reinterpret_cast<float*>(base + off) = v;
 }
+
+// 16-byte asynchronous global->shared copy; src_bytes = 0 writes zeros
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                 :: "r"(tc::smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 __global__ void __launch_bounds__(pf::NT, 1)
 prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
@@ -174,23 +180,45 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     };
 
     const int n_groups = (T + GRP - 1) / GRP;
-    for (int grp = 0; grp < n_groups; ++grp) {
-        const int t0 = grp * GRP;
-
-        // ---- phase 0: raw tile inputs (bf16) into shared memory, zero past T
-        for (int idx = tid; idx < 4 * GRP * (D / 8); idx += NT) {
+    // asynchronous copy of group `gi`'s q, k, v, g rows into raw buffer gi & 1
+    auto issue_raw = [&](int gi) {
+        const int tb = gi * GRP;
+        unsigned char* dst0 = sm + RAW + (gi & 1) * RAW_SZ;
+#pragma unroll
+        for (int it = 0; it < (4 * GRP * (D / 8)) / NT; ++it) {
+            const int idx = tid + it * NT;
             const int tensor = idx / (GRP * (D / 8));
             const int rem = idx % (GRP * (D / 8));
             const int r = rem / (D / 8), vec = rem % (D / 8);
             const __nv_bfloat16* src = tensor == 0 ? qh : tensor == 1 ? kh : tensor == 2 ? vh : gh;
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (t0 + r < T) val = *reinterpret_cast<const uint4*>(src + (int64_t)(t0 + r) * row_stride + vec * 8);
-            *reinterpret_cast<uint4*>(sm + RAW_Q + tensor * (GRP * D * 2) + (r * D + vec * 8) * 2) = val;
+            const bool in = tb + r < T;
+            cp_async16(dst0 + tensor * (GRP * D * 2) + (r * D + vec * 8) * 2,
+                       in ? (const void*)(src + (int64_t)(tb + r) * row_stride + vec * 8) : (const void*)src,
+                       in ? 16u : 0u);
         }
-        if (tid < GRP)
-            reinterpret_cast<float*>(sm + BETA)[tid] =
-                (t0 + tid < T) ? to_f32(bh[(int64_t)(t0 + tid) * H]) : 0.f;
+    };
+    float beta_cur = 0.f;
+    if (n_groups > 0) {
+        issue_raw(0);
+        cp_async_commit();
+        beta_cur = (tid < GRP && tid < T) ? to_f32(bh[(int64_t)tid * H]) : 0.f;
+    }
+    for (int grp = 0; grp < n_groups; ++grp) {
+        const int t0 = grp * GRP;
+
+        // ---- phase 0: prefetch the next group's inputs; wait for this one's
+        if (grp + 1 < n_groups) issue_raw(grp + 1);
+        cp_async_commit();
+        const float beta_next = (grp + 1 < n_groups && tid < GRP && t0 + GRP + tid < T)
+                                    ? to_f32(bh[(int64_t)(t0 + GRP + tid) * H]) : 0.f;
+        cp_async_wait_1();
+        if (tid < GRP) reinterpret_cast<float*>(sm + BETA)[tid] = beta_cur;
+        beta_cur = beta_next;
         __syncthreads();
+        const uint32_t RAW_Q = RAW + (grp & 1) * RAW_SZ;
+        const uint32_t RAW_K = RAW_Q + GRP * D * 2;
+        const uint32_t RAW_V = RAW_K + GRP * D * 2;
+        const uint32_t RAW_G = RAW_V + GRP * D * 2;
 
         // ---- phase 1: decay scaling; thread c = key channel -----------------
         {
@@ -346,13 +374,21 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
 #pragma unroll 1
         for (int t = 0; t < 2; ++t) {
             if (tid == 0) {
-                const uint32_t id = idesc_tf32(128, 32, false, false);
+                // W part (rows 0-15 of B1) first: the chain waits only on it
+                const uint32_t id = idesc_tf32(128, 16, false, false);
 #pragma unroll 1
                 for (int ks = 0; ks < D / 8; ++ks) {
                     const uint64_t bd = sdesc(smem_u32(sm + B1 + t * B1_SZ) + ks * 2 * PAD_LBO, PAD_LBO, GA_SBO);
                     mma_tf32_ts(tm + T_DX, tm + T_AS + ks * 8, bd, id, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(bar);
+                // Qt part (rows 16-31): completes behind the U computation
+#pragma unroll 1
+                for (int ks = 0; ks < D / 8; ++ks) {
+                    const uint64_t bd = sdesc(smem_u32(sm + B1 + t * B1_SZ + 2 * GA_SBO) + ks * 2 * PAD_LBO,
+                                              PAD_LBO, GA_SBO);
+                    mma_tf32_ts(tm + T_DX + TILE, tm + T_AS + ks * 8, bd, id, ks > 0 ? 1u : 0u);
+                }
             }
             __syncwarp();
             wait_mma();
