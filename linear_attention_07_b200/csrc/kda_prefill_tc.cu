@@ -81,10 +81,11 @@ constexpr uint32_t PMS = AMS + C * LD * 4;                     // P
 constexpr uint32_t XMS = PMS + C * LD * 4;                     // diagonal-block inverses
 constexpr uint32_t TMS = XMS + C * LD * 4;                     // T
 constexpr uint32_t YMS = TMS + C * LD * 4;                     // A_10 X_00 (16 x 17)
-constexpr uint32_t SMEM_BYTES = YMS + TILE * (TILE + 1) * 4;
+constexpr uint32_t OST = YMS + TILE * (TILE + 1) * 4;           // o staging, 32 x 128 bf16
+constexpr uint32_t SMEM_BYTES = OST + C * D * 2;
 
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(GA % 16 == 0 && GB % 16 == 0 && WA % 16 == 0 && VA % 16 == 0 && TB % 16 == 0 &&
+static_assert(OST % 16 == 0 && GA % 16 == 0 && GB % 16 == 0 && WA % 16 == 0 && VA % 16 == 0 && TB % 16 == 0 &&
               B1 % 16 == 0 && B2 % 16 == 0 && B3 % 16 == 0, "descriptor alignment");
 
 // tensor memory columns (512 allocated)
@@ -198,21 +199,17 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             named_bar(BAR_READY, NT);
             fence_after_sync();
             if (s_abort) break;
-            // X = S^T [W | Qt]^T: the W half first (the chain waits on it only)
+            // X = S^T [W | Qt]^T  (one N = 64 MMA per K step; the issue loop is
+            // unrolled with constant descriptor increments: the per-instruction
+            // issue cost, not the math, bounds these small-N MMAs)
             if (j == 0) {
-                const uint32_t id = idesc_tf32(128, 32, false, false);
-#pragma unroll 1
-                for (int ks = 0; ks < D / 8; ++ks) {
-                    const uint64_t bd = sdesc(smem_u32(sm + B1) + ks * 2 * PAD_LBO, PAD_LBO, SBO_K128P);
-                    mma_tf32_ts(tm + T_DX, tm + T_AS + ks * 8, bd, id, ks > 0 ? 1u : 0u);
-                }
+                const uint32_t id = idesc_tf32(128, 2 * C, false, false);
+                const uint64_t bd0 = sdesc(smem_u32(sm + B1), PAD_LBO, SBO_K128P);
+#pragma unroll
+                for (int ks = 0; ks < D / 8; ++ks)
+                    mma_tf32_ts(tm + T_DX, tm + T_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                id, ks > 0 ? 1u : 0u);
                 mma_commit(bar);
-#pragma unroll 1
-                for (int ks = 0; ks < D / 8; ++ks) {
-                    const uint64_t bd = sdesc(smem_u32(sm + B1 + 4 * SBO_K128P) + ks * 2 * PAD_LBO,
-                                              PAD_LBO, SBO_K128P);
-                    mma_tf32_ts(tm + T_DX + C, tm + T_AS + ks * 8, bd, id, ks > 0 ? 1u : 0u);
-                }
             }
             __syncwarp();
             wait_mma();
@@ -235,44 +232,61 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             if (j == 0) {
                 const uint32_t id2 = idesc_tf32(128, 128, false, false);
                 const uint32_t id3 = idesc_tf32(128, 32, false, false);
-#pragma unroll 1
+                const uint64_t b20 = sdesc(smem_u32(sm + B2), LBO, SBO_K32);
+                const uint64_t b30 = sdesc(smem_u32(sm + B3), PAD_LBO, SBO_K32P);
+#pragma unroll
                 for (int ks = 0; ks < C / 8; ++ks) {
-                    const uint64_t b2 = sdesc(smem_u32(sm + B2) + ks * 2 * LBO, LBO, SBO_K32);
-                    const uint64_t b3 = sdesc(smem_u32(sm + B3) + ks * 2 * PAD_LBO, PAD_LBO, SBO_K32P);
-                    mma_tf32_ts(tm + T_DKU, tm + T_AU + ks * 8, b2, id2, ks > 0 ? 1u : 0u);
-                    mma_tf32_ts(tm + T_DX + C, tm + T_AU + ks * 8, b3, id3, 1u);
+                    mma_tf32_ts(tm + T_DKU, tm + T_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                id2, ks > 0 ? 1u : 0u);
+                    mma_tf32_ts(tm + T_DX + C, tm + T_AU + ks * 8, b30 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                id3, 1u);
                 }
                 mma_commit(bar);
             }
             __syncwarp();
             wait_mma();
             {   // S <- Diag(gamma_C) S + Kb^T U ; refresh the tf32 copy; emit o
-                const float* gam = reinterpret_cast<const float*>(sm + GAM);
+                const float4* gam4 = reinterpret_cast<const float4*>(sm + GAM);
 #pragma unroll
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     float d[32];
                     tmem_ld32(tm + lane_base + T_DKU + c0, d);
                     wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        S[c0 + i] = fmaf(gam[c0 + i], S[c0 + i], d[i]);
-                        d[i] = to_tf32(S[c0 + i]);
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 gv = gam4[(c0 >> 2) + i4];
+                        const float gg[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int i = i4 * 4 + u;
+                            S[c0 + i] = fmaf(gg[u], S[c0 + i], d[i]);
+                            d[i] = to_tf32(S[c0 + i]);
+                        }
                     }
                     tmem_st32(tm + lane_base + T_AS + c0, d);
                 }
-                const int tb = ch * C;
+                // o: column j of the chunk's 32 x 128 tile into shared memory,
+                // then whole rows to global memory in 16-byte vectors
+                __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OST);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     float ov[16];
                     tmem_ld16(tm + lane_base + T_DX + C + half * 16, ov);
                     wait_ld();
 #pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        const int t = tb + half * 16 + r;
-                        if (t < T) oh[(int64_t)t * row_stride + j] = __float2bfloat16_rn(ov[r]);
-                    }
+                    for (int r = 0; r < 16; ++r) ost[(half * 16 + r) * D + j] = __float2bfloat16_rn(ov[r]);
                 }
                 wait_st();
+                named_bar(BAR_CHAIN, 128);
+                const int tb = ch * C;
+#pragma unroll
+                for (int m = 0; m < (C * D / 8) / 128; ++m) {
+                    const int vi = j + m * 128;
+                    const int r = vi / (D / 8), cv = vi % (D / 8);
+                    if (tb + r < T)
+                        *reinterpret_cast<uint4*>(oh + (int64_t)(tb + r) * row_stride + cv * 8) =
+                            *reinterpret_cast<const uint4*>(ost + r * D + cv * 8);
+                }
             }
         }
         if (hT && !s_abort) {
@@ -342,12 +356,22 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                 const __nv_bfloat162* rk = reinterpret_cast<const __nv_bfloat162*>(sm + RAW + 1 * RAW_T);
                 const __nv_bfloat162* rv = reinterpret_cast<const __nv_bfloat162*>(sm + RAW + 2 * RAW_T);
                 const __nv_bfloat162* rg = reinterpret_cast<const __nv_bfloat162*>(sm + RAW + 3 * RAW_T);
+                // all shared-memory reads of this slice first (independent of the
+                // stores below, so they are not ordered behind them)
+                __nv_bfloat162 Rq[TILE], Rk[TILE], Rv[TILE], Rg[TILE];
+#pragma unroll
+                for (int rr = 0; rr < TILE; ++rr) {
+                    const int idx = ((tau * TILE + rr) * D + c0) >> 1;
+                    Rq[rr] = rq[idx];
+                    Rk[rr] = rk[idx];
+                    Rv[rr] = rv[idx];
+                    Rg[rr] = rg[idx];
+                }
                 float a0[TILE], a1[TILE];
                 float e0 = 1.f, e1 = 1.f;
 #pragma unroll
                 for (int rr = 0; rr < TILE; ++rr) {
-                    const int r = tau * TILE + rr;
-                    const float2 gg = __bfloat1622float2(rg[(r * D + c0) >> 1]);
+                    const float2 gg = __bfloat1622float2(Rg[rr]);
                     a0[rr] = __expf(gg.x);
                     a1[rr] = __expf(gg.y);
                     e0 *= a0[rr];
@@ -371,8 +395,8 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                     const int r = tau * TILE + rr;
                     p0 *= a0[rr];
                     p1 *= a1[rr];
-                    const float2 kk = __bfloat1622float2(rk[(r * D + c0) >> 1]);
-                    const float2 qq = __bfloat1622float2(rq[(r * D + c0) >> 1]);
+                    const float2 kk = __bfloat1622float2(Rk[rr]);
+                    const float2 qq = __bfloat1622float2(Rq[rr]);
                     const float kt0 = kk.x * p0, kt1 = kk.y * p1;
                     const float qt0 = qq.x * p0, qt1 = qq.y * p1;
                     st_f32x2(sm, GB + off_kmajor(r, c0, PAD_LBO, SBO_K128P), to_tf32(kt0), to_tf32(kt1));
@@ -394,7 +418,7 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
 #pragma unroll
                 for (int rr = TILE - 1; rr >= 0; --rr) {
                     const int r = tau * TILE + rr;
-                    const float2 kk = __bfloat1622float2(rk[(r * D + c0) >> 1]);
+                    const float2 kk = __bfloat1622float2(Rk[rr]);
                     const float kb0 = kk.x * s0, kb1 = kk.y * s1;
                     st_f32x2(sm, GA + off_kmajor(r, c0, PAD_LBO, SBO_K128P), to_tf32(kb0 * i0), to_tf32(kb1 * i1));
                     if (tau == 0)
@@ -410,7 +434,7 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                     const int r = tau * TILE + rr;
                     float2 vv[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) vv[u] = __bfloat1622float2(rv[((r + u) * D + c0) >> 1]);
+                    for (int u = 0; u < 4; ++u) vv[u] = __bfloat1622float2(Rv[rr + u]);
                     st_f32x4(sm, VA + off_kmajor(c0, r, LBO, SBO_K32),
                              to_tf32(vv[0].x), to_tf32(vv[1].x), to_tf32(vv[2].x), to_tf32(vv[3].x));
                     st_f32x4(sm, VA + off_kmajor(c0 + 1, r, LBO, SBO_K32),
@@ -426,11 +450,12 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             // ---- Gram: D_G = [Kh_0; Kh_1; Kb_0; pad] [Kt_0 Kt_1 | Qt_0 Qt_1]^T
             if (pt == 0) {
                 const uint32_t id = idesc_tf32(64, 64, false, false);
-#pragma unroll 1
+                const uint64_t ad0 = sdesc(smem_u32(sm + GA), PAD_LBO, SBO_K128P);
+                const uint64_t bd0 = sdesc(smem_u32(sm + GB), PAD_LBO, SBO_K128P);
+#pragma unroll
                 for (int ks = 0; ks < D / 8; ++ks) {
-                    const uint64_t ad = sdesc(smem_u32(sm + GA) + ks * 2 * PAD_LBO, PAD_LBO, SBO_K128P);
-                    const uint64_t bd = sdesc(smem_u32(sm + GB) + ks * 2 * PAD_LBO, PAD_LBO, SBO_K128P);
-                    mma_tf32_ss(tm + T_DG, ad, bd, id, ks > 0 ? 1u : 0u);
+                    const uint64_t step = (uint64_t)((ks * 2 * PAD_LBO) >> 4);
+                    mma_tf32_ss(tm + T_DG, ad0 + step, bd0 + step, id, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(bar);
             }
@@ -530,13 +555,16 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             // ---- W^T = Kt^T T^T and U'^T = V^T T^T  (M 128, N 32, K 32)
             if (pt == 0) {
                 const uint32_t id = idesc_tf32(128, 32, false, false);
-#pragma unroll 1
+                const uint64_t bd0 = sdesc(smem_u32(sm + TB), PAD_LBO, SBO_K32P);
+                const uint64_t aw0 = sdesc(smem_u32(sm + WA), LBO, SBO_K32);
+                const uint64_t av0 = sdesc(smem_u32(sm + VA), LBO, SBO_K32);
+                const uint32_t du = tm + T_DU + (ch & 1) * C;
+#pragma unroll
                 for (int ks = 0; ks < C / 8; ++ks) {
-                    const uint64_t bd = sdesc(smem_u32(sm + TB) + ks * 2 * PAD_LBO, PAD_LBO, SBO_K32P);
-                    const uint64_t aw = sdesc(smem_u32(sm + WA) + ks * 2 * LBO, LBO, SBO_K32);
-                    const uint64_t av = sdesc(smem_u32(sm + VA) + ks * 2 * LBO, LBO, SBO_K32);
-                    mma_tf32_ss(tm + T_DW, aw, bd, id, ks > 0 ? 1u : 0u);
-                    mma_tf32_ss(tm + T_DU + (ch & 1) * C, av, bd, id, ks > 0 ? 1u : 0u);
+                    const uint64_t bstep = (uint64_t)((ks * 2 * PAD_LBO) >> 4);
+                    const uint64_t astep = (uint64_t)((ks * 2 * LBO) >> 4);
+                    mma_tf32_ss(tm + T_DW, aw0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                    mma_tf32_ss(du, av0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
                 }
                 mma_commit(bar);
             }
