@@ -42,6 +42,9 @@
 // Shared-memory operands use the no-swizzle K-major layout; when the thread
 // that produces a value owns the K index, the K-direction core-matrix stride
 // is padded to 144 B so that a warp's scalar stores hit distinct banks.
+#include <cuda.h>
+#include <string.h>
+
 #include "kda_common.cuh"
 #include "kda_tc.cuh"
 
@@ -52,7 +55,9 @@ namespace pf {
 constexpr int D = 128;         // d_k = d_v
 constexpr int TILE = 16;
 constexpr int C = 32;          // tokens per chunk (two tiles)
-constexpr int NT = 256;        // threads per CTA: chain + prep warpgroups
+constexpr int NCH = 256;       // chain threads (warps 0-7)
+constexpr int NPREP = 256;     // prep threads (warps 8-15)
+constexpr int NT = NCH + NPREP;
 
 constexpr uint32_t PAD_LBO = 144;            // padded K-direction core-matrix stride
 constexpr uint32_t LBO = 128;                // dense K-direction core-matrix stride
@@ -74,9 +79,9 @@ constexpr uint32_t TB = VA + (D / 8) * SBO_K32;                // T:    N 32 x K
 constexpr uint32_t B1 = TB + (C / 8) * SBO_K32P;               // [W | Qt]: N 64 x K 128 (padded)
 constexpr uint32_t B2 = B1 + 8 * SBO_K128P;                    // Kb:   N 128 x K 32
 constexpr uint32_t B3 = B2 + (D / 8) * SBO_K32;                // P:    N 32 x K 32 (padded)
-constexpr uint32_t GAM = B3 + (C / 8) * SBO_K32P;              // gamma_C, 128 fp32
+constexpr uint32_t GAM = B3 + (C / 8) * SBO_K32P;              // gamma_C, 2 x 128 fp32 (by chunk parity)
 constexpr int LD = C + 1;                                      // scratch row stride (floats)
-constexpr uint32_t AMS = GAM + D * 4;                          // A (32 x 33 fp32)
+constexpr uint32_t AMS = GAM + 2 * D * 4;                          // A (32 x 33 fp32)
 constexpr uint32_t PMS = AMS + C * LD * 4;                     // P
 constexpr uint32_t XMS = PMS + C * LD * 4;                     // diagonal-block inverses
 constexpr uint32_t TMS = XMS + C * LD * 4;                     // T
@@ -119,17 +124,14 @@ __device__ __forceinline__ void st_f32x4(unsigned char* base, uint32_t off, floa
 __device__ __forceinline__ void named_bar(uint32_t id, uint32_t count) {
     asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(count) : "memory");
 }
-// 16-byte asynchronous global->shared copy; src_bytes = 0 writes zeros
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-                 :: "r"(tc::smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
+
+__device__ __forceinline__ void named_arrive(uint32_t id, uint32_t count) {
+    asm volatile("bar.arrive %0, %1;" :: "r"(id), "r"(count) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __global__ void __launch_bounds__(pf::NT, 1)
-prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                  const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ g,
+prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                   const __nv_bfloat16* __restrict__ beta, const float* h0,
                   __nv_bfloat16* __restrict__ o, float* hT, int T, int H)
 {
@@ -137,7 +139,7 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     using namespace tc;
     extern __shared__ __align__(1024) unsigned char sm[];
     __shared__ uint32_t s_taddr;
-    __shared__ __align__(8) uint64_t s_bar[2];     // [0] chain MMAs, [1] prep MMAs
+    __shared__ __align__(8) uint64_t s_bar[3];     // chain MMAs, prep MMAs, input loads
     __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -153,6 +155,7 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     if (tid == 0) {
         mbar_init(smem_u32(&s_bar[0]), 1);
         mbar_init(smem_u32(&s_bar[1]), 1);
+        mbar_init(smem_u32(&s_bar[2]), 1);
         fence_mbar_init();
         s_abort = 0;
     }
@@ -160,34 +163,43 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     __syncthreads();
     fence_after_sync();
     const uint32_t tm = s_taddr;
-    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's TMEM lanes
+    const int sp = warp & 3;                                   // TMEM sub-partition of this warp
+    const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
     const int n_chunks = (T + C - 1) / C;
+    // A wait that expired sets s_abort; from then on both roles skip all MMA
+    // work but keep the barrier protocol, so the CTA winds down without
+    // further waits and reports KDA_ERR_TIMEOUT.
+    auto expired = [&]() {
+        s_abort = 1;
+        atomicExch(&g_prefill_status, (int)KDA_ERR_TIMEOUT);
+    };
 
-    if (warp < 4) {
-        // =================================================== chain warpgroup ==
-        const int j = tid;
+    if (tid < NCH) {
+        // =================================================== chain warpgroups ==
+        // thread: state column j (tensor-memory lane), key rows [64 hh, 64 hh + 64)
+        const int j = 32 * sp + lane;
+        const int hh = warp >> 2;
         const uint32_t bar = smem_u32(&s_bar[0]);
         uint32_t phase = 0;
+        // one thread polls the MMA barrier; the others block on a named barrier
         auto wait_mma = [&]() {
-            const bool ok = mbar_wait(bar, phase & 1u, WAIT_NS);
+            if (tid == 0 && !s_abort && !mbar_wait(bar, phase & 1u, WAIT_NS)) expired();
             ++phase;
-            if (!ok) {
-                s_abort = 1;
-                atomicExch(&g_prefill_status, (int)KDA_ERR_TIMEOUT);
-            }
+            __syncwarp();
+            named_bar(BAR_CHAIN, NCH);
             fence_after_sync();
         };
-        float S[D];
+        float S[D / 2];
         {
             const float* h0h = h0 ? h0 + head_off * D * D : nullptr;
 #pragma unroll
-            for (int c = 0; c < D; ++c) S[c] = h0h ? h0h[(int64_t)c * D + j] : 0.f;
+            for (int i = 0; i < D / 2; ++i) S[i] = h0h ? h0h[(int64_t)(64 * hh + i) * D + j] : 0.f;
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = 0; c0 < D / 2; c0 += 32) {
                 float t32[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) t32[i] = to_tf32(S[c0 + i]);
-                tmem_st32(tm + lane_base + T_AS + c0, t32);
+                tmem_st32(tm + lane_base + T_AS + 64 * hh + c0, t32);
             }
             wait_st();
         }
@@ -195,14 +207,12 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
 #pragma unroll 1
         for (int ch = 0; ch < n_chunks; ++ch) {
             fence_before_sync();
-            named_bar(BAR_FREE, NT);
-            named_bar(BAR_READY, NT);
+            named_bar(BAR_READY, NT);        // this chunk's operands are in place
             fence_after_sync();
-            if (s_abort) break;
             // X = S^T [W | Qt]^T  (one N = 64 MMA per K step; the issue loop is
             // unrolled with constant descriptor increments: the per-instruction
             // issue cost, not the math, bounds these small-N MMAs)
-            if (j == 0) {
+            if (tid == 0 && !s_abort) {
                 const uint32_t id = idesc_tf32(128, 2 * C, false, false);
                 const uint64_t bd0 = sdesc(smem_u32(sm + B1), PAD_LBO, SBO_K128P);
 #pragma unroll
@@ -211,25 +221,21 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                                 id, ks > 0 ? 1u : 0u);
                 mma_commit(bar);
             }
-            __syncwarp();
             wait_mma();
-            {   // U = U' - W S (thread j: 32 tokens)
+            {   // U = U' - W S  (this half: tokens [16 hh, 16 hh + 16))
                 float x[16], up[16];
+                tmem_ld16(tm + lane_base + T_DX + 16 * hh, x);
+                tmem_ld16(tm + lane_base + T_DU + (ch & 1) * C + 16 * hh, up);
+                wait_ld();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld16(tm + lane_base + T_DX + half * 16, x);
-                    tmem_ld16(tm + lane_base + T_DU + (ch & 1) * C + half * 16, up);
-                    wait_ld();
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) x[r] = to_tf32(up[r] - x[r]);
-                    tmem_st16(tm + lane_base + T_AU + half * 16, x);
-                }
+                for (int r = 0; r < 16; ++r) x[r] = to_tf32(up[r] - x[r]);
+                tmem_st16(tm + lane_base + T_AU + 16 * hh, x);
                 wait_st();
             }
             fence_before_sync();
-            named_bar(BAR_CHAIN, 128);
+            named_bar(BAR_CHAIN, NCH);
             fence_after_sync();
-            if (j == 0) {
+            if (tid == 0 && !s_abort) {
                 const uint32_t id2 = idesc_tf32(128, 128, false, false);
                 const uint32_t id3 = idesc_tf32(128, 32, false, false);
                 const uint64_t b20 = sdesc(smem_u32(sm + B2), LBO, SBO_K32);
@@ -243,95 +249,90 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                 }
                 mma_commit(bar);
             }
-            __syncwarp();
             wait_mma();
+            // B1, B2, B3 are no longer read: the prep may fill the next chunk's
+            // while the state update and the output store run
+            if (ch + 1 < n_chunks) named_arrive(BAR_FREE, NT);
             {   // S <- Diag(gamma_C) S + Kb^T U ; refresh the tf32 copy; emit o
-                const float4* gam4 = reinterpret_cast<const float4*>(sm + GAM);
+                const float4* gam4 = reinterpret_cast<const float4*>(sm + GAM + (ch & 1) * D * 4) + 16 * hh;
 #pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    float d[32];
-                    tmem_ld32(tm + lane_base + T_DKU + c0, d);
+                for (int c0 = 0; c0 < D / 2; c0 += 16) {
+                    float d[16];
+                    tmem_ld16(tm + lane_base + T_DKU + 64 * hh + c0, d);
                     wait_ld();
 #pragma unroll
-                    for (int i4 = 0; i4 < 8; ++i4) {
+                    for (int i4 = 0; i4 < 4; ++i4) {
                         const float4 gv = gam4[(c0 >> 2) + i4];
                         const float gg[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            const int i = i4 * 4 + u;
-                            S[c0 + i] = fmaf(gg[u], S[c0 + i], d[i]);
-                            d[i] = to_tf32(S[c0 + i]);
+                            const int i = c0 + i4 * 4 + u;
+                            S[i] = fmaf(gg[u], S[i], d[i - c0]);
+                            d[i - c0] = to_tf32(S[i]);
                         }
                     }
-                    tmem_st32(tm + lane_base + T_AS + c0, d);
+                    tmem_st16(tm + lane_base + T_AS + 64 * hh + c0, d);
                 }
-                // o: column j of the chunk's 32 x 128 tile into shared memory,
-                // then whole rows to global memory in 16-byte vectors
+                // o: this half's 16 tokens of column j into shared memory, then
+                // whole rows to global memory in 16-byte vectors
                 __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OST);
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
+                {
                     float ov[16];
-                    tmem_ld16(tm + lane_base + T_DX + C + half * 16, ov);
+                    tmem_ld16(tm + lane_base + T_DX + C + 16 * hh, ov);
                     wait_ld();
 #pragma unroll
-                    for (int r = 0; r < 16; ++r) ost[(half * 16 + r) * D + j] = __float2bfloat16_rn(ov[r]);
+                    for (int r = 0; r < 16; ++r) ost[(16 * hh + r) * D + j] = __float2bfloat16_rn(ov[r]);
                 }
                 wait_st();
-                named_bar(BAR_CHAIN, 128);
+                named_bar(BAR_CHAIN, NCH);
                 const int tb = ch * C;
 #pragma unroll
-                for (int m = 0; m < (C * D / 8) / 128; ++m) {
-                    const int vi = j + m * 128;
+                for (int m = 0; m < (C * D / 8) / NCH; ++m) {
+                    const int vi = tid + m * NCH;
                     const int r = vi / (D / 8), cv = vi % (D / 8);
                     if (tb + r < T)
                         *reinterpret_cast<uint4*>(oh + (int64_t)(tb + r) * row_stride + cv * 8) =
                             *reinterpret_cast<const uint4*>(ost + r * D + cv * 8);
                 }
+                named_bar(BAR_CHAIN, NCH);   // staging read before the next chunk writes it
             }
         }
         if (hT && !s_abort) {
             float* hTh = hT + head_off * D * D;
 #pragma unroll
-            for (int c = 0; c < D; ++c) hTh[(int64_t)c * D + j] = S[c];
+            for (int i = 0; i < D / 2; ++i) hTh[(int64_t)(64 * hh + i) * D + j] = S[i];
         }
     } else {
-        // ==================================================== prep warpgroup ==
-        const int pt = tid - 128;                  // 0..127
-        const int sp = warp & 3;                   // TMEM sub-partition of this warp
+        // ==================================================== prep warpgroups ==
+        const int pt = tid - NCH;                  // 0..255
+        const int pw = pt >> 5;                    // prep warp 0..7
         const uint32_t bar = smem_u32(&s_bar[1]);
-        uint32_t phase = 0;
+        const uint32_t rbar = smem_u32(&s_bar[2]);
+        uint32_t phase = 0, rphase = 0;
         auto wait_mma = [&]() {
-            const bool ok = mbar_wait(bar, phase & 1u, WAIT_NS);
+            if (pt == 0 && !s_abort && !mbar_wait(bar, phase & 1u, WAIT_NS)) expired();
             ++phase;
-            if (!ok) {
-                s_abort = 1;
-                atomicExch(&g_prefill_status, (int)KDA_ERR_TIMEOUT);
-            }
+            __syncwarp();
+            named_bar(BAR_PREP, NPREP);
             fence_after_sync();
         };
-        auto prep_sync = [&]() { named_bar(BAR_PREP, 128); };
-        auto issue_raw = [&](int ci) {   // cp.async of chunk ci's q, k, v, g rows
-            const int tb = ci * C;
-#pragma unroll
-            for (int it = 0; it < (4 * C * (D / 8)) / 128; ++it) {
-                const int idx = pt + it * 128;
-                const int tensor = idx / (C * (D / 8));
-                const int rem = idx % (C * (D / 8));
-                const int r = rem / (D / 8), vec = rem % (D / 8);
-                const bool in = tb + r < T;
-                const __nv_bfloat16* src = (tensor == 0 ? q : tensor == 1 ? k : tensor == 2 ? v : g) + base;
-                cp_async16(sm + RAW + tensor * RAW_T + (r * D + vec * 8) * 2,
-                           in ? (const void*)(src + (int64_t)(tb + r) * row_stride + vec * 8)
-                              : (const void*)src,
-                           in ? 16u : 0u);
+        auto prep_sync = [&]() { named_bar(BAR_PREP, NPREP); };
+        // TMA: chunk ci's q, k, v, g rows (32 x 128 bf16 each; rows past T are zero)
+        auto issue_raw = [&](int ci) {
+            if (pt == 0) {
+                mbar_arrive_expect_tx(rbar, 4 * RAW_T);
+                tma_load_3d(smem_u32(sm + RAW + 0 * RAW_T), &tm_q, h * D, ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + RAW + 1 * RAW_T), &tm_k, h * D, ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + RAW + 2 * RAW_T), &tm_v, h * D, ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + RAW + 3 * RAW_T), &tm_g, h * D, ci * C, b, rbar);
             }
-            cp_async_commit();
         };
         if (n_chunks > 0) issue_raw(0);
+        float beta_next = (pt < C && pt < T) ? to_f32(beta[((int64_t)b * T + pt) * H + h]) : 0.f;
 
-        // this thread's decay-scaling slice: tile tau, channels c0, c0 + 1
-        const int tau = pt >> 6;
-        const int c0 = (pt & 63) * 2;
+        // decay-scaling slice of this thread: tile tau, key channel c
+        const int tau = pt >> 7;
+        const int c = pt & 127;
         float* am = reinterpret_cast<float*>(sm + AMS);
         float* pm = reinterpret_cast<float*>(sm + PMS);
         float* xm = reinterpret_cast<float*>(sm + XMS);
@@ -340,115 +341,84 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         const float* bt = reinterpret_cast<const float*>(sm + BETA);
 #pragma unroll 1
         for (int ch = 0; ch < n_chunks; ++ch) {
-            const int t0 = ch * C;
-            // ---- inputs of this chunk
-            if (pt < C)
-                reinterpret_cast<float*>(sm + BETA)[pt] =
-                    (t0 + pt < T) ? to_f32(beta[((int64_t)b * T + t0 + pt) * H + h]) : 0.f;
-            cp_async_wait_all();
+            // ---- inputs of this chunk (beta prefetched one chunk ahead)
+            if (pt < C) {
+                reinterpret_cast<float*>(sm + BETA)[pt] = beta_next;
+                const int tn = (ch + 1) * C + pt;
+                beta_next = (tn < T) ? to_f32(beta[((int64_t)b * T + tn) * H + h]) : 0.f;
+            }
+            if (pt == 0 && !s_abort && !mbar_wait(rbar, rphase & 1u, WAIT_NS)) expired();
+            ++rphase;
+            __syncwarp();
             prep_sync();
 
-            // ---- decay scaling (thread: 16 tokens of tile tau x 2 channels)
-            float qtv[2][TILE], kbv[2][TILE];       // kept for the operand fill
-            float gam_c0, gam_c1;
+            // ---- decay scaling (thread: 16 tokens of tile tau, channel c)
+            float gam_c, fq, fk;                    // chunk-relative factors for the fill
+            float vr[TILE];
             {
-                const __nv_bfloat162* rq = reinterpret_cast<const __nv_bfloat162*>(sm + RAW + 0 * RAW_T);
-                const __nv_bfloat162* rk = reinterpret_cast<const __nv_bfloat162*>(sm + RAW + 1 * RAW_T);
-                const __nv_bfloat162* rv = reinterpret_cast<const __nv_bfloat162*>(sm + RAW + 2 * RAW_T);
-                const __nv_bfloat162* rg = reinterpret_cast<const __nv_bfloat162*>(sm + RAW + 3 * RAW_T);
-                // all shared-memory reads of this slice first (independent of the
-                // stores below, so they are not ordered behind them)
-                __nv_bfloat162 Rq[TILE], Rk[TILE], Rv[TILE], Rg[TILE];
+                const __nv_bfloat16* __restrict__ rq = reinterpret_cast<const __nv_bfloat16*>(sm + RAW + 0 * RAW_T);
+                const __nv_bfloat16* __restrict__ rk = reinterpret_cast<const __nv_bfloat16*>(sm + RAW + 1 * RAW_T);
+                const __nv_bfloat16* __restrict__ rv = reinterpret_cast<const __nv_bfloat16*>(sm + RAW + 2 * RAW_T);
+                const __nv_bfloat16* __restrict__ rg = reinterpret_cast<const __nv_bfloat16*>(sm + RAW + 3 * RAW_T);
+                // every shared-memory read of the slice first: later loads would
+                // otherwise be ordered behind the operand stores
+                float a[TILE], kr[TILE], qr[TILE];
 #pragma unroll
                 for (int rr = 0; rr < TILE; ++rr) {
-                    const int idx = ((tau * TILE + rr) * D + c0) >> 1;
-                    Rq[rr] = rq[idx];
-                    Rk[rr] = rk[idx];
-                    Rv[rr] = rv[idx];
-                    Rg[rr] = rg[idx];
+                    const int idx = (tau * TILE + rr) * D + c;
+                    kr[rr] = to_f32(rk[idx]);
+                    qr[rr] = to_f32(rq[idx]);
+                    vr[rr] = to_f32(rv[idx]);
+                    a[rr] = to_f32(rg[idx]);
                 }
-                float a0[TILE], a1[TILE];
-                float e0 = 1.f, e1 = 1.f;
+                float e = 1.f;
 #pragma unroll
                 for (int rr = 0; rr < TILE; ++rr) {
-                    const float2 gg = __bfloat1622float2(Rg[rr]);
-                    a0[rr] = __expf(gg.x);
-                    a1[rr] = __expf(gg.y);
-                    e0 *= a0[rr];
-                    e1 *= a1[rr];
+                    a[rr] = __expf(a[rr]);
+                    e *= a[rr];
                 }
                 float* gex = reinterpret_cast<float*>(sm + GEX);
-                gex[tau * D + c0] = e0;
-                gex[tau * D + c0 + 1] = e1;
+                gex[tau * D + c] = e;
                 prep_sync();
-                const float o0 = gex[(1 - tau) * D + c0], o1 = gex[(1 - tau) * D + c0 + 1];
-                // chunk-relative factors: tile 1 rows carry tile 0's decay
-                const float f0 = tau ? o0 : 1.f, f1 = tau ? o1 : 1.f;
-                gam_c0 = e0 * o0;
-                gam_c1 = e1 * o1;
-                // forward: Kt, Qt (tile-relative) for the Gram; Kt (chunk) for W;
-                // Qt (chunk) kept for the state product's B operand
-                float p0 = 1.f, p1 = 1.f;
-                float kc0[4], kc1[4];
+                const float oe = gex[(1 - tau) * D + c];
+                const float f = tau ? oe : 1.f;          // chunk-relative factor of tile 1 rows
+                gam_c = e * oe;
+                fq = f;
+                fk = tau ? e : oe;                       // Kb (chunk) from the stored Kh (tile 1) or Kb_0 (tile 0)
+                // forward: Kt, Qt (tile-relative) for the Gram; Kt (chunk) for W
+                float p = 1.f;
+                float kc[4];
 #pragma unroll
                 for (int rr = 0; rr < TILE; ++rr) {
                     const int r = tau * TILE + rr;
-                    p0 *= a0[rr];
-                    p1 *= a1[rr];
-                    const float2 kk = __bfloat1622float2(Rk[rr]);
-                    const float2 qq = __bfloat1622float2(Rq[rr]);
-                    const float kt0 = kk.x * p0, kt1 = kk.y * p1;
-                    const float qt0 = qq.x * p0, qt1 = qq.y * p1;
-                    st_f32x2(sm, GB + off_kmajor(r, c0, PAD_LBO, SBO_K128P), to_tf32(kt0), to_tf32(kt1));
-                    st_f32x2(sm, GB + off_kmajor(C + r, c0, PAD_LBO, SBO_K128P), to_tf32(qt0), to_tf32(qt1));
-                    qtv[0][rr] = to_tf32(qt0 * f0);
-                    qtv[1][rr] = to_tf32(qt1 * f1);
-                    kc0[rr & 3] = to_tf32(kt0 * f0);
-                    kc1[rr & 3] = to_tf32(kt1 * f1);
-                    if ((rr & 3) == 3) {
-                        st_f32x4(sm, WA + off_kmajor(c0, r - 3, LBO, SBO_K32), kc0[0], kc0[1], kc0[2], kc0[3]);
-                        st_f32x4(sm, WA + off_kmajor(c0 + 1, r - 3, LBO, SBO_K32), kc1[0], kc1[1], kc1[2], kc1[3]);
-                    }
+                    p *= a[rr];
+                    const float kt = kr[rr] * p;
+                    const float qt = qr[rr] * p;
+                    st_f32(sm, GB + off_kmajor(r, c, PAD_LBO, SBO_K128P), to_tf32(kt));
+                    st_f32(sm, GB + off_kmajor(C + r, c, PAD_LBO, SBO_K128P), to_tf32(qt));
+                    kc[rr & 3] = to_tf32(kt * f);
+                    if ((rr & 3) == 3)
+                        st_f32x4(sm, WA + off_kmajor(c, r - 3, LBO, SBO_K32), kc[0], kc[1], kc[2], kc[3]);
                 }
-                // backward: Kb (tile-relative suffix), Kh = Kb / gamma_tile,
-                // Kb (chunk-relative) kept for the update's B operand
-                const float i0 = 1.f / e0, i1 = 1.f / e1;
-                const float h0f = tau ? 1.f : o0, h1f = tau ? 1.f : o1;   // tile 0 rows carry tile 1's decay
-                float s0 = 1.f, s1 = 1.f;
+                // backward: Kb (tile-relative suffix) and Kh = Kb / gamma_tile
+                const float inv = 1.f / e;
+                float sgm = 1.f;
 #pragma unroll
                 for (int rr = TILE - 1; rr >= 0; --rr) {
                     const int r = tau * TILE + rr;
-                    const float2 kk = __bfloat1622float2(Rk[rr]);
-                    const float kb0 = kk.x * s0, kb1 = kk.y * s1;
-                    st_f32x2(sm, GA + off_kmajor(r, c0, PAD_LBO, SBO_K128P), to_tf32(kb0 * i0), to_tf32(kb1 * i1));
-                    if (tau == 0)
-                        st_f32x2(sm, GA + off_kmajor(C + rr, c0, PAD_LBO, SBO_K128P), to_tf32(kb0), to_tf32(kb1));
-                    kbv[0][rr] = to_tf32(kb0 * h0f);
-                    kbv[1][rr] = to_tf32(kb1 * h1f);
-                    s0 *= a0[rr];
-                    s1 *= a1[rr];
-                }
-                // V^T: thread's two value columns over its 16 tokens
-#pragma unroll
-                for (int rr = 0; rr < TILE; rr += 4) {
-                    const int r = tau * TILE + rr;
-                    float2 vv[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) vv[u] = __bfloat1622float2(Rv[rr + u]);
-                    st_f32x4(sm, VA + off_kmajor(c0, r, LBO, SBO_K32),
-                             to_tf32(vv[0].x), to_tf32(vv[1].x), to_tf32(vv[2].x), to_tf32(vv[3].x));
-                    st_f32x4(sm, VA + off_kmajor(c0 + 1, r, LBO, SBO_K32),
-                             to_tf32(vv[0].y), to_tf32(vv[1].y), to_tf32(vv[2].y), to_tf32(vv[3].y));
+                    const float kb = kr[rr] * sgm;
+                    st_f32(sm, GA + off_kmajor(r, c, PAD_LBO, SBO_K128P), to_tf32(kb * inv));
+                    if (tau == 0) st_f32(sm, GA + off_kmajor(C + rr, c, PAD_LBO, SBO_K128P), to_tf32(kb));
+                    sgm *= a[rr];
                 }
             }
             fence_smem_to_async();
             fence_before_sync();
-            prep_sync();                     // raw buffer consumed, operands written
+            prep_sync();                     // raw buffer consumed, Gram operands written
             fence_after_sync();
-            if (ch + 1 < n_chunks) issue_raw(ch + 1);
-
-            // ---- Gram: D_G = [Kh_0; Kh_1; Kb_0; pad] [Kt_0 Kt_1 | Qt_0 Qt_1]^T
-            if (pt == 0) {
+            // ---- Gram: D_G = [Kh_0; Kh_1; Kb_0; pad] [Kt_0 Kt_1 | Qt_0 Qt_1]^T,
+            // and the next chunk's inputs; V^T is written while the MMA runs
+            if (pt == 0 && !s_abort) {
                 const uint32_t id = idesc_tf32(64, 64, false, false);
                 const uint64_t ad0 = sdesc(smem_u32(sm + GA), PAD_LBO, SBO_K128P);
                 const uint64_t bd0 = sdesc(smem_u32(sm + GB), PAD_LBO, SBO_K128P);
@@ -459,11 +429,16 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                 }
                 mma_commit(bar);
             }
-            __syncwarp();
+            if (ch + 1 < n_chunks) issue_raw(ch + 1);
+#pragma unroll
+            for (int rr = 0; rr < TILE; rr += 4)
+                st_f32x4(sm, VA + off_kmajor(c, tau * TILE + rr, LBO, SBO_K32),
+                         to_tf32(vr[rr]), to_tf32(vr[rr + 1]), to_tf32(vr[rr + 2]), to_tf32(vr[rr + 3]));
+            fence_smem_to_async();
             wait_mma();
 
             // ---- A and P (32 x 32) into scratch; row m of D_G is lane (m % 16) + 32 (m / 16)
-            if (sp < 3) {
+            if (pw < 3) {
                 // sp 0: rows Kh_0 (cols Kt_0, Qt_0); sp 1: rows Kh_1 (cols Kt_1, Qt_1);
                 // sp 2: rows Kb_0 (cols Kt_1, Qt_1): the block between the tiles
                 const int colK = (sp == 0) ? 0 : TILE;
@@ -491,69 +466,57 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
             }
             prep_sync();
             // ---- diagonal blocks: X = (I + A_tt)^-1, column by column (right-looking)
-            if (sp < 2 && lane < TILE) {
-                const int off = sp * TILE;
+            if (pw < 2 && lane < TILE) {
+                const int off = pw * TILE;
                 const int i = lane;
                 float x[TILE];
 #pragma unroll
                 for (int r = 0; r < TILE; ++r) x[r] = (r == i) ? 1.f : 0.f;
 #pragma unroll
-                for (int s = 0; s < TILE; ++s) {
+                for (int s2 = 0; s2 < TILE; ++s2) {
 #pragma unroll
-                    for (int r = s + 1; r < TILE; ++r)
-                        x[r] = fmaf(-am[(off + r) * LD + off + s], x[s], x[r]);
+                    for (int r = s2 + 1; r < TILE; ++r)
+                        x[r] = fmaf(-am[(off + r) * LD + off + s2], x[s2], x[r]);
                 }
                 const float bi = bt[off + i];
 #pragma unroll
                 for (int r = 0; r < TILE; ++r) {
                     xm[(off + r) * LD + off + i] = x[r];
                     tmx[(off + r) * LD + off + i] = x[r] * bi;            // T_tt = X_tt diag(b)
-                    if (sp == 1) tmx[r * LD + off + i] = 0.f;            // T_01 = 0
+                    if (pw == 1) tmx[r * LD + off + i] = 0.f;            // T_01 = 0
                 }
             }
             prep_sync();
             // ---- off-diagonal block: T_10 = -X_11 (A_10 X_00) diag(b_0)
             {
-                const int r = pt >> 3, i = (pt & 7) * 2;
-                float y0 = 0.f, y1 = 0.f;
+                const int r = pt >> 4, i = pt & 15;
+                float y = 0.f;
 #pragma unroll
-                for (int s = 0; s < TILE; ++s) {
-                    const float a = am[(TILE + r) * LD + s];
-                    y0 = fmaf(a, xm[s * LD + i], y0);
-                    y1 = fmaf(a, xm[s * LD + i + 1], y1);
-                }
-                ym[r * (TILE + 1) + i] = y0;
-                ym[r * (TILE + 1) + i + 1] = y1;
+                for (int s2 = 0; s2 < TILE; ++s2) y = fmaf(am[(TILE + r) * LD + s2], xm[s2 * LD + i], y);
+                ym[r * (TILE + 1) + i] = y;
             }
             prep_sync();
             {
-                const int r = pt >> 3, i = (pt & 7) * 2;
-                float z0 = 0.f, z1 = 0.f;
+                const int r = pt >> 4, i = pt & 15;
+                float z = 0.f;
 #pragma unroll
-                for (int s = 0; s < TILE; ++s) {
-                    const float x = xm[(TILE + r) * LD + TILE + s];
-                    z0 = fmaf(x, ym[s * (TILE + 1) + i], z0);
-                    z1 = fmaf(x, ym[s * (TILE + 1) + i + 1], z1);
-                }
-                tmx[(TILE + r) * LD + i] = -z0 * bt[i];
-                tmx[(TILE + r) * LD + i + 1] = -z1 * bt[i + 1];
+                for (int s2 = 0; s2 < TILE; ++s2) z = fmaf(xm[(TILE + r) * LD + TILE + s2], ym[s2 * (TILE + 1) + i], z);
+                tmx[(TILE + r) * LD + i] = -z * bt[i];
             }
             prep_sync();
             // ---- T into the B operand of the W / U' products: element (n = r, k = i)
             {
-                const int r = pt >> 2, i = (pt & 3) * 8;
+                const int r = pt >> 3, i = (pt & 7) * 4;
                 const float* row = tmx + r * LD + i;
                 st_f32x4(sm, TB + off_kmajor(r, i, PAD_LBO, SBO_K32P),
                          to_tf32(row[0]), to_tf32(row[1]), to_tf32(row[2]), to_tf32(row[3]));
-                st_f32x4(sm, TB + off_kmajor(r, i + 4, PAD_LBO, SBO_K32P),
-                         to_tf32(row[4]), to_tf32(row[5]), to_tf32(row[6]), to_tf32(row[7]));
             }
             fence_smem_to_async();
             fence_before_sync();
             prep_sync();
             fence_after_sync();
             // ---- W^T = Kt^T T^T and U'^T = V^T T^T  (M 128, N 32, K 32)
-            if (pt == 0) {
+            if (pt == 0 && !s_abort) {
                 const uint32_t id = idesc_tf32(128, 32, false, false);
                 const uint64_t bd0 = sdesc(smem_u32(sm + TB), PAD_LBO, SBO_K32P);
                 const uint64_t aw0 = sdesc(smem_u32(sm + WA), LBO, SBO_K32);
@@ -568,65 +531,87 @@ prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
                 }
                 mma_commit(bar);
             }
-            __syncwarp();
+            // operands of the fill that do not come from the W MMA, read now
+            const float* gaf = reinterpret_cast<const float*>(sm + GA);
+            const float* gbf = reinterpret_cast<const float*>(sm + GB);
+            float qf[TILE], kf[TILE];
+#pragma unroll
+            for (int rr = 0; rr < TILE; ++rr) {
+                const int r = tau * TILE + rr;
+                qf[rr] = to_tf32(gbf[off_kmajor(C + r, c, PAD_LBO, SBO_K128P) >> 2] * fq);
+                const int row = tau ? (TILE + rr) : (C + rr);
+                kf[rr] = to_tf32(gaf[off_kmajor(row, c, PAD_LBO, SBO_K128P) >> 2] * fk);
+            }
+            float pf4[4];
+            {
+                const int r = pt >> 3, i = (pt & 7) * 4;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) pf4[u] = to_tf32(pm[r * LD + i + u]);
+            }
             wait_mma();
+            float w[16];
+            tmem_ld16(tm + lane_base + T_DW + 16 * tau, w);
+            wait_ld();
 
             // ---- hand the chunk's operands to the chain
-            fence_before_sync();
-            named_bar(BAR_FREE, NT);         // the chain no longer reads B1, B2, B3, GAM
-            fence_after_sync();
+            if (ch > 0) {
+                fence_before_sync();
+                named_bar(BAR_FREE, NT);     // the chain no longer reads B1, B2, B3
+                fence_after_sync();
+            }
             {
-                // W (thread = key channel pt): rows 0-31 of B1
-                float w[16];
+                // W (key channel c = TMEM lane, tokens [16 tau, 16 tau + 16)): rows 0-31 of B1
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld16(tm + lane_base + T_DW + half * 16, w);
-                    wait_ld();
-#pragma unroll
-                    for (int r = 0; r < 16; ++r)
-                        st_f32(sm, B1 + off_kmajor(half * 16 + r, pt, PAD_LBO, SBO_K128P), to_tf32(w[r]));
-                }
+                for (int r = 0; r < 16; ++r)
+                    st_f32(sm, B1 + off_kmajor(16 * tau + r, c, PAD_LBO, SBO_K128P), to_tf32(w[r]));
                 // Qt (chunk-relative): rows 32-63 of B1; Kb (chunk-relative): B2
 #pragma unroll
-                for (int rr = 0; rr < TILE; ++rr) {
-                    const int r = tau * TILE + rr;
-                    st_f32x2(sm, B1 + off_kmajor(C + r, c0, PAD_LBO, SBO_K128P), qtv[0][rr], qtv[1][rr]);
-                }
+                for (int rr = 0; rr < TILE; ++rr)
+                    st_f32(sm, B1 + off_kmajor(C + tau * TILE + rr, c, PAD_LBO, SBO_K128P), qf[rr]);
 #pragma unroll
-                for (int rr = 0; rr < TILE; rr += 4) {
-                    const int r = tau * TILE + rr;
-                    st_f32x4(sm, B2 + off_kmajor(c0, r, LBO, SBO_K32),
-                             kbv[0][rr], kbv[0][rr + 1], kbv[0][rr + 2], kbv[0][rr + 3]);
-                    st_f32x4(sm, B2 + off_kmajor(c0 + 1, r, LBO, SBO_K32),
-                             kbv[1][rr], kbv[1][rr + 1], kbv[1][rr + 2], kbv[1][rr + 3]);
-                }
+                for (int rr = 0; rr < TILE; rr += 4)
+                    st_f32x4(sm, B2 + off_kmajor(c, tau * TILE + rr, LBO, SBO_K32),
+                             kf[rr], kf[rr + 1], kf[rr + 2], kf[rr + 3]);
                 // P: element (n = r, k = i)
                 {
-                    const int r = pt >> 2, i = (pt & 3) * 8;
-                    const float* row = pm + r * LD + i;
-                    st_f32x4(sm, B3 + off_kmajor(r, i, PAD_LBO, SBO_K32P),
-                             to_tf32(row[0]), to_tf32(row[1]), to_tf32(row[2]), to_tf32(row[3]));
-                    st_f32x4(sm, B3 + off_kmajor(r, i + 4, PAD_LBO, SBO_K32P),
-                             to_tf32(row[4]), to_tf32(row[5]), to_tf32(row[6]), to_tf32(row[7]));
+                    const int r = pt >> 3, i = (pt & 7) * 4;
+                    st_f32x4(sm, B3 + off_kmajor(r, i, PAD_LBO, SBO_K32P), pf4[0], pf4[1], pf4[2], pf4[3]);
                 }
-                if (tau == 0) {
-                    float* gam = reinterpret_cast<float*>(sm + GAM);
-                    gam[c0] = gam_c0;
-                    gam[c0 + 1] = gam_c1;
-                }
+                if (tau == 0) reinterpret_cast<float*>(sm + GAM + (ch & 1) * D * 4)[c] = gam_c;
             }
             fence_smem_to_async();
             fence_before_sync();
-            named_bar(BAR_READY, NT);
-            fence_after_sync();
-            if (s_abort) break;
+            named_arrive(BAR_READY, NT);
         }
-        cp_async_wait_all();
     }
 
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, TMEM_COLS);
+}
+
+static bool make_map(CUtensorMap* map, const void* base, int B, int T, int H)
+{
+    typedef CUresult (*encode_fn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static encode_fn encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return false;
+        encode = (encode_fn)fn;
+    }
+    // [B][T][H * 128] bf16, box 128 x 32 x 1 (one head's 32 token rows)
+    const cuuint64_t dims[3] = {(cuuint64_t)H * pf::D, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)H * pf::D * 2, (cuuint64_t)T * H * pf::D * 2};
+    const cuuint32_t box[3] = {pf::D, pf::C, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
@@ -641,10 +626,18 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
+    CUtensorMap mq, mk, mv, mg;
+    if (T > 0) {
+        if (!make_map(&mq, q, B, T, H) || !make_map(&mk, k, B, T, H) ||
+            !make_map(&mv, v, B, T, H) || !make_map(&mg, g, B, T, H))
+            return cudaErrorInvalidValue;
+    } else {   // no chunk, no load: the kernel only carries h0 to hT
+        memset(&mq, 0, sizeof(mq)); memset(&mk, 0, sizeof(mk));
+        memset(&mv, 0, sizeof(mv)); memset(&mg, 0, sizeof(mg));
+    }
     dim3 grid(H, B);
     prefill_tc_kernel<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(
-        (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-        (const __nv_bfloat16*)g, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
+        mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
     note_launches(1);
     return cudaGetLastError();
 }

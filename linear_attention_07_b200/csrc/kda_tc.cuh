@@ -131,7 +131,7 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t saddr, uint32_t parit
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 100000;\n\t"
         "selp.b32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok) : "r"(saddr), "r"(parity) : "memory");
     return ok;
@@ -141,7 +141,9 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
     return t;
 }
-// Wait for phase `parity` to complete, giving up after `limit_ns`.
+// Wait for phase `parity` to complete, giving up after `limit_ns`.  Each
+// try_wait may suspend the thread (up to a 100 us hint) until the phase
+// completes, so a waiting thread does not spin on the issue slots.
 // Returns true on success, false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(saddr, parity)) return true;
@@ -150,6 +152,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, uint6
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }
     return true;
+}
+
+// ------------------------------------------------------------------ TMA --
+
+// Arrive on an mbarrier and add `bytes` to the transaction count it expects.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t saddr, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 :: "r"(saddr), "r"(bytes) : "memory");
+}
+// Tiled 3-D tensor load (no multicast) into shared memory; completion is
+// signalled as transaction bytes on the mbarrier.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst_saddr, const void* tmap, int x, int y, int z,
+                                            uint32_t mbar_saddr) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4}], [%5];"
+        :: "r"(dst_saddr), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z),
+           "r"(mbar_saddr) : "memory");
 }
 
 // ------------------------------------------------------ TMEM <-> registers --
@@ -220,11 +240,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
         : "memory");
 }
 
-// Round an fp32 value to tf32 (nearest, ties away), low 13 bits cleared.
+// Round an fp32 value to tf32 (nearest, ties away from zero): add half of the
+// last kept unit to the magnitude bits and clear the 13 dropped bits.
 __device__ __forceinline__ float to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
 
 }  // namespace tc
