@@ -110,6 +110,16 @@ int kda_decode_step(const void* q, const void* k, const void* v, const void* g,
  */
 int kda_device_status(kda_stream_t stream);
 
+/*
+ * kda_selftest_bounded_wait -- launches a one-warp kernel whose device-side
+ * wait can never be satisfied; the wait gives up after `limit_ns`
+ * (1 <= limit_ns <= 1e9) and sets the status word that kda_device_status
+ * reports as KDA_ERR_TIMEOUT.  Lets callers check, without any fault, that
+ * an expired wait ends the kernel cleanly and leaves the context usable.
+ * KDA_ERR_INVALID_ARG for a limit outside that range (nothing launched).
+ */
+int kda_selftest_bounded_wait(uint64_t limit_ns, kda_stream_t stream);
+
 /* Human-readable name of a kda_status value (static storage). */
 const char* kda_status_string(int status);
 

@@ -29,8 +29,8 @@ KDA_ERR_TIMEOUT = -4
 KDA_ERR_NO_MEMORY = -5
 
 EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_f32", "kda_decode_step",
-            "kda_device_status", "kda_status_string", "kda_launch_count",
-            "kda_version")
+            "kda_device_status", "kda_selftest_bounded_wait",
+            "kda_status_string", "kda_launch_count", "kda_version")
 
 
 class KdaLibraryError(RuntimeError):
@@ -68,6 +68,8 @@ def load_library(path: str = LIB_PATH):
     lib.kda_decode_step.restype = i
     lib.kda_device_status.argtypes = [vp]
     lib.kda_device_status.restype = i
+    lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
+    lib.kda_selftest_bounded_wait.restype = i
     lib.kda_status_string.argtypes = [i]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_launch_count.argtypes = []

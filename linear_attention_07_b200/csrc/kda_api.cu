@@ -18,6 +18,7 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
                               const void* beta, const float* h0, void* o, float* hT,
                               int B, int T, int H, cudaStream_t stream);
 int prefill_device_status(cudaStream_t stream);
+cudaError_t bounded_wait_selftest_launch(uint64_t limit_ns, cudaStream_t stream);
 
 template <typename Tin, typename Tout>
 cudaError_t prefill_serial_launch(const void* q, const void* k, const void* v,
@@ -125,6 +126,12 @@ const char* kda_status_string(int status)
 int kda_device_status(kda_stream_t stream)
 {
     return prefill_device_status((cudaStream_t)stream);
+}
+
+int kda_selftest_bounded_wait(uint64_t limit_ns, kda_stream_t stream)
+{
+    if (limit_ns == 0 || limit_ns > 1000000000ull) return KDA_ERR_INVALID_ARG;
+    return status_of(bounded_wait_selftest_launch(limit_ns, (cudaStream_t)stream));
 }
 
 uint64_t kda_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

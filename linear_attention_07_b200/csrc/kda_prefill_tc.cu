@@ -642,6 +642,28 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
     return cudaGetLastError();
 }
 
+// Self-test of the bounded waits: one warp waits on an mbarrier that nothing
+// completes, gives up after limit_ns and records KDA_ERR_TIMEOUT exactly as
+// the prefill kernel does.  No fault, trap or unbounded wait is involved.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(tc::smem_u32(&bar), 1);
+        tc::fence_mbar_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0 && !tc::mbar_wait(tc::smem_u32(&bar), 0, limit_ns))
+        atomicExch(&g_prefill_status, (int)KDA_ERR_TIMEOUT);
+}
+
+cudaError_t bounded_wait_selftest_launch(uint64_t limit_ns, cudaStream_t stream)
+{
+    bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
 // Reads and clears the timeout flag of the prefill kernels (blocking).
 int prefill_device_status(cudaStream_t stream)
 {

@@ -106,6 +106,13 @@ def test_decode_argument_errors(lib):
     assert lib.kda_launch_count() == n0
 
 
+def test_selftest_limit_checked_on_host(lib):
+    n0 = lib.kda_launch_count()
+    assert lib.kda_selftest_bounded_wait(0, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_selftest_bounded_wait(2_000_000_000, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_launch_count() == n0
+
+
 def test_binding_requires_cuda_tensors():
     import torch
     x = torch.zeros(1, 4, 1, 128, dtype=torch.bfloat16)

@@ -231,3 +231,21 @@ def test_workload_decode_256_sampled():
                               sel(d["beta"]), S0)
     assert err_out(o_all.transpose(0, 1), o_ref) <= TOL_BF16
     assert err_state(S[reqs], S_ref) <= 1e-4
+
+
+# ---------------------------------------------------- failure detection ---
+
+def test_bounded_wait_expiry_is_reported_and_context_survives():
+    """A device wait that nothing satisfies gives up after its limit, the
+    status word reports KDA_ERR_TIMEOUT once, and the context keeps working."""
+    stream = torch.cuda.current_stream(DEV)
+    assert kda.device_status() == kda.KDA_OK
+    lib = kda.load_library()
+    import ctypes
+    assert lib.kda_selftest_bounded_wait(20_000_000, ctypes.c_void_p(stream.cuda_stream)) == kda.KDA_OK
+    assert kda.device_status() == kda.KDA_ERR_TIMEOUT
+    assert kda.device_status() == kda.KDA_OK            # read and cleared
+    x = prefill_inputs(1, 40, 2, 128, 128, seed=41, h0_std=0.1)
+    o, hT = run_prefill(x)
+    check_prefill(x, o, hT, TOL_BF16)
+    assert kda.device_status() == kda.KDA_OK
