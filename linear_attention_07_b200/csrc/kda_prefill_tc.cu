@@ -328,7 +328,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
         };
         if (n_chunks > 0) issue_raw(0);
-        float beta_next = (pt < C && pt < T) ? to_f32(beta[((int64_t)b * T + pt) * H + h]) : 0.f;
+        // beta one chunk ahead, kept as raw bf16 bits until it is stored (a
+        // conversion right after the load would stall on the load)
+        const __nv_bfloat16 bzero = __float2bfloat16_rn(0.f);
+        __nv_bfloat16 beta_next = (pt < C && pt < T) ? beta[((int64_t)b * T + pt) * H + h] : bzero;
 
         // decay-scaling slice of this thread: tile tau, key channel c
         const int tau = pt >> 7;
@@ -343,9 +346,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int ch = 0; ch < n_chunks; ++ch) {
             // ---- inputs of this chunk (beta prefetched one chunk ahead)
             if (pt < C) {
-                reinterpret_cast<float*>(sm + BETA)[pt] = beta_next;
+                reinterpret_cast<float*>(sm + BETA)[pt] = to_f32(beta_next);
                 const int tn = (ch + 1) * C + pt;
-                beta_next = (tn < T) ? to_f32(beta[((int64_t)b * T + tn) * H + h]) : 0.f;
+                beta_next = (tn < T) ? beta[((int64_t)b * T + tn) * H + h] : bzero;
             }
             if (pt == 0 && !s_abort && !mbar_wait(rbar, rphase & 1u, WAIT_NS)) expired();
             ++rphase;
