@@ -32,16 +32,18 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 BYTES_BF16 = 2
+METRIC = ("KDA prefill tokens/s on 1 B200 (workload in config; default B1 H32 T8192 "
+          "d128 bf16); decode steps/s and both rooflines reported alongside")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
 
 # ------------------------------------------------------------ accounting --
 
-def prefill_alg_bytes(B, T, H, dk, dv, with_h0=True, with_hT=True):
+def prefill_alg_bytes(B, T, H, dk, dv, with_h0=True, with_hT=True, elem=BYTES_BF16):
     """Algorithmic HBM bytes of one prefill: q, k, g, v, beta read once, o
-    written once, h0 read and hT written once (fp32)."""
-    per_token_head = (3 * dk + dv + 1) * BYTES_BF16 + dv * BYTES_BF16
+    written once (elem bytes each), h0 read and hT written once (fp32)."""
+    per_token_head = (3 * dk + dv + 1) * elem + dv * elem
     state = dk * dv * 4
     return B * T * H * per_token_head + B * H * state * (int(with_h0) + int(with_hT))
 
@@ -205,13 +207,15 @@ def bench_kda(args, rank, world, local):
     sets = [prefill_inputs(B, T, H, dk, dv, seed=rank_seed(w.seed + 17 * i, rank),
                            device=dev, h0_std=w.h0_std, pin_frac=w.pin_frac)
             for i in range(2)]
-    outs = [(torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev),
+    outs = [(torch.empty((B, T, H, dv), dtype=w.dtype, device=dev),
              torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)) for _ in range(2)]
+    fwd = kda.chunk_fwd_f32 if w.dtype == torch.float32 else kda.chunk_fwd
+    set_bytes = sum(t.numel() * t.element_size() for t in sets[0].values() if t is not None)
 
     def step(i):
         x = sets[i % 2]
         o, hT = outs[i % 2]
-        kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"], o=o, hT=hT)
+        fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"], o=o, hT=hT)
 
     for i in range(args.warmup):
         step(i)
@@ -239,7 +243,8 @@ def bench_kda(args, rank, world, local):
 
     # roofline of the prefill kernel (one launch per step)
     hbm_gbs, bf16_tf, peak_src = load_peaks()
-    alg_b = prefill_alg_bytes(B, T, H, dk, dv, with_h0=w.h0_std > 0)
+    alg_b = prefill_alg_bytes(B, T, H, dk, dv, with_h0=w.h0_std > 0,
+                              elem=4 if w.dtype == torch.float32 else BYTES_BF16)
     alg_f = prefill_alg_flops(B, T, H, dk, dv)
     launch_ms = statistics.mean(per_step)
     achieved_gbs = alg_b / (launch_ms / 1e3) / 1e9
@@ -253,16 +258,18 @@ def bench_kda(args, rank, world, local):
                 "tensor_frac_alg": round(alg_f / (launch_ms / 1e3) / 1e12 / bf16_tf, 4)}
 
     result = {
-        "metric": "KDA prefill tokens/s on 1 B200 (B1 H32 T8192 d128 bf16); decode steps/s under 'decode'",
+        "metric": METRIC,
         "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if w.dtype == torch.float32 else "bf16",
         "data": "synthetic",
         "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
                    "global_batch": B * world, "seq_len": T,
                    "parallelism": "dp%d" % world,
-                   "l2": "two 269 MB input sets alternate (inputs > L2)"},
+                   "l2": "two %.0f MB input sets alternate (%s)" % (
+                       set_bytes / 1e6, "inputs > L2" if set_bytes > 126e6 else "inputs fit in L2")},
         "roofline": roofline,
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
@@ -270,7 +277,7 @@ def bench_kda(args, rank, world, local):
 
     # end to end through the public API: pinned host inputs -> device ->
     # kda_chunk_fwd -> o and hT back to pinned host memory, every step
-    result["e2e"] = bench_e2e(args, kda, sets, dev, B, T, world)
+    result["e2e"] = bench_e2e(args, kda, sets, dev, B, T, world, fwd, w.dtype)
 
     if args.decode:
         result["decode"] = bench_decode(args, kda, dev, rank, world, hbm_gbs, peak_src)
@@ -279,25 +286,25 @@ def bench_kda(args, rank, world, local):
     return result
 
 
-def bench_e2e(args, kda, sets, dev, B, T, world):
+def bench_e2e(args, kda, sets, dev, B, T, world, fwd, dtype):
     import torch
     host = []
     for x in sets:
         host.append({k: (None if t is None else t.cpu().pin_memory()) for k, t in x.items()})
     dbuf = {k: (None if t is None else torch.empty_like(t)) for k, t in sets[0].items()}
-    o_h = torch.empty(tuple(sets[0]["v"].shape), dtype=torch.bfloat16).pin_memory()
+    o_h = torch.empty(tuple(sets[0]["v"].shape), dtype=dtype).pin_memory()
     s_h = torch.empty(tuple(dbuf["h0"].shape) if dbuf["h0"] is not None else
                       (B, sets[0]["q"].shape[2], sets[0]["q"].shape[3], sets[0]["v"].shape[3]),
                       dtype=torch.float32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host[0].values() if t is not None)
-    d2h = o_h.numel() * 2 + s_h.numel() * 4
+    d2h = o_h.numel() * o_h.element_size() + s_h.numel() * 4
 
     def step(i):
         hx = host[i % 2]
         for k2, t in hx.items():
             if t is not None:
                 dbuf[k2].copy_(t, non_blocking=True)
-        o, hT = kda.chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], dbuf["h0"])
+        o, hT = fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["g"], dbuf["beta"], dbuf["h0"])
         o_h.copy_(o, non_blocking=True)
         s_h.copy_(hT, non_blocking=True)
 
@@ -408,7 +415,7 @@ def bench_reference(args, rank, world):
         toks += args.ref_heads * w.T / w.H
     total = sum(times)
     value = toks / total
-    return {"metric": "KDA prefill tokens/s on 1 B200 (B1 H32 T8192 d128 bf16); decode steps/s under 'decode'",
+    return {"metric": METRIC,
             "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total / args.steps * 1e3, 2), "higher_is_better": True,
