@@ -43,6 +43,7 @@
 // that produces a value owns the K index, the K-direction core-matrix stride
 // is padded to 144 B so that a warp's scalar stores hit distinct banks.
 #include <cuda.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "kda_common.cuh"
@@ -593,6 +594,504 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 0) tmem_dealloc(tm, TMEM_COLS);
 }
 
+// ============================================================================
+// Cluster variant for few heads (B * H small next to the SM count): each head
+// gets a cluster of three CTAs on three SMs.  Rank 0 runs the chain; ranks 1
+// and 2 prepare the chunks of even and odd index, each in its own SM, and push
+// every prepared chunk (the chain's operands and U') into one of two slots of
+// rank 0's shared memory with a single bulk copy (shared::cta ->
+// shared::cluster, no multicast).  FULL[slot] (rank 0) counts the copy's
+// bytes; EMPTY (the preparing CTA) is arrived on by rank 0 once the slot has
+// been read.  The arithmetic is the one of prefill_tc_kernel.
+namespace pc {
+using namespace pf;
+constexpr int NTH = 256;                                      // threads per CTA (both roles)
+// slot / staging layout (identical in rank 0's slots and a preparer's staging)
+constexpr uint32_t S_B1 = 0;                                   // [W | Qt]: N 64 x K 128 (padded)
+constexpr uint32_t S_B2 = S_B1 + 8 * SBO_K128P;                // Kb: N 128 x K 32
+constexpr uint32_t S_B3 = S_B2 + (D / 8) * SBO_K32;            // P: N 32 x K 32 (padded)
+constexpr uint32_t S_GAM = S_B3 + (C / 8) * SBO_K32P;          // gamma_C, 128 fp32
+constexpr uint32_t S_UP = S_GAM + D * 4;                       // U' [32 tokens][128] fp32
+constexpr uint32_t SLOT = S_UP + C * D * 4;                    // bytes per chunk
+static_assert(SLOT % 16 == 0, "bulk copy size");
+// rank 0 (chain)
+constexpr uint32_t C_SLOT0 = 0;
+constexpr uint32_t C_OST = 2 * SLOT;
+constexpr uint32_t C_BYTES = C_OST + C * D * 2;
+// ranks 1, 2 (preparation)
+constexpr uint32_t P_RAW = 0;
+constexpr uint32_t P_BETA = P_RAW + 4 * RAW_T;
+constexpr uint32_t P_GEX = P_BETA + C * 4;
+constexpr uint32_t P_GA = P_GEX + 2 * D * 4;
+constexpr uint32_t P_GB = P_GA + 6 * SBO_K128P;
+constexpr uint32_t P_WA = P_GB + 8 * SBO_K128P;
+constexpr uint32_t P_VA = P_WA + (D / 8) * SBO_K32;
+constexpr uint32_t P_TB = P_VA + (D / 8) * SBO_K32;
+constexpr uint32_t P_ST = P_TB + (C / 8) * SBO_K32P;           // staging of one slot
+constexpr uint32_t P_AMS = P_ST + SLOT;
+constexpr uint32_t P_PMS = P_AMS + C * LD * 4;
+constexpr uint32_t P_XMS = P_PMS + C * LD * 4;
+constexpr uint32_t P_TMS = P_XMS + C * LD * 4;
+constexpr uint32_t P_YMS = P_TMS + C * LD * 4;
+constexpr uint32_t P_BYTES = P_YMS + TILE * (TILE + 1) * 4;
+constexpr uint32_t SMEM_BYTES = P_BYTES > C_BYTES ? P_BYTES : C_BYTES;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(P_ST % 16 == 0 && P_GA % 16 == 0 && P_GB % 16 == 0 && P_WA % 16 == 0 && P_VA % 16 == 0 &&
+              P_TB % 16 == 0 && C_OST % 16 == 0 && SLOT % 16 == 0, "alignment");
+// tensor memory: rank 0 uses 352 columns (512 allocated), ranks 1-2 use 128
+constexpr uint32_t CT_AS = 0, CT_AU = 128, CT_DX = 160, CT_DKU = 224;
+constexpr uint32_t PT_DG = 0, PT_DW = 64, PT_DU = 96;
+}  // namespace pc
+
+__global__ void __cluster_dims__(3, 1, 1) __launch_bounds__(pc::NTH, 1)
+prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                       const __nv_bfloat16* __restrict__ beta, const float* h0,
+                       __nv_bfloat16* __restrict__ o, float* hT, int T, int H)
+{
+    using namespace pc;
+    using namespace tc;
+    extern __shared__ __align__(1024) unsigned char sm[];
+    __shared__ uint32_t s_taddr;
+    __shared__ __align__(8) uint64_t s_bar[3];   // rank 0: FULL[0], FULL[1], MMA; ranks 1-2: EMPTY, MMA, input loads
+    __shared__ int s_abort;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int h = blockIdx.x / 3, b = blockIdx.y;
+    const int64_t head_off = (int64_t)b * H + h;
+    const int64_t row_stride = (int64_t)H * D;
+    const int64_t base = ((int64_t)b * T * H + h) * D;
+    const int n_chunks = (T + C - 1) / C;
+    const uint32_t ncols = rank == 0 ? 512u : 128u;
+
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&s_taddr), ncols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
+        fence_mbar_init();
+        s_abort = 0;
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    cluster_sync();                    // every CTA's barriers exist before any remote arrive
+    const uint32_t tm = s_taddr;
+    const int sp = warp & 3;
+    const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
+    auto expired = [&]() {
+        s_abort = 1;
+        atomicExch(&g_prefill_status, (int)KDA_ERR_TIMEOUT);
+    };
+
+    if (rank == 0) {
+        // ========================================================= chain CTA ==
+        const int j = 32 * sp + lane;
+        const int hh = warp >> 2;
+        const uint32_t mbar = smem_u32(&s_bar[2]);
+        uint32_t phase = 0;
+        auto cta_bar = [&]() { __syncthreads(); };
+        auto wait_mma = [&]() {
+            if (tid == 0 && !s_abort && !mbar_wait(mbar, phase & 1u, WAIT_NS)) expired();
+            ++phase;
+            __syncwarp();
+            cta_bar();
+            fence_after_sync();
+        };
+        float S[D / 2];
+        {
+            const float* h0h = h0 ? h0 + head_off * D * D : nullptr;
+#pragma unroll
+            for (int i = 0; i < D / 2; ++i) S[i] = h0h ? h0h[(int64_t)(64 * hh + i) * D + j] : 0.f;
+#pragma unroll
+            for (int c0 = 0; c0 < D / 2; c0 += 32) {
+                float t32[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) t32[i] = to_tf32(S[c0 + i]);
+                tmem_st32(tm + lane_base + CT_AS + 64 * hh + c0, t32);
+            }
+            wait_st();
+        }
+        __nv_bfloat16* oh = o + base;
+#pragma unroll 1
+        for (int ch = 0; ch < n_chunks; ++ch) {
+            const int slot = ch & 1;
+            const uint32_t sb = C_SLOT0 + slot * SLOT;
+            if (tid == 0 && !s_abort && !mbar_wait_cluster(smem_u32(&s_bar[slot]), (ch >> 1) & 1, WAIT_NS))
+                expired();
+            __syncwarp();
+            cta_bar();
+            fence_after_sync();
+            if (tid == 0 && !s_abort) {
+                const uint32_t id = idesc_tf32(128, 2 * C, false, false);
+                const uint64_t bd0 = sdesc(smem_u32(sm + sb + S_B1), PAD_LBO, SBO_K128P);
+#pragma unroll
+                for (int ks = 0; ks < D / 8; ++ks)
+                    mma_tf32_ts(tm + CT_DX, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                id, ks > 0 ? 1u : 0u);
+                mma_commit(mbar);
+            }
+            wait_mma();
+            {   // U = U' - W S  (this half: tokens [16 hh, 16 hh + 16))
+                const float* up = reinterpret_cast<const float*>(sm + sb + S_UP);
+                float x[16];
+                tmem_ld16(tm + lane_base + CT_DX + 16 * hh, x);
+                wait_ld();
+#pragma unroll
+                for (int r = 0; r < 16; ++r) x[r] = to_tf32(up[(16 * hh + r) * D + j] - x[r]);
+                tmem_st16(tm + lane_base + CT_AU + 16 * hh, x);
+                wait_st();
+            }
+            fence_before_sync();
+            cta_bar();
+            fence_after_sync();
+            if (tid == 0 && !s_abort) {
+                const uint32_t id2 = idesc_tf32(128, 128, false, false);
+                const uint32_t id3 = idesc_tf32(128, 32, false, false);
+                const uint64_t b20 = sdesc(smem_u32(sm + sb + S_B2), LBO, SBO_K32);
+                const uint64_t b30 = sdesc(smem_u32(sm + sb + S_B3), PAD_LBO, SBO_K32P);
+#pragma unroll
+                for (int ks = 0; ks < C / 8; ++ks) {
+                    mma_tf32_ts(tm + CT_DKU, tm + CT_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                id2, ks > 0 ? 1u : 0u);
+                    mma_tf32_ts(tm + CT_DX + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                id3, 1u);
+                }
+                mma_commit(mbar);
+            }
+            wait_mma();
+            {   // S <- Diag(gamma_C) S + Kb^T U ; refresh the tf32 copy
+                const float4* gam4 = reinterpret_cast<const float4*>(sm + sb + S_GAM) + 16 * hh;
+#pragma unroll
+                for (int c0 = 0; c0 < D / 2; c0 += 16) {
+                    float d[16];
+                    tmem_ld16(tm + lane_base + CT_DKU + 64 * hh + c0, d);
+                    wait_ld();
+#pragma unroll
+                    for (int i4 = 0; i4 < 4; ++i4) {
+                        const float4 gv = gam4[(c0 >> 2) + i4];
+                        const float gg[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int i = c0 + i4 * 4 + u;
+                            S[i] = fmaf(gg[u], S[i], d[i - c0]);
+                            d[i - c0] = to_tf32(S[i]);
+                        }
+                    }
+                    tmem_st16(tm + lane_base + CT_AS + 64 * hh + c0, d);
+                }
+            }
+            // o of this chunk, then release the slot to its preparer
+            __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
+            {
+                float ov[16];
+                tmem_ld16(tm + lane_base + CT_DX + C + 16 * hh, ov);
+                wait_ld();
+#pragma unroll
+                for (int r = 0; r < 16; ++r) ost[(16 * hh + r) * D + j] = __float2bfloat16_rn(ov[r]);
+            }
+            wait_st();
+            fence_before_sync();
+            cta_bar();
+            if (tid == 0) mbar_arrive_remote(map_to_rank(smem_u32(&s_bar[0]), 1u + (uint32_t)slot));
+            const int tb = ch * C;
+#pragma unroll
+            for (int m = 0; m < (C * D / 8) / NTH; ++m) {
+                const int vi = tid + m * NTH;
+                const int r = vi / (D / 8), cv = vi % (D / 8);
+                if (tb + r < T)
+                    *reinterpret_cast<uint4*>(oh + (int64_t)(tb + r) * row_stride + cv * 8) =
+                        *reinterpret_cast<const uint4*>(ost + r * D + cv * 8);
+            }
+            cta_bar();                         // staging read before the next chunk writes it
+        }
+        if (hT && !s_abort) {
+            float* hTh = hT + head_off * D * D;
+#pragma unroll
+            for (int i = 0; i < D / 2; ++i) hTh[(int64_t)(64 * hh + i) * D + j] = S[i];
+        }
+    } else {
+        // ================================================== preparing CTAs ==
+        const int par = (int)rank - 1;             // chunks ch with ch % 2 == par
+        const int pt = tid;
+        const int pw = warp;
+        const uint32_t ebar = smem_u32(&s_bar[0]);
+        const uint32_t mbar = smem_u32(&s_bar[1]);
+        const uint32_t rbar = smem_u32(&s_bar[2]);
+        uint32_t phase = 0, rphase = 0, ephase = 0;
+        auto prep_sync = [&]() { __syncthreads(); };
+        auto wait_mma = [&]() {
+            if (pt == 0 && !s_abort && !mbar_wait(mbar, phase & 1u, WAIT_NS)) expired();
+            ++phase;
+            __syncwarp();
+            prep_sync();
+            fence_after_sync();
+        };
+        auto issue_raw = [&](int ci) {
+            if (pt == 0) {
+                mbar_arrive_expect_tx(rbar, 4 * RAW_T);
+                tma_load_3d(smem_u32(sm + P_RAW + 0 * RAW_T), &tm_q, h * D, ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + P_RAW + 1 * RAW_T), &tm_k, h * D, ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + P_RAW + 2 * RAW_T), &tm_v, h * D, ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + P_RAW + 3 * RAW_T), &tm_g, h * D, ci * C, b, rbar);
+            }
+        };
+        if (par < n_chunks) issue_raw(par);
+        const __nv_bfloat16 bzero = __float2bfloat16_rn(0.f);
+        __nv_bfloat16 beta_next = (pt < C && par * C + pt < T) ? beta[((int64_t)b * T + par * C + pt) * H + h] : bzero;
+        const int tau = pt >> 7;
+        const int c = pt & 127;
+        float* am = reinterpret_cast<float*>(sm + P_AMS);
+        float* pm = reinterpret_cast<float*>(sm + P_PMS);
+        float* xm = reinterpret_cast<float*>(sm + P_XMS);
+        float* tmx = reinterpret_cast<float*>(sm + P_TMS);
+        float* ym = reinterpret_cast<float*>(sm + P_YMS);
+        const float* bt = reinterpret_cast<const float*>(sm + P_BETA);
+        unsigned char* st = sm + P_ST;
+        const uint32_t full_remote = map_to_rank(smem_u32(&s_bar[par]), 0u);
+        const uint32_t slot_remote = map_to_rank(smem_u32(sm + C_SLOT0 + par * SLOT), 0u);
+#pragma unroll 1
+        for (int ch = par; ch < n_chunks; ch += 2) {
+            if (pt < C) {
+                reinterpret_cast<float*>(sm + P_BETA)[pt] = to_f32(beta_next);
+                const int tn = (ch + 2) * C + pt;
+                beta_next = (tn < T) ? beta[((int64_t)b * T + tn) * H + h] : bzero;
+            }
+            if (pt == 0 && !s_abort && !mbar_wait(rbar, rphase & 1u, WAIT_NS)) expired();
+            ++rphase;
+            __syncwarp();
+            prep_sync();
+            float gam_c, fq, fk;
+            float vr[TILE];
+            {
+                const __nv_bfloat16* __restrict__ rq = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW + 0 * RAW_T);
+                const __nv_bfloat16* __restrict__ rk = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW + 1 * RAW_T);
+                const __nv_bfloat16* __restrict__ rv = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW + 2 * RAW_T);
+                const __nv_bfloat16* __restrict__ rg = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW + 3 * RAW_T);
+                float a[TILE], kr[TILE], qr[TILE];
+#pragma unroll
+                for (int rr = 0; rr < TILE; ++rr) {
+                    const int idx = (tau * TILE + rr) * D + c;
+                    kr[rr] = to_f32(rk[idx]);
+                    qr[rr] = to_f32(rq[idx]);
+                    vr[rr] = to_f32(rv[idx]);
+                    a[rr] = to_f32(rg[idx]);
+                }
+                float e = 1.f;
+#pragma unroll
+                for (int rr = 0; rr < TILE; ++rr) {
+                    a[rr] = __expf(a[rr]);
+                    e *= a[rr];
+                }
+                float* gex = reinterpret_cast<float*>(sm + P_GEX);
+                gex[tau * D + c] = e;
+                prep_sync();
+                const float oe = gex[(1 - tau) * D + c];
+                const float f = tau ? oe : 1.f;
+                gam_c = e * oe;
+                fq = f;
+                fk = tau ? e : oe;
+                float p = 1.f;
+                float kc[4];
+#pragma unroll
+                for (int rr = 0; rr < TILE; ++rr) {
+                    const int r = tau * TILE + rr;
+                    p *= a[rr];
+                    const float kt = kr[rr] * p;
+                    const float qt = qr[rr] * p;
+                    st_f32(sm, P_GB + off_kmajor(r, c, PAD_LBO, SBO_K128P), to_tf32(kt));
+                    st_f32(sm, P_GB + off_kmajor(C + r, c, PAD_LBO, SBO_K128P), to_tf32(qt));
+                    kc[rr & 3] = to_tf32(kt * f);
+                    if ((rr & 3) == 3)
+                        st_f32x4(sm, P_WA + off_kmajor(c, r - 3, LBO, SBO_K32), kc[0], kc[1], kc[2], kc[3]);
+                }
+                const float inv = 1.f / e;
+                float sgm = 1.f;
+#pragma unroll
+                for (int rr = TILE - 1; rr >= 0; --rr) {
+                    const int r = tau * TILE + rr;
+                    const float kb = kr[rr] * sgm;
+                    st_f32(sm, P_GA + off_kmajor(r, c, PAD_LBO, SBO_K128P), to_tf32(kb * inv));
+                    if (tau == 0) st_f32(sm, P_GA + off_kmajor(C + rr, c, PAD_LBO, SBO_K128P), to_tf32(kb));
+                    sgm *= a[rr];
+                }
+            }
+            fence_smem_to_async();
+            fence_before_sync();
+            prep_sync();
+            fence_after_sync();
+            if (pt == 0 && !s_abort) {
+                const uint32_t id = idesc_tf32(64, 64, false, false);
+                const uint64_t ad0 = sdesc(smem_u32(sm + P_GA), PAD_LBO, SBO_K128P);
+                const uint64_t bd0 = sdesc(smem_u32(sm + P_GB), PAD_LBO, SBO_K128P);
+#pragma unroll
+                for (int ks = 0; ks < D / 8; ++ks) {
+                    const uint64_t step = (uint64_t)((ks * 2 * PAD_LBO) >> 4);
+                    mma_tf32_ss(tm + PT_DG, ad0 + step, bd0 + step, id, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(mbar);
+            }
+            if (ch + 2 < n_chunks) issue_raw(ch + 2);
+#pragma unroll
+            for (int rr = 0; rr < TILE; rr += 4)
+                st_f32x4(sm, P_VA + off_kmajor(c, tau * TILE + rr, LBO, SBO_K32),
+                         to_tf32(vr[rr]), to_tf32(vr[rr + 1]), to_tf32(vr[rr + 2]), to_tf32(vr[rr + 3]));
+            fence_smem_to_async();
+            wait_mma();
+            // A and P into scratch (row m of D_G is lane (m % 16) + 32 (m / 16))
+            if (pw < 3) {
+                const int colK = (sp == 0) ? 0 : TILE;
+                float gk[16], gq[16];
+                tmem_ld16(tm + lane_base + PT_DG + colK, gk);
+                tmem_ld16(tm + lane_base + PT_DG + C + colK, gq);
+                wait_ld();
+                if (lane < TILE) {
+                    const int i = (sp == 1 ? TILE : 0) + lane;
+                    const int rbase = (sp == 0) ? 0 : TILE;
+#pragma unroll
+                    for (int r = 0; r < TILE; ++r) {
+                        const int rg = rbase + r;
+                        am[rg * LD + i] = (rg > i) ? bt[rg] * gk[r] : 0.f;
+                        pm[rg * LD + i] = (rg >= i) ? gq[r] : 0.f;
+                    }
+                    if (sp == 1) {
+#pragma unroll
+                        for (int r = 0; r < TILE; ++r) {
+                            am[r * LD + i] = 0.f;
+                            pm[r * LD + i] = 0.f;
+                        }
+                    }
+                }
+            }
+            prep_sync();
+            if (pw < 2 && lane < TILE) {
+                const int off = pw * TILE;
+                const int i = lane;
+                float x[TILE];
+#pragma unroll
+                for (int r = 0; r < TILE; ++r) x[r] = (r == i) ? 1.f : 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < TILE; ++s2) {
+#pragma unroll
+                    for (int r = s2 + 1; r < TILE; ++r)
+                        x[r] = fmaf(-am[(off + r) * LD + off + s2], x[s2], x[r]);
+                }
+                const float bi = bt[off + i];
+#pragma unroll
+                for (int r = 0; r < TILE; ++r) {
+                    xm[(off + r) * LD + off + i] = x[r];
+                    tmx[(off + r) * LD + off + i] = x[r] * bi;
+                    if (pw == 1) tmx[r * LD + off + i] = 0.f;
+                }
+            }
+            prep_sync();
+            {
+                const int r = pt >> 4, i = pt & 15;
+                float y = 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < TILE; ++s2) y = fmaf(am[(TILE + r) * LD + s2], xm[s2 * LD + i], y);
+                ym[r * (TILE + 1) + i] = y;
+            }
+            prep_sync();
+            {
+                const int r = pt >> 4, i = pt & 15;
+                float z = 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < TILE; ++s2) z = fmaf(xm[(TILE + r) * LD + TILE + s2], ym[s2 * (TILE + 1) + i], z);
+                tmx[(TILE + r) * LD + i] = -z * bt[i];
+            }
+            prep_sync();
+            {
+                const int r = pt >> 3, i = (pt & 7) * 4;
+                const float* row = tmx + r * LD + i;
+                st_f32x4(sm, P_TB + off_kmajor(r, i, PAD_LBO, SBO_K32P),
+                         to_tf32(row[0]), to_tf32(row[1]), to_tf32(row[2]), to_tf32(row[3]));
+            }
+            fence_smem_to_async();
+            fence_before_sync();
+            prep_sync();
+            fence_after_sync();
+            if (pt == 0 && !s_abort) {
+                const uint32_t id = idesc_tf32(128, 32, false, false);
+                const uint64_t bd0 = sdesc(smem_u32(sm + P_TB), PAD_LBO, SBO_K32P);
+                const uint64_t aw0 = sdesc(smem_u32(sm + P_WA), LBO, SBO_K32);
+                const uint64_t av0 = sdesc(smem_u32(sm + P_VA), LBO, SBO_K32);
+#pragma unroll
+                for (int ks = 0; ks < C / 8; ++ks) {
+                    const uint64_t bstep = (uint64_t)((ks * 2 * PAD_LBO) >> 4);
+                    const uint64_t astep = (uint64_t)((ks * 2 * LBO) >> 4);
+                    mma_tf32_ss(tm + PT_DW, aw0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                    mma_tf32_ss(tm + PT_DU, av0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(mbar);
+            }
+            const float* gaf = reinterpret_cast<const float*>(sm + P_GA);
+            const float* gbf = reinterpret_cast<const float*>(sm + P_GB);
+            float qf[TILE], kf[TILE];
+#pragma unroll
+            for (int rr = 0; rr < TILE; ++rr) {
+                const int r = tau * TILE + rr;
+                qf[rr] = to_tf32(gbf[off_kmajor(C + r, c, PAD_LBO, SBO_K128P) >> 2] * fq);
+                const int row = tau ? (TILE + rr) : (C + rr);
+                kf[rr] = to_tf32(gaf[off_kmajor(row, c, PAD_LBO, SBO_K128P) >> 2] * fk);
+            }
+            float pf4[4];
+            {
+                const int r = pt >> 3, i = (pt & 7) * 4;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) pf4[u] = to_tf32(pm[r * LD + i + u]);
+            }
+            // the previous chunk's bulk copy has finished reading the staging
+            if (pt == 0) bulk_wait_read_all();
+            wait_mma();
+            {
+                float w[16], upv[16];
+                tmem_ld16(tm + lane_base + PT_DW + 16 * tau, w);
+                tmem_ld16(tm + lane_base + PT_DU + 16 * tau, upv);
+                wait_ld();
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    st_f32(st, S_B1 + off_kmajor(16 * tau + r, c, PAD_LBO, SBO_K128P), to_tf32(w[r]));
+                    reinterpret_cast<float*>(st + S_UP)[(16 * tau + r) * D + c] = upv[r];
+                }
+#pragma unroll
+                for (int rr = 0; rr < TILE; ++rr)
+                    st_f32(st, S_B1 + off_kmajor(C + tau * TILE + rr, c, PAD_LBO, SBO_K128P), qf[rr]);
+#pragma unroll
+                for (int rr = 0; rr < TILE; rr += 4)
+                    st_f32x4(st, S_B2 + off_kmajor(c, tau * TILE + rr, LBO, SBO_K32),
+                             kf[rr], kf[rr + 1], kf[rr + 2], kf[rr + 3]);
+                {
+                    const int r = pt >> 3, i = (pt & 7) * 4;
+                    st_f32x4(st, S_B3 + off_kmajor(r, i, PAD_LBO, SBO_K32P), pf4[0], pf4[1], pf4[2], pf4[3]);
+                }
+                if (tau == 0) reinterpret_cast<float*>(st + S_GAM)[c] = gam_c;
+            }
+            fence_smem_to_async();
+            fence_before_sync();
+            prep_sync();
+            if (pt == 0) {
+                // the chain has released this slot (its previous use, chunk ch - 2)
+                if (ch >= 2 && !s_abort && !mbar_wait_cluster(ebar, ephase & 1u, WAIT_NS)) expired();
+                if (ch >= 2) ++ephase;
+                if (!s_abort) {
+                    mbar_arrive_expect_tx_remote(full_remote, SLOT);
+                    bulk_copy_to_rank(slot_remote, smem_u32(st), SLOT, full_remote);
+                    bulk_commit();
+                }
+            }
+        }
+        if (pt == 0) bulk_wait_read_all();
+    }
+
+    fence_before_sync();
+    __syncthreads();
+    cluster_sync();                    // no CTA leaves while another may still touch its memory
+    if (warp == 0) tmem_dealloc(tm, ncols);
+}
+
 static bool make_map(CUtensorMap* map, const void* base, int B, int T, int H)
 {
     typedef CUresult (*encode_fn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -617,6 +1116,17 @@ static bool make_map(CUtensorMap* map, const void* base, int B, int T, int H)
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Three SMs per head pay off while the heads alone leave most SMs idle:
+// up to 48 heads (144 of the 148 SMs); larger batches use one SM per head.
+// KDA_PREFILL_VARIANT=fused|cluster overrides the choice (for measurement).
+static bool use_cluster_variant(int B, int H)
+{
+    const char* env = getenv("KDA_PREFILL_VARIANT");
+    if (env && strcmp(env, "cluster") == 0) return true;
+    if (env && strcmp(env, "fused") == 0) return false;
+    return (int64_t)B * H * 3 <= 144;
+}
+
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, const float* h0, void* o, float* hT,
                               int B, int T, int H, cudaStream_t stream)
@@ -638,9 +1148,23 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
         memset(&mq, 0, sizeof(mq)); memset(&mk, 0, sizeof(mk));
         memset(&mv, 0, sizeof(mv)); memset(&mg, 0, sizeof(mg));
     }
-    dim3 grid(H, B);
-    prefill_tc_kernel<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(
-        mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
+    if (use_cluster_variant(B, H)) {
+        static bool cattr_set = false;
+        if (!cattr_set) {
+            cudaError_t e = cudaFuncSetAttribute(prefill_cluster_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)pc::SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+            cattr_set = true;
+        }
+        dim3 grid(3 * H, B);
+        prefill_cluster_kernel<<<grid, pc::NTH, pc::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
+    } else {
+        dim3 grid(H, B);
+        prefill_tc_kernel<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
+    }
     note_launches(1);
     return cudaGetLastError();
 }

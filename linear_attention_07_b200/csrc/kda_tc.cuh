@@ -172,6 +172,65 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst_saddr, const void* tmap
            "r"(mbar_saddr) : "memory");
 }
 
+// --------------------------------------------------------------- cluster --
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Whole cluster barrier (all threads of all CTAs); release/acquire ordering.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared-memory address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+// Arrive on an mbarrier of another CTA of the cluster (release, cluster scope).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_saddr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
+                 :: "r"(cluster_saddr) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_saddr, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
+                 :: "r"(cluster_saddr), "r"(bytes) : "memory");
+}
+// Cluster-scope acquiring wait (data written by other CTAs of the cluster).
+__device__ __forceinline__ uint32_t mbar_try_wait_cluster(uint32_t saddr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, 100000;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok) : "r"(saddr), "r"(parity) : "memory");
+    return ok;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t saddr, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_try_wait_cluster(saddr, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_cluster(saddr, parity)) {
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory to
+// another CTA's shared memory in the cluster (no multicast); completion is
+// counted as transaction bytes on the destination CTA's mbarrier.
+__device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster_saddr, uint32_t src_saddr,
+                                                  uint32_t bytes, uint32_t mbar_cluster_saddr) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(dst_cluster_saddr), "r"(src_saddr), "r"(bytes), "r"(mbar_cluster_saddr) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until the source buffers of all committed bulk copies may be reused.
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // ------------------------------------------------------ TMEM <-> registers --
 // 32x32b shapes: thread l of warp w reads/writes lane 32 (w % 4) + l,
 // columns [col, col + N).

@@ -138,6 +138,17 @@ def test_bf16_split_resume_and_determinism():
     assert err_state(h_b, h_ref) <= TOL_BF16
 
 
+@pytest.mark.parametrize("variant", ["fused", "cluster"])
+@pytest.mark.parametrize("T", [1, 31, 33, 95, 300])
+def test_bf16_both_prefill_variants(monkeypatch, variant, T):
+    """The one-SM-per-head kernel and the three-SM cluster kernel, each forced."""
+    monkeypatch.setenv("KDA_PREFILL_VARIANT", variant)
+    x = prefill_inputs(2, T, 3, 128, 128, seed=500 + T, h0_std=0.1)
+    o, hT = run_prefill(x)
+    check_prefill(x, o, hT, TOL_BF16)
+    assert kda.device_status() == kda.KDA_OK
+
+
 # ------------------------------------------------------- full workloads ---
 
 def _sampled_heads_check(w, d, o, hT, heads):
