@@ -596,27 +596,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
 // ============================================================================
 // Cluster variant for few heads (B * H small next to the SM count): each head
-// gets a cluster of three CTAs on three SMs.  Rank 0 runs the chain; ranks 1
-// and 2 prepare the chunks of even and odd index, each in its own SM, and push
-// every prepared chunk (the chain's operands and U') into one of two slots of
-// rank 0's shared memory with a single bulk copy (shared::cta ->
-// shared::cluster, no multicast).  FULL[slot] (rank 0) counts the copy's
-// bytes; EMPTY (the preparing CTA) is arrived on by rank 0 once the slot has
-// been read.  The arithmetic is the one of prefill_tc_kernel.
+// gets a cluster of four CTAs on four SMs.  Rank 0 runs the chain; ranks 1-3
+// prepare the chunks ch with ch % 3 == rank - 1, each in its own SM, and push
+// every prepared chunk (the chain's operands and U') into slot ch % 3 of rank
+// 0's shared memory with a single bulk copy (shared::cta -> shared::cluster,
+// no multicast).  FULL[slot] (rank 0) counts the copy's bytes; EMPTY (the
+// preparing CTA) is arrived on by rank 0 as soon as the chunk's state update
+// has consumed the slot.  o is written with a TMA store from a staging
+// buffer, one chunk late, while the next chunk's first MMA runs.
+// The arithmetic is the one of prefill_tc_kernel.
 namespace pc {
 using namespace pf;
 constexpr int NTH = 256;                                      // threads per CTA (both roles)
+constexpr int NPREPCTA = 3;                                   // preparing CTAs per cluster (= slots)
 // slot / staging layout (identical in rank 0's slots and a preparer's staging)
 constexpr uint32_t S_B1 = 0;                                   // [W | Qt]: N 64 x K 128 (padded)
 constexpr uint32_t S_B2 = S_B1 + 8 * SBO_K128P;                // Kb: N 128 x K 32
-constexpr uint32_t S_B3 = S_B2 + (D / 8) * SBO_K32;            // P: N 32 x K 32 (padded)
-constexpr uint32_t S_GAM = S_B3 + (C / 8) * SBO_K32P;          // gamma_C, 128 fp32
+constexpr uint32_t S_B3 = S_B2 + (D / 8) * SBO_K32;            // P: N 32 x K 32 (dense: vector stores)
+constexpr uint32_t S_GAM = S_B3 + (C / 8) * SBO_K32;           // gamma_C, 128 fp32
 constexpr uint32_t S_UP = S_GAM + D * 4;                       // U' [32 tokens][128] fp32
 constexpr uint32_t SLOT = S_UP + C * D * 4;                    // bytes per chunk
 static_assert(SLOT % 16 == 0, "bulk copy size");
-// rank 0 (chain)
+// rank 0 (chain): NPREPCTA slots and the o staging of one chunk
 constexpr uint32_t C_SLOT0 = 0;
-constexpr uint32_t C_OST = 2 * SLOT;
+constexpr uint32_t C_OST = NPREPCTA * SLOT;
 constexpr uint32_t C_BYTES = C_OST + C * D * 2;
 // ranks 1, 2 (preparation)
 constexpr uint32_t P_RAW = 0;
@@ -637,15 +640,16 @@ constexpr uint32_t P_BYTES = P_YMS + TILE * (TILE + 1) * 4;
 constexpr uint32_t SMEM_BYTES = P_BYTES > C_BYTES ? P_BYTES : C_BYTES;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(P_ST % 16 == 0 && P_GA % 16 == 0 && P_GB % 16 == 0 && P_WA % 16 == 0 && P_VA % 16 == 0 &&
-              P_TB % 16 == 0 && C_OST % 16 == 0 && SLOT % 16 == 0, "alignment");
-// tensor memory: rank 0 uses 352 columns (512 allocated), ranks 1-2 use 128
-constexpr uint32_t CT_AS = 0, CT_AU = 128, CT_DX = 160, CT_DKU = 224;
+              P_TB % 16 == 0 && SLOT % 16 == 0 && C_OST % 16 == 0, "alignment");
+// tensor memory: rank 0 uses 416 columns (512 allocated), ranks 1-3 use 128
+constexpr uint32_t CT_AS = 0, CT_AU = 128, CT_DX0 = 160, CT_DKU = 224, CT_DX1 = 352;
 constexpr uint32_t PT_DG = 0, PT_DW = 64, PT_DU = 96;
 }  // namespace pc
 
-__global__ void __cluster_dims__(3, 1, 1) __launch_bounds__(pc::NTH, 1)
+__global__ void __cluster_dims__(pc::NPREPCTA + 1, 1, 1) __launch_bounds__(pc::NTH, 1)
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                       const __grid_constant__ CUtensorMap tm_o,
                        const __nv_bfloat16* __restrict__ beta, const float* h0,
                        __nv_bfloat16* __restrict__ o, float* hT, int T, int H)
 {
@@ -653,15 +657,13 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     using namespace tc;
     extern __shared__ __align__(1024) unsigned char sm[];
     __shared__ uint32_t s_taddr;
-    __shared__ __align__(8) uint64_t s_bar[3];   // rank 0: FULL[0], FULL[1], MMA; ranks 1-2: EMPTY, MMA, input loads
+    __shared__ __align__(8) uint64_t s_bar[4];   // rank 0: FULL[0..2], MMA; ranks 1-3: EMPTY, MMA, input loads
     __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
-    const int h = blockIdx.x / 3, b = blockIdx.y;
+    const int h = blockIdx.x / (NPREPCTA + 1), b = blockIdx.y;
     const int64_t head_off = (int64_t)b * H + h;
-    const int64_t row_stride = (int64_t)H * D;
-    const int64_t base = ((int64_t)b * T * H + h) * D;
     const int n_chunks = (T + C - 1) / C;
     const uint32_t ncols = rank == 0 ? 512u : 128u;
 
@@ -670,7 +672,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
+        for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
         fence_mbar_init();
         s_abort = 0;
     }
@@ -688,9 +690,13 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
     if (rank == 0) {
         // ========================================================= chain CTA ==
+        // Chunk ch: FULL wait, X = S^T [W | Qt]^T, U, the update MMAs and the
+        // state update.  The output of chunk ch - 1 (its X buffer is the other
+        // of two) is read out, staged and stored while chunk ch's first MMA
+        // runs, so it stays off the sequential path.
         const int j = 32 * sp + lane;
         const int hh = warp >> 2;
-        const uint32_t mbar = smem_u32(&s_bar[2]);
+        const uint32_t mbar = smem_u32(&s_bar[3]);
         uint32_t phase = 0;
         auto cta_bar = [&]() { __syncthreads(); };
         auto wait_mma = [&]() {
@@ -714,30 +720,56 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             }
             wait_st();
         }
-        __nv_bfloat16* oh = o + base;
+        // o of chunk cp (X buffer cp & 1) -> staging -> one TMA store (thread
+        // 32, whose previous store has read the staging before the last CTA
+        // barrier)
+        auto emit_output = [&](int cp) {
+            const uint32_t dx = (cp & 1) ? CT_DX1 : CT_DX0;
+            __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
+            float ov[16];
+            tmem_ld16(tm + lane_base + dx + C + 16 * hh, ov);
+            wait_ld();
+#pragma unroll
+            for (int r = 0; r < 16; ++r) ost[(16 * hh + r) * D + j] = __float2bfloat16_rn(ov[r]);
+            fence_smem_to_async();
+            fence_before_sync();
+            cta_bar();
+            fence_after_sync();
+            if (tid == 32) {
+                tma_store_3d(&tm_o, h * D, cp * C, b, smem_u32(ost));
+                bulk_commit();
+            }
+        };
 #pragma unroll 1
         for (int ch = 0; ch < n_chunks; ++ch) {
-            const int slot = ch & 1;
+            const int slot = ch % NPREPCTA;
             const uint32_t sb = C_SLOT0 + slot * SLOT;
-            if (tid == 0 && !s_abort && !mbar_wait_cluster(smem_u32(&s_bar[slot]), (ch >> 1) & 1, WAIT_NS))
+            const uint32_t dx = (ch & 1) ? CT_DX1 : CT_DX0;
+            if (tid == 32) bulk_wait_read_all();      // the o staging is free again
+            if (tid == 0 && !s_abort &&
+                !mbar_wait_cluster(smem_u32(&s_bar[slot]), (uint32_t)(ch / NPREPCTA) & 1u, WAIT_NS))
                 expired();
             __syncwarp();
             cta_bar();
             fence_after_sync();
+            // chunk ch - 1 has consumed its slot entirely: give it back to its preparer
+            if (tid == 32 && ch > 0)
+                mbar_arrive_remote(map_to_rank(smem_u32(&s_bar[0]), 1u + (uint32_t)((ch - 1) % NPREPCTA)));
             if (tid == 0 && !s_abort) {
                 const uint32_t id = idesc_tf32(128, 2 * C, false, false);
                 const uint64_t bd0 = sdesc(smem_u32(sm + sb + S_B1), PAD_LBO, SBO_K128P);
 #pragma unroll
                 for (int ks = 0; ks < D / 8; ++ks)
-                    mma_tf32_ts(tm + CT_DX, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                    mma_tf32_ts(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
                                 id, ks > 0 ? 1u : 0u);
                 mma_commit(mbar);
             }
+            if (ch > 0) emit_output(ch - 1);
             wait_mma();
             {   // U = U' - W S  (this half: tokens [16 hh, 16 hh + 16))
                 const float* up = reinterpret_cast<const float*>(sm + sb + S_UP);
                 float x[16];
-                tmem_ld16(tm + lane_base + CT_DX + 16 * hh, x);
+                tmem_ld16(tm + lane_base + dx + 16 * hh, x);
                 wait_ld();
 #pragma unroll
                 for (int r = 0; r < 16; ++r) x[r] = to_tf32(up[(16 * hh + r) * D + j] - x[r]);
@@ -751,12 +783,12 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const uint32_t id2 = idesc_tf32(128, 128, false, false);
                 const uint32_t id3 = idesc_tf32(128, 32, false, false);
                 const uint64_t b20 = sdesc(smem_u32(sm + sb + S_B2), LBO, SBO_K32);
-                const uint64_t b30 = sdesc(smem_u32(sm + sb + S_B3), PAD_LBO, SBO_K32P);
+                const uint64_t b30 = sdesc(smem_u32(sm + sb + S_B3), LBO, SBO_K32);
 #pragma unroll
                 for (int ks = 0; ks < C / 8; ++ks) {
                     mma_tf32_ts(tm + CT_DKU, tm + CT_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
                                 id2, ks > 0 ? 1u : 0u);
-                    mma_tf32_ts(tm + CT_DX + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                    mma_tf32_ts(tm + dx + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * LBO) >> 4),
                                 id3, 1u);
                 }
                 mma_commit(mbar);
@@ -782,31 +814,14 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     }
                     tmem_st16(tm + lane_base + CT_AS + 64 * hh + c0, d);
                 }
+                wait_st();
             }
-            // o of this chunk, then release the slot to its preparer
-            __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
-            {
-                float ov[16];
-                tmem_ld16(tm + lane_base + CT_DX + C + 16 * hh, ov);
-                wait_ld();
-#pragma unroll
-                for (int r = 0; r < 16; ++r) ost[(16 * hh + r) * D + j] = __float2bfloat16_rn(ov[r]);
-            }
-            wait_st();
             fence_before_sync();
-            cta_bar();
-            if (tid == 0) mbar_arrive_remote(map_to_rank(smem_u32(&s_bar[0]), 1u + (uint32_t)slot));
-            const int tb = ch * C;
-#pragma unroll
-            for (int m = 0; m < (C * D / 8) / NTH; ++m) {
-                const int vi = tid + m * NTH;
-                const int r = vi / (D / 8), cv = vi % (D / 8);
-                if (tb + r < T)
-                    *reinterpret_cast<uint4*>(oh + (int64_t)(tb + r) * row_stride + cv * 8) =
-                        *reinterpret_cast<const uint4*>(ost + r * D + cv * 8);
-            }
-            cta_bar();                         // staging read before the next chunk writes it
         }
+        if (tid == 32) bulk_wait_read_all();
+        cta_bar();
+        if (n_chunks > 0) emit_output(n_chunks - 1);
+        if (tid == 32) bulk_wait_all();       // the last o stores have landed
         if (hT && !s_abort) {
             float* hTh = hT + head_off * D * D;
 #pragma unroll
@@ -814,7 +829,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         }
     } else {
         // ================================================== preparing CTAs ==
-        const int par = (int)rank - 1;             // chunks ch with ch % 2 == par
+        const int par = (int)rank - 1;             // chunks ch with ch % NPREPCTA == par
         const int pt = tid;
         const int pw = warp;
         const uint32_t ebar = smem_u32(&s_bar[0]);
@@ -853,10 +868,10 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         const uint32_t full_remote = map_to_rank(smem_u32(&s_bar[par]), 0u);
         const uint32_t slot_remote = map_to_rank(smem_u32(sm + C_SLOT0 + par * SLOT), 0u);
 #pragma unroll 1
-        for (int ch = par; ch < n_chunks; ch += 2) {
+        for (int ch = par; ch < n_chunks; ch += NPREPCTA) {
             if (pt < C) {
                 reinterpret_cast<float*>(sm + P_BETA)[pt] = to_f32(beta_next);
-                const int tn = (ch + 2) * C + pt;
+                const int tn = (ch + NPREPCTA) * C + pt;
                 beta_next = (tn < T) ? beta[((int64_t)b * T + tn) * H + h] : bzero;
             }
             if (pt == 0 && !s_abort && !mbar_wait(rbar, rphase & 1u, WAIT_NS)) expired();
@@ -933,7 +948,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 }
                 mma_commit(mbar);
             }
-            if (ch + 2 < n_chunks) issue_raw(ch + 2);
+            if (ch + NPREPCTA < n_chunks) issue_raw(ch + NPREPCTA);
 #pragma unroll
             for (int rr = 0; rr < TILE; rr += 4)
                 st_f32x4(sm, P_VA + off_kmajor(c, tau * TILE + rr, LBO, SBO_K32),
@@ -1039,7 +1054,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             }
             float pf4[4];
             {
-                const int r = pt >> 3, i = (pt & 7) * 4;
+                const int r = pt & 31, i = (pt >> 5) * 4;     // lane = row: no bank conflicts
 #pragma unroll
                 for (int u = 0; u < 4; ++u) pf4[u] = to_tf32(pm[r * LD + i + u]);
             }
@@ -1064,8 +1079,8 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     st_f32x4(st, S_B2 + off_kmajor(c, tau * TILE + rr, LBO, SBO_K32),
                              kf[rr], kf[rr + 1], kf[rr + 2], kf[rr + 3]);
                 {
-                    const int r = pt >> 3, i = (pt & 7) * 4;
-                    st_f32x4(st, S_B3 + off_kmajor(r, i, PAD_LBO, SBO_K32P), pf4[0], pf4[1], pf4[2], pf4[3]);
+                    const int r = pt & 31, i = (pt >> 5) * 4;
+                    st_f32x4(st, S_B3 + off_kmajor(r, i, LBO, SBO_K32), pf4[0], pf4[1], pf4[2], pf4[3]);
                 }
                 if (tau == 0) reinterpret_cast<float*>(st + S_GAM)[c] = gam_c;
             }
@@ -1073,9 +1088,9 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             fence_before_sync();
             prep_sync();
             if (pt == 0) {
-                // the chain has released this slot (its previous use, chunk ch - 2)
-                if (ch >= 2 && !s_abort && !mbar_wait_cluster(ebar, ephase & 1u, WAIT_NS)) expired();
-                if (ch >= 2) ++ephase;
+                // the chain has released this slot (its previous use, chunk ch - NPREPCTA)
+                if (ch >= NPREPCTA && !s_abort && !mbar_wait_cluster(ebar, ephase & 1u, WAIT_NS)) expired();
+                if (ch >= NPREPCTA) ++ephase;
                 if (!s_abort) {
                     mbar_arrive_expect_tx_remote(full_remote, SLOT);
                     bulk_copy_to_rank(slot_remote, smem_u32(st), SLOT, full_remote);
@@ -1116,15 +1131,15 @@ static bool make_map(CUtensorMap* map, const void* base, int B, int T, int H)
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Three SMs per head pay off while the heads alone leave most SMs idle:
-// up to 48 heads (144 of the 148 SMs); larger batches use one SM per head.
+// Four SMs per head pay off while the heads alone leave most SMs idle:
+// up to 37 heads (148 SMs); larger batches use one SM per head.
 // KDA_PREFILL_VARIANT=fused|cluster overrides the choice (for measurement).
 static bool use_cluster_variant(int B, int H)
 {
     const char* env = getenv("KDA_PREFILL_VARIANT");
     if (env && strcmp(env, "cluster") == 0) return true;
     if (env && strcmp(env, "fused") == 0) return false;
-    return (int64_t)B * H * 3 <= 144;
+    return (int64_t)B * H * (pc::NPREPCTA + 1) <= 148;
 }
 
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
@@ -1139,14 +1154,14 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    CUtensorMap mq, mk, mv, mg;
+    CUtensorMap mq, mk, mv, mg, mo;
     if (T > 0) {
         if (!make_map(&mq, q, B, T, H) || !make_map(&mk, k, B, T, H) ||
-            !make_map(&mv, v, B, T, H) || !make_map(&mg, g, B, T, H))
+            !make_map(&mv, v, B, T, H) || !make_map(&mg, g, B, T, H) || !make_map(&mo, o, B, T, H))
             return cudaErrorInvalidValue;
     } else {   // no chunk, no load: the kernel only carries h0 to hT
         memset(&mq, 0, sizeof(mq)); memset(&mk, 0, sizeof(mk));
-        memset(&mv, 0, sizeof(mv)); memset(&mg, 0, sizeof(mg));
+        memset(&mv, 0, sizeof(mv)); memset(&mg, 0, sizeof(mg)); memset(&mo, 0, sizeof(mo));
     }
     if (use_cluster_variant(B, H)) {
         static bool cattr_set = false;
@@ -1157,9 +1172,9 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
             if (e != cudaSuccess) return e;
             cattr_set = true;
         }
-        dim3 grid(3 * H, B);
+        dim3 grid((pc::NPREPCTA + 1) * H, B);
         prefill_cluster_kernel<<<grid, pc::NTH, pc::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
+            mq, mk, mv, mg, mo, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
     } else {
         dim3 grid(H, B);
         prefill_tc_kernel<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(
