@@ -130,6 +130,12 @@ __device__ __forceinline__ void named_arrive(uint32_t id, uint32_t count) {
     asm volatile("bar.arrive %0, %1;" :: "r"(id), "r"(count) : "memory");
 }
 
+// A shared flag read once by lane 0 and broadcast: the same value in every
+// lane, so a whole-warp MMA issue never diverges on it.
+__device__ __forceinline__ bool warp_flag(const int& flag) {
+    return __shfl_sync(0xffffffffu, *(const volatile int*)&flag, 0) != 0;
+}
+
 __global__ void __launch_bounds__(pf::NT, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -213,14 +219,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             // X = S^T [W | Qt]^T  (one N = 64 MMA per K step; the issue loop is
             // unrolled with constant descriptor increments: the per-instruction
             // issue cost, not the math, bounds these small-N MMAs)
-            if (tid == 0 && !s_abort) {
+            if (warp == 0 && !warp_flag(s_abort)) {
                 const uint32_t id = idesc_tf32(128, 2 * C, false, false);
                 const uint64_t bd0 = sdesc(smem_u32(sm + B1), PAD_LBO, SBO_K128P);
 #pragma unroll
                 for (int ks = 0; ks < D / 8; ++ks)
-                    mma_tf32_ts(tm + T_DX, tm + T_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
-                                id, ks > 0 ? 1u : 0u);
-                mma_commit(bar);
+                    mma_tf32_ts_w(tm + T_DX, tm + T_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                  id, ks > 0 ? 1u : 0u);
+                mma_commit_w(bar);
             }
             wait_mma();
             {   // U = U' - W S  (this half: tokens [16 hh, 16 hh + 16))
@@ -236,19 +242,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             fence_before_sync();
             named_bar(BAR_CHAIN, NCH);
             fence_after_sync();
-            if (tid == 0 && !s_abort) {
+            if (warp == 0 && !warp_flag(s_abort)) {
                 const uint32_t id2 = idesc_tf32(128, 128, false, false);
                 const uint32_t id3 = idesc_tf32(128, 32, false, false);
                 const uint64_t b20 = sdesc(smem_u32(sm + B2), LBO, SBO_K32);
                 const uint64_t b30 = sdesc(smem_u32(sm + B3), PAD_LBO, SBO_K32P);
 #pragma unroll
                 for (int ks = 0; ks < C / 8; ++ks) {
-                    mma_tf32_ts(tm + T_DKU, tm + T_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
-                                id2, ks > 0 ? 1u : 0u);
-                    mma_tf32_ts(tm + T_DX + C, tm + T_AU + ks * 8, b30 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
-                                id3, 1u);
+                    mma_tf32_ts_w(tm + T_DKU, tm + T_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                  id2, ks > 0 ? 1u : 0u);
+                    mma_tf32_ts_w(tm + T_DX + C, tm + T_AU + ks * 8, b30 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                  id3, 1u);
                 }
-                mma_commit(bar);
+                mma_commit_w(bar);
             }
             wait_mma();
             // B1, B2, B3 are no longer read: the prep may fill the next chunk's
@@ -422,16 +428,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             fence_after_sync();
             // ---- Gram: D_G = [Kh_0; Kh_1; Kb_0; pad] [Kt_0 Kt_1 | Qt_0 Qt_1]^T,
             // and the next chunk's inputs; V^T is written while the MMA runs
-            if (pt == 0 && !s_abort) {
+            if (pw == 0 && !warp_flag(s_abort)) {
                 const uint32_t id = idesc_tf32(64, 64, false, false);
                 const uint64_t ad0 = sdesc(smem_u32(sm + GA), PAD_LBO, SBO_K128P);
                 const uint64_t bd0 = sdesc(smem_u32(sm + GB), PAD_LBO, SBO_K128P);
 #pragma unroll
                 for (int ks = 0; ks < D / 8; ++ks) {
                     const uint64_t step = (uint64_t)((ks * 2 * PAD_LBO) >> 4);
-                    mma_tf32_ss(tm + T_DG, ad0 + step, bd0 + step, id, ks > 0 ? 1u : 0u);
+                    mma_tf32_ss_w(tm + T_DG, ad0 + step, bd0 + step, id, ks > 0 ? 1u : 0u);
                 }
-                mma_commit(bar);
+                mma_commit_w(bar);
             }
             if (ch + 1 < n_chunks) issue_raw(ch + 1);
 #pragma unroll
@@ -520,7 +526,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             prep_sync();
             fence_after_sync();
             // ---- W^T = Kt^T T^T and U'^T = V^T T^T  (M 128, N 32, K 32)
-            if (pt == 0 && !s_abort) {
+            if (pw == 0 && !warp_flag(s_abort)) {
                 const uint32_t id = idesc_tf32(128, 32, false, false);
                 const uint64_t bd0 = sdesc(smem_u32(sm + TB), PAD_LBO, SBO_K32P);
                 const uint64_t aw0 = sdesc(smem_u32(sm + WA), LBO, SBO_K32);
@@ -530,10 +536,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int ks = 0; ks < C / 8; ++ks) {
                     const uint64_t bstep = (uint64_t)((ks * 2 * PAD_LBO) >> 4);
                     const uint64_t astep = (uint64_t)((ks * 2 * LBO) >> 4);
-                    mma_tf32_ss(tm + T_DW, aw0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
-                    mma_tf32_ss(du, av0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                    mma_tf32_ss_w(tm + T_DW, aw0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                    mma_tf32_ss_w(du, av0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
                 }
-                mma_commit(bar);
+                mma_commit_w(bar);
             }
             // operands of the fill that do not come from the W MMA, read now
             const float* gaf = reinterpret_cast<const float*>(sm + GA);
@@ -607,7 +613,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // The arithmetic is the one of prefill_tc_kernel.
 namespace pc {
 using namespace pf;
-constexpr int NTH = 256;                                      // threads per CTA (both roles)
+constexpr int NCW = 256;                                      // compute threads per CTA (both roles)
+constexpr int NX = NCW + 32;                                  // compute warps + one helper warp (hand-overs)
+constexpr int NTH = NCW + 64;                                 // plus an issuer warp and a remote-traffic warp
+// named barriers (0 is __syncthreads): issuer hand-overs and compute-warp syncs
+constexpr uint32_t NB_ASA = 1, NB_ASB = 2, NB_U = 3, NB_CW = 4;                 // chain CTA
+constexpr uint32_t NB_G = 5, NB_TB = 6, NB_STFREE = 7, NB_FILL = 8;              // preparing CTAs
 constexpr int NPREPCTA = 3;                                   // preparing CTAs per cluster (= slots)
 // slot / staging layout (identical in rank 0's slots and a preparer's staging)
 constexpr uint32_t S_B1 = 0;                                   // [W | Qt]: N 64 x K 128 (padded)
@@ -657,7 +668,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     using namespace tc;
     extern __shared__ __align__(1024) unsigned char sm[];
     __shared__ uint32_t s_taddr;
-    __shared__ __align__(8) uint64_t s_bar[4];   // rank 0: FULL[0..2], MMA; ranks 1-3: EMPTY, MMA, input loads
+    __shared__ __align__(8) uint64_t s_bar[5];   // rank 0: FULL[0..2], MMA, o; ranks 1-3: EMPTY, MMA, input loads
     __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -672,7 +683,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
+        for (int i = 0; i < 5; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
         fence_mbar_init();
         s_abort = 0;
     }
@@ -690,116 +701,115 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
     if (rank == 0) {
         // ========================================================= chain CTA ==
-        // Chunk ch: FULL wait, X = S^T [W | Qt]^T, U, the update MMAs and the
-        // state update.  The output of chunk ch - 1 (its X buffer is the other
-        // of two) is read out, staged and stored while chunk ch's first MMA
-        // runs, so it stays off the sequential path.
-        const int j = 32 * sp + lane;
-        const int hh = warp >> 2;
-        const uint32_t mbar = smem_u32(&s_bar[3]);
-        uint32_t phase = 0;
-        auto cta_bar = [&]() { __syncthreads(); };
-        auto wait_mma = [&]() {
-            if (tid == 0 && !s_abort && !mbar_wait(mbar, phase & 1u, WAIT_NS)) expired();
-            ++phase;
-            __syncwarp();
-            cta_bar();
-            fence_after_sync();
-        };
-        float S[D / 2];
-        {
-            const float* h0h = h0 ? h0 + head_off * D * D : nullptr;
-#pragma unroll
-            for (int i = 0; i < D / 2; ++i) S[i] = h0h ? h0h[(int64_t)(64 * hh + i) * D + j] : 0.f;
-#pragma unroll
-            for (int c0 = 0; c0 < D / 2; c0 += 32) {
-                float t32[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) t32[i] = to_tf32(S[c0 + i]);
-                tmem_st32(tm + lane_base + CT_AS + 64 * hh + c0, t32);
-            }
-            wait_st();
-        }
-        // o of chunk cp (X buffer cp & 1) -> staging -> one TMA store (thread
-        // 32, whose previous store has read the staging before the last CTA
-        // barrier)
-        auto emit_output = [&](int cp) {
-            const uint32_t dx = (cp & 1) ? CT_DX1 : CT_DX0;
-            __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
-            float ov[16];
-            tmem_ld16(tm + lane_base + dx + C + 16 * hh, ov);
-            wait_ld();
-#pragma unroll
-            for (int r = 0; r < 16; ++r) ost[(16 * hh + r) * D + j] = __float2bfloat16_rn(ov[r]);
-            fence_smem_to_async();
-            fence_before_sync();
-            cta_bar();
-            fence_after_sync();
-            if (tid == 32) {
-                tma_store_3d(&tm_o, h * D, cp * C, b, smem_u32(ost));
-                bulk_commit();
-            }
-        };
+        const uint32_t mbar = smem_u32(&s_bar[3]);   // X, then Kb^T U, of each chunk
+        const uint32_t obar = smem_u32(&s_bar[4]);   // P U of each chunk (its output complete)
+        if (warp == NCW / 32) {
+            // ------------------------------------------------------ issuer warp --
+            // Chunk ch: X = S^T [W | Qt]^T in two d_k halves (each as soon as
+            // the compute warps have written that half of the tf32 state), then
+            // Kb^T U and P U once U is in tensor memory.
+            const uint32_t id1 = idesc_tf32(128, 2 * C, false, false);
+            const uint32_t id2 = idesc_tf32(128, 128, false, false);
+            const uint32_t id3 = idesc_tf32(128, 32, false, false);
 #pragma unroll 1
-        for (int ch = 0; ch < n_chunks; ++ch) {
-            const int slot = ch % NPREPCTA;
-            const uint32_t sb = C_SLOT0 + slot * SLOT;
-            const uint32_t dx = (ch & 1) ? CT_DX1 : CT_DX0;
-            if (tid == 32) bulk_wait_read_all();      // the o staging is free again
-            if (tid == 0 && !s_abort &&
-                !mbar_wait_cluster(smem_u32(&s_bar[slot]), (uint32_t)(ch / NPREPCTA) & 1u, WAIT_NS))
-                expired();
-            __syncwarp();
-            cta_bar();
-            fence_after_sync();
-            // chunk ch - 1 has consumed its slot entirely: give it back to its preparer
-            if (tid == 32 && ch > 0)
-                mbar_arrive_remote(map_to_rank(smem_u32(&s_bar[0]), 1u + (uint32_t)((ch - 1) % NPREPCTA)));
-            if (tid == 0 && !s_abort) {
-                const uint32_t id = idesc_tf32(128, 2 * C, false, false);
+            for (int ch = 0; ch < n_chunks; ++ch) {
+                const int slot = ch % NPREPCTA;
+                const uint32_t sb = C_SLOT0 + slot * SLOT;
+                const uint32_t dx = (ch & 1) ? CT_DX1 : CT_DX0;
                 const uint64_t bd0 = sdesc(smem_u32(sm + sb + S_B1), PAD_LBO, SBO_K128P);
+                if (lane == 0 && !s_abort &&
+                    !mbar_wait_cluster(smem_u32(&s_bar[slot]), (uint32_t)(ch / NPREPCTA) & 1u, WAIT_NS))
+                    expired();
+                __syncwarp();
+                named_bar(NB_ASA, NX);
+                fence_after_sync();
+                if (!warp_flag(s_abort)) {
 #pragma unroll
-                for (int ks = 0; ks < D / 8; ++ks)
-                    mma_tf32_ts(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
-                                id, ks > 0 ? 1u : 0u);
-                mma_commit(mbar);
+                    for (int ks = 0; ks < D / 16; ++ks)
+                        mma_tf32_ts_w(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                      id1, ks > 0 ? 1u : 0u);
+                }
+                __syncwarp();
+                named_bar(NB_ASB, NX);
+                fence_after_sync();
+                if (!warp_flag(s_abort)) {
+#pragma unroll
+                    for (int ks = D / 16; ks < D / 8; ++ks)
+                        mma_tf32_ts_w(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                      id1, 1u);
+                    mma_commit_w(mbar);
+                }
+                __syncwarp();
+                named_bar(NB_U, NX);
+                fence_after_sync();
+                if (!warp_flag(s_abort)) {
+                    const uint64_t b20 = sdesc(smem_u32(sm + sb + S_B2), LBO, SBO_K32);
+                    const uint64_t b30 = sdesc(smem_u32(sm + sb + S_B3), LBO, SBO_K32);
+#pragma unroll
+                    for (int ks = 0; ks < C / 8; ++ks)
+                        mma_tf32_ts_w(tm + CT_DKU, tm + CT_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                      id2, ks > 0 ? 1u : 0u);
+                    mma_commit_w(mbar);
+#pragma unroll
+                    for (int ks = 0; ks < C / 8; ++ks)
+                        mma_tf32_ts_w(tm + dx + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                      id3, 1u);
+                    mma_commit_w(obar);
+                }
+                __syncwarp();
             }
-            if (ch > 0) emit_output(ch - 1);
-            wait_mma();
-            {   // U = U' - W S  (this half: tokens [16 hh, 16 hh + 16))
-                const float* up = reinterpret_cast<const float*>(sm + sb + S_UP);
-                float x[16];
-                tmem_ld16(tm + lane_base + dx + 16 * hh, x);
-                wait_ld();
+        } else if (warp == NCW / 32 + 1) {
+            // ------------------------------------------------------ release warp --
+            // Once the last MMA of chunk ch - 1 (P U) is done, nothing reads its
+            // slot any more: hand it back to its preparer.  A remote arrive is
+            // slow, so it stays off the issuer's and the compute warps' path.
+#pragma unroll 1
+            for (int ch = 1; ch < n_chunks; ++ch) {
+                if (lane == 0) {
+                    if (!s_abort && !mbar_wait(obar, (uint32_t)(ch - 1) & 1u, WAIT_NS)) expired();
+                    mbar_arrive_remote(map_to_rank(smem_u32(&s_bar[0]), 1u + (uint32_t)((ch - 1) % NPREPCTA)));
+                }
+                __syncwarp();
+            }
+        } else {
+            // ----------------------------------------------------- compute warps --
+            // Per chunk ch: the state update of chunk ch - 1 by d_k halves (each
+            // half handed to the issuer as soon as it is in tensor memory), the
+            // output of chunk ch - 1 (staged and written by TMA while X of chunk
+            // ch is computed), then U = U' - W S.
+            const int j = 32 * sp + lane;                // dv row = TMEM lane
+            const int hh = warp >> 2;                     // d_k columns [32 hh, +32) and [64 + 32 hh, +32)
+            uint32_t phase = 0;
+            auto cw_bar = [&]() { named_bar(NB_CW, NCW); };
+            auto wait_bar = [&](uint32_t bar, uint32_t parity) {
+                if (tid == 0 && !s_abort && !mbar_wait(bar, parity, WAIT_NS)) expired();
+                __syncwarp();
+                cw_bar();
+                fence_after_sync();
+            };
+            // S[32 q + i] holds d_k column 64 q + 32 hh + i of this thread's dv row
+            float S[D / 2];
+            {
+                const float* h0h = h0 ? h0 + head_off * D * D : nullptr;
 #pragma unroll
-                for (int r = 0; r < 16; ++r) x[r] = to_tf32(up[(16 * hh + r) * D + j] - x[r]);
-                tmem_st16(tm + lane_base + CT_AU + 16 * hh, x);
+                for (int q2 = 0; q2 < 2; ++q2) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        S[32 * q2 + i] = h0h ? h0h[(int64_t)(64 * q2 + 32 * hh + i) * D + j] : 0.f;
+                    float t32[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) t32[i] = to_tf32(S[32 * q2 + i]);
+                    tmem_st32(tm + lane_base + CT_AS + 64 * q2 + 32 * hh, t32);
+                }
                 wait_st();
             }
-            fence_before_sync();
-            cta_bar();
-            fence_after_sync();
-            if (tid == 0 && !s_abort) {
-                const uint32_t id2 = idesc_tf32(128, 128, false, false);
-                const uint32_t id3 = idesc_tf32(128, 32, false, false);
-                const uint64_t b20 = sdesc(smem_u32(sm + sb + S_B2), LBO, SBO_K32);
-                const uint64_t b30 = sdesc(smem_u32(sm + sb + S_B3), LBO, SBO_K32);
+            // S <- Diag(gamma_C) S + Kb^T U on d_k half q2 (gamma of the slot at sbp)
+            auto state_half = [&](int q2, uint32_t sbp) {
+                const float4* gam4 = reinterpret_cast<const float4*>(sm + sbp + S_GAM) + 16 * q2 + 8 * hh;
 #pragma unroll
-                for (int ks = 0; ks < C / 8; ++ks) {
-                    mma_tf32_ts(tm + CT_DKU, tm + CT_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
-                                id2, ks > 0 ? 1u : 0u);
-                    mma_tf32_ts(tm + dx + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * LBO) >> 4),
-                                id3, 1u);
-                }
-                mma_commit(mbar);
-            }
-            wait_mma();
-            {   // S <- Diag(gamma_C) S + Kb^T U ; refresh the tf32 copy
-                const float4* gam4 = reinterpret_cast<const float4*>(sm + sb + S_GAM) + 16 * hh;
-#pragma unroll
-                for (int c0 = 0; c0 < D / 2; c0 += 16) {
+                for (int c0 = 0; c0 < 32; c0 += 16) {
                     float d[16];
-                    tmem_ld16(tm + lane_base + CT_DKU + 64 * hh + c0, d);
+                    tmem_ld16(tm + lane_base + CT_DKU + 64 * q2 + 32 * hh + c0, d);
                     wait_ld();
 #pragma unroll
                     for (int i4 = 0; i4 < 4; ++i4) {
@@ -808,35 +818,174 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             const int i = c0 + i4 * 4 + u;
-                            S[i] = fmaf(gg[u], S[i], d[i - c0]);
-                            d[i - c0] = to_tf32(S[i]);
+                            S[32 * q2 + i] = fmaf(gg[u], S[32 * q2 + i], d[i - c0]);
+                            d[i - c0] = to_tf32(S[32 * q2 + i]);
                         }
                     }
-                    tmem_st16(tm + lane_base + CT_AS + 64 * hh + c0, d);
+                    tmem_st16(tm + lane_base + CT_AS + 64 * q2 + 32 * hh + c0, d);
                 }
                 wait_st();
-            }
-            fence_before_sync();
-        }
-        if (tid == 32) bulk_wait_read_all();
-        cta_bar();
-        if (n_chunks > 0) emit_output(n_chunks - 1);
-        if (tid == 32) bulk_wait_all();       // the last o stores have landed
-        if (hT && !s_abort) {
-            float* hTh = hT + head_off * D * D;
+            };
+            // o of chunk cp (X buffer cp & 1, complete once obar's phase cp has
+            // passed) -> staging -> one TMA store by thread 0
+            auto emit_output = [&](int cp) {
+                const uint32_t dx = (cp & 1) ? CT_DX1 : CT_DX0;
+                __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
+                if (tid == 0) bulk_wait_read_all();   // the previous store has read the staging
+                wait_bar(obar, (uint32_t)cp & 1u);
+                float ov[16];
+                tmem_ld16(tm + lane_base + dx + C + 16 * hh, ov);
+                wait_ld();
 #pragma unroll
-            for (int i = 0; i < D / 2; ++i) hTh[(int64_t)(64 * hh + i) * D + j] = S[i];
+                for (int r = 0; r < 16; ++r) ost[(16 * hh + r) * D + j] = __float2bfloat16_rn(ov[r]);
+                fence_smem_to_async();
+                cw_bar();
+                if (tid == 0) {
+                    tma_store_3d(&tm_o, h * D, cp * C, b, smem_u32(ost));
+                    bulk_commit();
+                }
+            };
+            fence_before_sync();
+            if (n_chunks > 0) {                       // the initial state for chunk 0
+                named_arrive(NB_ASA, NX);
+                named_arrive(NB_ASB, NX);
+            }
+#pragma unroll 1
+            for (int ch = 0; ch < n_chunks; ++ch) {
+                const int slot = ch % NPREPCTA;
+                const uint32_t sb = C_SLOT0 + slot * SLOT;
+                const uint32_t dx = (ch & 1) ? CT_DX1 : CT_DX0;
+                if (ch > 0) {
+                    const uint32_t sbp = C_SLOT0 + ((ch - 1) % NPREPCTA) * SLOT;
+                    state_half(0, sbp);
+                    fence_before_sync();
+                    named_arrive(NB_ASA, NX);
+                    state_half(1, sbp);
+                    fence_before_sync();
+                    named_arrive(NB_ASB, NX);
+                    emit_output(ch - 1);
+                }
+                // X of chunk ch (U' of this chunk is in the slot once its FULL phase passed)
+                if (tid == 0 && !s_abort &&
+                    !mbar_wait_cluster(smem_u32(&s_bar[slot]), (uint32_t)(ch / NPREPCTA) & 1u, WAIT_NS))
+                    expired();
+                wait_bar(mbar, phase & 1u);
+                ++phase;
+                {   // U = U' - W S  (this thread: tokens [16 hh, 16 hh + 16))
+                    const float* up = reinterpret_cast<const float*>(sm + sb + S_UP);
+                    float x[16];
+                    tmem_ld16(tm + lane_base + dx + 16 * hh, x);
+                    wait_ld();
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) x[r] = to_tf32(up[(16 * hh + r) * D + j] - x[r]);
+                    tmem_st16(tm + lane_base + CT_AU + 16 * hh, x);
+                    wait_st();
+                }
+                fence_before_sync();
+                named_arrive(NB_U, NX);
+                wait_bar(mbar, phase & 1u);           // Kb^T U of chunk ch
+                ++phase;
+            }
+            if (n_chunks > 0) {
+                const uint32_t sbp = C_SLOT0 + ((n_chunks - 1) % NPREPCTA) * SLOT;
+                state_half(0, sbp);
+                state_half(1, sbp);
+                emit_output(n_chunks - 1);
+            }
+            if (tid == 0) bulk_wait_all();           // the last o stores have landed
+            if (hT && !s_abort) {
+                float* hTh = hT + head_off * D * D;
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) hTh[(int64_t)(64 * q2 + 32 * hh + i) * D + j] = S[32 * q2 + i];
+            }
         }
     } else {
         // ================================================== preparing CTAs ==
         const int par = (int)rank - 1;             // chunks ch with ch % NPREPCTA == par
-        const int pt = tid;
-        const int pw = warp;
         const uint32_t ebar = smem_u32(&s_bar[0]);
         const uint32_t mbar = smem_u32(&s_bar[1]);
         const uint32_t rbar = smem_u32(&s_bar[2]);
-        uint32_t phase = 0, rphase = 0, ephase = 0;
-        auto prep_sync = [&]() { __syncthreads(); };
+        unsigned char* st = sm + P_ST;
+        if (warp == NCW / 32) {
+            // ------------------------------------------------------ issuer warp --
+            // MMAs and input loads: the compute warps hand over at named
+            // barriers and never wait on an issue.
+            auto issue_raw = [&](int ci) {
+                mbar_arrive_expect_tx(rbar, 4 * RAW_T);
+                tma_load_3d(smem_u32(sm + P_RAW + 0 * RAW_T), &tm_q, h * D, ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + P_RAW + 1 * RAW_T), &tm_k, h * D, ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + P_RAW + 2 * RAW_T), &tm_v, h * D, ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + P_RAW + 3 * RAW_T), &tm_g, h * D, ci * C, b, rbar);
+            };
+            if (lane == 0 && par < n_chunks) issue_raw(par);
+#pragma unroll 1
+            for (int ch = par; ch < n_chunks; ch += NPREPCTA) {
+                __syncwarp();
+                named_bar(NB_G, NX);                  // Gram operands written, raw inputs consumed
+                fence_after_sync();
+                if (!warp_flag(s_abort)) {
+                    const uint32_t id = idesc_tf32(64, 64, false, false);
+                    const uint64_t ad0 = sdesc(smem_u32(sm + P_GA), PAD_LBO, SBO_K128P);
+                    const uint64_t bd0 = sdesc(smem_u32(sm + P_GB), PAD_LBO, SBO_K128P);
+#pragma unroll
+                    for (int ks = 0; ks < D / 8; ++ks) {
+                        const uint64_t step = (uint64_t)((ks * 2 * PAD_LBO) >> 4);
+                        mma_tf32_ss_w(tm + PT_DG, ad0 + step, bd0 + step, id, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit_w(mbar);
+                }
+                if (lane == 0 && ch + NPREPCTA < n_chunks) issue_raw(ch + NPREPCTA);
+                __syncwarp();
+                named_bar(NB_TB, NX);                 // T, K~ f and V staged
+                fence_after_sync();
+                if (!warp_flag(s_abort)) {
+                    const uint32_t id = idesc_tf32(128, 32, false, false);
+                    const uint64_t bd0 = sdesc(smem_u32(sm + P_TB), PAD_LBO, SBO_K32P);
+                    const uint64_t aw0 = sdesc(smem_u32(sm + P_WA), LBO, SBO_K32);
+                    const uint64_t av0 = sdesc(smem_u32(sm + P_VA), LBO, SBO_K32);
+#pragma unroll
+                    for (int ks = 0; ks < C / 8; ++ks) {
+                        const uint64_t bstep = (uint64_t)((ks * 2 * PAD_LBO) >> 4);
+                        const uint64_t astep = (uint64_t)((ks * 2 * LBO) >> 4);
+                        mma_tf32_ss_w(tm + PT_DW, aw0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                        mma_tf32_ss_w(tm + PT_DU, av0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit_w(mbar);
+                }
+            }
+        } else if (warp == NCW / 32 + 1) {
+            // --------------------------------------------------------- push warp --
+            // Each prepared chunk goes to its slot in the chain CTA as one bulk
+            // copy, once the chain has released the slot; then the staging is
+            // handed back to the compute warps.
+            uint32_t ephase = 0;
+            const uint32_t full_remote = map_to_rank(smem_u32(&s_bar[par]), 0u);
+            const uint32_t slot_remote = map_to_rank(smem_u32(sm + C_SLOT0 + par * SLOT), 0u);
+#pragma unroll 1
+            for (int ch = par; ch < n_chunks; ch += NPREPCTA) {
+                named_bar(NB_FILL, NX);               // the staging holds chunk ch
+                if (lane == 0) {
+                    // the chain has released this slot (its previous use, chunk ch - NPREPCTA)
+                    if (ch >= NPREPCTA && !s_abort && !mbar_wait_cluster(ebar, ephase & 1u, WAIT_NS)) expired();
+                    if (ch >= NPREPCTA) ++ephase;
+                    if (!s_abort) {
+                        mbar_arrive_expect_tx_remote(full_remote, SLOT);
+                        bulk_copy_to_rank(slot_remote, smem_u32(st), SLOT, full_remote);
+                        bulk_commit();
+                    }
+                    bulk_wait_read_all();             // the copy has read the staging
+                }
+                __syncwarp();
+                if (ch + NPREPCTA < n_chunks) named_arrive(NB_STFREE, NX);
+            }
+        } else {
+        // ---------------------------------------------------------- compute warps --
+        const int pt = tid;
+        const int pw = warp;
+        uint32_t phase = 0, rphase = 0;
+        auto prep_sync = [&]() { named_bar(NB_CW, NCW); };
         auto wait_mma = [&]() {
             if (pt == 0 && !s_abort && !mbar_wait(mbar, phase & 1u, WAIT_NS)) expired();
             ++phase;
@@ -844,16 +993,6 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             prep_sync();
             fence_after_sync();
         };
-        auto issue_raw = [&](int ci) {
-            if (pt == 0) {
-                mbar_arrive_expect_tx(rbar, 4 * RAW_T);
-                tma_load_3d(smem_u32(sm + P_RAW + 0 * RAW_T), &tm_q, h * D, ci * C, b, rbar);
-                tma_load_3d(smem_u32(sm + P_RAW + 1 * RAW_T), &tm_k, h * D, ci * C, b, rbar);
-                tma_load_3d(smem_u32(sm + P_RAW + 2 * RAW_T), &tm_v, h * D, ci * C, b, rbar);
-                tma_load_3d(smem_u32(sm + P_RAW + 3 * RAW_T), &tm_g, h * D, ci * C, b, rbar);
-            }
-        };
-        if (par < n_chunks) issue_raw(par);
         const __nv_bfloat16 bzero = __float2bfloat16_rn(0.f);
         __nv_bfloat16 beta_next = (pt < C && par * C + pt < T) ? beta[((int64_t)b * T + par * C + pt) * H + h] : bzero;
         const int tau = pt >> 7;
@@ -864,9 +1003,6 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         float* tmx = reinterpret_cast<float*>(sm + P_TMS);
         float* ym = reinterpret_cast<float*>(sm + P_YMS);
         const float* bt = reinterpret_cast<const float*>(sm + P_BETA);
-        unsigned char* st = sm + P_ST;
-        const uint32_t full_remote = map_to_rank(smem_u32(&s_bar[par]), 0u);
-        const uint32_t slot_remote = map_to_rank(smem_u32(sm + C_SLOT0 + par * SLOT), 0u);
 #pragma unroll 1
         for (int ch = par; ch < n_chunks; ch += NPREPCTA) {
             if (pt < C) {
@@ -935,20 +1071,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             }
             fence_smem_to_async();
             fence_before_sync();
-            prep_sync();
-            fence_after_sync();
-            if (pt == 0 && !s_abort) {
-                const uint32_t id = idesc_tf32(64, 64, false, false);
-                const uint64_t ad0 = sdesc(smem_u32(sm + P_GA), PAD_LBO, SBO_K128P);
-                const uint64_t bd0 = sdesc(smem_u32(sm + P_GB), PAD_LBO, SBO_K128P);
-#pragma unroll
-                for (int ks = 0; ks < D / 8; ++ks) {
-                    const uint64_t step = (uint64_t)((ks * 2 * PAD_LBO) >> 4);
-                    mma_tf32_ss(tm + PT_DG, ad0 + step, bd0 + step, id, ks > 0 ? 1u : 0u);
-                }
-                mma_commit(mbar);
-            }
-            if (ch + NPREPCTA < n_chunks) issue_raw(ch + NPREPCTA);
+            named_arrive(NB_G, NX);
 #pragma unroll
             for (int rr = 0; rr < TILE; rr += 4)
                 st_f32x4(sm, P_VA + off_kmajor(c, tau * TILE + rr, LBO, SBO_K32),
@@ -1026,22 +1149,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             }
             fence_smem_to_async();
             fence_before_sync();
-            prep_sync();
-            fence_after_sync();
-            if (pt == 0 && !s_abort) {
-                const uint32_t id = idesc_tf32(128, 32, false, false);
-                const uint64_t bd0 = sdesc(smem_u32(sm + P_TB), PAD_LBO, SBO_K32P);
-                const uint64_t aw0 = sdesc(smem_u32(sm + P_WA), LBO, SBO_K32);
-                const uint64_t av0 = sdesc(smem_u32(sm + P_VA), LBO, SBO_K32);
-#pragma unroll
-                for (int ks = 0; ks < C / 8; ++ks) {
-                    const uint64_t bstep = (uint64_t)((ks * 2 * PAD_LBO) >> 4);
-                    const uint64_t astep = (uint64_t)((ks * 2 * LBO) >> 4);
-                    mma_tf32_ss(tm + PT_DW, aw0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
-                    mma_tf32_ss(tm + PT_DU, av0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
-                }
-                mma_commit(mbar);
-            }
+            named_arrive(NB_TB, NX);
             const float* gaf = reinterpret_cast<const float*>(sm + P_GA);
             const float* gbf = reinterpret_cast<const float*>(sm + P_GB);
             float qf[TILE], kf[TILE];
@@ -1059,8 +1167,8 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 for (int u = 0; u < 4; ++u) pf4[u] = to_tf32(pm[r * LD + i + u]);
             }
             // the previous chunk's bulk copy has finished reading the staging
-            if (pt == 0) bulk_wait_read_all();
             wait_mma();
+            if (ch != par) named_bar(NB_STFREE, NX);  // the previous push has read the staging
             {
                 float w[16], upv[16];
                 tmem_ld16(tm + lane_base + PT_DW + 16 * tau, w);
@@ -1085,20 +1193,9 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 if (tau == 0) reinterpret_cast<float*>(st + S_GAM)[c] = gam_c;
             }
             fence_smem_to_async();
-            fence_before_sync();
-            prep_sync();
-            if (pt == 0) {
-                // the chain has released this slot (its previous use, chunk ch - NPREPCTA)
-                if (ch >= NPREPCTA && !s_abort && !mbar_wait_cluster(ebar, ephase & 1u, WAIT_NS)) expired();
-                if (ch >= NPREPCTA) ++ephase;
-                if (!s_abort) {
-                    mbar_arrive_expect_tx_remote(full_remote, SLOT);
-                    bulk_copy_to_rank(slot_remote, smem_u32(st), SLOT, full_remote);
-                    bulk_commit();
-                }
-            }
+            named_arrive(NB_FILL, NX);
         }
-        if (pt == 0) bulk_wait_read_all();
+        }
     }
 
     fence_before_sync();
