@@ -606,11 +606,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // prepare the chunks ch with ch % 3 == rank - 1, each in its own SM, and push
 // every prepared chunk (the chain's operands and U') into slot ch % 3 of rank
 // 0's shared memory with a single bulk copy (shared::cta -> shared::cluster,
-// no multicast).  FULL[slot] (rank 0) counts the copy's bytes; EMPTY (the
-// preparing CTA) is arrived on by rank 0 as soon as the chunk's state update
-// has consumed the slot.  o is written with a TMA store from a staging
-// buffer, one chunk late, while the next chunk's first MMA runs.
-// The arithmetic is the one of prefill_tc_kernel.
+// no multicast).  FULL[slot] (rank 0) counts the copy's bytes and is armed by
+// rank 0 itself when it hands the slot back; EMPTY (the preparing CTA) is
+// arrived on by rank 0 once the chunk's MMAs are done and its decay applied.
+// o of a chunk is written from registers, one chunk late, while the next
+// chunk's first MMA runs.  The arithmetic is the one of prefill_tc_kernel.
 namespace pc {
 using namespace pf;
 constexpr int NCW = 256;                                      // compute threads per CTA (both roles)
@@ -628,10 +628,9 @@ constexpr uint32_t S_GAM = S_B3 + (C / 8) * SBO_K32;           // gamma_C, 128 f
 constexpr uint32_t S_UP = S_GAM + D * 4;                       // U' [32 tokens][128] fp32
 constexpr uint32_t SLOT = S_UP + C * D * 4;                    // bytes per chunk
 static_assert(SLOT % 16 == 0, "bulk copy size");
-// rank 0 (chain): NPREPCTA slots and the o staging of one chunk
+// rank 0 (chain): NPREPCTA slots
 constexpr uint32_t C_SLOT0 = 0;
-constexpr uint32_t C_OST = NPREPCTA * SLOT;
-constexpr uint32_t C_BYTES = C_OST + C * D * 2;
+constexpr uint32_t C_BYTES = NPREPCTA * SLOT;
 // ranks 1, 2 (preparation)
 constexpr uint32_t P_RAW = 0;
 constexpr uint32_t P_BETA = P_RAW + 4 * RAW_T;
@@ -651,7 +650,7 @@ constexpr uint32_t P_BYTES = P_YMS + TILE * (TILE + 1) * 4;
 constexpr uint32_t SMEM_BYTES = P_BYTES > C_BYTES ? P_BYTES : C_BYTES;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(P_ST % 16 == 0 && P_GA % 16 == 0 && P_GB % 16 == 0 && P_WA % 16 == 0 && P_VA % 16 == 0 &&
-              P_TB % 16 == 0 && SLOT % 16 == 0 && C_OST % 16 == 0, "alignment");
+              P_TB % 16 == 0 && SLOT % 16 == 0, "alignment");
 // tensor memory: rank 0 uses 416 columns (512 allocated), ranks 1-3 use 128
 constexpr uint32_t CT_AS = 0, CT_AU = 128, CT_DX0 = 160, CT_DKU = 224, CT_DX1 = 352;
 constexpr uint32_t PT_DG = 0, PT_DW = 64, PT_DU = 96;
@@ -660,7 +659,6 @@ constexpr uint32_t PT_DG = 0, PT_DW = 64, PT_DU = 96;
 __global__ void __cluster_dims__(pc::NPREPCTA + 1, 1, 1) __launch_bounds__(pc::NTH, 1)
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                       const __grid_constant__ CUtensorMap tm_o,
                        const __nv_bfloat16* __restrict__ beta, const float* h0,
                        __nv_bfloat16* __restrict__ o, float* hT, int T, int H)
 {
@@ -668,8 +666,9 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     using namespace tc;
     extern __shared__ __align__(1024) unsigned char sm[];
     __shared__ uint32_t s_taddr;
-    __shared__ __align__(8) uint64_t s_bar[5];   // rank 0: FULL[0..2], MMA, o; ranks 1-3: EMPTY, MMA, input loads
+    __shared__ __align__(8) uint64_t s_bar[4];   // rank 0: FULL[0..2], MMA; ranks 1-3: EMPTY, MMA, input loads
     __shared__ int s_abort;
+    __shared__ uint32_t s_odone;                 // rank 0: chunks whose slot is consumed
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
@@ -683,9 +682,14 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
+        for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
         fence_mbar_init();
         s_abort = 0;
+        s_odone = 0;
+        // rank 0: FULL[s] expects the bytes of chunk s's push; later uses are
+        // armed when the slot is released (the push itself carries no arrive)
+        if (rank == 0)
+            for (int i = 0; i < NPREPCTA && i < n_chunks; ++i) mbar_arrive_expect_tx(smem_u32(&s_bar[i]), SLOT);
     }
     fence_before_sync();
     __syncthreads();
@@ -701,13 +705,12 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
     if (rank == 0) {
         // ========================================================= chain CTA ==
-        const uint32_t mbar = smem_u32(&s_bar[3]);   // X, then Kb^T U, of each chunk
-        const uint32_t obar = smem_u32(&s_bar[4]);   // P U of each chunk (its output complete)
+        const uint32_t mbar = smem_u32(&s_bar[3]);   // X, then [Kb^T U, P U], of each chunk
         if (warp == NCW / 32) {
             // ------------------------------------------------------ issuer warp --
             // Chunk ch: X = S^T [W | Qt]^T in two d_k halves (each as soon as
             // the compute warps have written that half of the tf32 state), then
-            // Kb^T U and P U once U is in tensor memory.
+            // Kb^T U and P U (one commit) once U is in tensor memory.
             const uint32_t id1 = idesc_tf32(128, 2 * C, false, false);
             const uint32_t id2 = idesc_tf32(128, 128, false, false);
             const uint32_t id3 = idesc_tf32(128, 32, false, false);
@@ -749,34 +752,40 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     for (int ks = 0; ks < C / 8; ++ks)
                         mma_tf32_ts_w(tm + CT_DKU, tm + CT_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
                                       id2, ks > 0 ? 1u : 0u);
-                    mma_commit_w(mbar);
 #pragma unroll
                     for (int ks = 0; ks < C / 8; ++ks)
                         mma_tf32_ts_w(tm + dx + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * LBO) >> 4),
                                       id3, 1u);
-                    mma_commit_w(obar);
+                    mma_commit_w(mbar);
                 }
                 __syncwarp();
             }
         } else if (warp == NCW / 32 + 1) {
             // ------------------------------------------------------ release warp --
-            // Once the last MMA of chunk ch - 1 (P U) is done, nothing reads its
-            // slot any more: hand it back to its preparer.  A remote arrive is
-            // slow, so it stays off the issuer's and the compute warps' path.
+            // Once chunk ch - 1's last MMAs are done (and its decay applied),
+            // nothing reads its slot any more: hand it back to its preparer.
+            // A remote arrive is slow, so it stays off the issuer's and the
+            // compute warps' path.  Completion comes from a counter that the
+            // compute warps advance in order; a counter cannot be misread by a
+            // reader that lags.
 #pragma unroll 1
             for (int ch = 1; ch < n_chunks; ++ch) {
                 if (lane == 0) {
-                    if (!s_abort && !mbar_wait(obar, (uint32_t)(ch - 1) & 1u, WAIT_NS)) expired();
-                    mbar_arrive_remote(map_to_rank(smem_u32(&s_bar[0]), 1u + (uint32_t)((ch - 1) % NPREPCTA)));
+                    if (!s_abort && !counter_wait(smem_u32(&s_odone), (uint32_t)ch, WAIT_NS)) expired();
+                    const int cn = ch - 1 + NPREPCTA;        // the chunk that will reuse this slot
+                    if (cn < n_chunks) mbar_arrive_expect_tx(smem_u32(&s_bar[(ch - 1) % NPREPCTA]), SLOT);
+                    mbar_arrive_remote_relaxed(map_to_rank(smem_u32(&s_bar[0]), 1u + (uint32_t)((ch - 1) % NPREPCTA)));
                 }
                 __syncwarp();
             }
         } else {
             // ----------------------------------------------------- compute warps --
-            // Per chunk ch: the state update of chunk ch - 1 by d_k halves (each
-            // half handed to the issuer as soon as it is in tensor memory), the
-            // output of chunk ch - 1 (staged and written by TMA while X of chunk
-            // ch is computed), then U = U' - W S.
+            // Per chunk ch: the state increment of chunk ch - 1 by d_k halves
+            // (each half handed to the issuer as soon as it is in tensor
+            // memory), the output of chunk ch - 1 (staged and written by TMA
+            // while X of chunk ch is computed), then U = U' - W S, and the
+            // decay S <- Diag(gamma_C) S while Kb^T U and P U run.  Chunk ch's
+            // slot is then consumed and goes back to its preparer.
             const int j = 32 * sp + lane;                // dv row = TMEM lane
             const int hh = warp >> 2;                     // d_k columns [32 hh, +32) and [64 + 32 hh, +32)
             uint32_t phase = 0;
@@ -803,47 +812,46 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 }
                 wait_st();
             }
-            // S <- Diag(gamma_C) S + Kb^T U on d_k half q2 (gamma of the slot at sbp)
-            auto state_half = [&](int q2, uint32_t sbp) {
-                const float4* gam4 = reinterpret_cast<const float4*>(sm + sbp + S_GAM) + 16 * q2 + 8 * hh;
+            // S <- S + Kb^T U on d_k half q2 (the decay is already applied)
+            auto state_half = [&](int q2) {
+                float d[32];
+                tmem_ld32(tm + lane_base + CT_DKU + 64 * q2 + 32 * hh, d);
+                wait_ld();
 #pragma unroll
-                for (int c0 = 0; c0 < 32; c0 += 16) {
-                    float d[16];
-                    tmem_ld16(tm + lane_base + CT_DKU + 64 * q2 + 32 * hh + c0, d);
-                    wait_ld();
-#pragma unroll
-                    for (int i4 = 0; i4 < 4; ++i4) {
-                        const float4 gv = gam4[(c0 >> 2) + i4];
-                        const float gg[4] = {gv.x, gv.y, gv.z, gv.w};
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int i = c0 + i4 * 4 + u;
-                            S[32 * q2 + i] = fmaf(gg[u], S[32 * q2 + i], d[i - c0]);
-                            d[i - c0] = to_tf32(S[32 * q2 + i]);
-                        }
-                    }
-                    tmem_st16(tm + lane_base + CT_AS + 64 * q2 + 32 * hh + c0, d);
+                for (int i = 0; i < 32; ++i) {
+                    S[32 * q2 + i] += d[i];
+                    d[i] = to_tf32(S[32 * q2 + i]);
                 }
+                tmem_st32(tm + lane_base + CT_AS + 64 * q2 + 32 * hh, d);
                 wait_st();
             };
-            // o of chunk cp (X buffer cp & 1, complete once obar's phase cp has
-            // passed) -> staging -> one TMA store by thread 0
+            // S <- Diag(gamma_C) S with gamma of the slot at sb
+            auto decay = [&](uint32_t sb) {
+                const float4* gam4 = reinterpret_cast<const float4*>(sm + sb + S_GAM);
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        const float4 gv = gam4[16 * q2 + 8 * hh + i4];
+                        S[32 * q2 + 4 * i4 + 0] *= gv.x;
+                        S[32 * q2 + 4 * i4 + 1] *= gv.y;
+                        S[32 * q2 + 4 * i4 + 2] *= gv.z;
+                        S[32 * q2 + 4 * i4 + 3] *= gv.w;
+                    }
+            };
+            // o of chunk cp (X buffer cp & 1, complete since chunk cp's last
+            // MMA wait), written from registers: lanes hold adjacent dv
+            // columns, so each warp store covers 64 contiguous bytes of a row
             auto emit_output = [&](int cp) {
                 const uint32_t dx = (cp & 1) ? CT_DX1 : CT_DX0;
-                __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
-                if (tid == 0) bulk_wait_read_all();   // the previous store has read the staging
-                wait_bar(obar, (uint32_t)cp & 1u);
                 float ov[16];
                 tmem_ld16(tm + lane_base + dx + C + 16 * hh, ov);
                 wait_ld();
+                const int t0 = cp * C + 16 * hh;
+                __nv_bfloat16* op = o + ((int64_t)b * T + t0) * (int64_t)H * D + (int64_t)h * D + j;
 #pragma unroll
-                for (int r = 0; r < 16; ++r) ost[(16 * hh + r) * D + j] = __float2bfloat16_rn(ov[r]);
-                fence_smem_to_async();
-                cw_bar();
-                if (tid == 0) {
-                    tma_store_3d(&tm_o, h * D, cp * C, b, smem_u32(ost));
-                    bulk_commit();
-                }
+                for (int r = 0; r < 16; ++r)
+                    if (t0 + r < T) op[(int64_t)r * H * D] = __float2bfloat16_rn(ov[r]);
             };
             fence_before_sync();
             if (n_chunks > 0) {                       // the initial state for chunk 0
@@ -856,11 +864,10 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const uint32_t sb = C_SLOT0 + slot * SLOT;
                 const uint32_t dx = (ch & 1) ? CT_DX1 : CT_DX0;
                 if (ch > 0) {
-                    const uint32_t sbp = C_SLOT0 + ((ch - 1) % NPREPCTA) * SLOT;
-                    state_half(0, sbp);
+                    state_half(0);
                     fence_before_sync();
                     named_arrive(NB_ASA, NX);
-                    state_half(1, sbp);
+                    state_half(1);
                     fence_before_sync();
                     named_arrive(NB_ASB, NX);
                     emit_output(ch - 1);
@@ -883,16 +890,16 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 }
                 fence_before_sync();
                 named_arrive(NB_U, NX);
-                wait_bar(mbar, phase & 1u);           // Kb^T U of chunk ch
+                decay(sb);                            // while Kb^T U and P U run
+                wait_bar(mbar, phase & 1u);           // Kb^T U and P U of chunk ch
                 ++phase;
+                if (tid == 0) counter_publish(smem_u32(&s_odone), (uint32_t)ch + 1u);
             }
             if (n_chunks > 0) {
-                const uint32_t sbp = C_SLOT0 + ((n_chunks - 1) % NPREPCTA) * SLOT;
-                state_half(0, sbp);
-                state_half(1, sbp);
+                state_half(0);
+                state_half(1);
                 emit_output(n_chunks - 1);
             }
-            if (tid == 0) bulk_wait_all();           // the last o stores have landed
             if (hT && !s_abort) {
                 float* hTh = hT + head_off * D * D;
 #pragma unroll
@@ -970,8 +977,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     // the chain has released this slot (its previous use, chunk ch - NPREPCTA)
                     if (ch >= NPREPCTA && !s_abort && !mbar_wait_cluster(ebar, ephase & 1u, WAIT_NS)) expired();
                     if (ch >= NPREPCTA) ++ephase;
-                    if (!s_abort) {
-                        mbar_arrive_expect_tx_remote(full_remote, SLOT);
+                    if (!s_abort) {                   // FULL was armed by the chain
                         bulk_copy_to_rank(slot_remote, smem_u32(st), SLOT, full_remote);
                         bulk_commit();
                     }
@@ -1251,14 +1257,14 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    CUtensorMap mq, mk, mv, mg, mo;
+    CUtensorMap mq, mk, mv, mg;
     if (T > 0) {
         if (!make_map(&mq, q, B, T, H) || !make_map(&mk, k, B, T, H) ||
-            !make_map(&mv, v, B, T, H) || !make_map(&mg, g, B, T, H) || !make_map(&mo, o, B, T, H))
+            !make_map(&mv, v, B, T, H) || !make_map(&mg, g, B, T, H))
             return cudaErrorInvalidValue;
     } else {   // no chunk, no load: the kernel only carries h0 to hT
         memset(&mq, 0, sizeof(mq)); memset(&mk, 0, sizeof(mk));
-        memset(&mv, 0, sizeof(mv)); memset(&mg, 0, sizeof(mg)); memset(&mo, 0, sizeof(mo));
+        memset(&mv, 0, sizeof(mv)); memset(&mg, 0, sizeof(mg));
     }
     if (use_cluster_variant(B, H)) {
         static bool cattr_set = false;
@@ -1271,7 +1277,7 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
         }
         dim3 grid((pc::NPREPCTA + 1) * H, B);
         prefill_cluster_kernel<<<grid, pc::NTH, pc::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mg, mo, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
+            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
     } else {
         dim3 grid(H, B);
         prefill_tc_kernel<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(

@@ -163,7 +163,7 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t saddr, uint32_t parit
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 100000;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.b32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok) : "r"(saddr), "r"(parity) : "memory");
     return ok;
@@ -174,14 +174,37 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 // Wait for phase `parity` to complete, giving up after `limit_ns`.  Each
-// try_wait may suspend the thread (up to a 100 us hint) until the phase
-// completes, so a waiting thread does not spin on the issue slots.
-// Returns true on success, false on timeout.
+// try_wait may block for a short, implementation-defined time before it
+// returns false.  No suspend-time hint is given: with a long hint the waiting
+// thread wakes measurably later (a few hundred cycles) after the phase
+// completes.  Returns true on success, false on timeout.
 __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(saddr, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(saddr, parity)) {
         if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
+// A monotonic counter in shared memory, published with release and read with
+// acquire semantics (CTA scope).  Unlike an mbarrier phase parity, a reader
+// that falls behind by several steps still reads the right value.
+__device__ __forceinline__ void counter_publish(uint32_t saddr, uint32_t v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" :: "r"(saddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t counter_read(uint32_t saddr) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(saddr) : "memory");
+    return v;
+}
+// Wait until the counter reaches `target`; false once limit_ns has passed.
+__device__ __forceinline__ bool counter_wait(uint32_t saddr, uint32_t target, uint64_t limit_ns) {
+    if (counter_read(saddr) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (counter_read(saddr) < target) {
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+        __nanosleep(64);
     }
     return true;
 }
@@ -226,6 +249,13 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_saddr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
                  :: "r"(cluster_saddr) : "memory");
 }
+// Relaxed form: signals an event that orders no data (for example "this
+// buffer may be overwritten" once every read of it has completed); much
+// cheaper than the release form.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_saddr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];"
+                 :: "r"(cluster_saddr) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_saddr, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
                  :: "r"(cluster_saddr), "r"(bytes) : "memory");
@@ -235,7 +265,7 @@ __device__ __forceinline__ uint32_t mbar_try_wait_cluster(uint32_t saddr, uint32
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, 100000;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.b32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok) : "r"(saddr), "r"(parity) : "memory");
     return ok;
@@ -256,20 +286,6 @@ __device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster_saddr, ui
     asm volatile(
         "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         :: "r"(dst_cluster_saddr), "r"(src_saddr), "r"(bytes), "r"(mbar_cluster_saddr) : "memory");
-}
-// Tiled 3-D tensor store (shared -> global); rows outside the tensor are not written.
-__device__ __forceinline__ void tma_store_3d(const void* tmap, int x, int y, int z, uint32_t src_saddr) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];"
-        :: "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(src_saddr) : "memory");
-}
-// Wait until at most one committed bulk group still reads its source.
-__device__ __forceinline__ void bulk_wait_read_1() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
-// Wait until every committed bulk group has completed (writes included).
-__device__ __forceinline__ void bulk_wait_all() {
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the source buffers of all committed bulk copies may be reused.
