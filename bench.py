@@ -62,9 +62,10 @@ def decode_alg_bytes(N, H, dk, dv):
     return N * H * (2 * dk * dv * 4 + (3 * dk + dv + 1 + dv) * BYTES_BF16)
 
 
-def measured_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernel's source has changed since the capture."""
+def measured_traffic(kernel, workload):
+    """DRAM bytes per launch for this kernel on this workload from the
+    committed ncu summary, or None when there is no such line or when the
+    kernel's sources have changed since the capture."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
@@ -73,11 +74,13 @@ def measured_traffic(kernel):
                 if line.startswith("#") or not line.strip():
                     continue
                 parts = line.split()
-                if parts[0] != kernel:
+                if parts[0] != kernel or parts[4] != workload:
                     continue
-                with open(os.path.join(ROOT, parts[1]), "rb") as src:
-                    sha = hashlib.sha256(src.read()).hexdigest()[:16]
-                return int(parts[3]) if sha == parts[2] else None
+                h = hashlib.sha256()
+                for rel in parts[1].split(","):        # every source the kernel is built from
+                    with open(os.path.join(ROOT, rel), "rb") as src:
+                        h.update(src.read())
+                return int(parts[3]) if h.hexdigest()[:16] == parts[2] else None
     except Exception:
         return None
     return None
@@ -251,7 +254,7 @@ def bench_kda(args, rank, world, local):
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1),
                 "peak": hbm_gbs, "unit": "GB/s",
                 "frac": round(achieved_gbs / hbm_gbs, 4),
-                "traffic": measured_traffic("kda_chunk_fwd") if args.workload == "prefill_8k" else None, "peak_source": peak_src + " hbm_gbs (burst copy)",
+                "traffic": measured_traffic("kda_chunk_fwd", args.workload), "peak_source": peak_src + " hbm_gbs (burst copy)",
                 "alg_bytes_per_launch": alg_b,
                 "kernel": "kda_chunk_fwd",
                 "tensor_alg_tflops": round(alg_f / (launch_ms / 1e3) / 1e12, 2),
@@ -357,7 +360,7 @@ def bench_decode(args, kda, dev, rank, world, hbm_gbs, peak_src):
            "ms_per_step_p99": round(per[int(len(per) * 0.99) - 1], 5),
            "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_gbs,
                         "unit": "GB/s", "frac": round(ach / hbm_gbs, 4),
-                        "traffic": measured_traffic("kda_decode_step"),
+                        "traffic": measured_traffic("kda_decode_step", "decode_256"),
                         "peak_source": peak_src + " hbm_gbs (burst copy)",
                         "alg_bytes_per_launch": alg, "kernel": "kda_decode_step"}}
     del d

@@ -44,7 +44,9 @@ class Workload:
 
 
 # The five workloads: a tiny fp32 case, an 8K prefill, a batch of 64K
-# pre-training sequences, a million-token prefill and a batched decode run.
+# pre-training sequences, a million-token prefill and a batched decode run;
+# plus a profiling size for the one-SM-per-head prefill path (the 64K batch
+# scaled down in T so that a full profiler capture stays at about 1 GB).
 WORKLOADS = {
     "tiny_fp32": Workload("tiny_fp32", "prefill", 1, 64, 2, 32, 32,
                           torch.float32, 1001,
@@ -59,6 +61,10 @@ WORKLOADS = {
     "prefill_1m": Workload("prefill_1m", "prefill", 1, 1048576, 32, 128, 128,
                            torch.bfloat16, 1004,
                            note="B1 H32 T1048576 d128 bf16, h0=0"),
+    "pretrain_8k_b4": Workload("pretrain_8k_b4", "prefill", 4, 8192, 32, 128, 128,
+                               torch.bfloat16, 1006, pin_frac=0.1,
+                               note="B4 H32 T8192 d128 bf16, 10%+10% of g channels "
+                                    "pinned at -5 and 0, h0=0 (profiling size)"),
     "decode_256": Workload("decode_256", "decode", 256, 1000, 32, 128, 128,
                            torch.bfloat16, 1005, h0_std=0.1,
                            note="256 requests x H32 d128, fp32 state "
