@@ -28,7 +28,10 @@
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers, owned by the caller, 16-byte
  *     aligned, densely packed in the row-major layouts given per function.
- *     No entry point allocates, frees or keeps a pointer after it returns.
+ *     No entry point keeps a pointer after it returns.  Only kda_chunk_fwd
+ *     takes memory of its own, and only on its segment-scan path (see
+ *     there): stream-ordered workspace (cudaMallocAsync / cudaFreeAsync on
+ *     `stream`), returned before the call's work completes.
  *   - Calls are asynchronous on `stream` (0 = legacy default stream) and do
  *     no host synchronisation.  Asynchronous device errors surface at the
  *     caller's next synchronisation, as for any CUDA launch.
@@ -55,7 +58,7 @@ typedef enum {
     KDA_ERR_UNSUPPORTED = -2,  /* valid but unsupported shape (dk, dv)      */
     KDA_ERR_CUDA = -3,         /* a CUDA launch or runtime call failed      */
     KDA_ERR_TIMEOUT = -4,      /* a bounded device wait expired (see below) */
-    KDA_ERR_NO_MEMORY = -5     /* reserved                                  */
+    KDA_ERR_NO_MEMORY = -5     /* workspace allocation failed               */
 } kda_status;
 
 /*
@@ -71,6 +74,17 @@ typedef enum {
  * done in 16-token tiles on the tensor cores with an fp32 master state (the
  * "T11E1" transcript's log-decay-bound turn is what makes the diagonal tiles
  * dense).  Returns KDA_ERR_UNSUPPORTED for other dk/dv.
+ *
+ * Segment scan: with B*H <= 8 and T >= 4096 each sequence is cut into P
+ * segments that run in parallel (P about 148 / (B*H), at least 256 tokens
+ * each): a pass over all segments from a zero state and from the identity
+ * (with v = 0) gives, per segment, the state it reaches from zero and its
+ * transition matrix; a short chain over the segments gives each segment's
+ * true start state; a last pass writes o.  This path takes 3 * B * P * H *
+ * dk * dv * 4 bytes of stream-ordered workspace (at most 28.4 MB) and
+ * returns KDA_ERR_NO_MEMORY if it cannot.  The environment variable
+ * KDA_PREFILL_VARIANT = fused | cluster | segmented forces one path
+ * (measurement and tests; "segmented" needs T >= 512).
  */
 int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
                   const void* beta, const float* h0, void* o, float* hT,

@@ -39,7 +39,11 @@ static bool sizes_ok(int64_t a, int64_t b, int64_t c, int64_t d)
            (double)a * (double)b * (double)c * (double)d < 4.0e18;
 }
 
-static int status_of(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+static int status_of(cudaError_t e)
+{
+    if (e == cudaSuccess) return KDA_OK;
+    return e == cudaErrorMemoryAllocation ? KDA_ERR_NO_MEMORY : KDA_ERR_CUDA;
+}
 
 // Common checks of the two prefill entry points.
 static int check_prefill(const void* q, const void* k, const void* v, const void* g,

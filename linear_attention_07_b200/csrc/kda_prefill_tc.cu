@@ -109,6 +109,10 @@ constexpr uint32_t BAR_FREE = 1, BAR_READY = 2, BAR_CHAIN = 3, BAR_PREP = 4;
 
 constexpr uint64_t WAIT_NS = 2000000000ull;   // bounded waits: 2 s
 
+// Launch flags (segment scan passes): treat v as zero, start from h0 = I
+// (ignore h0), skip the o stores.
+constexpr uint32_t SEG_V_ZERO = 1u, SEG_H0_EYE = 2u, SEG_NO_O = 4u;
+
 }  // namespace pf
 
 __device__ int g_prefill_status;   // set to KDA_ERR_TIMEOUT by a wait that expired
@@ -140,7 +144,8 @@ __global__ void __launch_bounds__(pf::NT, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                   const __nv_bfloat16* __restrict__ beta, const float* h0,
-                  __nv_bfloat16* __restrict__ o, float* hT, int T, int H)
+                  __nv_bfloat16* __restrict__ o, float* hT, int T, int H,
+                  int seg_len, int n_seg, uint32_t flags)
 {
     using namespace pf;
     using namespace tc;
@@ -150,10 +155,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __shared__ int s_abort;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x, b = blockIdx.y;
-    const int64_t head_off = (int64_t)b * H + h;
+    // grid.y = B * n_seg: sequence b, segment [ts, ts + Tl) of it (n_seg = 1: the whole sequence)
+    const int h = blockIdx.x, bb = blockIdx.y;
+    const int b = bb / n_seg;
+    const int ts = (bb - b * n_seg) * seg_len;
+    const int Tl = max(0, min(seg_len, T - ts));
+    const int64_t head_off = (int64_t)bb * H + h;          // h0 / hT: [B * n_seg][H][D][D]
     const int64_t row_stride = (int64_t)H * D;            // elements between tokens
-    const int64_t base = ((int64_t)b * T * H + h) * D;    // token 0 of this head
+    const int64_t base = (((int64_t)b * T + ts) * H + h) * D;    // token ts of this head
 
     if (warp == 0) {
         tmem_alloc(smem_u32(&s_taddr), TMEM_COLS);
@@ -172,7 +181,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t tm = s_taddr;
     const int sp = warp & 3;                                   // TMEM sub-partition of this warp
     const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
-    const int n_chunks = (T + C - 1) / C;
+    const int n_chunks = (Tl + C - 1) / C;
     // A wait that expired sets s_abort; from then on both roles skip all MMA
     // work but keep the barrier protocol, so the CTA winds down without
     // further waits and reports KDA_ERR_TIMEOUT.
@@ -198,9 +207,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         };
         float S[D / 2];
         {
-            const float* h0h = h0 ? h0 + head_off * D * D : nullptr;
+            const float* h0h = (h0 && !(flags & SEG_H0_EYE)) ? h0 + head_off * D * D : nullptr;
 #pragma unroll
-            for (int i = 0; i < D / 2; ++i) S[i] = h0h ? h0h[(int64_t)(64 * hh + i) * D + j] : 0.f;
+            for (int i = 0; i < D / 2; ++i)
+                S[i] = (flags & SEG_H0_EYE) ? (64 * hh + i == j ? 1.f : 0.f)
+                                            : (h0h ? h0h[(int64_t)(64 * hh + i) * D + j] : 0.f);
 #pragma unroll
             for (int c0 = 0; c0 < D / 2; c0 += 32) {
                 float t32[32];
@@ -297,7 +308,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int m = 0; m < (C * D / 8) / NCH; ++m) {
                     const int vi = tid + m * NCH;
                     const int r = vi / (D / 8), cv = vi % (D / 8);
-                    if (tb + r < T)
+                    if (tb + r < Tl && !(flags & SEG_NO_O))
                         *reinterpret_cast<uint4*>(oh + (int64_t)(tb + r) * row_stride + cv * 8) =
                             *reinterpret_cast<const uint4*>(ost + r * D + cv * 8);
                 }
@@ -328,17 +339,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         auto issue_raw = [&](int ci) {
             if (pt == 0) {
                 mbar_arrive_expect_tx(rbar, 4 * RAW_T);
-                tma_load_3d(smem_u32(sm + RAW + 0 * RAW_T), &tm_q, h * D, ci * C, b, rbar);
-                tma_load_3d(smem_u32(sm + RAW + 1 * RAW_T), &tm_k, h * D, ci * C, b, rbar);
-                tma_load_3d(smem_u32(sm + RAW + 2 * RAW_T), &tm_v, h * D, ci * C, b, rbar);
-                tma_load_3d(smem_u32(sm + RAW + 3 * RAW_T), &tm_g, h * D, ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + RAW + 0 * RAW_T), &tm_q, h * D, ts + ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + RAW + 1 * RAW_T), &tm_k, h * D, ts + ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + RAW + 2 * RAW_T), &tm_v, h * D, ts + ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + RAW + 3 * RAW_T), &tm_g, h * D, ts + ci * C, b, rbar);
             }
         };
         if (n_chunks > 0) issue_raw(0);
         // beta one chunk ahead, kept as raw bf16 bits until it is stored (a
         // conversion right after the load would stall on the load)
         const __nv_bfloat16 bzero = __float2bfloat16_rn(0.f);
-        __nv_bfloat16 beta_next = (pt < C && pt < T) ? beta[((int64_t)b * T + pt) * H + h] : bzero;
+        __nv_bfloat16 beta_next = (pt < C && pt < Tl) ? beta[((int64_t)b * T + ts + pt) * H + h] : bzero;
 
         // decay-scaling slice of this thread: tile tau, key channel c
         const int tau = pt >> 7;
@@ -355,7 +366,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (pt < C) {
                 reinterpret_cast<float*>(sm + BETA)[pt] = to_f32(beta_next);
                 const int tn = (ch + 1) * C + pt;
-                beta_next = (tn < T) ? beta[((int64_t)b * T + tn) * H + h] : bzero;
+                beta_next = (tn < Tl) ? beta[((int64_t)b * T + ts + tn) * H + h] : bzero;
             }
             if (pt == 0 && !s_abort && !mbar_wait(rbar, rphase & 1u, WAIT_NS)) expired();
             ++rphase;
@@ -378,7 +389,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const int idx = (tau * TILE + rr) * D + c;
                     kr[rr] = to_f32(rk[idx]);
                     qr[rr] = to_f32(rq[idx]);
-                    vr[rr] = to_f32(rv[idx]);
+                    vr[rr] = (flags & SEG_V_ZERO) ? 0.f : to_f32(rv[idx]);
                     a[rr] = to_f32(rg[idx]);
                 }
                 float e = 1.f;
@@ -660,7 +671,8 @@ __global__ void __cluster_dims__(pc::NPREPCTA + 1, 1, 1) __launch_bounds__(pc::N
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                        const __nv_bfloat16* __restrict__ beta, const float* h0,
-                       __nv_bfloat16* __restrict__ o, float* hT, int T, int H)
+                       __nv_bfloat16* __restrict__ o, float* hT, int T, int H,
+                       int seg_len, int n_seg, uint32_t flags)
 {
     using namespace pc;
     using namespace tc;
@@ -672,9 +684,13 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
-    const int h = blockIdx.x / (NPREPCTA + 1), b = blockIdx.y;
-    const int64_t head_off = (int64_t)b * H + h;
-    const int n_chunks = (T + C - 1) / C;
+    // grid.y = B * n_seg: sequence b, segment [ts, ts + Tl) of it (n_seg = 1: the whole sequence)
+    const int h = blockIdx.x / (NPREPCTA + 1), bb = blockIdx.y;
+    const int b = bb / n_seg;
+    const int ts = (bb - b * n_seg) * seg_len;
+    const int Tl = max(0, min(seg_len, T - ts));
+    const int64_t head_off = (int64_t)bb * H + h;          // h0 / hT: [B * n_seg][H][D][D]
+    const int n_chunks = (Tl + C - 1) / C;
     const uint32_t ncols = rank == 0 ? 512u : 128u;
 
     if (warp == 0) {
@@ -799,12 +815,15 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             // S[32 q + i] holds d_k column 64 q + 32 hh + i of this thread's dv row
             float S[D / 2];
             {
-                const float* h0h = h0 ? h0 + head_off * D * D : nullptr;
+                const float* h0h = (h0 && !(flags & SEG_H0_EYE)) ? h0 + head_off * D * D : nullptr;
 #pragma unroll
                 for (int q2 = 0; q2 < 2; ++q2) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        S[32 * q2 + i] = h0h ? h0h[(int64_t)(64 * q2 + 32 * hh + i) * D + j] : 0.f;
+                    for (int i = 0; i < 32; ++i) {
+                        const int row = 64 * q2 + 32 * hh + i;
+                        S[32 * q2 + i] = (flags & SEG_H0_EYE) ? (row == j ? 1.f : 0.f)
+                                                              : (h0h ? h0h[(int64_t)row * D + j] : 0.f);
+                    }
                     float t32[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) t32[i] = to_tf32(S[32 * q2 + i]);
@@ -847,11 +866,13 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 float ov[16];
                 tmem_ld16(tm + lane_base + dx + C + 16 * hh, ov);
                 wait_ld();
-                const int t0 = cp * C + 16 * hh;
-                __nv_bfloat16* op = o + ((int64_t)b * T + t0) * (int64_t)H * D + (int64_t)h * D + j;
+                const int tt = cp * C + 16 * hh;              // token of ov[0] within the segment
+                __nv_bfloat16* op = o + ((int64_t)b * T + ts + tt) * (int64_t)H * D + (int64_t)h * D + j;
+                if (!(flags & SEG_NO_O)) {
 #pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    if (t0 + r < T) op[(int64_t)r * H * D] = __float2bfloat16_rn(ov[r]);
+                    for (int r = 0; r < 16; ++r)
+                        if (tt + r < Tl) op[(int64_t)r * H * D] = __float2bfloat16_rn(ov[r]);
+                }
             };
             fence_before_sync();
             if (n_chunks > 0) {                       // the initial state for chunk 0
@@ -921,10 +942,10 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             // barriers and never wait on an issue.
             auto issue_raw = [&](int ci) {
                 mbar_arrive_expect_tx(rbar, 4 * RAW_T);
-                tma_load_3d(smem_u32(sm + P_RAW + 0 * RAW_T), &tm_q, h * D, ci * C, b, rbar);
-                tma_load_3d(smem_u32(sm + P_RAW + 1 * RAW_T), &tm_k, h * D, ci * C, b, rbar);
-                tma_load_3d(smem_u32(sm + P_RAW + 2 * RAW_T), &tm_v, h * D, ci * C, b, rbar);
-                tma_load_3d(smem_u32(sm + P_RAW + 3 * RAW_T), &tm_g, h * D, ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + P_RAW + 0 * RAW_T), &tm_q, h * D, ts + ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + P_RAW + 1 * RAW_T), &tm_k, h * D, ts + ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + P_RAW + 2 * RAW_T), &tm_v, h * D, ts + ci * C, b, rbar);
+                tma_load_3d(smem_u32(sm + P_RAW + 3 * RAW_T), &tm_g, h * D, ts + ci * C, b, rbar);
             };
             if (lane == 0 && par < n_chunks) issue_raw(par);
 #pragma unroll 1
@@ -1000,7 +1021,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             fence_after_sync();
         };
         const __nv_bfloat16 bzero = __float2bfloat16_rn(0.f);
-        __nv_bfloat16 beta_next = (pt < C && par * C + pt < T) ? beta[((int64_t)b * T + par * C + pt) * H + h] : bzero;
+        __nv_bfloat16 beta_next = (pt < C && par * C + pt < Tl) ? beta[((int64_t)b * T + ts + par * C + pt) * H + h] : bzero;
         const int tau = pt >> 7;
         const int c = pt & 127;
         float* am = reinterpret_cast<float*>(sm + P_AMS);
@@ -1014,7 +1035,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             if (pt < C) {
                 reinterpret_cast<float*>(sm + P_BETA)[pt] = to_f32(beta_next);
                 const int tn = (ch + NPREPCTA) * C + pt;
-                beta_next = (tn < T) ? beta[((int64_t)b * T + tn) * H + h] : bzero;
+                beta_next = (tn < Tl) ? beta[((int64_t)b * T + ts + tn) * H + h] : bzero;
             }
             if (pt == 0 && !s_abort && !mbar_wait(rbar, rphase & 1u, WAIT_NS)) expired();
             ++rphase;
@@ -1033,7 +1054,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     const int idx = (tau * TILE + rr) * D + c;
                     kr[rr] = to_f32(rk[idx]);
                     qr[rr] = to_f32(rq[idx]);
-                    vr[rr] = to_f32(rv[idx]);
+                    vr[rr] = (flags & SEG_V_ZERO) ? 0.f : to_f32(rv[idx]);
                     a[rr] = to_f32(rg[idx]);
                 }
                 float e = 1.f;
@@ -1236,24 +1257,177 @@ static bool make_map(CUtensorMap* map, const void* base, int B, int T, int H)
 
 // Four SMs per head pay off while the heads alone leave most SMs idle:
 // up to 37 heads (148 SMs); larger batches use one SM per head.
-// KDA_PREFILL_VARIANT=fused|cluster overrides the choice (for measurement).
-static bool use_cluster_variant(int B, int H)
+static bool cluster_fits(int64_t heads) { return heads * (pc::NPREPCTA + 1) <= 148; }
+
+// One launch of either variant over B * n_seg segment-sequences of length
+// seg_len (n_seg = 1, seg_len = T: the plain prefill).
+static cudaError_t launch_pass(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                               const CUtensorMap& mg, const void* beta, const float* h0, void* o, float* hT,
+                               int B, int T, int H, int seg_len, int n_seg, uint32_t flags, bool cluster,
+                               cudaStream_t stream)
 {
+    if (cluster) {
+        dim3 grid((pc::NPREPCTA + 1) * H, B * n_seg);
+        prefill_cluster_kernel<<<grid, pc::NTH, pc::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags);
+    } else {
+        dim3 grid(H, B * n_seg);
+        prefill_tc_kernel<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(
+            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags);
+    }
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Segment scan (for very few heads on long sequences).  The sequence of each
+// head is cut into n_seg segments of seg_len tokens (a multiple of the
+// 32-token chunk).  The recurrence is affine in the state, so over a segment
+// S_end = M_p S_start + N_p, with M_p the product of the segment's per-token
+// transitions (I - b k k^T) Diag(exp g) and N_p the state the segment reaches
+// from zero.  Pass 1 runs every segment at once twice: from S = 0 (giving
+// N_p) and from S = I with v = 0 (giving M_p, since each state column evolves
+// on its own).  Pass 2 chains S_{p+1} = M_p S_p + N_p over the segments.
+// Pass 3 reruns every segment from its true S_p and writes o.
+constexpr int SEG_MAX_HEADS = 8;      // B * H up to this: the segment scan
+constexpr int SEG_MIN_CHUNKS = 8;     // chunks per segment at least
+constexpr int SEG_MIN_T_CHUNKS = 128; // and a sequence of at least 128 chunks
+constexpr int SEG_COLS = 16;          // state columns per combine CTA
+
+// S_{p+1} = M_p S_p + N_p for the segments of one (b, h), in fp32 on CUDA
+// cores (columns of S are independent: one CTA per group of 16 columns).
+// Writes S_p, the start state of segment p, for pass 3, and the final state.
+// M, N, S0: [B * n_seg][H][D][D]; h0, hT: [B][H][D][D] (either may be null;
+// hT may equal h0).
+__global__ void __launch_bounds__(256)
+segment_combine_kernel(const float* __restrict__ M, const float* __restrict__ N, float* __restrict__ S0,
+                       const float* h0, float* hT, int H, int n_seg)
+{
+    constexpr int D = pf::D;
+    __shared__ __align__(16) float s[D][SEG_COLS];
+    const int bh = blockIdx.y, b = bh / H, h = bh - b * H;
+    const int tid = threadIdx.x;
+    const int i = tid >> 1, jh = (tid & 1) * 8;              // row i, columns [col0, col0 + 8)
+    const int col0 = blockIdx.x * SEG_COLS + jh;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) s[i][jh + c] = h0 ? h0[(int64_t)bh * D * D + (int64_t)i * D + col0 + c] : 0.f;
+    __syncthreads();
+#pragma unroll 1
+    for (int p = 0; p < n_seg; ++p) {
+        const int64_t sp = ((int64_t)(b * n_seg + p) * H + h) * D * D + (int64_t)i * D + col0;
+        float acc[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            S0[sp + c] = s[i][jh + c];
+            acc[c] = N[sp + c];
+        }
+        const float4* mrow = reinterpret_cast<const float4*>(M + (sp - col0));
+#pragma unroll 4
+        for (int k4 = 0; k4 < D / 4; ++k4) {
+            const float4 m = mrow[k4];
+            const float mk[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const float4 a0 = *reinterpret_cast<const float4*>(&s[4 * k4 + kk][jh]);
+                const float4 a1 = *reinterpret_cast<const float4*>(&s[4 * k4 + kk][jh + 4]);
+                acc[0] = fmaf(mk[kk], a0.x, acc[0]); acc[1] = fmaf(mk[kk], a0.y, acc[1]);
+                acc[2] = fmaf(mk[kk], a0.z, acc[2]); acc[3] = fmaf(mk[kk], a0.w, acc[3]);
+                acc[4] = fmaf(mk[kk], a1.x, acc[4]); acc[5] = fmaf(mk[kk], a1.y, acc[5]);
+                acc[6] = fmaf(mk[kk], a1.z, acc[6]); acc[7] = fmaf(mk[kk], a1.w, acc[7]);
+            }
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < 8; ++c) s[i][jh + c] = acc[c];
+        __syncthreads();
+    }
+    if (hT) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) hT[(int64_t)bh * D * D + (int64_t)i * D + col0 + c] = s[i][jh + c];
+    }
+}
+
+enum class PrefillPath { OneSm, Cluster, Segmented };
+
+// KDA_PREFILL_VARIANT=fused|cluster|segmented overrides the choice (for
+// measurement and tests).
+static PrefillPath choose_path(int B, int T, int H)
+{
+    const int64_t heads = (int64_t)B * H;
+    const int n_chunks = (T + pf::C - 1) / pf::C;
+    const bool seg_ok = n_chunks >= 2 * SEG_MIN_CHUNKS;
     const char* env = getenv("KDA_PREFILL_VARIANT");
-    if (env && strcmp(env, "cluster") == 0) return true;
-    if (env && strcmp(env, "fused") == 0) return false;
-    return (int64_t)B * H * (pc::NPREPCTA + 1) <= 148;
+    if (env && strcmp(env, "cluster") == 0) return PrefillPath::Cluster;
+    if (env && strcmp(env, "fused") == 0) return PrefillPath::OneSm;
+    if (env && strcmp(env, "segmented") == 0 && seg_ok) return PrefillPath::Segmented;
+    if (heads <= SEG_MAX_HEADS && n_chunks >= SEG_MIN_T_CHUNKS) return PrefillPath::Segmented;
+    return cluster_fits(heads) ? PrefillPath::Cluster : PrefillPath::OneSm;
+}
+
+// Segments: about one wave of segment-heads, at least SEG_MIN_CHUNKS chunks
+// each, at least two.
+static void segment_plan(int B, int T, int H, int* seg_len, int* n_seg)
+{
+    const int64_t heads = (int64_t)B * H;
+    const int n_chunks = (T + pf::C - 1) / pf::C;
+    int64_t P = 148 / (heads > 0 ? heads : 1);
+    P = P < (int64_t)(n_chunks / SEG_MIN_CHUNKS) ? P : (int64_t)(n_chunks / SEG_MIN_CHUNKS);
+    if (P < 2) P = 2;
+    const int seg_chunks = (int)((n_chunks + P - 1) / P);
+    *seg_len = seg_chunks * pf::C;
+    *n_seg = (T + *seg_len - 1) / *seg_len;
+}
+
+static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                                    const CUtensorMap& mg, const void* beta, const float* h0, void* o,
+                                    float* hT, int B, int T, int H, cudaStream_t stream)
+{
+    int seg_len = 0, n_seg = 0;
+    segment_plan(B, T, H, &seg_len, &n_seg);
+    const size_t states = (size_t)B * n_seg * H * pf::D * pf::D;     // floats per array
+    static bool pool_set = false;   // keep freed workspace in the pool between calls
+    if (!pool_set) {
+        int dev = 0;
+        cudaMemPool_t pool;
+        if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+            uint64_t keep = UINT64_MAX;
+            cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        }
+        pool_set = true;
+    }
+    float* ws = nullptr;
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), 3 * states * sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+    float* Mw = ws;
+    float* Nw = ws + states;
+    float* Sw = ws + 2 * states;
+    const bool cl = cluster_fits((int64_t)B * n_seg * H);
+    e = launch_pass(mq, mk, mv, mg, beta, nullptr, o, Nw, B, T, H, seg_len, n_seg, pf::SEG_NO_O, cl, stream);
+    if (e == cudaSuccess)
+        e = launch_pass(mq, mk, mv, mg, beta, nullptr, o, Mw, B, T, H, seg_len, n_seg,
+                        pf::SEG_V_ZERO | pf::SEG_H0_EYE | pf::SEG_NO_O, cl, stream);
+    if (e == cudaSuccess) {
+        segment_combine_kernel<<<dim3(pf::D / SEG_COLS, B * H), 256, 0, stream>>>(Mw, Nw, Sw, h0, hT, H, n_seg);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess)
+        e = launch_pass(mq, mk, mv, mg, beta, Sw, o, nullptr, B, T, H, seg_len, n_seg, 0u, cl, stream);
+    const cudaError_t ef = cudaFreeAsync(ws, stream);
+    if (e == cudaSuccess) e = ef;
+    note_launches(4);
+    return e;
 }
 
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, const float* h0, void* o, float* hT,
                               int B, int T, int H, cudaStream_t stream)
 {
-    static bool attr_set = false;   // idempotent; races only repeat the same call
+    static bool attr_set = false;   // idempotent; races only repeat the same calls
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)pf::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)pc::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
@@ -1266,25 +1440,13 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
         memset(&mq, 0, sizeof(mq)); memset(&mk, 0, sizeof(mk));
         memset(&mv, 0, sizeof(mv)); memset(&mg, 0, sizeof(mg));
     }
-    if (use_cluster_variant(B, H)) {
-        static bool cattr_set = false;
-        if (!cattr_set) {
-            cudaError_t e = cudaFuncSetAttribute(prefill_cluster_kernel,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)pc::SMEM_BYTES);
-            if (e != cudaSuccess) return e;
-            cattr_set = true;
-        }
-        dim3 grid((pc::NPREPCTA + 1) * H, B);
-        prefill_cluster_kernel<<<grid, pc::NTH, pc::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
-    } else {
-        dim3 grid(H, B);
-        prefill_tc_kernel<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H);
-    }
+    const PrefillPath path = choose_path(B, T, H);
+    if (path == PrefillPath::Segmented)
+        return launch_segmented(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, stream);
+    const cudaError_t e = launch_pass(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, T, 1, 0u,
+                                      path == PrefillPath::Cluster, stream);
     note_launches(1);
-    return cudaGetLastError();
+    return e;
 }
 
 // Self-test of the bounded waits: one warp waits on an mbarrier that nothing

@@ -46,7 +46,8 @@ class Workload:
 # The five workloads: a tiny fp32 case, an 8K prefill, a batch of 64K
 # pre-training sequences, a million-token prefill and a batched decode run;
 # plus a profiling size for the one-SM-per-head prefill path (the 64K batch
-# scaled down in T so that a full profiler capture stays at about 1 GB).
+# scaled down in T so that a full profiler capture stays at about 1 GB) and a
+# million-token context with only two heads (the segment-scan path).
 WORKLOADS = {
     "tiny_fp32": Workload("tiny_fp32", "prefill", 1, 64, 2, 32, 32,
                           torch.float32, 1001,
@@ -65,6 +66,10 @@ WORKLOADS = {
                                torch.bfloat16, 1006, pin_frac=0.1,
                                note="B4 H32 T8192 d128 bf16, 10%+10% of g channels "
                                     "pinned at -5 and 0, h0=0 (profiling size)"),
+    "prefill_1m_h2": Workload("prefill_1m_h2", "prefill", 1, 1048576, 2, 128, 128,
+                              torch.bfloat16, 1007,
+                              note="B1 H2 T1048576 d128 bf16, h0=0 (few heads, long "
+                                   "context: the segment-scan path)"),
     "decode_256": Workload("decode_256", "decode", 256, 1000, 32, 128, 128,
                            torch.bfloat16, 1005, h0_std=0.1,
                            note="256 requests x H32 d128, fp32 state "

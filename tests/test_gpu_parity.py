@@ -149,6 +149,53 @@ def test_bf16_both_prefill_variants(monkeypatch, variant, T):
     assert kda.device_status() == kda.KDA_OK
 
 
+# ------------------------------------------------------ segment scan ---
+
+@pytest.mark.parametrize("B,H,T,pin", [(1, 1, 5000, 0.0), (1, 2, 4096, 0.1), (2, 1, 6173, 0.0)])
+def test_bf16_segment_scan_chosen(B, H, T, pin):
+    """Very few heads on a long sequence: the segment scan is chosen by itself
+    (pass 1 from S = 0 and from S = I with v = 0, the segment chain, pass 3)."""
+    x = prefill_inputs(B, T, H, 128, 128, seed=700 + T + H, h0_std=0.0 if pin else 0.1, pin_frac=pin)
+    o, hT = run_prefill(x)
+    check_prefill(x, o, hT, TOL_BF16)
+    assert kda.device_status() == kda.KDA_OK
+
+
+@pytest.mark.parametrize("T", [512, 1000, 2048, 3000])
+def test_bf16_segment_scan_forced(monkeypatch, T):
+    """Forced at more heads: segments that end on the last token and ragged
+    last segments; the per-pass kernel is the cluster variant (up to 37
+    segment-heads) or the one-SM variant."""
+    monkeypatch.setenv("KDA_PREFILL_VARIANT", "segmented")
+    x = prefill_inputs(2, T, 3, 128, 128, seed=800 + T, h0_std=0.1)
+    o, hT = run_prefill(x)
+    check_prefill(x, o, hT, TOL_BF16)
+    assert kda.device_status() == kda.KDA_OK
+
+
+@pytest.mark.slow
+def test_workload_prefill_1m_h2_sampled():
+    """A million-token context with two heads (segment scan, 74 segments per
+    head): one head checked over the full length."""
+    w = WORKLOADS["prefill_1m_h2"]
+    x = prefill_inputs(w.B, w.T, w.H, w.dk, w.dv, seed=w.seed, device=DEV)
+    o, hT = kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"])
+    torch.cuda.synchronize()
+    assert kda.device_status() == kda.KDA_OK
+    eo, eh = _sampled_heads_check(w, x, o, hT, [(0, 1)])
+    assert eo <= TOL_BF16 and eh <= TOL_BF16, f"err_o={eo:.3e} err_hT={eh:.3e}"
+
+
+def test_bf16_segment_scan_inplace_state():
+    """hT = h0 (in-place state update) through the segment scan."""
+    x = prefill_inputs(1, 4500, 1, 128, 128, seed=901, h0_std=0.1)
+    d = to_dev(x)
+    S = d["h0"].clone()
+    o, _ = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], S, hT=S)
+    torch.cuda.synchronize()
+    check_prefill(x, o, S, TOL_BF16)
+
+
 # ------------------------------------------------------- full workloads ---
 
 def _sampled_heads_check(w, d, o, hT, heads):
