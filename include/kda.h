@@ -31,7 +31,8 @@
  *     No entry point keeps a pointer after it returns.  Only kda_chunk_fwd
  *     takes memory of its own, and only on its segment-scan path (see
  *     there): stream-ordered workspace (cudaMallocAsync / cudaFreeAsync on
- *     `stream`), returned before the call's work completes.
+ *     `stream`).  kda_chunk_fwd_noalloc is the same call without any
+ *     allocation.
  *   - Calls are asynchronous on `stream` (0 = legacy default stream) and do
  *     no host synchronisation.  Asynchronous device errors surface at the
  *     caller's next synchronisation, as for any CUDA launch.
@@ -81,14 +82,32 @@ typedef enum {
  * (with v = 0) gives, per segment, the state it reaches from zero and its
  * transition matrix; a short chain over the segments gives each segment's
  * true start state; a last pass writes o.  This path takes 3 * B * P * H *
- * dk * dv * 4 bytes of stream-ordered workspace (at most 28.4 MB) and
- * returns KDA_ERR_NO_MEMORY if it cannot.  The environment variable
+ * dk * dv * 4 bytes of stream-ordered workspace (at most 29,097,984 bytes
+ * when the path is chosen by itself) and returns KDA_ERR_NO_MEMORY if it
+ * cannot.  The environment variable
  * KDA_PREFILL_VARIANT = fused | cluster | segmented forces one path
  * (measurement and tests; "segmented" needs T >= 512).
  */
 int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
                   const void* beta, const float* h0, void* o, float* hT,
                   int B, int T, int H, int dk, int dv, kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd that allocates nothing: on the
+ * segment-scan path its workspace is a fixed scratch array in the library's
+ * device memory (one copy per device, 29,097,984 bytes: three fp32 state
+ * arrays for up to 148 segment-heads, which covers every call that takes the
+ * segment scan by itself).  Arguments, layouts, results and the choice of
+ * path are those of kda_chunk_fwd (the same arithmetic, bit for bit).
+ * Returns KDA_ERR_NO_MEMORY, before anything is launched, when the call
+ * needs more scratch than that (possible only when the segment scan is
+ * forced through KDA_PREFILL_VARIANT).  Calls that take the segment-scan
+ * path share the one scratch of their device: order them (one stream, or
+ * events between streams); the other paths use no scratch.
+ */
+int kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const void* g,
+                          const void* beta, const float* h0, void* o, float* hT,
+                          int B, int T, int H, int dk, int dv, kda_stream_t stream);
 
 /*
  * kda_chunk_fwd_f32 -- the same recurrence with fp32 inputs and fp32 output,

@@ -28,7 +28,7 @@ KDA_ERR_CUDA = -3
 KDA_ERR_TIMEOUT = -4
 KDA_ERR_NO_MEMORY = -5
 
-EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_f32", "kda_decode_step",
+EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_f32", "kda_decode_step",
             "kda_device_status", "kda_selftest_bounded_wait",
             "kda_status_string", "kda_launch_count", "kda_version")
 
@@ -62,6 +62,8 @@ def load_library(path: str = LIB_PATH):
     vp, fp, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_fwd.restype = i
+    lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, vp]
+    lib.kda_chunk_fwd_noalloc.restype = i
     lib.kda_chunk_fwd_f32.argtypes = [fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_fwd_f32.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, fp, vp, i, i, i, i, vp]
@@ -163,6 +165,14 @@ def chunk_fwd(q, k, v, g, beta, h0=None, *, o=None, hT=None, output_final_state=
     """
     import torch
     return _prefill("kda_chunk_fwd", torch.bfloat16, q, k, v, g, beta, h0, o,
+                    hT, output_final_state)
+
+
+def chunk_fwd_noalloc(q, k, v, g, beta, h0=None, *, o=None, hT=None, output_final_state=True):
+    """chunk_fwd without any allocation in the library (kda_chunk_fwd_noalloc):
+    the segment-scan path uses the library's fixed device scratch."""
+    import torch
+    return _prefill("kda_chunk_fwd_noalloc", torch.bfloat16, q, k, v, g, beta, h0, o,
                     hT, output_final_state)
 
 

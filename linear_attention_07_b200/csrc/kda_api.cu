@@ -16,7 +16,7 @@ cudaError_t decode_step_launch(const void* q, const void* k, const void* v,
 
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, const float* h0, void* o, float* hT,
-                              int B, int T, int H, cudaStream_t stream);
+                              int B, int T, int H, bool no_alloc, cudaStream_t stream);
 int prefill_device_status(cudaStream_t stream);
 cudaError_t bounded_wait_selftest_launch(uint64_t limit_ns, cudaStream_t stream);
 
@@ -69,9 +69,9 @@ using namespace kda;
 
 extern "C" {
 
-int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
-                  const void* beta, const float* h0, void* o, float* hT,
-                  int B, int T, int H, int dk, int dv, kda_stream_t stream)
+static int chunk_fwd_bf16(const void* q, const void* k, const void* v, const void* g,
+                          const void* beta, const float* h0, void* o, float* hT,
+                          int B, int T, int H, int dk, int dv, bool no_alloc, kda_stream_t stream)
 {
     int st = check_prefill(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv);
     if (st != KDA_OK) return st;
@@ -79,8 +79,22 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
     if ((reinterpret_cast<uintptr_t>(beta) & 1u) != 0) return KDA_ERR_INVALID_ARG;
     if ((int64_t)B * H == 0) return KDA_OK;
     if (T == 0 && hT == nullptr) return KDA_OK;
-    return status_of(prefill_tc_launch(q, k, v, g, beta, h0, o, hT, B, T, H,
+    return status_of(prefill_tc_launch(q, k, v, g, beta, h0, o, hT, B, T, H, no_alloc,
                                        (cudaStream_t)stream));
+}
+
+int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
+                  const void* beta, const float* h0, void* o, float* hT,
+                  int B, int T, int H, int dk, int dv, kda_stream_t stream)
+{
+    return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, false, stream);
+}
+
+int kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const void* g,
+                          const void* beta, const float* h0, void* o, float* hT,
+                          int B, int T, int H, int dk, int dv, kda_stream_t stream)
+{
+    return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, true, stream);
 }
 
 int kda_chunk_fwd_f32(const float* q, const float* k, const float* v,

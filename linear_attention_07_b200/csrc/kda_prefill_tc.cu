@@ -1377,26 +1377,43 @@ static void segment_plan(int B, int T, int H, int* seg_len, int* n_seg)
     *n_seg = (T + *seg_len - 1) / *seg_len;
 }
 
+// Fixed scratch of the no-allocation entry point: the segment scan's three
+// state arrays for up to 148 segment-heads, which covers every call that
+// chooses the segment scan by itself (B * H * P <= 148).  One copy per device.
+constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)3 * 148 * pf::D * pf::D * sizeof(float);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
 static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                     const CUtensorMap& mg, const void* beta, const float* h0, void* o,
-                                    float* hT, int B, int T, int H, cudaStream_t stream)
+                                    float* hT, int B, int T, int H, bool no_alloc, cudaStream_t stream)
 {
     int seg_len = 0, n_seg = 0;
     segment_plan(B, T, H, &seg_len, &n_seg);
     const size_t states = (size_t)B * n_seg * H * pf::D * pf::D;     // floats per array
-    static bool pool_set = false;   // keep freed workspace in the pool between calls
-    if (!pool_set) {
-        int dev = 0;
-        cudaMemPool_t pool;
-        if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
-            uint64_t keep = UINT64_MAX;
-            cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-        }
-        pool_set = true;
-    }
+    const size_t bytes = 3 * states * sizeof(float);
     float* ws = nullptr;
-    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), 3 * states * sizeof(float), stream);
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
+    if (no_alloc) {
+        // nothing is launched when the fixed scratch is too small
+        if (bytes > NOALLOC_SCRATCH_BYTES) return cudaErrorMemoryAllocation;
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // this device's copy
+        if (e != cudaSuccess) return e;
+        ws = static_cast<float*>(p);
+    } else {
+        static bool pool_set = false;   // keep freed workspace in the pool between calls
+        if (!pool_set) {
+            int dev = 0;
+            cudaMemPool_t pool;
+            if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+                uint64_t keep = UINT64_MAX;
+                cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+            }
+            pool_set = true;
+        }
+        e = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
+        if (e != cudaSuccess) return e;
+    }
     float* Mw = ws;
     float* Nw = ws + states;
     float* Sw = ws + 2 * states;
@@ -1411,15 +1428,17 @@ static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk
     }
     if (e == cudaSuccess)
         e = launch_pass(mq, mk, mv, mg, beta, Sw, o, nullptr, B, T, H, seg_len, n_seg, 0u, cl, stream);
-    const cudaError_t ef = cudaFreeAsync(ws, stream);
-    if (e == cudaSuccess) e = ef;
+    if (!no_alloc) {
+        const cudaError_t ef = cudaFreeAsync(ws, stream);
+        if (e == cudaSuccess) e = ef;
+    }
     note_launches(4);
     return e;
 }
 
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, const float* h0, void* o, float* hT,
-                              int B, int T, int H, cudaStream_t stream)
+                              int B, int T, int H, bool no_alloc, cudaStream_t stream)
 {
     static bool attr_set = false;   // idempotent; races only repeat the same calls
     if (!attr_set) {
@@ -1442,7 +1461,7 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
     }
     const PrefillPath path = choose_path(B, T, H);
     if (path == PrefillPath::Segmented)
-        return launch_segmented(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, stream);
+        return launch_segmented(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, no_alloc, stream);
     const cudaError_t e = launch_pass(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, T, 1, 0u,
                                       path == PrefillPath::Cluster, stream);
     note_launches(1);
