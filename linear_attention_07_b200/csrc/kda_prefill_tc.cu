@@ -678,7 +678,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     using namespace tc;
     extern __shared__ __align__(1024) unsigned char sm[];
     __shared__ uint32_t s_taddr;
-    __shared__ __align__(8) uint64_t s_bar[4];   // rank 0: FULL[0..2], MMA; ranks 1-3: EMPTY, MMA, input loads
+    __shared__ __align__(8) uint64_t s_bar[6];   // rank 0: FULL[0..2], X, KU0, KU1; ranks 1-3: EMPTY, MMA, input loads
     __shared__ int s_abort;
     __shared__ uint32_t s_odone;                 // rank 0: chunks whose slot is consumed
 
@@ -698,7 +698,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         tmem_relinquish();
     }
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
+        for (int i = 0; i < 6; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
         fence_mbar_init();
         s_abort = 0;
         s_odone = 0;
@@ -721,14 +721,17 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
     if (rank == 0) {
         // ========================================================= chain CTA ==
-        const uint32_t mbar = smem_u32(&s_bar[3]);   // X, then [Kb^T U, P U], of each chunk
+        const uint32_t mbar = smem_u32(&s_bar[3]);   // X of each chunk
+        const uint32_t kbar0 = smem_u32(&s_bar[4]);  // Kb^T U, d_k columns [0, 64)
+        const uint32_t kbar1 = smem_u32(&s_bar[5]);  // Kb^T U, d_k columns [64, 128), and P U
         if (warp == NCW / 32) {
             // ------------------------------------------------------ issuer warp --
             // Chunk ch: X = S^T [W | Qt]^T in two d_k halves (each as soon as
-            // the compute warps have written that half of the tf32 state), then
-            // Kb^T U and P U (one commit) once U is in tensor memory.
+            // the compute warps have written that half of the tf32 state), then,
+            // once U is in tensor memory, Kb^T U by d_k halves (one commit each,
+            // so the next state update starts on the first half) and P U.
             const uint32_t id1 = idesc_tf32(128, 2 * C, false, false);
-            const uint32_t id2 = idesc_tf32(128, 128, false, false);
+            const uint32_t id2 = idesc_tf32(128, 64, false, false);
             const uint32_t id3 = idesc_tf32(128, 32, false, false);
 #pragma unroll 1
             for (int ch = 0; ch < n_chunks; ++ch) {
@@ -762,17 +765,24 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 named_bar(NB_U, NX);
                 fence_after_sync();
                 if (!warp_flag(s_abort)) {
+                    // Kb rows [64, 128) start 8 core-matrix rows of SBO_K32 further
                     const uint64_t b20 = sdesc(smem_u32(sm + sb + S_B2), LBO, SBO_K32);
+                    const uint64_t b21 = sdesc(smem_u32(sm + sb + S_B2 + 8 * SBO_K32), LBO, SBO_K32);
                     const uint64_t b30 = sdesc(smem_u32(sm + sb + S_B3), LBO, SBO_K32);
 #pragma unroll
                     for (int ks = 0; ks < C / 8; ++ks)
                         mma_tf32_ts_w(tm + CT_DKU, tm + CT_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
                                       id2, ks > 0 ? 1u : 0u);
+                    mma_commit_w(kbar0);
+#pragma unroll
+                    for (int ks = 0; ks < C / 8; ++ks)
+                        mma_tf32_ts_w(tm + CT_DKU + 64, tm + CT_AU + ks * 8, b21 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                      id2, ks > 0 ? 1u : 0u);
 #pragma unroll
                     for (int ks = 0; ks < C / 8; ++ks)
                         mma_tf32_ts_w(tm + dx + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * LBO) >> 4),
                                       id3, 1u);
-                    mma_commit_w(mbar);
+                    mma_commit_w(kbar1);
                 }
                 __syncwarp();
             }
@@ -888,6 +898,8 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     state_half(0);
                     fence_before_sync();
                     named_arrive(NB_ASA, NX);
+                    wait_bar(kbar1, (uint32_t)(ch - 1) & 1u);   // Kb^T U second half and P U of chunk ch - 1
+                    if (tid == 0) counter_publish(smem_u32(&s_odone), (uint32_t)ch);
                     state_half(1);
                     fence_before_sync();
                     named_arrive(NB_ASB, NX);
@@ -912,12 +924,11 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 fence_before_sync();
                 named_arrive(NB_U, NX);
                 decay(sb);                            // while Kb^T U and P U run
-                wait_bar(mbar, phase & 1u);           // Kb^T U and P U of chunk ch
-                ++phase;
-                if (tid == 0) counter_publish(smem_u32(&s_odone), (uint32_t)ch + 1u);
+                wait_bar(kbar0, (uint32_t)ch & 1u);   // Kb^T U, first d_k half, of chunk ch
             }
             if (n_chunks > 0) {
                 state_half(0);
+                wait_bar(kbar1, (uint32_t)(n_chunks - 1) & 1u);
                 state_half(1);
                 emit_output(n_chunks - 1);
             }
@@ -1297,49 +1308,73 @@ constexpr int SEG_COLS = 16;          // state columns per combine CTA
 // cores (columns of S are independent: one CTA per group of 16 columns).
 // Writes S_p, the start state of segment p, for pass 3, and the final state.
 // M, N, S0: [B * n_seg][H][D][D]; h0, hT: [B][H][D][D] (either may be null;
-// hT may equal h0).
+// hT may equal h0).  M_p goes to shared memory with cp.async, one segment
+// ahead (two buffers), rows padded to 132 floats (16-byte aligned; the 16
+// rows a warp reads at one k fall on 16 banks pairwise).
+constexpr int SEG_MLD = pf::D + 4;
+constexpr uint32_t SEG_COMBINE_SMEM = (uint32_t)(pf::D * SEG_COLS + 2 * pf::D * SEG_MLD) * 4;
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 :: "r"(tc::smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
 __global__ void __launch_bounds__(256)
 segment_combine_kernel(const float* __restrict__ M, const float* __restrict__ N, float* __restrict__ S0,
                        const float* h0, float* hT, int H, int n_seg)
 {
     constexpr int D = pf::D;
-    __shared__ __align__(16) float s[D][SEG_COLS];
+    extern __shared__ __align__(16) float csm[];
+    float (*s)[SEG_COLS] = reinterpret_cast<float (*)[SEG_COLS]>(csm);          // [D][SEG_COLS]
+    float* mb = csm + D * SEG_COLS;                                              // 2 x [D][SEG_MLD]
     const int bh = blockIdx.y, b = bh / H, h = bh - b * H;
     const int tid = threadIdx.x;
     const int i = tid >> 1, jh = (tid & 1) * 8;              // row i, columns [col0, col0 + 8)
     const int col0 = blockIdx.x * SEG_COLS + jh;
+    auto seg_base = [&](int p) { return ((int64_t)(b * n_seg + p) * H + h) * D * D; };
+    auto load_m = [&](int p) {                               // M_p -> buffer p & 1 (16 x 16 B per thread)
+        const float* src = M + seg_base(p);
+        float* dst = mb + (p & 1) * D * SEG_MLD;
+#pragma unroll
+        for (int u = 0; u < (D * D / 4) / 256; ++u) {
+            const int e = (u * 256 + tid) * 4;               // element of a row-major D x D matrix
+            cp_async16(dst + (e / D) * SEG_MLD + (e % D), src + e);
+        }
+        cp_async_commit();
+    };
+    load_m(0);
+    if (n_seg > 1) load_m(1); else cp_async_commit();
 #pragma unroll
     for (int c = 0; c < 8; ++c) s[i][jh + c] = h0 ? h0[(int64_t)bh * D * D + (int64_t)i * D + col0 + c] : 0.f;
-    __syncthreads();
 #pragma unroll 1
     for (int p = 0; p < n_seg; ++p) {
-        const int64_t sp = ((int64_t)(b * n_seg + p) * H + h) * D * D + (int64_t)i * D + col0;
+        const int64_t sp = seg_base(p) + (int64_t)i * D + col0;
         float acc[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            S0[sp + c] = s[i][jh + c];
-            acc[c] = N[sp + c];
-        }
-        const float4* mrow = reinterpret_cast<const float4*>(M + (sp - col0));
-#pragma unroll 4
-        for (int k4 = 0; k4 < D / 4; ++k4) {
-            const float4 m = mrow[k4];
-            const float mk[4] = {m.x, m.y, m.z, m.w};
+        for (int c = 0; c < 8; ++c) acc[c] = N[sp + c];
+        cp_async_wait_1();                                   // M_p has landed (M_{p+1} may be in flight)
+        __syncthreads();                                     // ... for every thread; s holds S_p
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const float4 a0 = *reinterpret_cast<const float4*>(&s[4 * k4 + kk][jh]);
-                const float4 a1 = *reinterpret_cast<const float4*>(&s[4 * k4 + kk][jh + 4]);
-                acc[0] = fmaf(mk[kk], a0.x, acc[0]); acc[1] = fmaf(mk[kk], a0.y, acc[1]);
-                acc[2] = fmaf(mk[kk], a0.z, acc[2]); acc[3] = fmaf(mk[kk], a0.w, acc[3]);
-                acc[4] = fmaf(mk[kk], a1.x, acc[4]); acc[5] = fmaf(mk[kk], a1.y, acc[5]);
-                acc[6] = fmaf(mk[kk], a1.z, acc[6]); acc[7] = fmaf(mk[kk], a1.w, acc[7]);
-            }
+        for (int c = 0; c < 8; ++c) S0[sp + c] = s[i][jh + c];
+        const float* mrow = mb + (p & 1) * D * SEG_MLD + i * SEG_MLD;
+#pragma unroll 8
+        for (int k = 0; k < D; ++k) {
+            const float m = mrow[k];
+            const float4 a0 = *reinterpret_cast<const float4*>(&s[k][jh]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&s[k][jh + 4]);
+            acc[0] = fmaf(m, a0.x, acc[0]); acc[1] = fmaf(m, a0.y, acc[1]);
+            acc[2] = fmaf(m, a0.z, acc[2]); acc[3] = fmaf(m, a0.w, acc[3]);
+            acc[4] = fmaf(m, a1.x, acc[4]); acc[5] = fmaf(m, a1.y, acc[5]);
+            acc[6] = fmaf(m, a1.z, acc[6]); acc[7] = fmaf(m, a1.w, acc[7]);
         }
-        __syncthreads();
+        __syncthreads();                                     // every read of S_p and of buffer p & 1 done
+        if (p + 2 < n_seg) load_m(p + 2); else cp_async_commit();
 #pragma unroll
         for (int c = 0; c < 8; ++c) s[i][jh + c] = acc[c];
-        __syncthreads();
     }
+    __syncthreads();
     if (hT) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) hT[(int64_t)bh * D * D + (int64_t)i * D + col0 + c] = s[i][jh + c];
@@ -1423,7 +1458,8 @@ static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk
         e = launch_pass(mq, mk, mv, mg, beta, nullptr, o, Mw, B, T, H, seg_len, n_seg,
                         pf::SEG_V_ZERO | pf::SEG_H0_EYE | pf::SEG_NO_O, cl, stream);
     if (e == cudaSuccess) {
-        segment_combine_kernel<<<dim3(pf::D / SEG_COLS, B * H), 256, 0, stream>>>(Mw, Nw, Sw, h0, hT, H, n_seg);
+        segment_combine_kernel<<<dim3(pf::D / SEG_COLS, B * H), 256, SEG_COMBINE_SMEM, stream>>>(
+            Mw, Nw, Sw, h0, hT, H, n_seg);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess)
@@ -1447,6 +1483,9 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(prefill_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)pc::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)SEG_COMBINE_SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
