@@ -93,6 +93,28 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
                   int B, int T, int H, int dk, int dv, kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_states -- kda_chunk_fwd that also writes intermediate states
+ * (prefix-cache blocks): the fp32 state after every `state_every` tokens,
+ *
+ *   states : fp32 [B][H][T / state_every][dk][dv],  states[b][h][s] = S after
+ *            token (s + 1) * state_every of sequence b, head h
+ *
+ * (floor division: a block that the sequence does not complete gets no
+ * state; with T a multiple of state_every the last one equals hT).
+ * state_every must be a positive multiple of 32 (the chunk of the state
+ * recurrence), else KDA_ERR_INVALID_ARG; states may be NULL only when
+ * T < state_every.  Same paths and arithmetic as kda_chunk_fwd (the states
+ * are the fp32 master state, not a rounded copy).  The "177: Kimi K3 in
+ * Detail" episode notes (Deep dive 10, 23) describe serving that keeps a
+ * long shared prefix and adds a few thousand tokens per turn; a state
+ * every block lets a later call resume from any block boundary.
+ */
+int kda_chunk_fwd_states(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const float* h0, void* o, float* hT,
+                         float* states, int state_every,
+                         int B, int T, int H, int dk, int dv, kda_stream_t stream);
+
+/*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd that allocates nothing: on the
  * segment-scan path its workspace is a fixed scratch array in the library's
  * device memory (one copy per device, 29,097,984 bytes: three fp32 state

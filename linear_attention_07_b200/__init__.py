@@ -28,7 +28,8 @@ KDA_ERR_CUDA = -3
 KDA_ERR_TIMEOUT = -4
 KDA_ERR_NO_MEMORY = -5
 
-EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_f32", "kda_decode_step",
+EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_states", "kda_chunk_fwd_f32",
+            "kda_decode_step",
             "kda_device_status", "kda_selftest_bounded_wait",
             "kda_status_string", "kda_launch_count", "kda_version")
 
@@ -64,6 +65,8 @@ def load_library(path: str = LIB_PATH):
     lib.kda_chunk_fwd.restype = i
     lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_fwd_noalloc.restype = i
+    lib.kda_chunk_fwd_states.argtypes = [vp, vp, vp, vp, vp, fp, vp, fp, fp, i, i, i, i, i, i, vp]
+    lib.kda_chunk_fwd_states.restype = i
     lib.kda_chunk_fwd_f32.argtypes = [fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_fwd_f32.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, fp, vp, i, i, i, i, vp]
@@ -174,6 +177,35 @@ def chunk_fwd_noalloc(q, k, v, g, beta, h0=None, *, o=None, hT=None, output_fina
     import torch
     return _prefill("kda_chunk_fwd_noalloc", torch.bfloat16, q, k, v, g, beta, h0, o,
                     hT, output_final_state)
+
+
+def chunk_fwd_states(q, k, v, g, beta, h0=None, *, state_every, o=None, hT=None, states=None):
+    """chunk_fwd that also returns the fp32 state after every `state_every`
+    tokens (kda_chunk_fwd_states): (o, hT, states), states [B, H, T //
+    state_every, dk, dv]."""
+    import torch
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    n = T // state_every if state_every > 0 else 0
+    if states is None:
+        states = torch.empty((B, H, n, dk, dv), dtype=torch.float32, device=q.device)
+    _check(states, "states", torch.float32, (B, H, n, dk, dv), q.device)
+    if o is None:
+        o = torch.empty_like(v)
+    if hT is None:
+        hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("g", g, (B, T, H, dk)),
+                         ("v", v, (B, T, H, dv)), ("beta", beta, (B, T, H)), ("o", o, (B, T, H, dv))):
+        _check(t, name, torch.bfloat16, shp, q.device)
+    _check(hT, "hT", torch.float32, (B, H, dk, dv), q.device)
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (B, H, dk, dv), q.device)
+    st = load_library().kda_chunk_fwd_states(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o), _ptr(hT),
+        _ptr(states) if n > 0 else None, int(state_every), B, T, H, dk, dv, _stream(q.device))
+    if st != KDA_OK:
+        raise KdaError("kda_chunk_fwd_states", st)
+    return o, hT, states
 
 
 def chunk_fwd_f32(q, k, v, g, beta, h0=None, *, o=None, hT=None, output_final_state=True):

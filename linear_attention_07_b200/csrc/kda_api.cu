@@ -16,7 +16,8 @@ cudaError_t decode_step_launch(const void* q, const void* k, const void* v,
 
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, const float* h0, void* o, float* hT,
-                              int B, int T, int H, bool no_alloc, cudaStream_t stream);
+                              int B, int T, int H, bool no_alloc, float* states, int snap_every,
+                              cudaStream_t stream);
 int prefill_device_status(cudaStream_t stream);
 cudaError_t bounded_wait_selftest_launch(uint64_t limit_ns, cudaStream_t stream);
 
@@ -71,7 +72,8 @@ extern "C" {
 
 static int chunk_fwd_bf16(const void* q, const void* k, const void* v, const void* g,
                           const void* beta, const float* h0, void* o, float* hT,
-                          int B, int T, int H, int dk, int dv, bool no_alloc, kda_stream_t stream)
+                          int B, int T, int H, int dk, int dv, bool no_alloc,
+                          float* states, int state_every, kda_stream_t stream)
 {
     int st = check_prefill(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv);
     if (st != KDA_OK) return st;
@@ -80,21 +82,33 @@ static int chunk_fwd_bf16(const void* q, const void* k, const void* v, const voi
     if ((int64_t)B * H == 0) return KDA_OK;
     if (T == 0 && hT == nullptr) return KDA_OK;
     return status_of(prefill_tc_launch(q, k, v, g, beta, h0, o, hT, B, T, H, no_alloc,
-                                       (cudaStream_t)stream));
+                                       states, state_every / 32, (cudaStream_t)stream));
 }
 
 int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
                   const void* beta, const float* h0, void* o, float* hT,
                   int B, int T, int H, int dk, int dv, kda_stream_t stream)
 {
-    return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, false, stream);
+    return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, false, nullptr, 0, stream);
+}
+
+int kda_chunk_fwd_states(const void* q, const void* k, const void* v, const void* g,
+                         const void* beta, const float* h0, void* o, float* hT,
+                         float* states, int state_every,
+                         int B, int T, int H, int dk, int dv, kda_stream_t stream)
+{
+    if (state_every <= 0 || state_every % 32 != 0) return KDA_ERR_INVALID_ARG;
+    const int64_t n_snap = T > 0 ? T / state_every : 0;
+    if (n_snap > 0 && (states == nullptr || !aligned16(states))) return KDA_ERR_INVALID_ARG;
+    return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, false,
+                          n_snap > 0 ? states : nullptr, state_every, stream);
 }
 
 int kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const void* g,
                           const void* beta, const float* h0, void* o, float* hT,
                           int B, int T, int H, int dk, int dv, kda_stream_t stream)
 {
-    return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, true, stream);
+    return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, true, nullptr, 0, stream);
 }
 
 int kda_chunk_fwd_f32(const float* q, const float* k, const float* v,

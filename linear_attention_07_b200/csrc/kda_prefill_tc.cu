@@ -134,6 +134,20 @@ __device__ __forceinline__ void named_arrive(uint32_t id, uint32_t count) {
     asm volatile("bar.arrive %0, %1;" :: "r"(id), "r"(count) : "memory");
 }
 
+// State snapshots (prefix-cache blocks): with snap_every > 0 chunks, the fp32
+// state after every snap_every * 32 tokens of the whole sequence is written
+// to states[b][h][s][D][D], s = 0 .. T / (snap_every * 32) - 1 (a block that
+// the sequence does not complete gets no snapshot).  gc is the index of the
+// chunk just completed, counted from the start of the sequence.
+__device__ __forceinline__ float* snapshot_slot(float* states, int snap_every, int gc, int T, int b, int H, int h)
+{
+    if (states == nullptr || snap_every <= 0 || (gc + 1) % snap_every != 0) return nullptr;
+    const int s = (gc + 1) / snap_every - 1;
+    const int n_snap = T / (snap_every * pf::C);
+    if (s >= n_snap) return nullptr;
+    return states + (((int64_t)b * H + h) * n_snap + s) * pf::D * pf::D;
+}
+
 // A shared flag read once by lane 0 and broadcast: the same value in every
 // lane, so a whole-warp MMA issue never diverges on it.
 __device__ __forceinline__ bool warp_flag(const int& flag) {
@@ -145,7 +159,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                   const __nv_bfloat16* __restrict__ beta, const float* h0,
                   __nv_bfloat16* __restrict__ o, float* hT, int T, int H,
-                  int seg_len, int n_seg, uint32_t flags)
+                  int seg_len, int n_seg, uint32_t flags, float* states, int snap_every)
 {
     using namespace pf;
     using namespace tc;
@@ -291,6 +305,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                     tmem_st16(tm + lane_base + T_AS + 64 * hh + c0, d);
                 }
+                if (float* snap = snapshot_slot(states, snap_every, ts / C + ch, T, b, H, h)) {
+#pragma unroll
+                    for (int i = 0; i < D / 2; ++i) snap[(int64_t)(64 * hh + i) * D + j] = S[i];
+                }
                 // o: this half's 16 tokens of column j into shared memory, then
                 // whole rows to global memory in 16-byte vectors
                 __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + OST);
@@ -416,7 +434,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const float kt = kr[rr] * p;
                     const float qt = qr[rr] * p;
                     st_f32(sm, GB + off_kmajor(r, c, PAD_LBO, SBO_K128P), to_tf32(kt));
-                    st_f32(sm, GB + off_kmajor(C + r, c, PAD_LBO, SBO_K128P), to_tf32(qt));
+                    st_f32(sm, GB + off_kmajor(C + r, c, PAD_LBO, SBO_K128P), qt);   // full fp32: see below
                     kc[rr & 3] = to_tf32(kt * f);
                     if ((rr & 3) == 3)
                         st_f32x4(sm, WA + off_kmajor(c, r - 3, LBO, SBO_K32), kc[0], kc[1], kc[2], kc[3]);
@@ -428,8 +446,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int rr = TILE - 1; rr >= 0; --rr) {
                     const int r = tau * TILE + rr;
                     const float kb = kr[rr] * sgm;
-                    st_f32(sm, GA + off_kmajor(r, c, PAD_LBO, SBO_K128P), to_tf32(kb * inv));
-                    if (tau == 0) st_f32(sm, GA + off_kmajor(C + rr, c, PAD_LBO, SBO_K128P), to_tf32(kb));
+                    // Qt (above), Kh and Kb_0 stay in full fp32: the operand fill
+                    // rescales them into the chunk-relative Qt and Kb and rounds
+                    // to tf32 once (rounding here too would round those twice);
+                    // the Gram MMA reads the rows as tf32 (low mantissa bits
+                    // ignored).
+                    st_f32(sm, GA + off_kmajor(r, c, PAD_LBO, SBO_K128P), kb * inv);
+                    if (tau == 0) st_f32(sm, GA + off_kmajor(C + rr, c, PAD_LBO, SBO_K128P), kb);
                     sgm *= a[rr];
                 }
             }
@@ -672,7 +695,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                        const __nv_bfloat16* __restrict__ beta, const float* h0,
                        __nv_bfloat16* __restrict__ o, float* hT, int T, int H,
-                       int seg_len, int n_seg, uint32_t flags)
+                       int seg_len, int n_seg, uint32_t flags, float* states, int snap_every)
 {
     using namespace pc;
     using namespace tc;
@@ -854,6 +877,16 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 tmem_st32(tm + lane_base + CT_AS + 64 * q2 + 32 * hh, d);
                 wait_st();
             };
+            // the fp32 state after chunk gc of the sequence, when it ends a snapshot block
+            auto snapshot = [&](int gc) {
+                if (float* snap = snapshot_slot(states, snap_every, gc, T, b, H, h)) {
+#pragma unroll
+                    for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            snap[(int64_t)(64 * q2 + 32 * hh + i) * D + j] = S[32 * q2 + i];
+                }
+            };
             // S <- Diag(gamma_C) S with gamma of the slot at sb
             auto decay = [&](uint32_t sb) {
                 const float4* gam4 = reinterpret_cast<const float4*>(sm + sb + S_GAM);
@@ -903,6 +936,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     state_half(1);
                     fence_before_sync();
                     named_arrive(NB_ASB, NX);
+                    snapshot(ts / C + ch - 1);                  // S after chunk ch - 1
                     emit_output(ch - 1);
                 }
                 // X of chunk ch (U' of this chunk is in the slot once its FULL phase passed)
@@ -930,6 +964,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 state_half(0);
                 wait_bar(kbar1, (uint32_t)(n_chunks - 1) & 1u);
                 state_half(1);
+                snapshot(ts / C + n_chunks - 1);
                 emit_output(n_chunks - 1);
             }
             if (hT && !s_abort) {
@@ -1091,7 +1126,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     const float kt = kr[rr] * p;
                     const float qt = qr[rr] * p;
                     st_f32(sm, P_GB + off_kmajor(r, c, PAD_LBO, SBO_K128P), to_tf32(kt));
-                    st_f32(sm, P_GB + off_kmajor(C + r, c, PAD_LBO, SBO_K128P), to_tf32(qt));
+                    st_f32(sm, P_GB + off_kmajor(C + r, c, PAD_LBO, SBO_K128P), qt);   // full fp32: see below
                     kc[rr & 3] = to_tf32(kt * f);
                     if ((rr & 3) == 3)
                         st_f32x4(sm, P_WA + off_kmajor(c, r - 3, LBO, SBO_K32), kc[0], kc[1], kc[2], kc[3]);
@@ -1102,8 +1137,13 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 for (int rr = TILE - 1; rr >= 0; --rr) {
                     const int r = tau * TILE + rr;
                     const float kb = kr[rr] * sgm;
-                    st_f32(sm, P_GA + off_kmajor(r, c, PAD_LBO, SBO_K128P), to_tf32(kb * inv));
-                    if (tau == 0) st_f32(sm, P_GA + off_kmajor(C + rr, c, PAD_LBO, SBO_K128P), to_tf32(kb));
+                    // Qt (above), Kh and Kb_0 stay in full fp32: the operand fill
+                    // rescales them into the chunk-relative Qt and Kb and rounds
+                    // to tf32 once (rounding here too would round those twice);
+                    // the Gram MMA reads the rows as tf32 (low mantissa bits
+                    // ignored).
+                    st_f32(sm, P_GA + off_kmajor(r, c, PAD_LBO, SBO_K128P), kb * inv);
+                    if (tau == 0) st_f32(sm, P_GA + off_kmajor(C + rr, c, PAD_LBO, SBO_K128P), kb);
                     sgm *= a[rr];
                 }
             }
@@ -1275,16 +1315,18 @@ static bool cluster_fits(int64_t heads) { return heads * (pc::NPREPCTA + 1) <= 1
 static cudaError_t launch_pass(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                const CUtensorMap& mg, const void* beta, const float* h0, void* o, float* hT,
                                int B, int T, int H, int seg_len, int n_seg, uint32_t flags, bool cluster,
-                               cudaStream_t stream)
+                               float* states, int snap_every, cudaStream_t stream)
 {
     if (cluster) {
         dim3 grid((pc::NPREPCTA + 1) * H, B * n_seg);
         prefill_cluster_kernel<<<grid, pc::NTH, pc::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags);
+            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags,
+            states, snap_every);
     } else {
         dim3 grid(H, B * n_seg);
         prefill_tc_kernel<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags);
+            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags,
+            states, snap_every);
     }
     return cudaGetLastError();
 }
@@ -1420,12 +1462,13 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH
 
 static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                     const CUtensorMap& mg, const void* beta, const float* h0, void* o,
-                                    float* hT, int B, int T, int H, bool no_alloc, cudaStream_t stream)
+                                    float* hT, int B, int T, int H, bool no_alloc, float* states,
+                                    int snap_every, cudaStream_t stream)
 {
     int seg_len = 0, n_seg = 0;
     segment_plan(B, T, H, &seg_len, &n_seg);
-    const size_t states = (size_t)B * n_seg * H * pf::D * pf::D;     // floats per array
-    const size_t bytes = 3 * states * sizeof(float);
+    const size_t n_state = (size_t)B * n_seg * H * pf::D * pf::D;    // floats per array
+    const size_t bytes = 3 * n_state * sizeof(float);
     float* ws = nullptr;
     cudaError_t e = cudaSuccess;
     if (no_alloc) {
@@ -1450,20 +1493,22 @@ static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk
         if (e != cudaSuccess) return e;
     }
     float* Mw = ws;
-    float* Nw = ws + states;
-    float* Sw = ws + 2 * states;
+    float* Nw = ws + n_state;
+    float* Sw = ws + 2 * n_state;
     const bool cl = cluster_fits((int64_t)B * n_seg * H);
-    e = launch_pass(mq, mk, mv, mg, beta, nullptr, o, Nw, B, T, H, seg_len, n_seg, pf::SEG_NO_O, cl, stream);
+    e = launch_pass(mq, mk, mv, mg, beta, nullptr, o, Nw, B, T, H, seg_len, n_seg, pf::SEG_NO_O, cl,
+                    nullptr, 0, stream);
     if (e == cudaSuccess)
         e = launch_pass(mq, mk, mv, mg, beta, nullptr, o, Mw, B, T, H, seg_len, n_seg,
-                        pf::SEG_V_ZERO | pf::SEG_H0_EYE | pf::SEG_NO_O, cl, stream);
+                        pf::SEG_V_ZERO | pf::SEG_H0_EYE | pf::SEG_NO_O, cl, nullptr, 0, stream);
     if (e == cudaSuccess) {
         segment_combine_kernel<<<dim3(pf::D / SEG_COLS, B * H), 256, SEG_COMBINE_SMEM, stream>>>(
             Mw, Nw, Sw, h0, hT, H, n_seg);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess)
-        e = launch_pass(mq, mk, mv, mg, beta, Sw, o, nullptr, B, T, H, seg_len, n_seg, 0u, cl, stream);
+        e = launch_pass(mq, mk, mv, mg, beta, Sw, o, nullptr, B, T, H, seg_len, n_seg, 0u, cl,
+                        states, snap_every, stream);
     if (!no_alloc) {
         const cudaError_t ef = cudaFreeAsync(ws, stream);
         if (e == cudaSuccess) e = ef;
@@ -1474,7 +1519,8 @@ static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk
 
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, const float* h0, void* o, float* hT,
-                              int B, int T, int H, bool no_alloc, cudaStream_t stream)
+                              int B, int T, int H, bool no_alloc, float* states, int snap_every,
+                              cudaStream_t stream)
 {
     static bool attr_set = false;   // idempotent; races only repeat the same calls
     if (!attr_set) {
@@ -1500,9 +1546,9 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
     }
     const PrefillPath path = choose_path(B, T, H);
     if (path == PrefillPath::Segmented)
-        return launch_segmented(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, no_alloc, stream);
+        return launch_segmented(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, no_alloc, states, snap_every, stream);
     const cudaError_t e = launch_pass(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, T, 1, 0u,
-                                      path == PrefillPath::Cluster, stream);
+                                      path == PrefillPath::Cluster, states, snap_every, stream);
     note_launches(1);
     return e;
 }

@@ -83,6 +83,21 @@ def test_prefill_argument_errors(lib, fn):
     assert lib.kda_launch_count() == n0
 
 
+def test_states_argument_errors(lib):
+    """kda_chunk_fwd_states: the block length and the states buffer are checked
+    on the host; nothing is launched on a bad argument."""
+    n0 = lib.kda_launch_count()
+    f = lib.kda_chunk_fwd_states
+    args = lambda states, every, T=64: (A, A, A, A, A2, NUL, A, NUL, states, every, 1, T, 2, 128, 128, None)
+    assert f(*args(A, 0)) == kda.KDA_ERR_INVALID_ARG          # no block length
+    assert f(*args(A, 48)) == kda.KDA_ERR_INVALID_ARG         # not a multiple of 32
+    assert f(*args(A, -32)) == kda.KDA_ERR_INVALID_ARG
+    assert f(*args(NUL, 32)) == kda.KDA_ERR_INVALID_ARG       # two states to write, no buffer
+    assert f(*args(MIS, 32)) == kda.KDA_ERR_INVALID_ARG       # misaligned buffer
+    assert f(*args(A, 32, T=64)[:1] + (NUL,) + args(A, 32)[2:]) == kda.KDA_ERR_INVALID_ARG   # k missing
+    assert lib.kda_launch_count() == n0
+
+
 def test_bf16_prefill_shape_support(lib):
     # the tensor-core path is specialised to d_k = d_v = 128
     assert prefill(lib, "kda_chunk_fwd", dk=64, dv=64) == kda.KDA_ERR_UNSUPPORTED

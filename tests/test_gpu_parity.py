@@ -196,6 +196,53 @@ def test_bf16_segment_scan_inplace_state():
     check_prefill(x, o, S, TOL_BF16)
 
 
+# -------------------------------------------------- intermediate states ---
+
+def _check_states(x, states, every, tol=TOL_BF16):
+    """states[:, :, s] against the oracle's final state on the prefix of
+    (s + 1) * every tokens."""
+    T = x["q"].shape[1]
+    assert states.shape[2] == T // every
+    pre = lambda t, n: t[:, :n]
+    for s in range(T // every):
+        n = (s + 1) * every
+        _, hT_ref = oracle.fwd(pre(x["q"], n), pre(x["k"], n), pre(x["v"], n), pre(x["g"], n),
+                               pre(x["beta"], n), x["h0"])
+        e = err_state(states[:, :, s], hT_ref)
+        assert e <= tol, f"state {s} (after {n} tokens): err={e:.3e}"
+
+
+@pytest.mark.parametrize("variant,B,H,T,every", [
+    ("fused", 2, 3, 1000, 256), ("cluster", 2, 3, 1000, 256), ("cluster", 1, 2, 300, 32),
+    ("segmented", 2, 3, 2000, 512), ("segmented", 1, 1, 1100, 96)])
+def test_bf16_intermediate_states(monkeypatch, variant, B, H, T, every):
+    """kda_chunk_fwd_states on every path: each state against the oracle on the
+    matching prefix; o and hT as kda_chunk_fwd's, bit for bit."""
+    monkeypatch.setenv("KDA_PREFILL_VARIANT", variant)
+    x = prefill_inputs(B, T, H, 128, 128, seed=1100 + T + every, h0_std=0.1)
+    d = to_dev(x)
+    o, hT, st = kda.chunk_fwd_states(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], state_every=every)
+    o2, hT2 = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"])
+    torch.cuda.synchronize()
+    assert kda.device_status() == kda.KDA_OK
+    assert torch.equal(o, o2) and torch.equal(hT, hT2)
+    _check_states(x, st.cpu(), every)
+    if T % every == 0:
+        assert torch.equal(st[:, :, -1], hT)
+
+
+def test_bf16_intermediate_states_chosen_segment_scan():
+    """Few heads on a long sequence (segment scan chosen by itself): states
+    come from pass 3, which starts each segment from its true state."""
+    x = prefill_inputs(1, 4608, 1, 128, 128, seed=1200, h0_std=0.1)
+    d = to_dev(x)
+    o, hT, st = kda.chunk_fwd_states(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"], state_every=512)
+    torch.cuda.synchronize()
+    check_prefill(x, o, hT, TOL_BF16)
+    _check_states(x, st.cpu(), 512)
+    assert torch.equal(st[:, :, -1], hT)
+
+
 # ------------------------------------------------------- full workloads ---
 
 def _sampled_heads_check(w, d, o, hT, heads):
