@@ -115,6 +115,37 @@ int kda_chunk_fwd_states(const void* q, const void* k, const void* v, const void
                          int B, int T, int H, int dk, int dv, kda_stream_t stream);
 
 /*
+ * kda_chunk_transition -- the transition of each sequence as a whole,
+ *
+ *   M[b][h] = prod_{t = T..1} (I - beta_t k_t k_t^T) Diag(exp g_t)   (d_k x d_k)
+ *
+ * so that running the sequence from any start state S0 ends at
+ * M S0 + (the state it reaches from zero).  Computed on the tensor cores as
+ * the state reached from S = I with v = 0 (every state column evolves on its
+ * own), no o written.  q, k, g: bf16 [B][T][H][dk]; beta: bf16 [B][T][H];
+ * M: fp32 [B][H][dk][dk] (T == 0: the identity).  Supported: dk == 128.
+ * With kda_state_chain this joins segments of one sequence that were run
+ * independently (for example one segment per GPU).
+ */
+int kda_chunk_transition(const void* q, const void* k, const void* g, const void* beta, float* M,
+                         int B, int T, int H, int dk, kda_stream_t stream);
+
+/*
+ * kda_state_chain -- joins P consecutive segments of each sequence: with
+ * M[b][p][h] a segment's transition (kda_chunk_transition) and N[b][p][h]
+ * the state it reaches from zero (kda_chunk_fwd with h0 = NULL),
+ *
+ *   S_0 = h0[b][h] (or zero),   S_{p+1} = M_p S_p + N_p,
+ *
+ * writes S_start[b][p][h] = S_p (the true start state of segment p) and
+ * hT[b][h] = S_P.  M, N, S_start: fp32 [B][P][H][dk][dv] (M's last two
+ * dimensions are dk x dk, with dk == dv); h0, hT: fp32 [B][H][dk][dv], either
+ * may be NULL; hT may equal h0.  fp32 arithmetic.  Supported: dk == dv == 128.
+ */
+int kda_state_chain(const float* M, const float* N, const float* h0, float* S_start, float* hT,
+                    int B, int P, int H, int dk, int dv, kda_stream_t stream);
+
+/*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd that allocates nothing: on the
  * segment-scan path its workspace is a fixed scratch array in the library's
  * device memory (one copy per device, 29,097,984 bytes: three fp32 state

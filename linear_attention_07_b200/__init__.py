@@ -29,7 +29,7 @@ KDA_ERR_TIMEOUT = -4
 KDA_ERR_NO_MEMORY = -5
 
 EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_states", "kda_chunk_fwd_f32",
-            "kda_decode_step",
+            "kda_chunk_transition", "kda_state_chain", "kda_decode_step",
             "kda_device_status", "kda_selftest_bounded_wait",
             "kda_status_string", "kda_launch_count", "kda_version")
 
@@ -67,6 +67,10 @@ def load_library(path: str = LIB_PATH):
     lib.kda_chunk_fwd_noalloc.restype = i
     lib.kda_chunk_fwd_states.argtypes = [vp, vp, vp, vp, vp, fp, vp, fp, fp, i, i, i, i, i, i, vp]
     lib.kda_chunk_fwd_states.restype = i
+    lib.kda_chunk_transition.argtypes = [vp, vp, vp, vp, fp, i, i, i, i, vp]
+    lib.kda_chunk_transition.restype = i
+    lib.kda_state_chain.argtypes = [fp, fp, fp, fp, fp, i, i, i, i, i, vp]
+    lib.kda_state_chain.restype = i
     lib.kda_chunk_fwd_f32.argtypes = [fp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, i, vp]
     lib.kda_chunk_fwd_f32.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, fp, vp, i, i, i, i, vp]
@@ -206,6 +210,49 @@ def chunk_fwd_states(q, k, v, g, beta, h0=None, *, state_every, o=None, hT=None,
     if st != KDA_OK:
         raise KdaError("kda_chunk_fwd_states", st)
     return o, hT, states
+
+
+def chunk_transition(q, k, g, beta, *, M=None):
+    """Transition M [B, H, dk, dk] (fp32) of each whole sequence
+    (kda_chunk_transition): running it from S0 ends at M S0 + (its state from zero)."""
+    import torch
+    B, T, H, dk = q.shape
+    dev = q.device
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("g", g, (B, T, H, dk)),
+                         ("beta", beta, (B, T, H))):
+        _check(t, name, torch.bfloat16, shp, dev)
+    if M is None:
+        M = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev)
+    _check(M, "M", torch.float32, (B, H, dk, dk), dev)
+    st = load_library().kda_chunk_transition(_ptr(q), _ptr(k), _ptr(g), _ptr(beta), _ptr(M),
+                                             B, T, H, dk, _stream(dev))
+    if st != KDA_OK:
+        raise KdaError("kda_chunk_transition", st)
+    return M
+
+
+def state_chain(M, N, h0=None, *, S_start=None, hT=None):
+    """S_0 = h0, S_{p+1} = M_p S_p + N_p over P segments (kda_state_chain).
+    M: [B, P, H, dk, dk]; N: [B, P, H, dk, dv]; h0: [B, H, dk, dv] or None.
+    Returns (S_start [B, P, H, dk, dv], hT [B, H, dk, dv])."""
+    import torch
+    B, P, H, dk, dv = N.shape
+    dev = N.device
+    _check(M, "M", torch.float32, (B, P, H, dk, dk), dev)
+    _check(N, "N", torch.float32, (B, P, H, dk, dv), dev)
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (B, H, dk, dv), dev)
+    if S_start is None:
+        S_start = torch.empty_like(N)
+    if hT is None:
+        hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    _check(S_start, "S_start", torch.float32, (B, P, H, dk, dv), dev)
+    _check(hT, "hT", torch.float32, (B, H, dk, dv), dev)
+    st = load_library().kda_state_chain(_ptr(M), _ptr(N), _ptr(h0), _ptr(S_start), _ptr(hT),
+                                        B, P, H, dk, dv, _stream(dev))
+    if st != KDA_OK:
+        raise KdaError("kda_state_chain", st)
+    return S_start, hT
 
 
 def chunk_fwd_f32(q, k, v, g, beta, h0=None, *, o=None, hT=None, output_final_state=True):

@@ -18,6 +18,10 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
                               const void* beta, const float* h0, void* o, float* hT,
                               int B, int T, int H, bool no_alloc, float* states, int snap_every,
                               cudaStream_t stream);
+cudaError_t prefill_transition_launch(const void* q, const void* k, const void* g, const void* beta,
+                                      float* M, int B, int T, int H, cudaStream_t stream);
+cudaError_t state_chain_launch(const float* M, const float* N, const float* h0, float* S_start, float* hT,
+                               int B, int P, int H, cudaStream_t stream);
 int prefill_device_status(cudaStream_t stream);
 cudaError_t bounded_wait_selftest_launch(uint64_t limit_ns, cudaStream_t stream);
 
@@ -102,6 +106,31 @@ int kda_chunk_fwd_states(const void* q, const void* k, const void* v, const void
     if (n_snap > 0 && (states == nullptr || !aligned16(states))) return KDA_ERR_INVALID_ARG;
     return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, false,
                           n_snap > 0 ? states : nullptr, state_every, stream);
+}
+
+int kda_chunk_transition(const void* q, const void* k, const void* g, const void* beta, float* M,
+                         int B, int T, int H, int dk, kda_stream_t stream)
+{
+    // the checks of a prefill, with v and o absent and M in the place of hT
+    int st = check_prefill(q, k, q, g, beta, nullptr, q, M, B, T, H, dk, dk);
+    if (st != KDA_OK) return st;
+    if (dk != 128) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * H == 0) return KDA_OK;
+    if (!ptr_ok(M)) return KDA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(beta) & 1u) != 0) return KDA_ERR_INVALID_ARG;
+    return status_of(prefill_transition_launch(q, k, g, beta, M, B, T, H, (cudaStream_t)stream));
+}
+
+int kda_state_chain(const float* M, const float* N, const float* h0, float* S_start, float* hT,
+                    int B, int P, int H, int dk, int dv, kda_stream_t stream)
+{
+    if (B < 0 || P < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+    if (!(dk == 128 && dv == 128)) return KDA_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * P * H == 0) return KDA_OK;
+    if (!ptr_ok(M) || !ptr_ok(N) || !ptr_ok(S_start) || !opt_ptr_ok(h0) || !opt_ptr_ok(hT))
+        return KDA_ERR_INVALID_ARG;
+    return status_of(state_chain_launch(M, N, h0, S_start, hT, B, P, H, (cudaStream_t)stream));
 }
 
 int kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const void* g,

@@ -1553,6 +1553,55 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
     return e;
 }
 
+// Transition of each whole sequence: M = prod_t (I - b_t k_t k_t^T) Diag(exp g_t)
+// (d_k x d_k), as the state reached from S = I with v = 0 (each state column
+// evolves on its own).  M: [B][H][D][D].  v is not read (its map reuses q's).
+cudaError_t prefill_transition_launch(const void* q, const void* k, const void* g, const void* beta,
+                                      float* M, int B, int T, int H, cudaStream_t stream)
+{
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)pf::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)pc::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap mq, mk, mg;
+    if (T > 0) {
+        if (!make_map(&mq, q, B, T, H) || !make_map(&mk, k, B, T, H) || !make_map(&mg, g, B, T, H))
+            return cudaErrorInvalidValue;
+    } else {
+        memset(&mq, 0, sizeof(mq)); memset(&mk, 0, sizeof(mk)); memset(&mg, 0, sizeof(mg));
+    }
+    const cudaError_t e = launch_pass(mq, mk, mq, mg, beta, nullptr, nullptr, M, B, T, H, T, 1,
+                                      pf::SEG_V_ZERO | pf::SEG_H0_EYE | pf::SEG_NO_O,
+                                      cluster_fits((int64_t)B * H), nullptr, 0, stream);
+    note_launches(1);
+    return e;
+}
+
+// S_{p+1} = M_p S_p + N_p over P consecutive segments of each (b, h):
+// M, N, S_start: [B][P][H][D][D]; h0, hT: [B][H][D][D] (either may be null).
+cudaError_t state_chain_launch(const float* M, const float* N, const float* h0, float* S_start, float* hT,
+                               int B, int P, int H, cudaStream_t stream)
+{
+    static bool attr_set = false;
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(segment_combine_kernel,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)SEG_COMBINE_SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    segment_combine_kernel<<<dim3(pf::D / SEG_COLS, B * H), 256, SEG_COMBINE_SMEM, stream>>>(
+        M, N, S_start, h0, hT, H, P);
+    note_launches(1);
+    return cudaGetLastError();
+}
+
 // Self-test of the bounded waits: one warp waits on an mbarrier that nothing
 // completes, gives up after limit_ns and records KDA_ERR_TIMEOUT exactly as
 // the prefill kernel does.  No fault, trap or unbounded wait is involved.
