@@ -62,6 +62,15 @@ def decode_alg_bytes(N, H, dk, dv):
     return N * H * (2 * dk * dv * 4 + (3 * dk + dv + 1 + dv) * BYTES_BF16)
 
 
+def code_only(text):
+    """C/C++/CUDA source without comments and with whitespace collapsed: what
+    decides whether a kernel has changed since its counters were taken."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def measured_traffic(kernel, workload):
     """DRAM bytes per launch for this kernel on this workload from the
     committed ncu summary, or None when there is no such line or when the
@@ -78,8 +87,8 @@ def measured_traffic(kernel, workload):
                     continue
                 h = hashlib.sha256()
                 for rel in parts[1].split(","):        # every source the kernel is built from
-                    with open(os.path.join(ROOT, rel), "rb") as src:
-                        h.update(src.read())
+                    with open(os.path.join(ROOT, rel), encoding="utf-8") as src:
+                        h.update(code_only(src.read()).encode())
                 return int(parts[3]) if h.hexdigest()[:16] == parts[2] else None
     except Exception:
         return None

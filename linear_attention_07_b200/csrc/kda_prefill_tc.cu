@@ -20,25 +20,29 @@
 // turn; subtitles, cue 14).  The block between the two tiles of a chunk uses
 // the tile boundary as reference: Kb_tile0 (<= 1) against Kt_tile1 (<= 1).
 //
-// One CTA of 256 threads per (batch, head), d_k = d_v = 128, two roles:
-//   * chain warpgroup (warps 0-3): thread j owns column j of the fp32 state S
-//     in registers.  Per chunk: X = S^T [W | Qt]^T (tf32 copy of S^T in tensor
-//     memory as the A operand, M 128, N 64, K 128), U^T = U'^T - X_W into
-//     tensor memory, S^T += U^T Kb (N 128, K 32) and O^T += U^T P^T (N 32,
-//     K 32), then the decay/update of S and the bf16 store of o.
-//   * prep warpgroup (warps 4-7): for the next chunk, the decay scaling
-//     (two channels per thread), the Gram MMA Kh' [Kt | Qt]^T (M 64: rows
-//     Kh of both tiles and Kb of tile 0), the 32x32 unit-triangular solve
-//     (block-wise, all 128 threads), and W^T = Kt^T T^T, U'^T = V^T T^T
-//     (M 128, N 32, K 32).  It then fills the chain's operand buffers.
-// The two roles meet at two named-barrier rendezvous per chunk: "free" (the
-// chain no longer reads the operand buffers) and "ready" (the next chunk's
-// operands are in place).  Inputs of the next chunk are prefetched with
-// cp.async while the current one is processed.
-//
-// All MMAs are tf32 with operands rounded to nearest (cvt.rna): bf16
-// operands would leave errors of a few percent of rms(o) on these products
-// (the q.k diagonal times a large u), tf32 leaves ~0.3%.
+// Three launch paths over this arithmetic (d_k = d_v = 128):
+//   * prefill_tc_kernel, one SM per (batch, head), 512 threads in two roles:
+//     chain warps 0-7 (thread (j, half) owns column j, rows [64 half, +64) of
+//     the fp32 state S in registers; per chunk X = S^T [W | Qt]^T with the
+//     tf32 copy of S^T in tensor memory as the A operand (M 128, N 64, K 128),
+//     U^T = U'^T - X_W, S^T += U^T Kb (N 128, K 32), O^T += U^T P^T (N 32,
+//     K 32), the decay/update of S and the bf16 store of o) and prep warps
+//     8-15 (for the next chunk: TMA loads of q, k, v, g, the decay scaling,
+//     the Gram MMA, the 32 x 32 unit-triangular solve, W^T = Kt^T T^T and
+//     U'^T = V^T T^T (M 128, N 32, K 32), and the fill of the chain's
+//     operand buffers).  The roles meet at named-barrier rendezvous.
+//   * prefill_cluster_kernel, a cluster of four SMs per head when the heads
+//     alone would leave most SMs idle: one chain CTA, three preparing CTAs
+//     that push each prepared chunk into the chain CTA's shared memory over
+//     DSMEM (description above the kernel).
+//   * the segment scan for very few heads on long sequences: every sequence
+//     cut into segments run in parallel by either kernel, joined through
+//     their transitions (description above launch_segmented).
+// Every MMA is tf32 (kind::tf32) with fp32 accumulation, issued by a whole
+// converged warp with elect.sync.  Operands are rounded to tf32 once, to
+// nearest (ties away from zero), by an integer add-and-mask: bf16 operands
+// would leave errors of a few percent of rms(o) on these products (the q.k
+// diagonal times a large u); tf32 leaves a few tenths of a percent.
 // Shared-memory operands use the no-swizzle K-major layout; when the thread
 // that produces a value owns the K index, the K-direction core-matrix stride
 // is padded to 144 B so that a warp's scalar stores hit distinct banks.
@@ -665,7 +669,7 @@ static_assert(SLOT % 16 == 0, "bulk copy size");
 // rank 0 (chain): NPREPCTA slots
 constexpr uint32_t C_SLOT0 = 0;
 constexpr uint32_t C_BYTES = NPREPCTA * SLOT;
-// ranks 1, 2 (preparation)
+// ranks 1-3 (preparation)
 constexpr uint32_t P_RAW = 0;
 constexpr uint32_t P_BETA = P_RAW + 4 * RAW_T;
 constexpr uint32_t P_GEX = P_BETA + C * 4;
