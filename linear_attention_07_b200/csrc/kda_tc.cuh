@@ -60,28 +60,10 @@ __host__ __device__ constexpr uint32_t off_mnmajor(int mn, int k, uint32_t lbo, 
 
 // ------------------------------------------------------------------- MMA --
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]
-__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n"
-        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 
-// D[tmem] (+)= A[tmem] * B[smem desc]   (A is K-major: lane = row, column = k)
-__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n"
-        :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 
+// D[tmem] (+)= A[smem desc or tmem] * B[smem desc], and the commit that
+// arrives on an mbarrier once every MMA issued before it has completed.
 // Whole-warp forms: every lane of a converged warp calls them with the same
 // (warp-uniform) arguments and one elected lane issues.  Issuing from a
 // converged warp keeps the descriptors warp-uniform; a single-lane branch
@@ -114,11 +96,6 @@ __device__ __forceinline__ void mma_commit_w(uint32_t mbar_saddr) {
         :: "r"(mbar_saddr) : "memory");
 }
 
-// Arrive on an mbarrier once every previously issued MMA of this thread is done.
-__device__ __forceinline__ void mma_commit(uint32_t mbar_saddr) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 :: "r"(mbar_saddr) : "memory");
-}
 
 // ---------------------------------------------------------------- fences --
 
@@ -244,21 +221,12 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
 }
-// Arrive on an mbarrier of another CTA of the cluster (release, cluster scope).
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_saddr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
-                 :: "r"(cluster_saddr) : "memory");
-}
-// Relaxed form: signals an event that orders no data (for example "this
-// buffer may be overwritten" once every read of it has completed); much
-// cheaper than the release form.
+// Arrive on an mbarrier of another CTA of the cluster, relaxed: signals an
+// event that orders no data (for example "this buffer may be overwritten"
+// once every read of it has completed); much cheaper than a release arrive.
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_saddr) {
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];"
                  :: "r"(cluster_saddr) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t cluster_saddr, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
-                 :: "r"(cluster_saddr), "r"(bytes) : "memory");
 }
 // Cluster-scope acquiring wait (data written by other CTAs of the cluster).
 __device__ __forceinline__ uint32_t mbar_try_wait_cluster(uint32_t saddr, uint32_t parity) {
