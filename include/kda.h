@@ -93,6 +93,20 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
                   int B, int T, int H, int dk, int dv, kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_raw -- kda_chunk_fwd with the prologue fused in: q_raw and
+ * k_raw are NOT normalised and z is the gate pre-activation.  Inside the
+ * kernel, per token and head, q and k are L2-normalised over the dk channels
+ * (in fp32; a zero vector stays zero) and the log-decay is g = -5 sigmoid(z)
+ * (the lower-bounded sigmoid decay of the "Kimi K3 goes trillion-scale ..."
+ * subtitles, cue 14, with the transcript's -5 floor), so no separate pass
+ * writes normalised q, k or g.  Layouts, paths, results otherwise as
+ * kda_chunk_fwd (z in the place of g).
+ */
+int kda_chunk_fwd_raw(const void* q_raw, const void* k_raw, const void* v, const void* z,
+                      const void* beta, const float* h0, void* o, float* hT,
+                      int B, int T, int H, int dk, int dv, kda_stream_t stream);
+
+/*
  * kda_chunk_fwd_states -- kda_chunk_fwd that also writes intermediate states
  * (prefix-cache blocks): the fp32 state after every `state_every` tokens,
  *
@@ -187,6 +201,14 @@ int kda_chunk_fwd_f32(const float* q, const float* k, const float* v,
 int kda_decode_step(const void* q, const void* k, const void* v, const void* g,
                     const void* beta, float* state, void* o,
                     int N, int H, int dk, int dv, kda_stream_t stream);
+
+/*
+ * kda_decode_step_raw -- kda_decode_step with the same fused prologue as
+ * kda_chunk_fwd_raw (q_raw, k_raw unnormalised; z the gate pre-activation).
+ */
+int kda_decode_step_raw(const void* q_raw, const void* k_raw, const void* v, const void* z,
+                        const void* beta, float* state, void* o,
+                        int N, int H, int dk, int dv, kda_stream_t stream);
 
 /*
  * kda_device_status -- KDA_OK, or KDA_ERR_TIMEOUT if a kernel of this

@@ -29,7 +29,8 @@ KDA_ERR_TIMEOUT = -4
 KDA_ERR_NO_MEMORY = -5
 
 EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_states", "kda_chunk_fwd_f32",
-            "kda_chunk_transition", "kda_state_chain", "kda_decode_step",
+            "kda_chunk_transition", "kda_state_chain", "kda_chunk_fwd_raw", "kda_decode_step",
+            "kda_decode_step_raw",
             "kda_device_status", "kda_selftest_bounded_wait",
             "kda_status_string", "kda_launch_count", "kda_version")
 
@@ -75,6 +76,10 @@ def load_library(path: str = LIB_PATH):
     lib.kda_chunk_fwd_f32.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, vp, vp, fp, vp, i, i, i, i, vp]
     lib.kda_decode_step.restype = i
+    lib.kda_chunk_fwd_raw.argtypes = [vp, vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, vp]
+    lib.kda_chunk_fwd_raw.restype = i
+    lib.kda_decode_step_raw.argtypes = [vp, vp, vp, vp, vp, fp, vp, i, i, i, i, vp]
+    lib.kda_decode_step_raw.restype = i
     lib.kda_device_status.argtypes = [vp]
     lib.kda_device_status.restype = i
     lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
@@ -175,6 +180,14 @@ def chunk_fwd(q, k, v, g, beta, h0=None, *, o=None, hT=None, output_final_state=
                     hT, output_final_state)
 
 
+def chunk_fwd_raw(q_raw, k_raw, v, z, beta, h0=None, *, o=None, hT=None, output_final_state=True):
+    """chunk_fwd with the prologue fused in (kda_chunk_fwd_raw): q_raw, k_raw
+    unnormalised, z the gate pre-activation (g = -5 sigmoid(z) in the kernel)."""
+    import torch
+    return _prefill("kda_chunk_fwd_raw", torch.bfloat16, q_raw, k_raw, v, z, beta, h0, o,
+                    hT, output_final_state)
+
+
 def chunk_fwd_noalloc(q, k, v, g, beta, h0=None, *, o=None, hT=None, output_final_state=True):
     """chunk_fwd without any allocation in the library (kda_chunk_fwd_noalloc):
     the segment-scan path uses the library's fixed device scratch."""
@@ -262,10 +275,7 @@ def chunk_fwd_f32(q, k, v, g, beta, h0=None, *, o=None, hT=None, output_final_st
                     hT, output_final_state)
 
 
-def decode_step(q, k, v, g, beta, state, *, o=None):
-    """One decode token per request; `state` [N, H, dk, dv] fp32 is updated
-    in place.  q, k, g: [N, H, dk]; v: [N, H, dv]; beta: [N, H] (bf16).
-    Returns o [N, H, dv] bf16."""
+def _decode(fn_name, q, k, v, g, beta, state, o):
     import torch
     N, H, dk = q.shape
     dv = v.shape[-1]
@@ -280,8 +290,23 @@ def decode_step(q, k, v, g, beta, state, *, o=None):
     if o is None:
         o = torch.empty((N, H, dv), dtype=torch.bfloat16, device=dev)
     _check(o, "o", torch.bfloat16, (N, H, dv), dev)
-    st = load_library().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+    st = getattr(load_library(), fn_name)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
                                         _ptr(state), _ptr(o), N, H, dk, dv, _stream(dev))
     if st != KDA_OK:
-        raise KdaError("kda_decode_step", st)
+        raise KdaError(fn_name, st)
     return o
+
+
+def decode_step(q, k, v, g, beta, state, *, o=None):
+    """One decode token per request; `state` [N, H, dk, dv] fp32 is updated
+    in place.  q, k, g: [N, H, dk]; v: [N, H, dv]; beta: [N, H] (bf16).
+    Returns o [N, H, dv] bf16."""
+    return _decode("kda_decode_step", q, k, v, g, beta, state, o)
+
+
+def decode_step_raw(q_raw, k_raw, v, z, beta, state, *, o=None):
+    """decode_step with the prologue fused in (kda_decode_step_raw): q_raw,
+    k_raw unnormalised, z the gate pre-activation."""
+    return _decode("kda_decode_step_raw", q_raw, k_raw, v, z, beta, state, o)
+
+

@@ -11,13 +11,13 @@ void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_
 
 cudaError_t decode_step_launch(const void* q, const void* k, const void* v,
                                const void* g, const void* beta, float* state,
-                               void* o, int64_t NH, int dk, int dv,
+                               void* o, int64_t NH, int dk, int dv, bool raw,
                                cudaStream_t stream);
 
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, const float* h0, void* o, float* hT,
                               int B, int T, int H, bool no_alloc, float* states, int snap_every,
-                              cudaStream_t stream);
+                              bool prologue, cudaStream_t stream);
 cudaError_t prefill_transition_launch(const void* q, const void* k, const void* g, const void* beta,
                                       float* M, int B, int T, int H, cudaStream_t stream);
 cudaError_t state_chain_launch(const float* M, const float* N, const float* h0, float* S_start, float* hT,
@@ -77,7 +77,7 @@ extern "C" {
 static int chunk_fwd_bf16(const void* q, const void* k, const void* v, const void* g,
                           const void* beta, const float* h0, void* o, float* hT,
                           int B, int T, int H, int dk, int dv, bool no_alloc,
-                          float* states, int state_every, kda_stream_t stream)
+                          float* states, int state_every, bool raw, kda_stream_t stream)
 {
     int st = check_prefill(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv);
     if (st != KDA_OK) return st;
@@ -86,14 +86,21 @@ static int chunk_fwd_bf16(const void* q, const void* k, const void* v, const voi
     if ((int64_t)B * H == 0) return KDA_OK;
     if (T == 0 && hT == nullptr) return KDA_OK;
     return status_of(prefill_tc_launch(q, k, v, g, beta, h0, o, hT, B, T, H, no_alloc,
-                                       states, state_every / 32, (cudaStream_t)stream));
+                                       states, state_every / 32, raw, (cudaStream_t)stream));
 }
 
 int kda_chunk_fwd(const void* q, const void* k, const void* v, const void* g,
                   const void* beta, const float* h0, void* o, float* hT,
                   int B, int T, int H, int dk, int dv, kda_stream_t stream)
 {
-    return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, false, nullptr, 0, stream);
+    return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, false, nullptr, 0, false, stream);
+}
+
+int kda_chunk_fwd_raw(const void* q_raw, const void* k_raw, const void* v, const void* z,
+                      const void* beta, const float* h0, void* o, float* hT,
+                      int B, int T, int H, int dk, int dv, kda_stream_t stream)
+{
+    return chunk_fwd_bf16(q_raw, k_raw, v, z, beta, h0, o, hT, B, T, H, dk, dv, false, nullptr, 0, true, stream);
 }
 
 int kda_chunk_fwd_states(const void* q, const void* k, const void* v, const void* g,
@@ -105,7 +112,7 @@ int kda_chunk_fwd_states(const void* q, const void* k, const void* v, const void
     const int64_t n_snap = T > 0 ? T / state_every : 0;
     if (n_snap > 0 && (states == nullptr || !aligned16(states))) return KDA_ERR_INVALID_ARG;
     return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, false,
-                          n_snap > 0 ? states : nullptr, state_every, stream);
+                          n_snap > 0 ? states : nullptr, state_every, false, stream);
 }
 
 int kda_chunk_transition(const void* q, const void* k, const void* g, const void* beta, float* M,
@@ -137,7 +144,7 @@ int kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const voi
                           const void* beta, const float* h0, void* o, float* hT,
                           int B, int T, int H, int dk, int dv, kda_stream_t stream)
 {
-    return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, true, nullptr, 0, stream);
+    return chunk_fwd_bf16(q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, true, nullptr, 0, false, stream);
 }
 
 int kda_chunk_fwd_f32(const float* q, const float* k, const float* v,
@@ -155,9 +162,9 @@ int kda_chunk_fwd_f32(const float* q, const float* k, const float* v,
         q, k, v, g, beta, h0, o, hT, B, T, H, dk, dv, (cudaStream_t)stream));
 }
 
-int kda_decode_step(const void* q, const void* k, const void* v, const void* g,
-                    const void* beta, float* state, void* o,
-                    int N, int H, int dk, int dv, kda_stream_t stream)
+static int decode_step_any(const void* q, const void* k, const void* v, const void* g,
+                           const void* beta, float* state, void* o,
+                           int N, int H, int dk, int dv, bool raw, kda_stream_t stream)
 {
     if (N < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
@@ -167,8 +174,22 @@ int kda_decode_step(const void* q, const void* k, const void* v, const void* g,
     if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) || !ptr_ok(state) || !ptr_ok(o))
         return KDA_ERR_INVALID_ARG;
     if (beta == nullptr || (reinterpret_cast<uintptr_t>(beta) & 1u) != 0) return KDA_ERR_INVALID_ARG;
-    return status_of(decode_step_launch(q, k, v, g, beta, state, o, NH, dk, dv,
+    return status_of(decode_step_launch(q, k, v, g, beta, state, o, NH, dk, dv, raw,
                                         (cudaStream_t)stream));
+}
+
+int kda_decode_step(const void* q, const void* k, const void* v, const void* g,
+                    const void* beta, float* state, void* o,
+                    int N, int H, int dk, int dv, kda_stream_t stream)
+{
+    return decode_step_any(q, k, v, g, beta, state, o, N, H, dk, dv, false, stream);
+}
+
+int kda_decode_step_raw(const void* q_raw, const void* k_raw, const void* v, const void* z,
+                        const void* beta, float* state, void* o,
+                        int N, int H, int dk, int dv, kda_stream_t stream)
+{
+    return decode_step_any(q_raw, k_raw, v, z, beta, state, o, N, H, dk, dv, true, stream);
 }
 
 const char* kda_status_string(int status)

@@ -15,13 +15,17 @@
 // vector access.  All ROWS loads are issued before any arithmetic so that
 // each thread has ROWS x 16 bytes in flight.  The two column reductions over
 // d_k (p and r) go through one shared-memory pass.
+//
+// RAW (the fused prologue): q and k arrive unnormalised and g holds the gate
+// pre-activation z; the step L2-normalises q and k (a zero vector stays
+// zero) and takes g = -5 sigmoid(z) before the recurrence.
 #include "kda_common.cuh"
 
 namespace kda {
 
 constexpr int kDecodeThreads = 256;
 
-template <int DK, int DV>
+template <int DK, int DV, bool RAW>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_step_kernel(const __nv_bfloat16* __restrict__ q,
                    const __nv_bfloat16* __restrict__ k,
@@ -38,6 +42,7 @@ decode_step_kernel(const __nv_bfloat16* __restrict__ q,
 
     __shared__ float s_a[DK], s_k[DK], s_q[DK];
     __shared__ float s_qk;
+    __shared__ float s_inv[2];                  // RAW: 1 / |q|, 1 / |k|
     __shared__ float4 s_red[2][RSTEP][CG];
 
     const int64_t nh = blockIdx.x;              // request * H + head
@@ -52,9 +57,34 @@ decode_step_kernel(const __nv_bfloat16* __restrict__ q,
 
     // small per-head vectors
     for (int i = tid; i < DK; i += kDecodeThreads) {
-        s_a[i] = expf(to_f32(g[nh * DK + i]));
+        const float gi = to_f32(g[nh * DK + i]);
+        s_a[i] = expf(RAW ? -5.f / (1.f + expf(-gi)) : gi);
         s_k[i] = to_f32(k[nh * DK + i]);
         s_q[i] = to_f32(q[nh * DK + i]);
+    }
+    if constexpr (RAW) {
+        __syncthreads();
+        if (tid < 32) {
+            float nq = 0.f, nk = 0.f;
+            for (int i = tid; i < DK; i += 32) {
+                nq = fmaf(s_q[i], s_q[i], nq);
+                nk = fmaf(s_k[i], s_k[i], nk);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                nq += __shfl_xor_sync(0xffffffffu, nq, off);
+                nk += __shfl_xor_sync(0xffffffffu, nk, off);
+            }
+            if (tid == 0) {
+                s_inv[0] = nq > 0.f ? rsqrtf(nq) : 0.f;
+                s_inv[1] = nk > 0.f ? rsqrtf(nk) : 0.f;
+            }
+        }
+        __syncthreads();
+        for (int i = tid; i < DK; i += kDecodeThreads) {
+            s_q[i] *= s_inv[0];
+            s_k[i] *= s_inv[1];
+        }
     }
     const float b = to_f32(beta[nh]);
     const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(v + nh * DV + 4 * cg);
@@ -112,12 +142,12 @@ decode_step_kernel(const __nv_bfloat16* __restrict__ q,
     }
 }
 
-template <int DK, int DV>
+template <int DK, int DV, bool RAW>
 static cudaError_t launch_decode(const void* q, const void* k, const void* v,
                                  const void* g, const void* beta, float* state,
                                  void* o, int64_t NH, cudaStream_t stream)
 {
-    decode_step_kernel<DK, DV><<<(unsigned)NH, kDecodeThreads, 0, stream>>>(
+    decode_step_kernel<DK, DV, RAW><<<(unsigned)NH, kDecodeThreads, 0, stream>>>(
         (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
         (const __nv_bfloat16*)g, (const __nv_bfloat16*)beta, state, (__nv_bfloat16*)o);
     note_launches(1);
@@ -126,11 +156,13 @@ static cudaError_t launch_decode(const void* q, const void* k, const void* v,
 
 cudaError_t decode_step_launch(const void* q, const void* k, const void* v,
                                const void* g, const void* beta, float* state,
-                               void* o, int64_t NH, int dk, int dv,
+                               void* o, int64_t NH, int dk, int dv, bool raw,
                                cudaStream_t stream)
 {
 #define KDA_DEC(DK_, DV_) \
-    if (dk == DK_ && dv == DV_) return launch_decode<DK_, DV_>(q, k, v, g, beta, state, o, NH, stream);
+    if (dk == DK_ && dv == DV_) \
+        return raw ? launch_decode<DK_, DV_, true>(q, k, v, g, beta, state, o, NH, stream) \
+                   : launch_decode<DK_, DV_, false>(q, k, v, g, beta, state, o, NH, stream);
     KDA_DEC(32, 32) KDA_DEC(32, 64) KDA_DEC(32, 128)
     KDA_DEC(64, 32) KDA_DEC(64, 64) KDA_DEC(64, 128)
     KDA_DEC(128, 32) KDA_DEC(128, 64) KDA_DEC(128, 128)

@@ -92,7 +92,9 @@ constexpr uint32_t XMS = PMS + C * LD * 4;                     // diagonal-block
 constexpr uint32_t TMS = XMS + C * LD * 4;                     // T
 constexpr uint32_t YMS = TMS + C * LD * 4;                     // A_10 X_00 (16 x 17)
 constexpr uint32_t OST = YMS + TILE * (TILE + 1) * 4;           // o staging, 32 x 128 bf16
-constexpr uint32_t SMEM_BYTES = OST + C * D * 2;
+constexpr uint32_t NRM = OST + C * D * 2;                      // prologue: per-warp squared norms
+constexpr uint32_t NRM_BYTES = 2 * 4 * 2 * TILE * 4;           // [tile][warp][q, k][token]
+constexpr uint32_t SMEM_BYTES = NRM + NRM_BYTES;
 
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(OST % 16 == 0 && GA % 16 == 0 && GB % 16 == 0 && WA % 16 == 0 && VA % 16 == 0 && TB % 16 == 0 &&
@@ -116,6 +118,10 @@ constexpr uint64_t WAIT_NS = 2000000000ull;   // bounded waits: 2 s
 // Launch flags (segment scan passes): treat v as zero, start from h0 = I
 // (ignore h0), skip the o stores.
 constexpr uint32_t SEG_V_ZERO = 1u, SEG_H0_EYE = 2u, SEG_NO_O = 4u;
+// Fused prologue: q, k arrive unnormalised and the g tensor holds the gate
+// pre-activation z; the kernel L2-normalises q and k per token and head (a
+// zero vector stays zero) and takes g = -5 sigmoid(z) (g = 0 past the end).
+constexpr uint32_t PROLOGUE = 8u;
 
 }  // namespace pf
 
@@ -152,12 +158,65 @@ __device__ __forceinline__ float* snapshot_slot(float* states, int snap_every, i
     return states + (((int64_t)b * H + h) * n_snap + s) * pf::D * pf::D;
 }
 
+// Prologue, part 1 (before the exponentials): a[] holds z and becomes
+// g = -5 sigmoid(z) (0 for tokens t0 + rr >= Tl, which leaves the state
+// alone); each warp writes the squared norms of q and k over its 32 channels
+// for the 16 tokens of its tile to nrm[tile][warp][q, k][token].
+__device__ __forceinline__ void prologue_gate_and_norms(float (&a)[pf::TILE], const float (&qr)[pf::TILE],
+                                                        const float (&kr)[pf::TILE], int t0, int Tl,
+                                                        float* nrm, int tau, int c)
+{
+    constexpr int TILE = pf::TILE;
+    float nq[TILE], nk[TILE];
+#pragma unroll
+    for (int rr = 0; rr < TILE; ++rr) {
+        a[rr] = (t0 + rr < Tl) ? -5.f / (1.f + __expf(-a[rr])) : 0.f;
+        nq[rr] = qr[rr] * qr[rr];
+        nk[rr] = kr[rr] * kr[rr];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int rr = 0; rr < TILE; ++rr) {
+            nq[rr] += __shfl_xor_sync(0xffffffffu, nq[rr], off);
+            nk[rr] += __shfl_xor_sync(0xffffffffu, nk[rr], off);
+        }
+    if ((c & 31) == 0) {
+        float* w = nrm + ((tau * 4 + (c >> 5)) * 2) * TILE;
+#pragma unroll
+        for (int rr = 0; rr < TILE; ++rr) {
+            w[rr] = nq[rr];
+            w[TILE + rr] = nk[rr];
+        }
+    }
+}
+
+// Prologue, part 2 (after a barrier): q, k of this thread's 16 tokens scaled
+// to unit norm over the 128 channels (zero vectors stay zero).
+__device__ __forceinline__ void prologue_normalise(float (&qr)[pf::TILE], float (&kr)[pf::TILE],
+                                                   const float* nrm, int tau)
+{
+    constexpr int TILE = pf::TILE;
+#pragma unroll
+    for (int rr = 0; rr < TILE; ++rr) {
+        float sq = 0.f, sk = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            sq += nrm[((tau * 4 + w) * 2) * TILE + rr];
+            sk += nrm[((tau * 4 + w) * 2) * TILE + TILE + rr];
+        }
+        qr[rr] *= sq > 0.f ? rsqrtf(sq) : 0.f;
+        kr[rr] *= sk > 0.f ? rsqrtf(sk) : 0.f;
+    }
+}
+
 // A shared flag read once by lane 0 and broadcast: the same value in every
 // lane, so a whole-warp MMA issue never diverges on it.
 __device__ __forceinline__ bool warp_flag(const int& flag) {
     return __shfl_sync(0xffffffffu, *(const volatile int*)&flag, 0) != 0;
 }
 
+template <bool PRO>       // PRO: the fused prologue (launch flag PROLOGUE)
 __global__ void __launch_bounds__(pf::NT, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -414,6 +473,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     vr[rr] = (flags & SEG_V_ZERO) ? 0.f : to_f32(rv[idx]);
                     a[rr] = to_f32(rg[idx]);
                 }
+                if constexpr (PRO) prologue_gate_and_norms(a, qr, kr, ch * C + tau * TILE, Tl,
+                                                            reinterpret_cast<float*>(sm + NRM), tau, c);
                 float e = 1.f;
 #pragma unroll
                 for (int rr = 0; rr < TILE; ++rr) {
@@ -423,6 +484,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 float* gex = reinterpret_cast<float*>(sm + GEX);
                 gex[tau * D + c] = e;
                 prep_sync();
+                if constexpr (PRO) prologue_normalise(qr, kr, reinterpret_cast<const float*>(sm + NRM), tau);
                 const float oe = gex[(1 - tau) * D + c];
                 const float f = tau ? oe : 1.f;          // chunk-relative factor of tile 1 rows
                 gam_c = e * oe;
@@ -684,7 +746,8 @@ constexpr uint32_t P_PMS = P_AMS + C * LD * 4;
 constexpr uint32_t P_XMS = P_PMS + C * LD * 4;
 constexpr uint32_t P_TMS = P_XMS + C * LD * 4;
 constexpr uint32_t P_YMS = P_TMS + C * LD * 4;
-constexpr uint32_t P_BYTES = P_YMS + TILE * (TILE + 1) * 4;
+constexpr uint32_t P_NRM = P_YMS + TILE * (TILE + 1) * 4;    // prologue: per-warp squared norms
+constexpr uint32_t P_BYTES = P_NRM + NRM_BYTES;
 constexpr uint32_t SMEM_BYTES = P_BYTES > C_BYTES ? P_BYTES : C_BYTES;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(P_ST % 16 == 0 && P_GA % 16 == 0 && P_GB % 16 == 0 && P_WA % 16 == 0 && P_VA % 16 == 0 &&
@@ -694,6 +757,7 @@ constexpr uint32_t CT_AS = 0, CT_AU = 128, CT_DX0 = 160, CT_DKU = 224, CT_DX1 = 
 constexpr uint32_t PT_DG = 0, PT_DW = 64, PT_DU = 96;
 }  // namespace pc
 
+template <bool PRO>       // PRO: the fused prologue (launch flag PROLOGUE)
 __global__ void __cluster_dims__(pc::NPREPCTA + 1, 1, 1) __launch_bounds__(pc::NTH, 1)
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -1107,6 +1171,8 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     vr[rr] = (flags & SEG_V_ZERO) ? 0.f : to_f32(rv[idx]);
                     a[rr] = to_f32(rg[idx]);
                 }
+                if constexpr (PRO) prologue_gate_and_norms(a, qr, kr, ch * C + tau * TILE, Tl,
+                                                            reinterpret_cast<float*>(sm + P_NRM), tau, c);
                 float e = 1.f;
 #pragma unroll
                 for (int rr = 0; rr < TILE; ++rr) {
@@ -1116,6 +1182,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 float* gex = reinterpret_cast<float*>(sm + P_GEX);
                 gex[tau * D + c] = e;
                 prep_sync();
+                if constexpr (PRO) prologue_normalise(qr, kr, reinterpret_cast<const float*>(sm + P_NRM), tau);
                 const float oe = gex[(1 - tau) * D + c];
                 const float f = tau ? oe : 1.f;
                 gam_c = e * oe;
@@ -1310,6 +1377,17 @@ static bool make_map(CUtensorMap* map, const void* base, int B, int T, int H)
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Dynamic shared memory of both kernels in both instantiations.
+static cudaError_t set_prefill_attributes()
+{
+    const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<false>, a, (int)pf::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_tc_kernel<true>, a, (int)pf::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_cluster_kernel<false>, a, (int)pc::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_cluster_kernel<true>, a, (int)pc::SMEM_BYTES);
+    return e;
+}
+
 // Four SMs per head pay off while the heads alone leave most SMs idle:
 // up to 37 heads (148 SMs); larger batches use one SM per head.
 static bool cluster_fits(int64_t heads) { return heads * (pc::NPREPCTA + 1) <= 148; }
@@ -1321,14 +1399,17 @@ static cudaError_t launch_pass(const CUtensorMap& mq, const CUtensorMap& mk, con
                                int B, int T, int H, int seg_len, int n_seg, uint32_t flags, bool cluster,
                                float* states, int snap_every, cudaStream_t stream)
 {
+    const bool pro = (flags & pf::PROLOGUE) != 0;
     if (cluster) {
         dim3 grid((pc::NPREPCTA + 1) * H, B * n_seg);
-        prefill_cluster_kernel<<<grid, pc::NTH, pc::SMEM_BYTES, stream>>>(
+        auto kern = pro ? prefill_cluster_kernel<true> : prefill_cluster_kernel<false>;
+        kern<<<grid, pc::NTH, pc::SMEM_BYTES, stream>>>(
             mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags,
             states, snap_every);
     } else {
         dim3 grid(H, B * n_seg);
-        prefill_tc_kernel<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(
+        auto kern = pro ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
+        kern<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(
             mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags,
             states, snap_every);
     }
@@ -1467,7 +1548,7 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH
 static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                     const CUtensorMap& mg, const void* beta, const float* h0, void* o,
                                     float* hT, int B, int T, int H, bool no_alloc, float* states,
-                                    int snap_every, cudaStream_t stream)
+                                    int snap_every, uint32_t base_flags, cudaStream_t stream)
 {
     int seg_len = 0, n_seg = 0;
     segment_plan(B, T, H, &seg_len, &n_seg);
@@ -1500,18 +1581,18 @@ static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk
     float* Nw = ws + n_state;
     float* Sw = ws + 2 * n_state;
     const bool cl = cluster_fits((int64_t)B * n_seg * H);
-    e = launch_pass(mq, mk, mv, mg, beta, nullptr, o, Nw, B, T, H, seg_len, n_seg, pf::SEG_NO_O, cl,
+    e = launch_pass(mq, mk, mv, mg, beta, nullptr, o, Nw, B, T, H, seg_len, n_seg, base_flags | pf::SEG_NO_O, cl,
                     nullptr, 0, stream);
     if (e == cudaSuccess)
         e = launch_pass(mq, mk, mv, mg, beta, nullptr, o, Mw, B, T, H, seg_len, n_seg,
-                        pf::SEG_V_ZERO | pf::SEG_H0_EYE | pf::SEG_NO_O, cl, nullptr, 0, stream);
+                        base_flags | pf::SEG_V_ZERO | pf::SEG_H0_EYE | pf::SEG_NO_O, cl, nullptr, 0, stream);
     if (e == cudaSuccess) {
         segment_combine_kernel<<<dim3(pf::D / SEG_COLS, B * H), 256, SEG_COMBINE_SMEM, stream>>>(
             Mw, Nw, Sw, h0, hT, H, n_seg);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess)
-        e = launch_pass(mq, mk, mv, mg, beta, Sw, o, nullptr, B, T, H, seg_len, n_seg, 0u, cl,
+        e = launch_pass(mq, mk, mv, mg, beta, Sw, o, nullptr, B, T, H, seg_len, n_seg, base_flags, cl,
                         states, snap_every, stream);
     if (!no_alloc) {
         const cudaError_t ef = cudaFreeAsync(ws, stream);
@@ -1524,15 +1605,12 @@ static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, const float* h0, void* o, float* hT,
                               int B, int T, int H, bool no_alloc, float* states, int snap_every,
-                              cudaStream_t stream)
+                              bool prologue, cudaStream_t stream)
 {
+    const uint32_t flags = prologue ? pf::PROLOGUE : 0u;
     static bool attr_set = false;   // idempotent; races only repeat the same calls
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)pf::SMEM_BYTES);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(prefill_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)pc::SMEM_BYTES);
+        cudaError_t e = set_prefill_attributes();
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)SEG_COMBINE_SMEM);
@@ -1550,8 +1628,9 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
     }
     const PrefillPath path = choose_path(B, T, H);
     if (path == PrefillPath::Segmented)
-        return launch_segmented(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, no_alloc, states, snap_every, stream);
-    const cudaError_t e = launch_pass(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, T, 1, 0u,
+        return launch_segmented(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, no_alloc, states, snap_every,
+                                flags, stream);
+    const cudaError_t e = launch_pass(mq, mk, mv, mg, beta, h0, o, hT, B, T, H, T, 1, flags,
                                       path == PrefillPath::Cluster, states, snap_every, stream);
     note_launches(1);
     return e;
@@ -1565,11 +1644,7 @@ cudaError_t prefill_transition_launch(const void* q, const void* k, const void* 
 {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)pf::SMEM_BYTES);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(prefill_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)pc::SMEM_BYTES);
+        cudaError_t e = set_prefill_attributes();
         if (e != cudaSuccess) return e;
         attr_set = true;
     }

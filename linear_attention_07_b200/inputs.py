@@ -115,6 +115,27 @@ def prefill_inputs(B: int, T: int, H: int, dk: int, dv: int, *, seed: int,
     return dict(q=q, k=k, v=v, g=g, beta=beta, h0=h0)
 
 
+def raw_inputs(shape_qk, shape_v, shape_beta, *, seed: int, device="cpu", zero_rows: int = 0):
+    """Inputs for the fused prologue: q and k as drawn (N(0, 1), not
+    normalised), the gate pre-activation z ~ N(0, 1) (the gate is
+    g = -5 sigmoid(z)), v ~ N(0, 1) and beta = sigmoid(N(0, 1)), all bf16.
+    q, k, z: shape_qk; v: shape_v; beta: shape_beta.  The first `zero_rows`
+    entries along the second axis of q and k are zero vectors (the degenerate
+    case of the normalisation)."""
+    gen = torch.Generator(device=device).manual_seed(int(seed))
+    f32 = dict(generator=gen, device=device, dtype=torch.float32)
+    q = torch.randn(shape_qk, **f32)
+    k = torch.randn(shape_qk, **f32)
+    if zero_rows > 0:
+        q[:, :zero_rows] = 0.0
+        k[:, :zero_rows] = 0.0
+    z = torch.randn(shape_qk, **f32)
+    v = torch.randn(shape_v, **f32)
+    beta = torch.sigmoid(torch.randn(shape_beta, **f32))
+    bf = lambda t: t.to(torch.bfloat16)
+    return dict(q=bf(q), k=bf(k), z=bf(z), v=bf(v), beta=bf(beta))
+
+
 def decode_inputs(N: int, H: int, dk: int, dv: int, steps: int, *, seed: int,
                   dtype: torch.dtype = torch.bfloat16, device="cpu",
                   state_std: float = 0.1):

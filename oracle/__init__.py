@@ -168,3 +168,33 @@ def fwd(*a, **kw):
 
 def decode_step(*a, **kw):
     return default().decode_step(*a, **kw)
+
+
+def prologue(q_raw, k_raw, z):
+    """The fused prologue by its definition, in fp64: q and k L2-normalised
+    over the key channels for every (token, head) (a zero vector stays zero),
+    and the log-decay g = -5 sigmoid(z) (the lower-bounded sigmoid decay of
+    the "Kimi K3 goes trillion-scale ..." subtitles, cue 14, with the -5 floor
+    of the "T11E1: K3 tech report" transcript).  Returns (q, k, g) in fp64.
+    """
+    q, k, z = map(_f64, (q_raw, k_raw, z))
+
+    def unit(x):
+        n = np.sqrt((x * x).sum(axis=-1, keepdims=True))
+        return np.where(n > 0.0, x / np.where(n > 0.0, n, 1.0), 0.0)
+
+    with np.errstate(over="ignore"):
+        g = -5.0 / (1.0 + np.exp(-z))
+    return unit(q), unit(k), g
+
+
+def fwd_raw(q_raw, k_raw, v, z, beta, h0=None, **kw):
+    """fwd after the prologue: raw q, k and gate pre-activation z."""
+    q, k, g = prologue(q_raw, k_raw, z)
+    return fwd(q, k, v, g, beta, h0, **kw)
+
+
+def decode_step_raw(q_raw, k_raw, v, z, beta, state, **kw):
+    """decode_step after the prologue."""
+    q, k, g = prologue(q_raw, k_raw, z)
+    return decode_step(q, k, v, g, beta, state, **kw)

@@ -243,6 +243,51 @@ def test_bf16_intermediate_states_chosen_segment_scan():
     assert torch.equal(st[:, :, -1], hT)
 
 
+# ------------------------------------------------------- fused prologue ---
+
+def _raw_prefill(B, T, H, seed, zero_rows=2):
+    from linear_attention_07_b200.inputs import raw_inputs
+    x = raw_inputs((B, T, H, 128), (B, T, H, 128), (B, T, H), seed=seed, zero_rows=zero_rows)
+    gen = torch.Generator().manual_seed(seed + 1)
+    x["h0"] = torch.randn((B, H, 128, 128), generator=gen) * 0.1
+    return x
+
+
+@pytest.mark.parametrize("variant,B,H,T", [("fused", 2, 3, 1000), ("fused", 1, 2, 77), ("cluster", 2, 3, 1000),
+                                           ("cluster", 1, 2, 77), ("segmented", 1, 2, 2100)])
+def test_bf16_fused_prologue(monkeypatch, variant, B, H, T):
+    """kda_chunk_fwd_raw (q, k normalised and g = -5 sigmoid(z) in the
+    kernel) against the oracle's prologue + recurrence, with zero q/k
+    vectors and ragged tails (g stays 0 past the end)."""
+    monkeypatch.setenv("KDA_PREFILL_VARIANT", variant)
+    x = _raw_prefill(B, T, H, seed=1800 + T + H)
+    d = to_dev(x)
+    o, hT = kda.chunk_fwd_raw(d["q"], d["k"], d["v"], d["z"], d["beta"], d["h0"])
+    torch.cuda.synchronize()
+    assert kda.device_status() == kda.KDA_OK
+    o_ref, hT_ref = oracle.fwd_raw(x["q"], x["k"], x["v"], x["z"], x["beta"], x["h0"])
+    eo, eh = err_out(o, o_ref), err_state(hT, hT_ref)
+    assert eo <= TOL_BF16 and eh <= TOL_BF16, f"err_o={eo:.3e} err_hT={eh:.3e}"
+
+
+def test_bf16_fused_prologue_decode():
+    """kda_decode_step_raw over 6 steps (state in place) against the oracle."""
+    from linear_attention_07_b200.inputs import raw_inputs
+    N, H, steps = 5, 3, 6
+    x = raw_inputs((steps, N, H, 128), (steps, N, H, 128), (steps, N, H), seed=1900, zero_rows=1)
+    gen = torch.Generator().manual_seed(1901)
+    state0 = torch.randn((N, H, 128, 128), generator=gen) * 0.1
+    S = state0.to(DEV)
+    S_ref = state0.double().numpy()
+    for t in range(steps):
+        o = kda.decode_step_raw(x["q"][t].to(DEV), x["k"][t].to(DEV), x["v"][t].to(DEV), x["z"][t].to(DEV),
+                                x["beta"][t].to(DEV), S)
+        o_ref, S_ref = oracle.decode_step_raw(x["q"][t], x["k"][t], x["v"][t], x["z"][t], x["beta"][t], S_ref)
+        torch.cuda.synchronize()
+        assert err_out(o, o_ref) <= TOL_BF16
+    assert err_state(S, S_ref) <= TOL_BF16
+
+
 # ------------------------------------------------------- full workloads ---
 
 def _sampled_heads_check(w, d, o, hT, heads):
