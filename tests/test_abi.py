@@ -98,6 +98,40 @@ def test_states_argument_errors(lib):
     assert lib.kda_launch_count() == n0
 
 
+def test_raw_entry_points_argument_errors(lib):
+    """The fused-prologue entry points check their arguments like the plain
+    ones; nothing is launched."""
+    n0 = lib.kda_launch_count()
+    assert prefill(lib, "kda_chunk_fwd_raw", q=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert prefill(lib, "kda_chunk_fwd_raw", g=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert prefill(lib, "kda_chunk_fwd_raw", dk=64, dv=64) == kda.KDA_ERR_UNSUPPORTED
+    assert prefill(lib, "kda_chunk_fwd_raw", B=0) == kda.KDA_OK
+    dec = lib.kda_decode_step_raw
+    assert dec(A, A, A, A, A2, A, A, 4, 2, 96, 128, None) == kda.KDA_ERR_UNSUPPORTED
+    assert dec(A, A, A, NUL, A2, A, A, 4, 2, 128, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert dec(A, A, A, A, A2, A, A, 0, 2, 128, 128, None) == kda.KDA_OK
+    assert lib.kda_launch_count() == n0
+
+
+def test_joining_entry_points_argument_errors(lib):
+    """kda_chunk_transition and kda_state_chain: host checks, no launch."""
+    n0 = lib.kda_launch_count()
+    tr = lib.kda_chunk_transition
+    assert tr(A, A, A, A2, NUL, 1, 16, 2, 128, None) == kda.KDA_ERR_INVALID_ARG     # no M
+    assert tr(A, A, A, A2, MIS, 1, 16, 2, 128, None) == kda.KDA_ERR_INVALID_ARG     # misaligned M
+    assert tr(NUL, A, A, A2, A, 1, 16, 2, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert tr(A, A, A, A2, A, 1, 16, 2, 64, None) == kda.KDA_ERR_UNSUPPORTED
+    assert tr(A, A, A, A2, A, 0, 16, 2, 128, None) == kda.KDA_OK                    # nothing to do
+    ch = lib.kda_state_chain
+    assert ch(NUL, A, NUL, A, NUL, 1, 3, 2, 128, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert ch(A, A, NUL, MIS, NUL, 1, 3, 2, 128, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert ch(A, A, MIS, A, NUL, 1, 3, 2, 128, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert ch(A, A, NUL, A, NUL, 1, 3, 2, 64, 64, None) == kda.KDA_ERR_UNSUPPORTED
+    assert ch(A, A, NUL, A, NUL, 1, -1, 2, 128, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert ch(NUL, NUL, NUL, NUL, NUL, 1, 0, 2, 128, 128, None) == kda.KDA_OK      # no segments
+    assert lib.kda_launch_count() == n0
+
+
 def test_bf16_prefill_shape_support(lib):
     # the tensor-core path is specialised to d_k = d_v = 128
     assert prefill(lib, "kda_chunk_fwd", dk=64, dv=64) == kda.KDA_ERR_UNSUPPORTED
