@@ -53,7 +53,7 @@ class OracleOps:
         return S_start, S
 
 
-def _cpu_worker(rank, world, port, seed, errs):
+def _cpu_worker(rank, world, port, seed, errs, cuts=None, with_h0=True):
     import torch.distributed as dist
     from linear_attention_07_b200.context_parallel import chunk_fwd_context_parallel
     os.environ["MASTER_ADDR"] = "127.0.0.1"
@@ -61,34 +61,48 @@ def _cpu_worker(rank, world, port, seed, errs):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         B, T, H, d = 2, 96, 2, 16
-        x = prefill_inputs(B, T, H, d, d, seed=seed, h0_std=0.1)
-        L = T // world
-        blk = {n: x[n][:, rank * L:(rank + 1) * L].contiguous() for n in ("q", "k", "v", "g", "beta")}
-        h0 = x["h0"].double()
+        x = prefill_inputs(B, T, H, d, d, seed=seed, h0_std=0.1 if with_h0 else 0.0)
+        cuts = cuts or [T * r // world for r in range(world + 1)]
+        lo, hi = cuts[rank], cuts[rank + 1]
+        blk = {n: x[n][:, lo:hi].contiguous() for n in ("q", "k", "v", "g", "beta")}
+        h0 = None if x["h0"] is None else x["h0"].double()
         o, hT = chunk_fwd_context_parallel(blk["q"], blk["k"], blk["v"], blk["g"], blk["beta"], h0,
                                            ops=OracleOps)
         o_ref, hT_ref = oracle.fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"])
-        eo = float(np.abs(o.numpy() - o_ref[:, rank * L:(rank + 1) * L]).max())
+        eo = float(np.abs(o.numpy() - o_ref[:, lo:hi]).max())
         eh = float(np.abs(hT.numpy() - hT_ref).max())
         errs[rank] = max(eo, eh)
     finally:
         dist.destroy_process_group()
 
 
-def test_context_parallel_orchestration_gloo():
-    """Two ranks, one sequence: each rank's o and the final state equal the
-    whole-sequence oracle (fp64 throughout, so to rounding)."""
+def _run_ranks(world, seed, cuts=None, with_h0=True):
     ctx = mp.get_context("spawn")
     errs = ctx.Manager().dict()
     port = _free_port()
-    procs = [ctx.Process(target=_cpu_worker, args=(r, 2, port, 1301, errs)) for r in range(2)]
+    procs = [ctx.Process(target=_cpu_worker, args=(r, world, port, seed, errs, cuts, with_h0))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(120)
         assert p.exitcode == 0
-    assert sorted(errs.keys()) == [0, 1]
-    assert max(errs.values()) < 1e-9, dict(errs)
+    assert sorted(errs.keys()) == list(range(world))
+    return dict(errs)
+
+
+def test_context_parallel_orchestration_gloo():
+    """Two ranks, one sequence: each rank's o and the final state equal the
+    whole-sequence oracle (fp64 throughout, so to rounding)."""
+    errs = _run_ranks(2, 1301)
+    assert max(errs.values()) < 1e-9, errs
+
+
+def test_context_parallel_uneven_blocks_three_ranks():
+    """Three ranks with blocks of 17, 50 and 29 tokens and no start state:
+    the exchanged (M, N) have fixed shapes, so the blocks need not match."""
+    errs = _run_ranks(3, 1302, cuts=[0, 17, 67, 96], with_h0=False)
+    assert max(errs.values()) < 1e-9, errs
 
 
 # ----------------------------------------------------------------- GPU ---
