@@ -48,3 +48,54 @@ def test_mutant_is_caught(tmp_path, desc, old, new):
         if not (err <= tol):
             caught.append(name)
     assert caught, f"no pin caught the planted mistake: {desc}"
+
+
+# (description, exact text in kda_oracle_bwd.c, replacement)
+BWD_MUTANTS = [
+    ("dq read from the decayed state, not the updated one",
+     "const double* row = S + (size_t)i * dv;\n                    for (int j = 0; j < dv; ++j) acc += row[j] * dO[t * dv + j];",
+     "const double* row = Sd + (size_t)i * dv;\n                    for (int j = 0; j < dv; ++j) acc += row[j] * dO[t * dv + j];"),
+    ("read not added to the state adjoint", "row[j] += qt[i] * dO[t * dv + j];",
+     "row[j] += 0.0 * qt[i] * dO[t * dv + j];"),
+    ("dk misses the write term", "dkt[i] = acc;", "dkt[i] = 0.0 * acc;"),
+    ("dk misses the recall term", "dkt[i] += acc;", "dkt[i] += 0.0 * acc;"),
+    ("dbeta from v instead of v - p", "db += du[j] * (vt[j] - p[j]);", "db += du[j] * vt[j];"),
+    ("sign of dp flipped", "dp[j] = -bt * du[j];", "dp[j] = bt * du[j];"),
+    ("dv without beta", "dvt[j] = bt * du[j];", "dvt[j] = du[j];"),
+    ("recall's state term dropped", "row[j] += kt[i] * dp[j];", "(void)row;"),
+    ("dg from the undecayed state",
+     "const double* srow = Sd + (size_t)i * dv;",
+     "const double* srow = seg + (size_t)(t - t0) * st + (size_t)i * dv;"),
+    ("state adjoint not decayed",
+     "                const double a = exp(gt[i]);\n                for (int j = 0; j < dv; ++j) row[j] *= a;",
+     "                const double a = 1.0;\n                for (int j = 0; j < dv; ++j) row[j] *= a;"),
+    ("segment recomputed from the previous checkpoint",
+     "memcpy(S, ck + (size_t)c * st, sizeof(double) * st);",
+     "memcpy(S, ck + (size_t)(c > 0 ? c - 1 : 0) * st, sizeof(double) * st);"),
+    ("dhT ignored", "if (dhT) memcpy(dS, dhT, sizeof(double) * st);",
+     "if (0) memcpy(dS, dhT, sizeof(double) * st);"),
+    ("transposed state index in dq",
+     "for (int j = 0; j < dv; ++j) acc += row[j] * dO[t * dv + j];",
+     "for (int j = 0; j < dv; ++j) acc += S[(size_t)(j % dk) * dv + (i % dv)] * dO[t * dv + j];"),
+]
+
+
+@pytest.mark.parametrize("desc,old,new", BWD_MUTANTS, ids=[m[0] for m in BWD_MUTANTS])
+def test_bwd_mutant_is_caught(tmp_path, desc, old, new):
+    import pins_bwd
+    with open(oracle.SOURCE_BWD) as f:
+        src = f.read()
+    assert src.count(old) == 1, f"mutation site not unique/found: {desc}"
+    path = tmp_path / "mutant_bwd.c"
+    path.write_text(src.replace(old, new))
+    lib = oracle.compile_c(str(path), str(tmp_path / "libmutant_bwd.so"))
+    orc = oracle.Oracle(oracle.build(), lib)
+    caught = []
+    for name, (fn, tol) in pins_bwd.ALL_PINS.items():
+        try:
+            err = fn(orc)
+        except Exception:  # a crash or shape error also counts as caught
+            err = float("inf")
+        if not (err <= tol):
+            caught.append(name)
+    assert caught, f"no pin caught the planted mistake: {desc}"
