@@ -3,12 +3,16 @@
 Thin ctypes binding over ``libkda.so`` (the C ABI declared in
 ``include/kda.h``).  Every step of the computation runs in the library's
 CUDA kernels; this module only checks tensors and passes pointers, sizes
-and the current CUDA stream.  PyTorch is used for device memory and streams.
+and the current CUDA stream of the tensors' device, which it makes the
+current device for the call.  PyTorch is used for device memory and streams.
 
-Raw C functions are exposed under their C names (``kda_chunk_fwd``,
-``kda_chunk_fwd_f32``, ``kda_decode_step``, ``kda_status_string``,
-``kda_launch_count``, ``kda_version``); the tensor-level helpers
-``chunk_fwd``, ``chunk_fwd_f32`` and ``decode_step`` wrap them.
+Raw C functions are exposed under their C names (every name in
+``EXPORTED``).  The tensor-level helpers wrap them: ``chunk_fwd``,
+``chunk_fwd_raw`` (prologue fused), ``chunk_fwd_noalloc``,
+``chunk_fwd_states`` (intermediate states), ``chunk_transition`` and
+``state_chain`` (the pieces of a split sequence), ``chunk_fwd_f32``,
+``decode_step`` and ``decode_step_raw``.  They accept only contiguous CUDA
+tensors of the documented dtypes and shapes.
 
 If the library is missing or cannot be loaded, every call raises
 ``KdaLibraryError``: there is no fallback implementation.
@@ -109,8 +113,9 @@ def device_status(device=None) -> int:
     """KDA_OK or KDA_ERR_TIMEOUT (a bounded device wait expired since the
     last call); synchronises the current stream and clears the flag."""
     import torch
-    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
-    return int(load_library().kda_device_status(_stream(dev)))
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(load_library().kda_device_status(_stream(dev)))
 
 
 def launch_count() -> int:
@@ -129,6 +134,12 @@ def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
+def _require_cuda(t, name="inputs"):
+    if t.device.type != "cuda":
+        raise ValueError("%s must be CUDA tensors, got %s" % (name, t.device))
+    return t.device
+
+
 def _check(t, name, dtype, shape, device):
     if t.dtype != dtype:
         raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
@@ -144,9 +155,7 @@ def _prefill(fn_name, dtype, q, k, v, g, beta, h0, o, hT, output_final_state):
     import torch
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    dev = q.device
-    if dev.type != "cuda":
-        raise ValueError("inputs must be CUDA tensors")
+    dev = _require_cuda(q)
     for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)),
                          ("g", g, (B, T, H, dk)), ("v", v, (B, T, H, dv)),
                          ("beta", beta, (B, T, H))):
@@ -161,8 +170,9 @@ def _prefill(fn_name, dtype, q, k, v, g, beta, h0, o, hT, output_final_state):
     if hT is not None:
         _check(hT, "hT", torch.float32, (B, H, dk, dv), dev)
     fn = getattr(load_library(), fn_name)
-    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o),
-            _ptr(hT), B, T, H, dk, dv, _stream(dev))
+    with torch.cuda.device(dev):
+        st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o),
+                _ptr(hT), B, T, H, dk, dv, _stream(dev))
     if st != KDA_OK:
         raise KdaError(fn_name, st)
     return o, hT
@@ -203,6 +213,7 @@ def chunk_fwd_states(q, k, v, g, beta, h0=None, *, state_every, o=None, hT=None,
     import torch
     B, T, H, dk = q.shape
     dv = v.shape[-1]
+    _require_cuda(q)
     n = T // state_every if state_every > 0 else 0
     if states is None:
         states = torch.empty((B, H, n, dk, dv), dtype=torch.float32, device=q.device)
@@ -217,9 +228,11 @@ def chunk_fwd_states(q, k, v, g, beta, h0=None, *, state_every, o=None, hT=None,
     _check(hT, "hT", torch.float32, (B, H, dk, dv), q.device)
     if h0 is not None:
         _check(h0, "h0", torch.float32, (B, H, dk, dv), q.device)
-    st = load_library().kda_chunk_fwd_states(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o), _ptr(hT),
-        _ptr(states) if n > 0 else None, int(state_every), B, T, H, dk, dv, _stream(q.device))
+    with torch.cuda.device(q.device):
+        st = load_library().kda_chunk_fwd_states(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0), _ptr(o), _ptr(hT),
+            _ptr(states) if n > 0 else None, int(state_every), B, T, H, dk, dv,
+            _stream(q.device))
     if st != KDA_OK:
         raise KdaError("kda_chunk_fwd_states", st)
     return o, hT, states
@@ -230,15 +243,16 @@ def chunk_transition(q, k, g, beta, *, M=None):
     (kda_chunk_transition): running it from S0 ends at M S0 + (its state from zero)."""
     import torch
     B, T, H, dk = q.shape
-    dev = q.device
+    dev = _require_cuda(q)
     for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("g", g, (B, T, H, dk)),
                          ("beta", beta, (B, T, H))):
         _check(t, name, torch.bfloat16, shp, dev)
     if M is None:
         M = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev)
     _check(M, "M", torch.float32, (B, H, dk, dk), dev)
-    st = load_library().kda_chunk_transition(_ptr(q), _ptr(k), _ptr(g), _ptr(beta), _ptr(M),
-                                             B, T, H, dk, _stream(dev))
+    with torch.cuda.device(dev):
+        st = load_library().kda_chunk_transition(_ptr(q), _ptr(k), _ptr(g), _ptr(beta), _ptr(M),
+                                                 B, T, H, dk, _stream(dev))
     if st != KDA_OK:
         raise KdaError("kda_chunk_transition", st)
     return M
@@ -250,7 +264,7 @@ def state_chain(M, N, h0=None, *, S_start=None, hT=None):
     Returns (S_start [B, P, H, dk, dv], hT [B, H, dk, dv])."""
     import torch
     B, P, H, dk, dv = N.shape
-    dev = N.device
+    dev = _require_cuda(N)
     _check(M, "M", torch.float32, (B, P, H, dk, dk), dev)
     _check(N, "N", torch.float32, (B, P, H, dk, dv), dev)
     if h0 is not None:
@@ -261,8 +275,9 @@ def state_chain(M, N, h0=None, *, S_start=None, hT=None):
         hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     _check(S_start, "S_start", torch.float32, (B, P, H, dk, dv), dev)
     _check(hT, "hT", torch.float32, (B, H, dk, dv), dev)
-    st = load_library().kda_state_chain(_ptr(M), _ptr(N), _ptr(h0), _ptr(S_start), _ptr(hT),
-                                        B, P, H, dk, dv, _stream(dev))
+    with torch.cuda.device(dev):
+        st = load_library().kda_state_chain(_ptr(M), _ptr(N), _ptr(h0), _ptr(S_start), _ptr(hT),
+                                            B, P, H, dk, dv, _stream(dev))
     if st != KDA_OK:
         raise KdaError("kda_state_chain", st)
     return S_start, hT
@@ -279,9 +294,7 @@ def _decode(fn_name, q, k, v, g, beta, state, o):
     import torch
     N, H, dk = q.shape
     dv = v.shape[-1]
-    dev = q.device
-    if dev.type != "cuda":
-        raise ValueError("inputs must be CUDA tensors")
+    dev = _require_cuda(q)
     for name, t, shp in (("q", q, (N, H, dk)), ("k", k, (N, H, dk)),
                          ("g", g, (N, H, dk)), ("v", v, (N, H, dv)),
                          ("beta", beta, (N, H))):
@@ -290,8 +303,9 @@ def _decode(fn_name, q, k, v, g, beta, state, o):
     if o is None:
         o = torch.empty((N, H, dv), dtype=torch.bfloat16, device=dev)
     _check(o, "o", torch.bfloat16, (N, H, dv), dev)
-    st = getattr(load_library(), fn_name)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
-                                        _ptr(state), _ptr(o), N, H, dk, dv, _stream(dev))
+    with torch.cuda.device(dev):
+        st = getattr(load_library(), fn_name)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                            _ptr(state), _ptr(o), N, H, dk, dv, _stream(dev))
     if st != KDA_OK:
         raise KdaError(fn_name, st)
     return o

@@ -2,14 +2,15 @@
 (context parallelism with one exchange step).
 
 Rank r holds the r-th contiguous block of tokens of every sequence (the blocks
-in rank order make up the sequence), with the same B, H and block length on
-every rank.  The recurrence is affine in the state, so a block run from a
+in rank order make up the sequence), with the same B and H on every rank;
+block lengths may differ between ranks, since M and N do not depend on them.  The recurrence is affine in the state, so a block run from a
 start state S ends at M S + N, with M the block's transition (the product of
 its per-token (I - b k k^T) Diag(exp g)) and N the state it reaches from zero.
 Each rank
 
   1. runs its block from zero (N_r) and computes its transition (M_r);
-  2. all-gathers (M_r, N_r) over the group: 2 x 64 KB per (b, h) per rank;
+  2. all-gathers (M_r, N_r) over the group in one collective: 2 x 64 KB per
+     (b, h) per rank;
   3. chains S_{p+1} = M_p S_p + N_p from h0 over the blocks (every rank the
      same small computation), which gives its own start state S_r and the
      final state hT;
@@ -51,10 +52,14 @@ def chunk_fwd_context_parallel(q, k, v, g, beta, h0=None, *, group=None, ops=Ker
     rank = dist.get_rank(group)
     _, N = ops.block_fwd(q, k, v, g, beta, None)
     M = ops.transition(q, k, g, beta)
-    Ms = [torch.empty_like(M) for _ in range(world)]
-    Ns = [torch.empty_like(N) for _ in range(world)]
-    dist.all_gather(Ms, M.contiguous(), group=group)
-    dist.all_gather(Ns, N.contiguous(), group=group)
-    S_start, hT = ops.state_chain(torch.stack(Ms, 1).contiguous(), torch.stack(Ns, 1).contiguous(), h0)
+    if M.shape != N.shape:
+        raise ValueError("the exchange step needs d_k == d_v, got M %s and N %s"
+                         % (tuple(M.shape), tuple(N.shape)))
+    MN = torch.stack([M, N])                       # [2, B, H, dk, dv]
+    parts = [torch.empty_like(MN) for _ in range(world)]
+    dist.all_gather(parts, MN, group=group)
+    Ms = torch.stack([p[0] for p in parts], 1).contiguous()
+    Ns = torch.stack([p[1] for p in parts], 1).contiguous()
+    S_start, hT = ops.state_chain(Ms, Ns, h0)
     o, _ = ops.block_fwd(q, k, v, g, beta, S_start[:, rank].contiguous())
     return o, hT

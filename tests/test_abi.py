@@ -162,12 +162,34 @@ def test_selftest_limit_checked_on_host(lib):
     assert lib.kda_launch_count() == n0
 
 
-def test_binding_requires_cuda_tensors():
+def test_binding_requires_cuda_tensors(lib):
+    """Every tensor-level wrapper refuses host tensors before any launch:
+    the library takes device pointers only."""
     import torch
-    x = torch.zeros(1, 4, 1, 128, dtype=torch.bfloat16)
-    b = torch.zeros(1, 4, 1, dtype=torch.bfloat16)
-    with pytest.raises(ValueError):
-        kda.chunk_fwd(x, x, x, x, b)
+    n0 = lib.kda_launch_count()
+    x = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16)
+    b = torch.zeros(1, 64, 1, dtype=torch.bfloat16)
+    xf = torch.zeros(1, 64, 1, 128)
+    bf = torch.zeros(1, 64, 1)
+    d = torch.zeros(2, 1, 128, dtype=torch.bfloat16)
+    db = torch.zeros(2, 1, dtype=torch.bfloat16)
+    st = torch.zeros(2, 1, 128, 128)
+    M = torch.zeros(1, 2, 1, 128, 128)
+    calls = [
+        lambda: kda.chunk_fwd(x, x, x, x, b),
+        lambda: kda.chunk_fwd_raw(x, x, x, x, b),
+        lambda: kda.chunk_fwd_noalloc(x, x, x, x, b),
+        lambda: kda.chunk_fwd_states(x, x, x, x, b, state_every=32),
+        lambda: kda.chunk_transition(x, x, x, b),
+        lambda: kda.state_chain(M, M),
+        lambda: kda.chunk_fwd_f32(xf, xf, xf, xf, bf),
+        lambda: kda.decode_step(d, d, d, d, db, st),
+        lambda: kda.decode_step_raw(d, d, d, d, db, st),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA"):
+            call()
+    assert lib.kda_launch_count() == n0
 
 
 def test_missing_library_fails_loudly(tmp_path):
