@@ -140,6 +140,20 @@ def barrier(device=None):
 
 # --------------------------------------------------------------- clocks ---
 
+def smi_gpu_id(cuda_index: int, visible=None) -> str:
+    """The nvidia-smi `-i` selector of the GPU that CUDA calls `cuda_index`
+    in this process: CUDA numbers only the devices in CUDA_VISIBLE_DEVICES
+    (indices or UUIDs, in that order), nvidia-smi numbers every device."""
+    if visible is None:
+        visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if visible is None or not visible.strip():
+        return str(cuda_index)
+    entries = [e.strip() for e in visible.split(",") if e.strip()]
+    if 0 <= cuda_index < len(entries):
+        return entries[cuda_index]
+    return str(cuda_index)
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during a region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -147,12 +161,14 @@ class ClockSampler:
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+        self.gpu = smi_gpu_id(gpu_index)
         self.proc = None
         self.lines = []
         self._t = None
 
     def __enter__(self):
+        # no sleep here: the caller keeps the GPU under load while the
+        # sampler starts (keep_busy), so the samples see the loaded clocks
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
@@ -160,7 +176,6 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
-            time.sleep(0.3)
         except Exception:
             self.proc = None
         return self
@@ -171,7 +186,6 @@ class ClockSampler:
 
     def __exit__(self, *exc):
         if self.proc is not None:
-            time.sleep(0.2)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -200,6 +214,25 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def keep_busy(step, seconds, sync, first=0, parity=2):
+    """Run untimed `step(i)` calls for about `seconds` of wall time (waiting
+    for the device every 8 calls, so the queue stays short), around a timed
+    region, so that clock samples taken meanwhile see the GPU under the same
+    load.  Makes a multiple of `parity` calls, indices first, first + 1, ...,
+    so with first = 0 the next call, step(0), uses the other input set than
+    the last one, as it does between timed steps.  Returns the number of
+    calls."""
+    t_end = time.perf_counter() + seconds
+    i = first
+    while time.perf_counter() < t_end or (i - first) % parity != 0:
+        step(i)
+        i += 1
+        if (i - first) % 8 == 0:
+            sync()
+    sync()
+    return i - first
 
 
 # ------------------------------------------------------------- kda arm ----
@@ -235,17 +268,19 @@ def bench_kda(args, rank, world, local):
 
     stream = torch.cuda.current_stream(dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    n0 = kda.launch_count()
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        keep_busy(step, 0.4, torch.cuda.synchronize)
         barrier(dev)
         torch.cuda.synchronize()
+        n0 = kda.launch_count()
         ev[0].record(stream)
         for i in range(args.steps):
             step(i)
             ev[i + 1].record(stream)
         torch.cuda.synchronize()
+        launches = kda.launch_count() - n0
         barrier(dev)
-    launches = kda.launch_count() - n0
+        keep_busy(step, 0.3, torch.cuda.synchronize, first=args.steps)
     per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
     total_ms = ev[0].elapsed_time(ev[-1])
     total_ms = max_over_ranks(total_ms, dev)

@@ -53,3 +53,40 @@ def test_alg_accounting():
     assert bench.prefill_alg_bytes(1, 1, 1, 128, 128, False, False) == (3 * 128 + 128 + 1 + 128) * 2
     b = bench.decode_alg_bytes(256, 32, 128, 128)
     assert b == 256 * 32 * 132354
+
+
+def test_clock_sampler_selects_the_process_gpu():
+    """nvidia-smi numbers every GPU; CUDA numbers those in
+    CUDA_VISIBLE_DEVICES.  The sampler must query the GPU the process uses."""
+    import bench
+    assert bench.smi_gpu_id(0, visible=None) == "0" or "CUDA_VISIBLE_DEVICES" in os.environ
+    assert bench.smi_gpu_id(0, visible="") == "0"
+    assert bench.smi_gpu_id(0, visible="5") == "5"
+    assert bench.smi_gpu_id(1, visible="3, 6") == "6"
+    assert bench.smi_gpu_id(0, visible="GPU-8a1c2f3e-aaaa-bbbb-cccc-0123456789ab") == \
+        "GPU-8a1c2f3e-aaaa-bbbb-cccc-0123456789ab"
+    assert bench.smi_gpu_id(2, visible="4") == "2"          # out of range: as given
+
+
+def test_keep_busy_alternates_and_syncs():
+    """The untimed load around the timed region: about the asked wall time,
+    an even number of calls (so step(0) follows a call on the other input
+    set), and a wait for the device every 8 calls and at the end."""
+    import time
+    import bench
+    calls, syncs = [], []
+
+    def step(i):
+        calls.append(i)
+        time.sleep(0.001)
+
+    t0 = time.perf_counter()
+    n = bench.keep_busy(step, 0.05, lambda: syncs.append(len(calls)))
+    assert time.perf_counter() - t0 >= 0.05
+    assert n == len(calls) and n % 2 == 0 and calls == list(range(n))
+    assert calls[-1] % 2 == 1
+    assert syncs[-1] == n and all(c % 8 == 0 for c in syncs[:-1])
+    calls.clear()
+    assert bench.keep_busy(step, 0.0, lambda: None) == 0 and calls == []
+    n = bench.keep_busy(step, 0.01, lambda: None, first=5)
+    assert n >= 2 and n % 2 == 0 and calls == list(range(5, 5 + n))
