@@ -28,18 +28,23 @@
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers, owned by the caller, 16-byte
  *     aligned, densely packed in the row-major layouts given per function.
- *     No entry point keeps a pointer after it returns.  Only kda_chunk_fwd
- *     takes memory of its own, and only on its segment-scan path (see
- *     there): stream-ordered workspace (cudaMallocAsync / cudaFreeAsync on
- *     `stream`).  kda_chunk_fwd_noalloc is the same call without any
- *     allocation.
+ *     No entry point keeps a pointer after it returns.  Only the bf16
+ *     prefill calls kda_chunk_fwd, kda_chunk_fwd_raw and kda_chunk_fwd_states
+ *     take memory of their own, and only on the segment-scan path (see
+ *     kda_chunk_fwd): stream-ordered workspace (cudaMallocAsync /
+ *     cudaFreeAsync on `stream`).  kda_chunk_fwd_noalloc is kda_chunk_fwd
+ *     without any allocation.
  *   - Calls are asynchronous on `stream` (0 = legacy default stream) and do
  *     no host synchronisation.  Asynchronous device errors surface at the
  *     caller's next synchronisation, as for any CUDA launch.
  *   - Return value: KDA_OK, or a negative kda_status.  Argument errors are
  *     detected on the host and return before anything is launched.
  *   - Inputs and outputs must not overlap, except that hT may equal h0.
- *   - Thread-safe: no global mutable state besides a launch counter.
+ *   - Thread-safe: calls may come from several host threads, on several
+ *     streams at once.  The library's global state is a launch counter
+ *     (atomic), one bounded-wait error word per device (kda_device_status)
+ *     and the scratch array of kda_chunk_fwd_noalloc, whose segment-scan
+ *     calls must be ordered with one another (see there).
  */
 #ifndef KDA_H
 #define KDA_H
