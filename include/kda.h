@@ -79,7 +79,10 @@ typedef enum {
  * o_t is written for every token; hT is S after the last token.  The work is
  * done in 16-token tiles on the tensor cores with an fp32 master state (the
  * "T11E1" transcript's log-decay-bound turn is what makes the diagonal tiles
- * dense).  Returns KDA_ERR_UNSUPPORTED for other dk/dv.
+ * dense): every MMA takes tf32 operands (each rounded once, to nearest) and
+ * accumulates in fp32, which keeps o within 1e-2 of the exact recurrence
+ * where bf16 operands would not.  Returns KDA_ERR_UNSUPPORTED for other
+ * dk/dv.
  *
  * Segment scan: with B*H <= 8 and T >= 4096 each sequence is cut into P
  * segments that run in parallel (P about 148 / (B*H), at least 256 tokens
