@@ -17,7 +17,8 @@ rank runs the same per-GPU workload on its own seed with no collective on
 the data path (weak scaling); the time is the max over ranks.
 
 --impl reference times the fp64 CPU oracle (the correctness reference) on
-this host's cores over a bounded sample of the same workload.
+this host's cores (one whole head per core) over a bounded sample of the same
+workload.
 """
 from __future__ import annotations
 
@@ -312,6 +313,7 @@ def bench_kda(args, rank, world, local):
         "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "ms_per_step_median": round(statistics.median(per_step), 4),
         "scaling": "weak", "vs_baseline": None,
         "dtype": "f32" if w.dtype == torch.float32 else "bf16",
         "data": "synthetic",
@@ -493,55 +495,77 @@ def bench_decode(args, kda, dev, rank, world, hbm_gbs, peak_src):
 
 # -------------------------------------------------------- oracle on CPU ---
 
-def oracle_sample(workload_name, heads, seed, budget_s=None):
-    """Time the fp64 oracle on `heads` whole (b, h) sequences of a prefill
-    workload on all host cores.  Returns (tokens_per_s, seconds, cores,
-    sample_description); tokens/s counts full tokens (all H heads), i.e.
-    sampled token-heads / H / seconds."""
-    import torch
+class OracleSample:
+    """`heads` whole (b, h) sequences of a prefill workload (its per-head
+    recipe), generated once, for timing the fp64 oracle on the host cores:
+    the oracle runs one head per thread.  Tokens/s counts full tokens (all H
+    heads of the workload), i.e. sampled token-heads / H / seconds."""
+
+    def __init__(self, workload_name, heads, seed):
+        import oracle
+        from linear_attention_07_b200.inputs import WORKLOADS, prefill_inputs
+        self.w = w = WORKLOADS[workload_name]
+        self.heads = heads
+        self.x = prefill_inputs(1, w.T, heads, w.dk, w.dv, seed=seed, dtype=w.dtype,
+                                h0_std=w.h0_std, pin_frac=w.pin_frac)
+        self.threads = min(heads, oracle.num_cores())
+        self.tokens = heads * w.T / w.H
+        self.desc = ("%d heads x %d tokens with the per-head recipe of %s (H = %d), fp64 "
+                     "token-by-token, one head per thread" % (heads, w.T, w.name, w.H))
+
+    def time(self):
+        """One timed oracle run over the whole sample: seconds."""
+        import oracle
+        x = self.x
+        t0 = time.perf_counter()
+        oracle.fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"])
+        return time.perf_counter() - t0
+
+
+def oracle_heads(requested):
+    """Heads per oracle sample: as asked, else one per host core (at most
+    256), so the oracle runs on every core as its thread pool is built to."""
+    if requested:
+        return int(requested)
     import oracle
-    from linear_attention_07_b200.inputs import WORKLOADS, prefill_inputs
-    w = WORKLOADS[workload_name]
-    x = prefill_inputs(1, w.T, heads, w.dk, w.dv, seed=seed, dtype=w.dtype,
-                       h0_std=w.h0_std, pin_frac=w.pin_frac)
-    t0 = time.perf_counter()
-    oracle.fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"])
-    dt = time.perf_counter() - t0
-    tok_s = heads * w.T / w.H / dt
-    desc = "%d of %d heads x %d tokens of %s, fp64 token-by-token, all cores" % (
-        heads, w.H, w.T, w.name)
-    return tok_s, dt, oracle.num_cores(), desc
+    return max(1, min(256, oracle.num_cores()))
+
+
+def cpu_model():
+    """The host CPU's model name (Linux), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def cpu_baseline(args, min_seconds=10.0, max_runs=40):
-    """The oracle, as it stands, on repeated whole-head samples until about
-    `min_seconds` of CPU work has been timed."""
-    total_t, total_tok, runs = 0.0, 0.0, 0
+    """The oracle, as it stands, timed on one sample of the workload, run
+    repeatedly until about `min_seconds` of oracle time has been timed."""
+    smp = OracleSample(args.workload, oracle_heads(args.cpu_heads), 4242)
+    total_t, runs = 0.0, 0
     while runs < max_runs and (runs == 0 or total_t < min_seconds):
-        tok_s, dt, cores, desc = oracle_sample(args.workload, args.cpu_heads, 4242 + runs)
-        total_t += dt
-        total_tok += tok_s * dt
+        total_t += smp.time()
         runs += 1
-    return {"value": round(total_tok / total_t, 2), "unit": "tokens/s", "cores": cores,
-            "kind": "oracle", "sample": "%d x (%s)" % (runs, desc),
-            "seconds": round(total_t, 2)}
+    return {"value": round(smp.tokens * runs / total_t, 2), "unit": "tokens/s",
+            "cores": smp.threads, "kind": "oracle", "sample": "%d x (%s)" % (runs, smp.desc),
+            "seconds": round(total_t, 2), "cpu_model": cpu_model()}
 
 
 def bench_reference(args, rank, world):
     if rank != 0:
         return None
-    import oracle
-    from linear_attention_07_b200.inputs import WORKLOADS
-    w = WORKLOADS[args.workload]
+    smp = OracleSample(args.workload, oracle_heads(args.ref_heads), 199)
+    w = smp.w
     for i in range(args.warmup):
-        oracle_sample(args.workload, args.ref_heads, 99 + i)
-    times, toks = [], 0
-    for i in range(args.steps):
-        tok_s, dt, cores, desc = oracle_sample(args.workload, args.ref_heads, 199 + i)
-        times.append(dt)
-        toks += args.ref_heads * w.T / w.H
-    total = sum(times)
-    value = toks / total
+        smp.time()
+    total = sum(smp.time() for _ in range(args.steps))
+    value = smp.tokens * args.steps / total
+    cores, desc = smp.threads, smp.desc
     return {"metric": METRIC,
             "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -552,7 +576,8 @@ def bench_reference(args, rank, world):
                        "dv": w.dv, "global_batch": w.B, "seq_len": w.T,
                        "parallelism": "host threads"},
             "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
-                             "kind": "oracle", "sample": "each step: " + desc},
+                             "kind": "oracle", "sample": "each step: " + desc,
+                             "cpu_model": cpu_model()},
             "e2e": {"value": round(value, 2), "unit": "tokens/s",
                     "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -568,8 +593,10 @@ def main(argv=None):
     ap.add_argument("--workload", default="prefill_8k")
     ap.add_argument("--no-decode", dest="decode", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_base", action="store_false")
-    ap.add_argument("--cpu-heads", type=int, default=32)
-    ap.add_argument("--ref-heads", type=int, default=4)
+    ap.add_argument("--cpu-heads", type=int, default=None,
+                    help="heads per oracle sample (default: one per host core)")
+    ap.add_argument("--ref-heads", type=int, default=None,
+                    help="heads per reference-arm step (default: one per host core)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
