@@ -3,13 +3,17 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
                     [--workload prefill_8k] [--no-decode] [--no-cpu-baseline]
+                    [--more-workloads pretrain_64k,prefill_1m] [--small-footprint]
 
 A step is one kda_chunk_fwd over one batch of the prefill workload (B=1,
 H=32, T=8192, d=128, bf16 inputs, fp32 state).  Two independent input sets
 of 269 MB each (together > 4x the 126 MB L2) alternate between steps, so no
 step starts with its inputs in L2.  The decode workload (256 requests x 32
 heads, 1000 successive kda_decode_step calls) is timed in the same run and
-reported under "decode".  "e2e" is the same prefill through the public API
+reported under "decode", and the other prefill workloads of the pages'
+length range (a batch of four 64K pre-training sequences and a
+million-token sequence, each 32 heads) under their own names, each with its
+tokens/s, roofline and clock record.  "e2e" is the same prefill through the public API
 with host buffers: every step uploads its inputs from pinned host memory and
 downloads o and hT, pipelined across steps on two copy streams.  Multi-GPU:
 one process per GPU (torchrun), every
@@ -107,6 +111,18 @@ def load_peaks():
         return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def tensor_fractions(alg_flops, launch_ms, bf16_tflops):
+    """Algorithmic tensor throughput of a prefill launch against the peak of
+    its own MMA type: every prefill MMA is kind::tf32, whose peak is taken as
+    half the measured bf16 peak (the nominal tf32 : bf16 ratio, 1 : 2)."""
+    tf = alg_flops / (launch_ms / 1e3) / 1e12
+    return {"tensor_alg_tflops": round(tf, 2),
+            "tensor_frac_tf32": round(tf / (bf16_tflops / 2.0), 4),
+            "tensor_peak_tf32": round(bf16_tflops / 2.0, 1),
+            "tensor_peak_note": "tf32 peak = measured bf16 peak x 1/2 (nominal tf32:bf16 ratio)",
+            "tensor_frac_bf16": round(tf / bf16_tflops, 4)}
 
 
 # ---------------------------------------------------------------- ranks ---
@@ -252,18 +268,21 @@ def bench_kda(args, rank, world, local):
     w = WORKLOADS[args.workload]
     B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
 
-    # two independent input sets, alternated between steps
+    # two independent input sets, alternated between steps (one set in the
+    # small-footprint mode for profiler captures: the timing there is the
+    # profiler's, not the bench's)
+    n_sets = 1 if args.small_footprint else 2
     sets = [prefill_inputs(B, T, H, dk, dv, seed=rank_seed(w.seed + 17 * i, rank),
                            device=dev, h0_std=w.h0_std, pin_frac=w.pin_frac)
-            for i in range(2)]
+            for i in range(n_sets)]
     outs = [(torch.empty((B, T, H, dv), dtype=w.dtype, device=dev),
-             torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)) for _ in range(2)]
+             torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)) for _ in range(n_sets)]
     fwd = kda.chunk_fwd_f32 if w.dtype == torch.float32 else kda.chunk_fwd
     set_bytes = sum(t.numel() * t.element_size() for t in sets[0].values() if t is not None)
 
     def step(i):
-        x = sets[i % 2]
-        o, hT = outs[i % 2]
+        x = sets[i % n_sets]
+        o, hT = outs[i % n_sets]
         fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"], o=o, hT=hT)
 
     for i in range(args.warmup):
@@ -305,8 +324,8 @@ def bench_kda(args, rank, world, local):
                 "traffic": measured_traffic("kda_chunk_fwd", args.workload), "peak_source": peak_src + " hbm_gbs (burst copy)",
                 "alg_bytes_per_launch": alg_b,
                 "kernel": "kda_chunk_fwd",
-                "tensor_alg_tflops": round(alg_f / (launch_ms / 1e3) / 1e12, 2),
-                "tensor_frac_alg": round(alg_f / (launch_ms / 1e3) / 1e12 / bf16_tf, 4)}
+                "variant": kda.prefill_path(B, T, H)}
+    roofline.update(tensor_fractions(alg_f, launch_ms, bf16_tf))
 
     result = {
         "metric": METRIC,
@@ -320,8 +339,10 @@ def bench_kda(args, rank, world, local):
         "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
                    "global_batch": B * world, "seq_len": T,
                    "parallelism": "dp%d" % world,
-                   "l2": "two %.0f MB input sets alternate (%s)" % (
-                       set_bytes / 1e6, "inputs > L2" if set_bytes > 126e6 else "inputs fit in L2")},
+                   "l2": "%s %.0f MB input set%s (%s)" % (
+                       "two" if n_sets == 2 else "one", set_bytes / 1e6,
+                       "s alternate" if n_sets == 2 else "",
+                       "inputs > L2" if set_bytes > 126e6 else "inputs fit in L2")},
         "roofline": roofline,
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
@@ -330,13 +351,81 @@ def bench_kda(args, rank, world, local):
     # end to end through the public API: pinned host inputs -> device ->
     # kda_chunk_fwd -> o and hT back to pinned host memory, every step
     # (pipelined across steps; see bench_e2e)
-    result["e2e"] = bench_e2e(args, kda, sets, dev, B, T, world, fwd, w.dtype)
+    if not args.small_footprint:
+        result["e2e"] = bench_e2e(args, kda, sets, dev, B, T, world, fwd, w.dtype)
+    del sets, outs
+    torch.cuda.empty_cache()
 
     if args.decode:
         result["decode"] = bench_decode(args, kda, dev, rank, world, hbm_gbs, peak_src)
-    del sets, outs
-    torch.cuda.empty_cache()
+    # the other prefill workloads of the pages' length range, each timed the
+    # same way on its own inputs (each input set is far larger than L2)
+    if not args.small_footprint:
+        for name in args.more_workloads:
+            if name and name != w.name:
+                result[name] = bench_prefill_workload(args, kda, dev, rank, world, name,
+                                                      hbm_gbs, bf16_tf, peak_src)
     return result
+
+
+def bench_prefill_workload(args, kda, dev, rank, world, name, hbm_gbs, bf16_tf, peak_src):
+    """One more prefill workload, timed like the main line (warm-up, CUDA
+    events around `steps` back-to-back launches, clocks sampled under load),
+    with one input set: each of these workloads is many times the size of
+    L2, so no step finds its inputs there."""
+    import torch
+    from linear_attention_07_b200.inputs import WORKLOADS, prefill_inputs
+    w = WORKLOADS[name]
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    x = prefill_inputs(B, T, H, dk, dv, seed=rank_seed(w.seed, rank), device=dev,
+                       h0_std=w.h0_std, pin_frac=w.pin_frac)
+    o = torch.empty((B, T, H, dv), dtype=w.dtype, device=dev)
+    hT = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    set_bytes = sum(t.numel() * t.element_size() for t in x.values() if t is not None)
+
+    def step(i):
+        kda.chunk_fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"], o=o, hT=hT)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        keep_busy(step, 0.3, torch.cuda.synchronize)
+        barrier(dev)
+        torch.cuda.synchronize()
+        n0 = kda.launch_count()
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step(i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        launches = kda.launch_count() - n0
+        barrier(dev)
+        keep_busy(step, 0.2, torch.cuda.synchronize)
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), dev)
+    launch_ms = statistics.mean(per_step)
+    alg_b = prefill_alg_bytes(B, T, H, dk, dv, with_h0=w.h0_std > 0)
+    ach = alg_b / (launch_ms / 1e3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_gbs, "unit": "GB/s",
+            "frac": round(ach / hbm_gbs, 4), "traffic": measured_traffic("kda_chunk_fwd", name),
+            "peak_source": peak_src + " hbm_gbs (burst copy)",
+            "alg_bytes_per_launch": alg_b, "kernel": "kda_chunk_fwd",
+            "variant": kda.prefill_path(B, T, H)}
+    roof.update(tensor_fractions(prefill_alg_flops(B, T, H, dk, dv), launch_ms, bf16_tf))
+    out = {"metric": "KDA prefill tokens/s (%s)" % w.note,
+           "value": round(B * T * world * args.steps / (total_ms / 1e3), 1), "unit": "tokens/s",
+           "ms_per_step": round(total_ms / args.steps, 4),
+           "ms_per_step_median": round(statistics.median(per_step), 4),
+           "steps": args.steps, "warmup": args.warmup,
+           "config": {"workload": w.name, "B": B, "T": T, "H": H, "dk": dk, "dv": dv,
+                      "l2": "one %.2f GB input set (inputs > L2)" % (set_bytes / 1e9)},
+           "roofline": roof, "gpu_launches": int(launches), "clocks": clk.summary()}
+    del x, o, hT
+    torch.cuda.empty_cache()
+    return out
 
 
 def bench_e2e(args, kda, sets, dev, B, T, world, fwd, dtype):
@@ -459,6 +548,8 @@ def bench_decode(args, kda, dev, rank, world, hbm_gbs, peak_src):
     from linear_attention_07_b200.inputs import WORKLOADS, decode_inputs
     w = WORKLOADS["decode_256"]
     N, H, dk, dv, steps = w.B, w.H, w.dk, w.dv, w.T
+    if args.small_footprint:
+        steps = 16            # profiler captures: 16 steps of inputs, not 1000 (8.4 GB)
     d = decode_inputs(N, H, dk, dv, steps, seed=rank_seed(w.seed, rank), device=dev,
                       state_std=w.h0_std)
     S = d["state"]
@@ -593,6 +684,13 @@ def main(argv=None):
     ap.add_argument("--workload", default="prefill_8k")
     ap.add_argument("--no-decode", dest="decode", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_base", action="store_false")
+    ap.add_argument("--more-workloads", default="pretrain_64k,prefill_1m",
+                    type=lambda x: [y for y in x.split(",") if y],
+                    help="other prefill workloads timed in the same run, reported as sub-objects "
+                         "(comma-separated names; empty: none)")
+    ap.add_argument("--small-footprint", action="store_true",
+                    help="for profiler captures: one prefill input set, 16 decode steps, "
+                         "no end-to-end leg and no other workloads")
     ap.add_argument("--cpu-heads", type=int, default=None,
                     help="heads per oracle sample (default: one per host core)")
     ap.add_argument("--ref-heads", type=int, default=None,

@@ -41,8 +41,11 @@
  *     detected on the host and return before anything is launched.
  *   - Inputs and outputs must not overlap, except that hT may equal h0.
  *   - Thread-safe: calls may come from several host threads, on several
- *     streams at once.  The library's global state is a launch counter
- *     (atomic), one bounded-wait error word per device (kda_device_status)
+ *     streams and devices at once.  A call runs on the current device.  The
+ *     library's global state is a launch counter (atomic), one-time set-up
+ *     per device (kernel shared-memory limits, the SM count, the memory
+ *     pool's release threshold; idempotent, done by the first call on each
+ *     device), one bounded-wait error word per device (kda_device_status)
  *     and the scratch array of kda_chunk_fwd_noalloc, whose segment-scan
  *     calls must be ordered with one another (see there).
  */
@@ -85,13 +88,13 @@ typedef enum {
  * dk/dv.
  *
  * Segment scan: with B*H <= 8 and T >= 4096 each sequence is cut into P
- * segments that run in parallel (P about 148 / (B*H), at least 256 tokens
+ * segments that run in parallel (P about SMs / (B*H), at least 256 tokens
  * each): a pass over all segments from a zero state and from the identity
  * (with v = 0) gives, per segment, the state it reaches from zero and its
  * transition matrix; a short chain over the segments gives each segment's
  * true start state; a last pass writes o.  This path takes 3 * B * P * H *
  * dk * dv * 4 bytes of stream-ordered workspace (at most 29,097,984 bytes
- * when the path is chosen by itself) and returns KDA_ERR_NO_MEMORY if it
+ * when the path is chosen by itself on a 148-SM B200) and returns KDA_ERR_NO_MEMORY if it
  * cannot.  The environment variable
  * KDA_PREFILL_VARIANT = fused | cluster | segmented forces one path
  * (measurement and tests; "segmented" needs T >= 512).
@@ -220,9 +223,12 @@ int kda_decode_step_raw(const void* q_raw, const void* k_raw, const void* v, con
 
 /*
  * kda_device_status -- KDA_OK, or KDA_ERR_TIMEOUT if a kernel of this
- * library gave up on a bounded device-side wait since the last call (the
- * kernel then returned early and its outputs are incomplete).  Reads and
- * clears the flag; synchronises `stream`.  KDA_ERR_CUDA if a CUDA call fails.
+ * library gave up on a bounded device-side wait since the last call (every
+ * wait between the roles of a prefill kernel gives up after 2 s).  The
+ * kernel then returns early and fills the o rows and hT of the affected
+ * heads with NaN (intermediate states, if asked for, are undefined), so a
+ * partial result never passes for a real one.  Reads and clears the flag;
+ * synchronises `stream`.  KDA_ERR_CUDA if a CUDA call fails.
  */
 int kda_device_status(kda_stream_t stream);
 
@@ -242,6 +248,16 @@ const char* kda_status_string(int status);
 /* Number of kernels this library has launched in this process (all entry
  * points, all devices); lets callers count launches in a timed region. */
 uint64_t kda_launch_count(void);
+
+/*
+ * kda_prefill_path -- which path a bf16 prefill call (kda_chunk_fwd and its
+ * variants) of this shape takes on the current device: 0 = one SM per
+ * (batch, head), 1 = a cluster of four SMs per head (when batch x heads x 4
+ * fits in the device's SMs), 2 = the segment scan (batch x heads <= 8 and
+ * T >= 4096), after any KDA_PREFILL_VARIANT override.  Launches nothing.
+ * KDA_ERR_INVALID_ARG for negative sizes.
+ */
+int kda_prefill_path(int B, int T, int H);
 
 /* ABI version: (major << 16) | minor. */
 int kda_version(void);

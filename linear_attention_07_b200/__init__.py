@@ -36,7 +36,7 @@ EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_states", "k
             "kda_chunk_transition", "kda_state_chain", "kda_chunk_fwd_raw", "kda_decode_step",
             "kda_decode_step_raw",
             "kda_device_status", "kda_selftest_bounded_wait",
-            "kda_status_string", "kda_launch_count", "kda_version")
+            "kda_status_string", "kda_launch_count", "kda_prefill_path", "kda_version")
 
 
 class KdaLibraryError(RuntimeError):
@@ -92,6 +92,8 @@ def load_library(path: str = LIB_PATH):
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_launch_count.argtypes = []
     lib.kda_launch_count.restype = ctypes.c_uint64
+    lib.kda_prefill_path.argtypes = [i, i, i]
+    lib.kda_prefill_path.restype = i
     lib.kda_version.argtypes = []
     lib.kda_version.restype = i
     _lib = lib
@@ -116,6 +118,17 @@ def device_status(device=None) -> int:
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     with torch.cuda.device(dev):
         return int(load_library().kda_device_status(_stream(dev)))
+
+
+PREFILL_PATHS = ("one SM per head", "cluster of four SMs per head", "segment scan")
+
+
+def prefill_path(B: int, T: int, H: int) -> str:
+    """The path a bf16 prefill of this shape takes on the current device."""
+    p = int(load_library().kda_prefill_path(int(B), int(T), int(H)))
+    if p < 0:
+        raise KdaError("kda_prefill_path", p)
+    return PREFILL_PATHS[p]
 
 
 def launch_count() -> int:

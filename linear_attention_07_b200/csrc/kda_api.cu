@@ -9,6 +9,19 @@ namespace kda {
 static std::atomic<uint64_t> g_launches{0};
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
+static std::atomic<int> g_sm_count[MAX_DEVICES];
+
+int current_sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const bool tracked = dev >= 0 && dev < MAX_DEVICES;
+    if (tracked && (n = g_sm_count[dev].load(std::memory_order_relaxed)) > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 0;
+    if (tracked) g_sm_count[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 cudaError_t decode_step_launch(const void* q, const void* k, const void* v,
                                const void* g, const void* beta, float* state,
                                void* o, int64_t NH, int dk, int dv, bool raw,
@@ -23,6 +36,7 @@ cudaError_t prefill_transition_launch(const void* q, const void* k, const void* 
 cudaError_t state_chain_launch(const float* M, const float* N, const float* h0, float* S_start, float* hT,
                                int B, int P, int H, cudaStream_t stream);
 int prefill_device_status(cudaStream_t stream);
+int prefill_path_of(int B, int T, int H);
 cudaError_t bounded_wait_selftest_launch(uint64_t limit_ns, cudaStream_t stream);
 
 template <typename Tin, typename Tout>
@@ -217,6 +231,12 @@ int kda_selftest_bounded_wait(uint64_t limit_ns, kda_stream_t stream)
 }
 
 uint64_t kda_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int kda_prefill_path(int B, int T, int H)
+{
+    if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+    return prefill_path_of(B, T, H);
+}
 
 int kda_version(void) { return (1 << 16) | 0; }
 

@@ -4,12 +4,40 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/kda.h"
 
 namespace kda {
 
 // Counts every kernel launch made by the library (kda_launch_count()).
 void note_launches(int n);
+
+// Kernel attributes (the dynamic shared-memory limit) and memory-pool
+// settings apply to one device only, so one-time setup is kept per device
+// ordinal.  The setup calls are idempotent: two host threads that race on a
+// device's first call may both run them, which is harmless.
+constexpr int MAX_DEVICES = 64;
+using DeviceFlags = std::atomic<bool>[MAX_DEVICES];
+
+// Runs setup(device) on the current device unless it has already succeeded
+// there; returns its error, or cudaSuccess.
+template <typename F>
+cudaError_t once_per_device(DeviceFlags& done, F&& setup)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const bool tracked = dev >= 0 && dev < MAX_DEVICES;
+    if (tracked && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = setup(dev);
+    if (e == cudaSuccess && tracked) done[dev].store(true, std::memory_order_release);
+    return e;
+}
+
+// Number of SMs of the current device (queried once per device); 0 if the
+// query fails.
+int current_sm_count();
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }

@@ -114,6 +114,10 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t BAR_FREE = 1, BAR_READY = 2, BAR_CHAIN = 3, BAR_PREP = 4;
 
 constexpr uint64_t WAIT_NS = 2000000000ull;   // bounded waits: 2 s
+// After an expired wait: how long a CTA lets a copy that was already issued
+// land before it gives up its shared memory (an issued copy lands within
+// microseconds; one that was never issued never does).
+constexpr uint64_t DRAIN_NS = 20000000ull;    // 20 ms
 
 // Launch flags (segment scan passes): treat v as zero, start from h0 = I
 // (ignore h0), skip the o stores.
@@ -208,6 +212,23 @@ __device__ __forceinline__ void prologue_normalise(float (&qr)[pf::TILE], float 
         qr[rr] *= sq > 0.f ? rsqrtf(sq) : 0.f;
         kr[rr] *= sk > 0.f ? rsqrtf(sk) : 0.f;
     }
+}
+
+// After a bounded wait expired anywhere in a CTA its o rows and hT are
+// incomplete: fill them with NaN so that a caller who never reads
+// kda_device_status cannot mistake a partial result for a real one.
+// o_head points at token 0 of this head's segment, rows row_stride apart.
+__device__ __forceinline__ void poison_head_outputs(__nv_bfloat16* o_head, int64_t row_stride, int Tl,
+                                                    bool write_o, float* hT_head, int tid, int nthr)
+{
+    const float qnan = __int_as_float(0x7fc00000);
+    if (write_o) {
+        const __nv_bfloat16 nb = __float2bfloat16_rn(qnan);
+        for (int64_t e = tid; e < (int64_t)Tl * pf::D; e += nthr)
+            o_head[(e / pf::D) * row_stride + (e % pf::D)] = nb;
+    }
+    if (hT_head)
+        for (int e = tid; e < pf::D * pf::D; e += nthr) hT_head[e] = qnan;
 }
 
 // A shared flag read once by lane 0 and broadcast: the same value in every
@@ -698,6 +719,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, TMEM_COLS);
+    if (*(volatile int*)&s_abort)
+        poison_head_outputs(o ? o + base : nullptr, row_stride, Tl, o && !(flags & SEG_NO_O),
+                            hT ? hT + head_off * D * D : nullptr, tid, NT);
 }
 
 // ============================================================================
@@ -772,6 +796,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     __shared__ __align__(8) uint64_t s_bar[6];   // rank 0: FULL[0..2], X, KU0, KU1; ranks 1-3: EMPTY, MMA, input loads
     __shared__ int s_abort;
     __shared__ uint32_t s_odone;                 // rank 0: chunks whose slot is consumed
+    __shared__ int s_last_armed[NPREPCTA];       // rank 0: last chunk whose bytes FULL[slot] expects
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
@@ -795,8 +820,12 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         s_odone = 0;
         // rank 0: FULL[s] expects the bytes of chunk s's push; later uses are
         // armed when the slot is released (the push itself carries no arrive)
+        for (int i = 0; i < NPREPCTA; ++i) s_last_armed[i] = -1;
         if (rank == 0)
-            for (int i = 0; i < NPREPCTA && i < n_chunks; ++i) mbar_arrive_expect_tx(smem_u32(&s_bar[i]), SLOT);
+            for (int i = 0; i < NPREPCTA && i < n_chunks; ++i) {
+                mbar_arrive_expect_tx(smem_u32(&s_bar[i]), SLOT);
+                s_last_armed[i] = i;
+            }
     }
     fence_before_sync();
     __syncthreads();
@@ -889,9 +918,19 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             for (int ch = 1; ch < n_chunks; ++ch) {
                 if (lane == 0) {
                     if (!s_abort && !counter_wait(smem_u32(&s_odone), (uint32_t)ch, WAIT_NS)) expired();
-                    const int cn = ch - 1 + NPREPCTA;        // the chunk that will reuse this slot
-                    if (cn < n_chunks) mbar_arrive_expect_tx(smem_u32(&s_bar[(ch - 1) % NPREPCTA]), SLOT);
-                    mbar_arrive_remote_relaxed(map_to_rank(smem_u32(&s_bar[0]), 1u + (uint32_t)((ch - 1) % NPREPCTA)));
+                    // After an expired wait no slot is handed back (its previous
+                    // bytes may still be on their way): the preparers then give up
+                    // on their own bounded waits, and at most one push per slot is
+                    // left to drain before the CTA exits.
+                    if (!*(volatile int*)&s_abort) {
+                        const int sl = (ch - 1) % NPREPCTA;
+                        const int cn = ch - 1 + NPREPCTA;    // the chunk that will reuse this slot
+                        if (cn < n_chunks) {
+                            mbar_arrive_expect_tx(smem_u32(&s_bar[sl]), SLOT);
+                            s_last_armed[sl] = cn;
+                        }
+                        mbar_arrive_remote_relaxed(map_to_rank(smem_u32(&s_bar[0]), 1u + (uint32_t)sl));
+                    }
                 }
                 __syncwarp();
             }
@@ -1349,8 +1388,21 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
     fence_before_sync();
     __syncthreads();
-    cluster_sync();                    // no CTA leaves while another may still touch its memory
+    cluster_sync();                    // every push that will be issued has been issued
+    if (rank == 0 && tid == 0 && *(volatile int*)&s_abort) {
+        // An expired wait let this CTA stop consuming slots: a push into a
+        // slot may still be landing.  Let each slot's last expected push land
+        // (or find that it was never sent) before the shared memory is given up.
+        for (int sl = 0; sl < NPREPCTA; ++sl)
+            if (s_last_armed[sl] >= 0)
+                mbar_wait_cluster(smem_u32(&s_bar[sl]), (uint32_t)(s_last_armed[sl] / NPREPCTA) & 1u, DRAIN_NS);
+    }
+    __syncthreads();
     if (warp == 0) tmem_dealloc(tm, ncols);
+    if (rank == 0 && tid < NCW && *(volatile int*)&s_abort)
+        poison_head_outputs(o ? o + ((int64_t)b * T + ts) * (int64_t)H * D + (int64_t)h * D : nullptr,
+                            (int64_t)H * D, Tl, o && !(flags & SEG_NO_O),
+                            hT ? hT + head_off * D * D : nullptr, tid, NCW);
 }
 
 static bool make_map(CUtensorMap* map, const void* base, int B, int T, int H)
@@ -1358,15 +1410,17 @@ static bool make_map(CUtensorMap* map, const void* base, int B, int T, int H)
     typedef CUresult (*encode_fn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-    static encode_fn encode = nullptr;
-    if (!encode) {
+    // looked up once per process (thread-safe static initialisation): the
+    // driver entry point is the same for every device
+    static const encode_fn encode = []() -> encode_fn {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess || !fn)
-            return false;
-        encode = (encode_fn)fn;
-    }
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return (encode_fn)fn;
+    }();
+    if (!encode) return false;
     // [B][T][H * 128] bf16, box 128 x 32 x 1 (one head's 32 token rows)
     const cuuint64_t dims[3] = {(cuuint64_t)H * pf::D, (cuuint64_t)T, (cuuint64_t)B};
     const cuuint64_t strides[2] = {(cuuint64_t)H * pf::D * 2, (cuuint64_t)T * H * pf::D * 2};
@@ -1377,20 +1431,34 @@ static bool make_map(CUtensorMap* map, const void* base, int B, int T, int H)
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Dynamic shared memory of both kernels in both instantiations.
+// Dynamic shared memory of every prefill kernel, set once per device (the
+// attribute applies to the current device only).
+static cudaError_t segment_combine_attribute();
+static DeviceFlags g_prefill_attr_done;
+
 static cudaError_t set_prefill_attributes()
 {
-    const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<false>, a, (int)pf::SMEM_BYTES);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_tc_kernel<true>, a, (int)pf::SMEM_BYTES);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_cluster_kernel<false>, a, (int)pc::SMEM_BYTES);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_cluster_kernel<true>, a, (int)pc::SMEM_BYTES);
-    return e;
+    return once_per_device(g_prefill_attr_done, [](int) {
+        const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+        cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<false>, a, (int)pf::SMEM_BYTES);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_tc_kernel<true>, a, (int)pf::SMEM_BYTES);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_cluster_kernel<false>, a, (int)pc::SMEM_BYTES);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_cluster_kernel<true>, a, (int)pc::SMEM_BYTES);
+        if (e == cudaSuccess) e = segment_combine_attribute();
+        return e;
+    });
+}
+
+// SMs of the current device (148 on a B200 if the query fails).
+static int64_t sm_count()
+{
+    const int n = current_sm_count();
+    return n > 0 ? n : 148;
 }
 
 // Four SMs per head pay off while the heads alone leave most SMs idle:
-// up to 37 heads (148 SMs); larger batches use one SM per head.
-static bool cluster_fits(int64_t heads) { return heads * (pc::NPREPCTA + 1) <= 148; }
+// up to SMs / 4 heads (37 on a B200); larger batches use one SM per head.
+static bool cluster_fits(int64_t heads) { return heads * (pc::NPREPCTA + 1) <= sm_count(); }
 
 // One launch of either variant over B * n_seg segment-sequences of length
 // seg_len (n_seg = 1, seg_len = T: the plain prefill).
@@ -1508,6 +1576,12 @@ segment_combine_kernel(const float* __restrict__ M, const float* __restrict__ N,
     }
 }
 
+static cudaError_t segment_combine_attribute()
+{
+    return cudaFuncSetAttribute(segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)SEG_COMBINE_SMEM);
+}
+
 enum class PrefillPath { OneSm, Cluster, Segmented };
 
 // KDA_PREFILL_VARIANT=fused|cluster|segmented overrides the choice (for
@@ -1531,7 +1605,7 @@ static void segment_plan(int B, int T, int H, int* seg_len, int* n_seg)
 {
     const int64_t heads = (int64_t)B * H;
     const int n_chunks = (T + pf::C - 1) / pf::C;
-    int64_t P = 148 / (heads > 0 ? heads : 1);
+    int64_t P = sm_count() / (heads > 0 ? heads : 1);
     P = P < (int64_t)(n_chunks / SEG_MIN_CHUNKS) ? P : (int64_t)(n_chunks / SEG_MIN_CHUNKS);
     if (P < 2) P = 2;
     const int seg_chunks = (int)((n_chunks + P - 1) / P);
@@ -1564,16 +1638,16 @@ static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk
         if (e != cudaSuccess) return e;
         ws = static_cast<float*>(p);
     } else {
-        static bool pool_set = false;   // keep freed workspace in the pool between calls
-        if (!pool_set) {
-            int dev = 0;
+        // keep freed workspace in this device's pool between calls
+        static DeviceFlags pool_done;
+        once_per_device(pool_done, [](int dev) {
             cudaMemPool_t pool;
-            if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+            if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
                 uint64_t keep = UINT64_MAX;
                 cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
             }
-            pool_set = true;
-        }
+            return cudaSuccess;   // a pool that keeps nothing only costs speed
+        });
         e = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
         if (e != cudaSuccess) return e;
     }
@@ -1602,20 +1676,22 @@ static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk
     return e;
 }
 
+// Which path a bf16 prefill of this shape takes on the current device
+// (0 one SM per head, 1 cluster of four SMs per head, 2 segment scan).
+int prefill_path_of(int B, int T, int H)
+{
+    return (int)choose_path(B, T, H);
+}
+
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, const float* h0, void* o, float* hT,
                               int B, int T, int H, bool no_alloc, float* states, int snap_every,
                               bool prologue, cudaStream_t stream)
 {
     const uint32_t flags = prologue ? pf::PROLOGUE : 0u;
-    static bool attr_set = false;   // idempotent; races only repeat the same calls
-    if (!attr_set) {
-        cudaError_t e = set_prefill_attributes();
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(segment_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)SEG_COMBINE_SMEM);
+    {
+        const cudaError_t e = set_prefill_attributes();
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     CUtensorMap mq, mk, mv, mg;
     if (T > 0) {
@@ -1642,11 +1718,9 @@ cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const
 cudaError_t prefill_transition_launch(const void* q, const void* k, const void* g, const void* beta,
                                       float* M, int B, int T, int H, cudaStream_t stream)
 {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = set_prefill_attributes();
+    {
+        const cudaError_t e = set_prefill_attributes();
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     CUtensorMap mq, mk, mg;
     if (T > 0) {
@@ -1667,13 +1741,9 @@ cudaError_t prefill_transition_launch(const void* q, const void* k, const void* 
 cudaError_t state_chain_launch(const float* M, const float* N, const float* h0, float* S_start, float* hT,
                                int B, int P, int H, cudaStream_t stream)
 {
-    static bool attr_set = false;
-    if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(segment_combine_kernel,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)SEG_COMBINE_SMEM);
+    {
+        const cudaError_t e = set_prefill_attributes();
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     segment_combine_kernel<<<dim3(pf::D / SEG_COLS, B * H), 256, SEG_COMBINE_SMEM, stream>>>(
         M, N, S_start, h0, hT, H, P);

@@ -10,6 +10,13 @@ err_out:   max_i |x_i - ref_i| / (rms(ref) + |ref_i|) -- the same bound in
            (up to 2^-8 relative) would exceed the plain max/rms form on the
            heavy tail; the allclose form still bounds every element by 1% of
            the larger of its own size and the typical size.
+bf16_floor: max|bf16(ref) - ref| / rms(ref): what rounding the exact result
+           to the output format costs in the plain metric, with no kernel
+           error at all.
+out_report / check_out: the three numbers for a bf16 output (plain, floor,
+           relaxed) and the checks on them: the relaxed form within the
+           tolerance, and the plain form within the tolerance of the floor
+           (the kernel's own error beyond what the format forces).
 """
 import numpy as np
 
@@ -35,12 +42,43 @@ def err_state(x, ref):
     return d / r if r > 0 else d
 
 
+err_plain = err_state
+
+
 def err_out(x, ref):
     x, ref = _np(x), _np(ref)
     if ref.size == 0:
         return 0.0
     r = rms(ref)
     return float(np.max(np.abs(x - ref) / (r + np.abs(ref))))
+
+
+def bf16_floor(ref):
+    """max|bf16(ref) - ref| / rms(ref), bf16 rounding to nearest even."""
+    import torch
+    ref = _np(ref)
+    if ref.size == 0:
+        return 0.0
+    rounded = torch.from_numpy(ref).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    return err_state(rounded, ref)
+
+
+def out_report(x, ref):
+    """(plain, floor, relaxed) for a bf16 output x against the exact ref."""
+    return err_state(x, ref), bf16_floor(ref), err_out(x, ref)
+
+
+def fmt_report(rep):
+    return "plain=%.3e floor=%.3e relaxed=%.3e" % rep
+
+
+def check_out(x, ref, tol, what="o"):
+    """Assert the bf16-output bounds; returns (plain, floor, relaxed)."""
+    rep = out_report(x, ref)
+    plain, floor, relaxed = rep
+    assert relaxed <= tol and plain <= floor + tol, \
+        "%s: %s (tol %.0e; plain must stay within tol of the floor)" % (what, fmt_report(rep), tol)
+    return rep
 
 
 TOL_BF16 = 1e-2
