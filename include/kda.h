@@ -222,6 +222,60 @@ int kda_decode_step_raw(const void* q_raw, const void* k_raw, const void* v, con
                         int N, int H, int dk, int dv, kda_stream_t stream);
 
 /*
+ * kda_chunk_bwd -- gradients of a kda_chunk_fwd call (training at the 8K-64K
+ * pre-training lengths of the "T11E1: K3 tech report" transcript, the
+ * context-length turn): with L = sum(dO * o) + sum(dhT * hT), the gradients
+ * of L with respect to q, k, v, g, beta and h0.  The pages give the forward
+ * only; the backward is its exact derivative (up to rounding).
+ *
+ *   q, k, g, v, beta, h0 : the forward's inputs (layouts of kda_chunk_fwd)
+ *   dO   : bf16 [B][T][H][dv], the gradient of o
+ *   dhT  : fp32 [B][H][dk][dv], the gradient of hT, or NULL (zero)
+ *   dq, dk, dg : bf16 [B][T][H][dk]     dv : bf16 [B][T][H][dv]
+ *   dbeta      : bf16 [B][T][H]         dh0 : fp32 [B][H][dk][dv], or NULL
+ *   Supported: d_k == d_v == 128.  T == 0: dh0 receives dhT (or zeros).
+ * Four launches on `stream`, fp32 arithmetic throughout (the gradient of the
+ * decay sums terms that nearly cancel, and tf32 state products would move
+ * it by about 1e-2 of its scale): per-chunk operands, the forward state
+ * chain, the reverse state chain, the chunk-local gradients.  Stream-ordered
+ * workspace of 209,408 bytes per 32-token chunk and head (about 6.5 KB per
+ * token and head; KDA_ERR_NO_MEMORY if it cannot be had).  Outputs must not
+ * overlap inputs or one another.
+ */
+int kda_chunk_bwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                  const float* h0, const void* dO, const float* dhT,
+                  void* dq, void* dk, void* dv, void* dg, void* dbeta, float* dh0,
+                  int B, int T, int H, int d_k, int d_v, kda_stream_t stream);
+
+/*
+ * kda_verify_fwd -- K consecutive tokens of each of N requests from a start
+ * state, keeping the state after EVERY token (speculative decoding: verify
+ * K drafted tokens, then continue from the state after the last accepted
+ * one).  The "177: Kimi K3 in Detail" episode notes (Deep dive 23) describe
+ * the rollback this serves: keep a checkpoint and a short log per step, and
+ * replay the accepted steps.
+ *
+ *   q, k, g : bf16 [N][K][H][dk]      v, o : bf16 [N][K][H][dv]
+ *   beta    : bf16 [N][K][H]
+ *   h0      : fp32 [N][H][dk][dv] start states, read only (NULL: zero)
+ *   states  : fp32 [N][K][H][dk][dv]; states[n][t] = S after token t + 1
+ *             of request n (all heads: one [H][dk][dv] block, the layout of
+ *             a kda_decode_step state, so rolling back to an accepted
+ *             prefix is one contiguous copy per request)
+ *   1 <= K <= KDA_VERIFY_MAX_TOKENS (else KDA_ERR_UNSUPPORTED; K == 0 is a
+ *   no-op).  Supported: dk, dv in {32, 64, 128}.
+ * Every token is the exact arithmetic of kda_decode_step (fp32, CUDA
+ * cores, the same operation order), so replaying the first j tokens from h0
+ * with kda_decode_step reproduces states[n][j - 1] bit for bit.  Memory
+ * bound: h0 read once, K states written.  o and states must not overlap
+ * the inputs; h0 may not alias states.
+ */
+#define KDA_VERIFY_MAX_TOKENS 64
+int kda_verify_fwd(const void* q, const void* k, const void* v, const void* g,
+                   const void* beta, const float* h0, void* o, float* states,
+                   int N, int K, int H, int dk, int dv, kda_stream_t stream);
+
+/*
  * kda_device_status -- KDA_OK, or KDA_ERR_TIMEOUT if a kernel of this
  * library gave up on a bounded device-side wait since the last call (every
  * wait between the roles of a prefill kernel gives up after 2 s).  The

@@ -11,7 +11,8 @@ Raw C functions are exposed under their C names (every name in
 ``chunk_fwd_raw`` (prologue fused), ``chunk_fwd_noalloc``,
 ``chunk_fwd_states`` (intermediate states), ``chunk_transition`` and
 ``state_chain`` (the pieces of a split sequence), ``chunk_fwd_f32``,
-``decode_step`` and ``decode_step_raw``.  They accept only contiguous CUDA
+``decode_step``, ``decode_step_raw``, ``verify_fwd`` (several tokens
+per request with the state after each) and ``chunk_bwd`` (the gradients).  They accept only contiguous CUDA
 tensors of the documented dtypes and shapes.
 
 If the library is missing or cannot be loaded, every call raises
@@ -34,7 +35,7 @@ KDA_ERR_NO_MEMORY = -5
 
 EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_states", "kda_chunk_fwd_f32",
             "kda_chunk_transition", "kda_state_chain", "kda_chunk_fwd_raw", "kda_decode_step",
-            "kda_decode_step_raw",
+            "kda_decode_step_raw", "kda_verify_fwd", "kda_chunk_bwd",
             "kda_device_status", "kda_selftest_bounded_wait",
             "kda_status_string", "kda_launch_count", "kda_prefill_path", "kda_version")
 
@@ -84,6 +85,11 @@ def load_library(path: str = LIB_PATH):
     lib.kda_chunk_fwd_raw.restype = i
     lib.kda_decode_step_raw.argtypes = [vp, vp, vp, vp, vp, fp, vp, i, i, i, i, vp]
     lib.kda_decode_step_raw.restype = i
+    lib.kda_chunk_bwd.argtypes = [vp, vp, vp, vp, vp, fp, vp, fp, vp, vp, vp, vp, vp, fp,
+                                  i, i, i, i, i, vp]
+    lib.kda_chunk_bwd.restype = i
+    lib.kda_verify_fwd.argtypes = [vp, vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, vp]
+    lib.kda_verify_fwd.restype = i
     lib.kda_device_status.argtypes = [vp]
     lib.kda_device_status.restype = i
     lib.kda_selftest_bounded_wait.argtypes = [ctypes.c_uint64, vp]
@@ -337,3 +343,67 @@ def decode_step_raw(q_raw, k_raw, v, z, beta, state, *, o=None):
     return _decode("kda_decode_step_raw", q_raw, k_raw, v, z, beta, state, o)
 
 
+
+
+VERIFY_MAX_TOKENS = 64
+
+
+def verify_fwd(q, k, v, g, beta, h0=None, *, o=None, states=None):
+    """K tokens per request from the start states h0, keeping the state after
+    every token (kda_verify_fwd).  q, k, g: [N, K, H, dk]; v: [N, K, H, dv];
+    beta: [N, K, H] (bf16); h0: [N, H, dk, dv] fp32 or None (read only).
+    Returns (o [N, K, H, dv] bf16, states [N, K, H, dk, dv] fp32), with
+    states[n, t] the state of request n after its token t + 1."""
+    import torch
+    N, K, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = _require_cuda(q)
+    for name, t, shp in (("q", q, (N, K, H, dk)), ("k", k, (N, K, H, dk)),
+                         ("g", g, (N, K, H, dk)), ("v", v, (N, K, H, dv)),
+                         ("beta", beta, (N, K, H))):
+        _check(t, name, torch.bfloat16, shp, dev)
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((N, K, H, dv), dtype=torch.bfloat16, device=dev)
+    if states is None:
+        states = torch.empty((N, K, H, dk, dv), dtype=torch.float32, device=dev)
+    _check(o, "o", torch.bfloat16, (N, K, H, dv), dev)
+    _check(states, "states", torch.float32, (N, K, H, dk, dv), dev)
+    with torch.cuda.device(dev):
+        st = load_library().kda_verify_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                           _ptr(h0), _ptr(o), _ptr(states), N, K, H, dk, dv,
+                                           _stream(dev))
+    if st != KDA_OK:
+        raise KdaError("kda_verify_fwd", st)
+    return o, states
+
+
+def chunk_bwd(q, k, v, g, beta, h0, dO, dhT=None, *, want_dh0=True):
+    """Gradients of chunk_fwd (kda_chunk_bwd): with L = sum(dO * o) +
+    sum(dhT * hT), returns (dq, dk, dv, dg, dbeta, dh0); dq, dk, dg, dv,
+    dbeta bf16 in the input layouts, dh0 [B, H, dk, dv] fp32 (None if
+    want_dh0 is False).  dO: [B, T, H, dv] bf16; dhT: [B, H, dk, dv] fp32 or
+    None; h0 as for chunk_fwd."""
+    import torch
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = _require_cuda(q)
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)),
+                         ("g", g, (B, T, H, dk)), ("v", v, (B, T, H, dv)),
+                         ("beta", beta, (B, T, H)), ("dO", dO, (B, T, H, dv))):
+        _check(t, name, torch.bfloat16, shp, dev)
+    for name, t in (("h0", h0), ("dhT", dhT)):
+        if t is not None:
+            _check(t, name, torch.float32, (B, H, dk, dv), dev)
+    gq, gk, gg = (torch.empty((B, T, H, dk), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    gv = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device=dev)
+    gb = torch.empty((B, T, H), dtype=torch.bfloat16, device=dev)
+    gh = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_dh0 else None
+    with torch.cuda.device(dev):
+        st = load_library().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                          _ptr(dO), _ptr(dhT), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gg),
+                                          _ptr(gb), _ptr(gh), B, T, H, dk, dv, _stream(dev))
+    if st != KDA_OK:
+        raise KdaError("kda_chunk_bwd", st)
+    return gq, gk, gv, gg, gb, gh

@@ -27,6 +27,14 @@ cudaError_t decode_step_launch(const void* q, const void* k, const void* v,
                                void* o, int64_t NH, int dk, int dv, bool raw,
                                cudaStream_t stream);
 
+cudaError_t verify_launch(const void* q, const void* k, const void* v, const void* g,
+                          const void* beta, const float* h0, void* o, float* states,
+                          int N, int K, int H, int dk, int dv, cudaStream_t stream);
+
+cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                             const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv,
+                             void* dg, void* dbeta, float* dh0, int B, int T, int H, cudaStream_t stream);
+
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, const float* h0, void* o, float* hT,
                               int B, int T, int H, bool no_alloc, float* states, int snap_every,
@@ -204,6 +212,43 @@ int kda_decode_step_raw(const void* q_raw, const void* k_raw, const void* v, con
                         int N, int H, int dk, int dv, kda_stream_t stream)
 {
     return decode_step_any(q_raw, k_raw, v, z, beta, state, o, N, H, dk, dv, true, stream);
+}
+
+int kda_chunk_bwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                  const float* h0, const void* dO, const float* dhT,
+                  void* dq, void* dk, void* dv, void* dg, void* dbeta, float* dh0,
+                  int B, int T, int H, int d_k, int d_v, kda_stream_t stream)
+{
+    int st = check_prefill(q, k, v, g, beta, h0, dO, dhT, B, T, H, d_k, d_v);
+    if (st != KDA_OK) return st;
+    if (!(d_k == 128 && d_v == 128)) return KDA_ERR_UNSUPPORTED;
+    if (!opt_ptr_ok(dh0)) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * T * H > 0) {
+        if (!ptr_ok(dq) || !ptr_ok(dk) || !ptr_ok(dv) || !ptr_ok(dg) || dbeta == nullptr)
+            return KDA_ERR_INVALID_ARG;
+        if (((reinterpret_cast<uintptr_t>(beta) | reinterpret_cast<uintptr_t>(dbeta)) & 1u) != 0)
+            return KDA_ERR_INVALID_ARG;
+    }
+    if ((int64_t)B * H == 0) return KDA_OK;
+    if (T == 0 && dh0 == nullptr) return KDA_OK;
+    return status_of(chunk_bwd_launch(q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, B, T, H,
+                                      (cudaStream_t)stream));
+}
+
+int kda_verify_fwd(const void* q, const void* k, const void* v, const void* g,
+                   const void* beta, const float* h0, void* o, float* states,
+                   int N, int K, int H, int dk, int dv, kda_stream_t stream)
+{
+    if (N < 0 || K < 0 || H < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (N > 65535 || H > 65535 || K > KDA_VERIFY_MAX_TOKENS) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)N * K * H == 0) return KDA_OK;
+    if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) || !ptr_ok(o) || !ptr_ok(states) ||
+        !opt_ptr_ok(h0))
+        return KDA_ERR_INVALID_ARG;
+    if (beta == nullptr || (reinterpret_cast<uintptr_t>(beta) & 1u) != 0) return KDA_ERR_INVALID_ARG;
+    return status_of(verify_launch(q, k, v, g, beta, h0, o, states, N, K, H, dk, dv,
+                                   (cudaStream_t)stream));
 }
 
 const char* kda_status_string(int status)

@@ -1,0 +1,848 @@
+// KDA backward (training): the gradients of L = sum(dO * o) + sum(dhT * hT)
+// with respect to q, k, v, g, beta and h0, for d_k = d_v = 128.
+//
+// The pages give the forward recurrence only ("T11E1: K3 tech report"
+// transcript, the KDA turn; "Kimi K3 goes trillion-scale ..." subtitles, cue
+// 14) and name 8K-64K pre-training lengths (transcript, the context-length
+// turn); the backward is the derivative of the chunked forward taken chunk by
+// chunk.  Per 32-token chunk with start state S0 (Gam the in-chunk running
+// sum of g, gam = exp(Gam), gC = gam of the last token):
+//     Kt = K gam, Qt = Q gam, Kb = K exp(Gam_C - Gam),
+//     A  = diag(beta) strict_lower(Araw),  Araw_ri = sum_c k_rc k_ic exp(Gam_rc - Gam_ic),
+//     P  = lower_incl(Praw),               Praw_ri = sum_c q_rc k_ic exp(Gam_rc - Gam_ic),
+//     X  = (I + A)^-1,  Tm = X diag(beta),  W = Tm Kt,  U = Tm V - W S0,
+//     O  = Qt S0 + P U,  S_C = Diag(gC) S0 + Kb^T U.
+// Backward, with dS = dL/dS_C:
+//     dU = P^T dO + Kb dS,   dS0 = Diag(gC) dS - W^T (Kb dS) + (Qt - P W)^T dO,
+// and the chunk-local gradients of Tm, W, U, P, Kt, Qt, Kb, V and the decay.
+// The decayed pair products (Araw, Praw and their gradients) are never formed
+// with a chunk-relative 1/gam, which leaves fp32 after 17 tokens at the -5
+// log-decay floor: a pair (r, i) inside one 16-token tile uses the tile start
+// as reference (factors <= 1 and <= e^80), a pair across the two tiles the
+// tile boundary (both factors <= 1) -- the bound of the transcript's
+// log-decay-bound turn.
+//
+// Four launches, all fp32 arithmetic on CUDA cores:
+//   1. bwd_prep_kernel     (one CTA per chunk): Araw, Praw, X, W, U' = Tm V,
+//                           Z = Qt - P W, Kb, gC -> workspace;
+//   2. bwd_chain_kernel<0> (one CTA per (b, h, 32 state columns)): the forward
+//                           state chain S <- Diag(gC) S + Kb^T (U' - W S),
+//                           writing every chunk's start state;
+//   3. bwd_chain_kernel<1> : the reverse chain dS <- Diag(gC) dS - W^T (Kb dS)
+//                           + Z^T dO, writing every chunk's end gradient and
+//                           dh0 (state columns are independent in both chains);
+//   4. bwd_local_kernel    (one CTA per chunk): dq, dk, dv, dg, dbeta.
+// The start states come from an fp32 chain rather than the tf32 forward
+// kernel: dg sums terms that nearly cancel, and state errors at the tf32
+// level (about 1e-3) move it by about 1e-2 of its scale.
+#include "kda_common.cuh"
+
+namespace kda {
+namespace bw {
+
+constexpr int D = 128, C = 32, TILE = 16, NT = 256;
+constexpr int LD = D + 1;        // odd row stride: conflict-free row and column walks
+constexpr int L32 = C + 1;
+constexpr int NS = 32;           // state columns per chain CTA
+constexpr int JB = 16;           // state columns per block in the local kernel
+constexpr int LJ = JB + 1;
+
+// per-chunk record written by the prep kernel (floats)
+constexpr int R_KB = 0, R_W = R_KB + C * D, R_UP = R_W + C * D, R_Z = R_UP + C * D, R_GC = R_Z + C * D,
+              R_A = R_GC + D, R_P = R_A + C * C, R_X = R_P + C * C, R_FLOATS = R_X + C * C;
+static_assert(R_FLOATS % 4 == 0, "records stay 16-byte aligned");
+
+__device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Rows [t0, t0 + C) of one head of a [B][T][H][D] bf16 tensor into shared
+// memory (row stride LD), zero past Tl.
+__device__ __forceinline__ void load_rows(float* dst, const __nv_bfloat16* __restrict__ src, int64_t row0,
+                                          int64_t row_stride, int n_valid)
+{
+    for (int v = threadIdx.x; v < C * (D / 8); v += NT) {
+        const int r = v / (D / 8), c8 = (v % (D / 8)) * 8;
+        float f[8];
+        if (r < n_valid) {
+            const uint4 u = *reinterpret_cast<const uint4*>(src + row0 + (int64_t)r * row_stride + c8);
+            const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 x = __bfloat1622float2(p[j]);
+                f[2 * j] = x.x;
+                f[2 * j + 1] = x.y;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] = 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dst[r * LD + c8 + j] = f[j];
+    }
+}
+
+// Running sum of g over the chunk, per channel, in place.
+__device__ __forceinline__ void running_sum(float* G)
+{
+    if (threadIdx.x < D) {
+        float s = 0.f;
+        for (int r = 0; r < C; ++r) {
+            s += G[r * LD + threadIdx.x];
+            G[r * LD + threadIdx.x] = s;
+        }
+    }
+}
+
+// Reference of the tile-relative factors of row r: Gam before its tile.
+__device__ __forceinline__ float tile_ref(const float* G, int r, int c)
+{
+    return r >= TILE ? G[(TILE - 1) * LD + c] : 0.f;
+}
+
+// Block GEMM on shared-memory operands, fp32 FMA, all NT threads:
+// out(m, n, sum_k a(m, k) b(k, n)) for an M x N result.  Thread (tm, tn)
+// computes rows tm * TM .. + TM - 1 and columns tn + NC j: consecutive
+// threads read consecutive columns of a row-major b (or one column each of
+// a transposed one; odd row strides keep both conflict-free) and share the
+// a values (broadcast).
+template <int M, int N, int K, int TM, int TN, typename FA, typename FB, typename FO>
+__device__ __forceinline__ void tgemm(FA a, FB b, FO out)
+{
+    constexpr int NC = N / TN, NR = M / TM;
+    static_assert(NC * NR == NT && NC * TN == N && NR * TM == M, "tile shape");
+    const int t = threadIdx.x, tn = t % NC, tm = t / NC;
+    float acc[TM][TN];
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        float av[TM], bv[TN];
+#pragma unroll
+        for (int i = 0; i < TM; ++i) av[i] = a(tm * TM + i, k);
+#pragma unroll
+        for (int j = 0; j < TN; ++j) bv[j] = b(k, tn + NC * j);
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) out(tm * TM + i, tn + NC * j, acc[i][j]);
+}
+
+// ---------------------------------------------------------------- prep --
+
+constexpr int PREP_BIG = 8;                                  // K, Q, V, G, four scratch
+constexpr size_t PREP_SMEM = (size_t)(PREP_BIG * C * LD + 4 * C * L32 + C) * sizeof(float);
+
+__global__ void __launch_bounds__(NT, 1)
+bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ g,
+                const __nv_bfloat16* __restrict__ beta, float* __restrict__ rec_all, int T, int H, int n_chunks)
+{
+    extern __shared__ __align__(16) float sm[];
+    float* sK = sm;
+    float* sQ = sK + C * LD;
+    float* sV = sQ + C * LD;
+    float* sG = sV + C * LD;
+    float* s1 = sG + C * LD;
+    float* s2 = s1 + C * LD;
+    float* s3 = s2 + C * LD;
+    float* s4 = s3 + C * LD;
+    float* sA = s4 + C * LD;       // Araw
+    float* sP = sA + C * L32;      // Praw (lower incl)
+    float* sX = sP + C * L32;      // (I + A)^-1
+    float* sT = sX + C * L32;      // Tm
+    float* sB = sT + C * L32;      // beta
+
+    const int c_idx = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int t0 = c_idx * C;
+    const int Tl = min(C, T - t0);
+    const int tid = threadIdx.x;
+    const int64_t rs = (int64_t)H * D;
+    const int64_t row0 = ((int64_t)b * T + t0) * rs + (int64_t)h * D;
+    float* rec = rec_all + (((int64_t)b * H + h) * n_chunks + c_idx) * R_FLOATS;
+
+    load_rows(sK, k, row0, rs, Tl);
+    load_rows(sQ, q, row0, rs, Tl);
+    load_rows(sV, v, row0, rs, Tl);
+    load_rows(sG, g, row0, rs, Tl);
+    if (tid < C) sB[tid] = tid < Tl ? bf(beta[((int64_t)b * T + t0 + tid) * H + h]) : 0.f;
+    __syncthreads();
+    running_sum(sG);
+    __syncthreads();
+    // tile-relative operands of the pair products
+    for (int e = tid; e < C * D; e += NT) {
+        const int r = e / D, c = e % D;
+        const float Gr = sG[r * LD + c], ref = tile_ref(sG, r, c);
+        const float kk = sK[r * LD + c];
+        const float a = __expf(Gr - ref);
+        s1[r * LD + c] = kk * a;                                  // Ka
+        s2[r * LD + c] = sQ[r * LD + c] * a;                      // Qa
+        s3[r * LD + c] = kk * __expf(ref - Gr);                   // Kf (<= e^80)
+        if (r < TILE) s4[r * LD + c] = kk * __expf(sG[(TILE - 1) * LD + c] - Gr);   // Kc (<= 1)
+    }
+    __syncthreads();
+    // Araw (strict lower) and Praw (lower incl): one warp per pair, lanes over channels
+    {
+        const int w = tid >> 5, lane = tid & 31;
+        for (int p = w; p < C * (C + 1) / 2; p += NT / 32) {
+            int r = 0, base = 0;
+            while (base + r + 1 <= p) { base += r + 1; ++r; }
+            const int i = p - base;                               // i <= r
+            const float* R = (r / TILE == i / TILE) ? s3 : s4;
+            float sa = 0.f, sp = 0.f;
+#pragma unroll
+            for (int j = 0; j < D / 32; ++j) {
+                const int c = lane + 32 * j;
+                const float rv = R[i * LD + c];
+                sa = fmaf(s1[r * LD + c], rv, sa);
+                sp = fmaf(s2[r * LD + c], rv, sp);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                sa += __shfl_xor_sync(0xffffffffu, sa, off);
+                sp += __shfl_xor_sync(0xffffffffu, sp, off);
+            }
+            if (lane == 0) {
+                sA[r * L32 + i] = i < r ? sa : 0.f;
+                sP[r * L32 + i] = sp;
+                if (i < r) {
+                    sA[i * L32 + r] = 0.f;
+                    sP[i * L32 + r] = 0.f;
+                }
+            }
+        }
+        if (tid < C) sA[tid * L32 + tid] = 0.f;
+    }
+    __syncthreads();
+    // X = (I + diag(beta) Araw)^-1 by forward substitution, one column per thread
+    if (tid < C) {
+        const int j = tid;
+        float x[C];
+#pragma unroll
+        for (int r = 0; r < C; ++r) {
+            float s = 0.f;
+#pragma unroll
+            for (int i = 0; i < r; ++i) s = fmaf(sA[r * L32 + i], x[i], s);
+            x[r] = (r == j) ? 1.f : (r > j ? -sB[r] * s : 0.f);
+        }
+#pragma unroll
+        for (int r = 0; r < C; ++r) {
+            sX[r * L32 + j] = x[r];
+            sT[r * L32 + j] = x[r] * sB[j];
+        }
+    }
+    __syncthreads();
+    // Kt = K gam into s3 (Kf no longer needed)
+    for (int e = tid; e < C * D; e += NT) {
+        const int r = e / D, c = e % D;
+        s3[r * LD + c] = sK[r * LD + c] * __expf(sG[r * LD + c]);
+    }
+    __syncthreads();
+    // W = Tm Kt -> s1;  U' = Tm V -> s2
+    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return sT[m * L32 + kk]; },
+                         [&](int kk, int n) { return s3[kk * LD + n]; },
+                         [&](int m, int n, float x) { s1[m * LD + n] = x; });
+    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return sT[m * L32 + kk]; },
+                         [&](int kk, int n) { return sV[kk * LD + n]; },
+                         [&](int m, int n, float x) { s2[m * LD + n] = x; });
+    __syncthreads();
+    // Z = Qt - P W -> global
+    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return sP[m * L32 + kk]; },
+                         [&](int kk, int n) { return s1[kk * LD + n]; },
+                         [&](int m, int n, float x) {
+                             rec[R_Z + m * D + n] = sQ[m * LD + n] * __expf(sG[m * LD + n]) - x;
+                         });
+    for (int e = tid; e < C * D; e += NT) {
+        const int r = e / D, c = e % D;
+        rec[R_KB + e] = sK[r * LD + c] * __expf(sG[(C - 1) * LD + c] - sG[r * LD + c]);
+        rec[R_W + e] = s1[r * LD + c];
+        rec[R_UP + e] = s2[r * LD + c];
+    }
+    if (tid < D) rec[R_GC + tid] = __expf(sG[(C - 1) * LD + tid]);
+    for (int e = tid; e < C * C; e += NT) {
+        const int r = e / C, i = e % C;
+        rec[R_A + e] = sA[r * L32 + i];
+        rec[R_P + e] = sP[r * L32 + i];
+        rec[R_X + e] = sX[r * L32 + i];
+    }
+}
+
+// --------------------------------------------------------------- chains --
+// Per (b, h, NS state columns): the forward chain (REV = false) writes the
+// start state of every chunk to S_all[b][h][c]; the reverse chain (REV =
+// true) writes the gradient at the end of every chunk to S_all[b][h][c] and
+// the start-state gradient to out_last (dh0).  The chunk operands of the
+// next chunk are prefetched with cp.async while this one is processed.
+
+constexpr int CLD = D + 4;        // operand rows: 528 B, 16-byte aligned
+constexpr int XLD = NS + 4;       // state / Y rows: 144 B
+constexpr int OPS = 3 * C * CLD + C * XLD + D;     // W, Kb, Z, (U' or dO) slice, gC: one buffer
+constexpr size_t CHAIN_SMEM = (size_t)(2 * OPS + D * XLD + C * XLD) * sizeof(float);
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 :: "r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+template <bool REV>
+__global__ void __launch_bounds__(NT, 1)
+bwd_chain_kernel(const float* __restrict__ rec_all, const __nv_bfloat16* __restrict__ dO,
+                 const float* __restrict__ S_init, float* __restrict__ S_all, float* __restrict__ out_last,
+                 int T, int H, int n_chunks)
+{
+    extern __shared__ __align__(16) float sm[];
+    float* sXs = sm + 2 * OPS;               // state slice [D][XLD]
+    float* sY = sXs + D * XLD;               // [C][XLD]
+    const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int j0 = s * NS;
+    const int tid = threadIdx.x;
+    const int64_t bh = (int64_t)b * H + h;
+    const float* rec_h = rec_all + bh * n_chunks * R_FLOATS;
+
+    // prefetch the operands of chunk c into buffer `buf`
+    auto prefetch = [&](int c, int buf) {
+        float* o = sm + buf * OPS;
+        const float* r = rec_h + (int64_t)c * R_FLOATS;
+        for (int e = tid; e < C * (D / 4); e += NT) {
+            const int row = e / (D / 4), c4 = (e % (D / 4)) * 4;
+            cp_async16(o + 0 * C * CLD + row * CLD + c4, r + R_W + row * D + c4);
+            cp_async16(o + 1 * C * CLD + row * CLD + c4, r + R_KB + row * D + c4);
+            if (REV) cp_async16(o + 2 * C * CLD + row * CLD + c4, r + R_Z + row * D + c4);
+        }
+        float* sl = o + 3 * C * CLD;
+        if (!REV) {
+            for (int e = tid; e < C * (NS / 4); e += NT) {
+                const int row = e / (NS / 4), c4 = (e % (NS / 4)) * 4;
+                cp_async16(sl + row * XLD + c4, r + R_UP + row * D + j0 + c4);
+            }
+        } else {
+            // dO slice: bf16 [C][NS] as raw bytes in the first half of each row
+            const int t0 = c * C;
+            for (int e = tid; e < C * (NS / 8); e += NT) {
+                const int row = e / (NS / 8), c8 = (e % (NS / 8)) * 8;
+                if (t0 + row < T)
+                    cp_async16(reinterpret_cast<__nv_bfloat16*>(sl + row * XLD) + c8,
+                               dO + (((int64_t)b * T + t0 + row) * H + h) * D + j0 + c8);
+                else
+                    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(sl + row * XLD) + c8) =
+                        make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        for (int e = tid; e < D / 4; e += NT)
+            cp_async16(o + 3 * C * CLD + C * XLD + 4 * e, r + R_GC + 4 * e);
+        cp_commit();
+    };
+
+    // state slice: thread (ig, cg) owns rows ig + 32 m, columns 4 cg .. 4 cg + 3
+    const int ig = tid / (NS / 4), cg = tid % (NS / 4);
+    float xr[4][4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+        const int i = ig + 32 * m;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (S_init) x = *reinterpret_cast<const float4*>(S_init + bh * D * D + (int64_t)i * D + j0 + 4 * cg);
+        xr[m][0] = x.x; xr[m][1] = x.y; xr[m][2] = x.z; xr[m][3] = x.w;
+        *reinterpret_cast<float4*>(sXs + i * XLD + 4 * cg) = x;
+    }
+    const int first = REV ? n_chunks - 1 : 0;
+    const int step = REV ? -1 : 1;
+    if (n_chunks > 0) prefetch(first, 0);
+#pragma unroll 1
+    for (int n = 0; n < n_chunks; ++n) {
+        const int c = first + step * n;
+        const int buf = n & 1;
+        // the state at this chunk boundary
+        float* dst = S_all + (bh * n_chunks + c) * D * D;
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            *reinterpret_cast<float4*>(dst + (int64_t)(ig + 32 * m) * D + j0 + 4 * cg) =
+                make_float4(xr[m][0], xr[m][1], xr[m][2], xr[m][3]);
+        if (n + 1 < n_chunks) prefetch(c + step, buf ^ 1); else cp_commit();
+        cp_wait_1();
+        __syncthreads();                     // chunk c's operands, the state in shared memory
+        const float* oW = sm + buf * OPS;
+        const float* oK = oW + C * CLD;
+        const float* oZ = oK + C * CLD;
+        const float* oS = oW + 3 * C * CLD;
+        const float* oG = oS + C * XLD;
+        {   // step 1: Y = U'_s - W X (forward) or Y = Kb X (reverse); thread (r, cg)
+            const int r = tid / (NS / 4);
+            const float* A1 = REV ? oK : oW;
+            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+            for (int i = 0; i < D; ++i) {
+                const float a = A1[r * CLD + i];
+                const float4 x = *reinterpret_cast<const float4*>(sXs + i * XLD + 4 * cg);
+                y.x = fmaf(a, x.x, y.x); y.y = fmaf(a, x.y, y.y);
+                y.z = fmaf(a, x.z, y.z); y.w = fmaf(a, x.w, y.w);
+            }
+            if (!REV) {
+                const float4 u = *reinterpret_cast<const float4*>(oS + r * XLD + 4 * cg);
+                y = make_float4(u.x - y.x, u.y - y.y, u.z - y.z, u.w - y.w);
+            } else {
+                y = make_float4(-y.x, -y.y, -y.z, -y.w);      // -(Kb dS): enters as -W^T (Kb dS)
+            }
+            *reinterpret_cast<float4*>(sY + r * XLD + 4 * cg) = y;
+        }
+        __syncthreads();
+        {   // step 2: X = Diag(gC) X + Kb^T Y (forward) or X = Diag(gC) X + W^T Y + Z^T dO (reverse)
+            const float* B1 = REV ? oW : oK;
+            float acc[4][4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float gcv = oG[ig + 32 * m];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[m][u] = gcv * xr[m][u];
+            }
+#pragma unroll 4
+            for (int r = 0; r < C; ++r) {
+                const float4 y = *reinterpret_cast<const float4*>(sY + r * XLD + 4 * cg);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const float bb = B1[r * CLD + ig + 32 * m];
+                    acc[m][0] = fmaf(bb, y.x, acc[m][0]); acc[m][1] = fmaf(bb, y.y, acc[m][1]);
+                    acc[m][2] = fmaf(bb, y.z, acc[m][2]); acc[m][3] = fmaf(bb, y.w, acc[m][3]);
+                }
+            }
+            if (REV) {
+                const __nv_bfloat16* dOs = reinterpret_cast<const __nv_bfloat16*>(oS);
+#pragma unroll 4
+                for (int r = 0; r < C; ++r) {
+                    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(dOs + r * 2 * XLD + 4 * cg);
+                    const float2 d01 = __bfloat1622float2(d2[0]), d23 = __bfloat1622float2(d2[1]);
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float z = oZ[r * CLD + ig + 32 * m];
+                        acc[m][0] = fmaf(z, d01.x, acc[m][0]); acc[m][1] = fmaf(z, d01.y, acc[m][1]);
+                        acc[m][2] = fmaf(z, d23.x, acc[m][2]); acc[m][3] = fmaf(z, d23.y, acc[m][3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) xr[m][u] = acc[m][u];
+                *reinterpret_cast<float4*>(sXs + (ig + 32 * m) * XLD + 4 * cg) =
+                    make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
+            }
+        }
+        __syncthreads();                     // state written; buffer `buf` free for the prefetch after next
+    }
+    if (out_last) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+            *reinterpret_cast<float4*>(out_last + bh * D * D + (int64_t)(ig + 32 * m) * D + j0 + 4 * cg) =
+                make_float4(xr[m][0], xr[m][1], xr[m][2], xr[m][3]);
+    }
+}
+
+// ---------------------------------------------------------- local grads --
+
+constexpr int LOC_BIG = 9;     // K, Q, V, dO, G, W, dKb, dQt, dW
+constexpr size_t LOC_SMEM = (size_t)(LOC_BIG * C * LD + 2 * D * LJ + 2 * C * LJ + 8 * C * L32 + 2 * C + 2 * D) *
+                            sizeof(float);
+
+__device__ __forceinline__ __nv_bfloat16 to_bf(float x) { return __float2bfloat16_rn(x); }
+
+__global__ void __launch_bounds__(NT, 1)
+bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                 const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ g,
+                 const __nv_bfloat16* __restrict__ beta, const __nv_bfloat16* __restrict__ dO,
+                 const float* __restrict__ rec_all, const float* __restrict__ S0_all,
+                 const float* __restrict__ dS_all,
+                 __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                 __nv_bfloat16* __restrict__ dg, __nv_bfloat16* __restrict__ dbeta, int T, int H, int n_chunks)
+{
+    extern __shared__ __align__(16) float sm[];
+    float* bK = sm;
+    float* bQ = bK + C * LD;       // Kb during the column blocks, then Q
+    float* bV = bQ + C * LD;       // V, then dGam
+    float* bDO = bV + C * LD;      // dO, then dKt (from W), then Kf
+    float* bG = bDO + C * LD;      // Gam
+    float* bW = bG + C * LD;       // W, then Kt, then Ka
+    float* bDKB = bW + C * LD;     // dKb -> dk
+    float* bDQT = bDKB + C * LD;   // dQt (direct) -> dq
+    float* bDW = bDQT + C * LD;    // dW, then Qa
+    float* bS0 = bDW + C * LD;     // [D][LJ] start-state block, then Kc
+    float* bDS = bS0 + D * LJ;     // [D][LJ] end-gradient block
+    float* bU = bDS + D * LJ;      // [C][LJ]
+    float* bDU = bU + C * LJ;      // [C][LJ]
+    float* sA = bDU + C * LJ;      // Araw
+    float* sP = sA + C * L32;      // Praw (lower incl)
+    float* sX = sP + C * L32;
+    float* sT = sX + C * L32;      // Tm
+    float* sdP = sT + C * L32;     // dO U^T (masked to lower incl after the blocks)
+    float* sdUV = sdP + C * L32;   // dU V^T
+    float* sdT = sdUV + C * L32;   // dTm, then dX, then dA (unscaled), then dAr
+    float* sY = sdT + C * L32;     // dX X^T
+    float* sB = sY + C * L32;      // beta [C]
+    float* sDB = sB + C;           // dbeta [C]
+    float* sRS = sDB + C;          // sum_j dS_ij S0_ij [D]
+    float* sKS = sRS + D;          // sum_r dKb_rc Kb_rc [D]
+
+    const int c_idx = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int t0 = c_idx * C;
+    const int Tl = min(C, T - t0);
+    const int tid = threadIdx.x;
+    const int64_t rs = (int64_t)H * D;
+    const int64_t row0 = ((int64_t)b * T + t0) * rs + (int64_t)h * D;
+    const int64_t bh = (int64_t)b * H + h;
+    const float* rec = rec_all + (bh * n_chunks + c_idx) * R_FLOATS;
+    const float* S0 = S0_all + (bh * n_chunks + c_idx) * D * D;
+    const float* dS = dS_all + (bh * n_chunks + c_idx) * D * D;
+
+    // ---- inputs, the prep record and the chunk's decay
+    load_rows(bK, k, row0, rs, Tl);
+    load_rows(bV, v, row0, rs, Tl);
+    load_rows(bDO, dO, row0, rs, Tl);
+    load_rows(bG, g, row0, rs, Tl);
+    if (tid < C) {
+        sB[tid] = tid < Tl ? bf(beta[((int64_t)b * T + t0 + tid) * H + h]) : 0.f;
+        sDB[tid] = 0.f;
+    }
+    for (int e = tid; e < C * D; e += NT) {
+        const int r = e / D, c = e % D;
+        bW[r * LD + c] = rec[R_W + e];
+        bDKB[r * LD + c] = 0.f;
+        bDQT[r * LD + c] = 0.f;
+        bDW[r * LD + c] = 0.f;
+    }
+    for (int e = tid; e < C * C; e += NT) {
+        const int r = e / C, i = e % C;
+        sA[r * L32 + i] = rec[R_A + e];
+        sP[r * L32 + i] = rec[R_P + e];
+        sX[r * L32 + i] = rec[R_X + e];
+        sdP[r * L32 + i] = 0.f;
+        sdUV[r * L32 + i] = 0.f;
+    }
+    if (tid < D) sRS[tid] = 0.f;
+    __syncthreads();
+    running_sum(bG);
+    for (int e = tid; e < C * C; e += NT) {
+        const int r = e / C, i = e % C;
+        sT[r * L32 + i] = sX[r * L32 + i] * sB[i];
+    }
+    __syncthreads();
+    for (int e = tid; e < C * D; e += NT) {                       // Kb = K exp(Gam_C - Gam)
+        const int r = e / D, c = e % D;
+        bQ[r * LD + c] = bK[r * LD + c] * __expf(bG[(C - 1) * LD + c] - bG[r * LD + c]);
+    }
+    __syncthreads();
+
+    // ---- the state-sized products, JB state columns at a time
+#pragma unroll 1
+    for (int jb = 0; jb < D; jb += JB) {
+        for (int e = tid; e < D * (JB / 4); e += NT) {
+            const int i = e / (JB / 4), c4 = (e % (JB / 4)) * 4;
+            const float4 s0 = *reinterpret_cast<const float4*>(S0 + (int64_t)i * D + jb + c4);
+            const float4 ds = *reinterpret_cast<const float4*>(dS + (int64_t)i * D + jb + c4);
+            float* p0 = bS0 + i * LJ + c4;
+            float* p1 = bDS + i * LJ + c4;
+            p0[0] = s0.x; p0[1] = s0.y; p0[2] = s0.z; p0[3] = s0.w;
+            p1[0] = ds.x; p1[1] = ds.y; p1[2] = ds.z; p1[3] = ds.w;
+        }
+        __syncthreads();
+        // U = Tm V - W S0 and dU = P^T dO + Kb dS on this block (K = 32 + 128)
+        tgemm<C, JB, C + D, 2, 1>(
+            [&](int m, int kk) { return kk < C ? sT[m * L32 + kk] : -bW[m * LD + kk - C]; },
+            [&](int kk, int n) { return kk < C ? bV[kk * LD + jb + n] : bS0[(kk - C) * LJ + n]; },
+            [&](int m, int n, float x) { bU[m * LJ + n] = x; });
+        tgemm<C, JB, C + D, 2, 1>(
+            [&](int m, int kk) { return kk < C ? sP[kk * L32 + m] : bQ[m * LD + kk - C]; },
+            [&](int kk, int n) { return kk < C ? bDO[kk * LD + jb + n] : bDS[(kk - C) * LJ + n]; },
+            [&](int m, int n, float x) { bDU[m * LJ + n] = x; });
+        if (tid < D) {
+            float acc = sRS[tid];
+#pragma unroll
+            for (int j = 0; j < JB; ++j) acc = fmaf(bDS[tid * LJ + j], bS0[tid * LJ + j], acc);
+            sRS[tid] = acc;
+        }
+        __syncthreads();
+        // accumulate over the block's columns j
+        tgemm<C, C, JB, 4, 1>([&](int m, int kk) { return bDO[m * LD + jb + kk]; },
+                              [&](int kk, int n) { return bU[n * LJ + kk]; },
+                              [&](int m, int n, float x) { sdP[m * L32 + n] += x; });
+        tgemm<C, C, JB, 4, 1>([&](int m, int kk) { return bDU[m * LJ + kk]; },
+                              [&](int kk, int n) { return bV[n * LD + jb + kk]; },
+                              [&](int m, int n, float x) { sdUV[m * L32 + n] += x; });
+        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bDO[m * LD + jb + kk]; },
+                              [&](int kk, int n) { return bS0[n * LJ + kk]; },
+                              [&](int m, int n, float x) { bDQT[m * LD + n] += x; });
+        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bU[m * LJ + kk]; },
+                              [&](int kk, int n) { return bDS[n * LJ + kk]; },
+                              [&](int m, int n, float x) { bDKB[m * LD + n] += x; });
+        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bDU[m * LJ + kk]; },
+                              [&](int kk, int n) { return bS0[n * LJ + kk]; },
+                              [&](int m, int n, float x) { bDW[m * LD + n] -= x; });
+        // dV = Tm^T dU on this block, straight to global memory
+        tgemm<C, JB, C, 2, 1>([&](int m, int kk) { return sT[kk * L32 + m]; },
+                              [&](int kk, int n) { return bDU[kk * LJ + n]; },
+                              [&](int m, int n, float x) {
+                                  if (m < Tl) dv[row0 + (int64_t)m * rs + jb + n] = to_bf(x);
+                              });
+        __syncthreads();
+    }
+
+    // ---- Q back in place of Kb; dGam from the direct terms; dq, dk partials
+    load_rows(bQ, q, row0, rs, Tl);
+    if (tid < D) {                                   // sum_r dKb_rc Kb_rc, before dKb is rescaled
+        const int c = tid;
+        const float gl = bG[(C - 1) * LD + c];
+        float acc = 0.f;
+        for (int r = 0; r < C; ++r)
+            acc = fmaf(bDKB[r * LD + c], bK[r * LD + c] * __expf(gl - bG[r * LD + c]), acc);
+        sKS[c] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < C * D; e += NT) {
+        const int r = e / D, c = e % D;
+        const float Gr = bG[r * LD + c];
+        const float gam = __expf(Gr), kbf = __expf(bG[(C - 1) * LD + c] - Gr);
+        const float kk = bK[r * LD + c], qq = bQ[r * LD + c];
+        const float dqt = bDQT[r * LD + c], dkb = bDKB[r * LD + c];
+        bV[r * LD + c] = dqt * qq * gam - dkb * kk * kbf;        // dGam (direct terms)
+        bDQT[r * LD + c] = dqt * gam;
+        bDKB[r * LD + c] = dkb * kbf;
+        bW[r * LD + c] = kk * gam;                               // Kt
+    }
+    __syncthreads();
+    // dTm = dW Kt^T + dU V^T;  dKt = Tm^T dW -> bDO
+    tgemm<C, C, D, 4, 1>([&](int m, int kk) { return bDW[m * LD + kk]; },
+                         [&](int kk, int n) { return bW[n * LD + kk]; },
+                         [&](int m, int n, float x) { sdT[m * L32 + n] = x + sdUV[m * L32 + n]; });
+    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return sT[kk * L32 + m]; },
+                         [&](int kk, int n) { return bDW[kk * LD + n]; },
+                         [&](int m, int n, float x) { bDO[m * LD + n] = x; });
+    __syncthreads();
+    for (int e = tid; e < C * D; e += NT) {
+        const int r = e / D, c = e % D;
+        const float dkt = bDO[r * LD + c];
+        bDKB[r * LD + c] += dkt * __expf(bG[r * LD + c]);
+        bV[r * LD + c] += dkt * bW[r * LD + c];
+    }
+    // dbeta (columns: sum_r dTm_ri X_ri), then dX = dTm diag(beta)
+    if (tid < C) {
+        float acc = 0.f;
+        for (int r = 0; r < C; ++r) acc = fmaf(sdT[r * L32 + tid], sX[r * L32 + tid], acc);
+        sDB[tid] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < C * C; e += NT) {
+        const int r = e / C, i = e % C;
+        sdT[r * L32 + i] *= sB[i];
+        if (i > r) sdP[r * L32 + i] = 0.f;            // P is lower triangular incl. the diagonal
+    }
+    __syncthreads();
+    // Y = dX X^T;  dA = -(X^T Y), strictly lower
+    tgemm<C, C, C, 4, 1>([&](int m, int kk) { return sdT[m * L32 + kk]; },
+                         [&](int kk, int n) { return sX[n * L32 + kk]; },
+                         [&](int m, int n, float x) { sY[m * L32 + n] = x; });
+    __syncthreads();
+    tgemm<C, C, C, 4, 1>([&](int m, int kk) { return sX[kk * L32 + m]; },
+                         [&](int kk, int n) { return sY[kk * L32 + n]; },
+                         [&](int m, int n, float x) { sdT[m * L32 + n] = n < m ? -x : 0.f; });
+    __syncthreads();
+    // dbeta (rows: sum_i dA_ri Araw_ri), then dAr = diag(beta) dA
+    if (tid < C) {
+        float acc = sDB[tid];
+        for (int i = 0; i < C; ++i) acc = fmaf(sdT[tid * L32 + i], sA[tid * L32 + i], acc);
+        sDB[tid] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < C * C; e += NT) {
+        const int r = e / C, i = e % C;
+        sdT[r * L32 + i] *= sB[r];
+    }
+    // tile-relative operands: Ka -> bW, Qa -> bDW, Kf -> bDO, Kc -> bS0 (tile 0 rows)
+    for (int e = tid; e < C * D; e += NT) {
+        const int r = e / D, c = e % D;
+        const float Gr = bG[r * LD + c], ref = tile_ref(bG, r, c);
+        const float kk = bK[r * LD + c], a = __expf(Gr - ref);
+        bW[r * LD + c] = kk * a;
+        bDW[r * LD + c] = bQ[r * LD + c] * a;
+        bDO[r * LD + c] = kk * __expf(ref - Gr);
+        if (r < TILE) bS0[r * LD + c] = kk * __expf(bG[(TILE - 1) * LD + c] - Gr);
+    }
+    __syncthreads();
+    // pair-product gradients: thread rows r0 .. r0 + 3 (one tile), channels lane + 32 j
+    {
+        const int r0 = 4 * (tid >> 5), lane = tid & 31;
+        const int tau = r0 / TILE;
+        const int i0 = tau * TILE;
+        float rk[4][4], rq[4][4], ck_s[4][4], ck_x[4][4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) rk[u][j] = rq[u][j] = ck_s[u][j] = ck_x[u][j] = 0.f;
+        // same tile: row role over columns i, column role over rows rr, both in [i0, i0 + 16)
+#pragma unroll 4
+        for (int ii = 0; ii < TILE; ++ii) {
+            const int i = i0 + ii;
+            float kf[4], ka[4], qa[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int c = lane + 32 * j;
+                kf[j] = bDO[i * LD + c];
+                ka[j] = bW[i * LD + c];
+                qa[j] = bDW[i * LD + c];
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float dar = sdT[(r0 + u) * L32 + i], dpr = sdP[(r0 + u) * L32 + i];   // (row r, col i)
+                const float dac = sdT[i * L32 + r0 + u], dpc = sdP[i * L32 + r0 + u];       // (row i, col r)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    rk[u][j] = fmaf(dar, kf[j], rk[u][j]);
+                    rq[u][j] = fmaf(dpr, kf[j], rq[u][j]);
+                    ck_s[u][j] = fmaf(dac, ka[j], fmaf(dpc, qa[j], ck_s[u][j]));
+                }
+            }
+        }
+        if (tau == 1) {       // rows of tile 1 against columns of tile 0 (row role)
+#pragma unroll 4
+            for (int i = 0; i < TILE; ++i) {
+                float kc[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) kc[j] = bS0[i * LD + lane + 32 * j];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float dar = sdT[(r0 + u) * L32 + i], dpr = sdP[(r0 + u) * L32 + i];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        rk[u][j] = fmaf(dar, kc[j], rk[u][j]);
+                        rq[u][j] = fmaf(dpr, kc[j], rq[u][j]);
+                    }
+                }
+            }
+        } else {              // columns of tile 0 against rows of tile 1 (column role)
+#pragma unroll 4
+            for (int rr = TILE; rr < C; ++rr) {
+                float ka[4], qa[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    ka[j] = bW[rr * LD + lane + 32 * j];
+                    qa[j] = bDW[rr * LD + lane + 32 * j];
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float dac = sdT[rr * L32 + r0 + u], dpc = sdP[rr * L32 + r0 + u];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) ck_x[u][j] = fmaf(dac, ka[j], fmaf(dpc, qa[j], ck_x[u][j]));
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = r0 + u;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int c = lane + 32 * j;
+                const float Gr = bG[r * LD + c], ref = tile_ref(bG, r, c);
+                const float a = __expf(Gr - ref), bfac = __expf(ref - Gr);
+                float colk = ck_s[u][j] * bfac;
+                if (tau == 0) colk = fmaf(ck_x[u][j], __expf(bG[(TILE - 1) * LD + c] - Gr), colk);
+                const float rowk = rk[u][j] * a, rowq = rq[u][j] * a;
+                const float kk = bK[r * LD + c], qq = bQ[r * LD + c];
+                bDKB[r * LD + c] += rowk + colk;
+                bDQT[r * LD + c] += rowq;
+                bV[r * LD + c] += kk * (rowk - colk) + qq * rowq;
+            }
+        }
+    }
+    __syncthreads();
+    // the chunk's last token carries the terms of Gam_C; dg = reverse running sum
+    if (tid < D) {
+        const int c = tid;
+        const float gl = bG[(C - 1) * LD + c];
+        bV[(C - 1) * LD + c] += sKS[c] + sRS[c] * __expf(gl);
+        float s = 0.f;
+        for (int r = C - 1; r >= 0; --r) {
+            s += bV[r * LD + c];
+            bV[r * LD + c] = s;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < C * D; e += NT) {
+        const int r = e / D, c = e % D;
+        if (r < Tl) {
+            const int64_t o = row0 + (int64_t)r * rs + c;
+            dq[o] = to_bf(bDQT[r * LD + c]);
+            dk[o] = to_bf(bDKB[r * LD + c]);
+            dg[o] = to_bf(bV[r * LD + c]);
+        }
+    }
+    if (tid < Tl) dbeta[((int64_t)b * T + t0 + tid) * H + h] = to_bf(sDB[tid]);
+}
+
+}  // namespace bw
+
+static DeviceFlags g_bwd_attr_done;
+
+cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                             const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv,
+                             void* dg, void* dbeta, float* dh0, int B, int T, int H, cudaStream_t stream)
+{
+    using namespace bw;
+    cudaError_t e = once_per_device(g_bwd_attr_done, [](int) {
+        const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+        cudaError_t r = cudaFuncSetAttribute(bwd_prep_kernel, a, (int)PREP_SMEM);
+        if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_chain_kernel<false>, a, (int)CHAIN_SMEM);
+        if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_chain_kernel<true>, a, (int)CHAIN_SMEM);
+        if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_local_kernel, a, (int)LOC_SMEM);
+        return r;
+    });
+    if (e != cudaSuccess) return e;
+    const size_t state_bytes = (size_t)D * D * sizeof(float);
+    if (T == 0) {        // no token: the start-state gradient is the end-state gradient
+        if (!dh0) return cudaSuccess;
+        return dhT ? cudaMemcpyAsync(dh0, dhT, (size_t)B * H * state_bytes, cudaMemcpyDeviceToDevice, stream)
+                   : cudaMemsetAsync(dh0, 0, (size_t)B * H * state_bytes, stream);
+    }
+    const int n_chunks = (T + C - 1) / C;
+    const size_t units = (size_t)B * H * n_chunks;
+    const size_t bytes = units * ((size_t)R_FLOATS * sizeof(float) + 2 * state_bytes);
+    float* ws = nullptr;
+    e = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
+    if (e != cudaSuccess) return e;
+    float* rec = ws;
+    float* S0_all = rec + units * R_FLOATS;
+    float* dS_all = S0_all + units * D * D;
+    const dim3 grid_c((unsigned)n_chunks, (unsigned)H, (unsigned)B);
+    const dim3 grid_s((unsigned)(D / NS), (unsigned)H, (unsigned)B);
+    const __nv_bfloat16* bq = (const __nv_bfloat16*)q;
+    const __nv_bfloat16* bk = (const __nv_bfloat16*)k;
+    const __nv_bfloat16* bv = (const __nv_bfloat16*)v;
+    const __nv_bfloat16* bg = (const __nv_bfloat16*)g;
+    const __nv_bfloat16* bb = (const __nv_bfloat16*)beta;
+    const __nv_bfloat16* bdo = (const __nv_bfloat16*)dO;
+    bwd_prep_kernel<<<grid_c, NT, PREP_SMEM, stream>>>(bq, bk, bv, bg, bb, rec, T, H, n_chunks);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) {
+        bwd_chain_kernel<false><<<grid_s, NT, CHAIN_SMEM, stream>>>(rec, bdo, h0, S0_all, nullptr, T, H, n_chunks);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) {
+        bwd_chain_kernel<true><<<grid_s, NT, CHAIN_SMEM, stream>>>(rec, bdo, dhT, dS_all, dh0, T, H, n_chunks);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) {
+        bwd_local_kernel<<<grid_c, NT, LOC_SMEM, stream>>>(
+            bq, bk, bv, bg, bb, bdo, rec, S0_all, dS_all, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk,
+            (__nv_bfloat16*)dv, (__nv_bfloat16*)dg, (__nv_bfloat16*)dbeta, T, H, n_chunks);
+        e = cudaGetLastError();
+    }
+    const cudaError_t ef = cudaFreeAsync(ws, stream);
+    if (e == cudaSuccess) e = ef;
+    note_launches(4);
+    return e;
+}
+
+}  // namespace kda

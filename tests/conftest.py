@@ -23,3 +23,20 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(autouse=True)
+def _name_reports(request):
+    import tolerance
+    tolerance.CURRENT_TEST[0] = request.node.nodeid
+    yield
+
+
+def pytest_terminal_summary(terminalreporter):
+    """The error report of every bf16 output checked in this session."""
+    import tolerance
+    if not tolerance.REPORTS:
+        return
+    terminalreporter.section("bf16 output errors (plain / floor / relaxed / excess)")
+    for test, what, rep in tolerance.REPORTS:
+        terminalreporter.write_line("%s [%s] %s" % (test, what, tolerance.fmt_report(rep)))

@@ -155,6 +155,66 @@ def test_decode_argument_errors(lib):
     assert lib.kda_launch_count() == n0
 
 
+def test_backward_argument_errors(lib):
+    """kda_chunk_bwd: host checks, no launch."""
+    n0 = lib.kda_launch_count()
+
+    def bwd(q=A, dO=A, dhT=NUL, dq=A, dk=A, dv=A, dg=A, dbeta=A2, dh0=A, B=1, T=64, H=2, d_k=128, d_v=128):
+        return lib.kda_chunk_bwd(q, A, A, A, A2, NUL, dO, dhT, dq, dk, dv, dg, dbeta, dh0,
+                                 B, T, H, d_k, d_v, None)
+
+    assert bwd(q=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(dO=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(dq=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(dg=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(dbeta=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(dbeta=ctypes.c_void_p(0x20001)) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(dh0=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(dhT=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(T=-1) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(d_k=64, d_v=64) == kda.KDA_ERR_UNSUPPORTED
+    assert bwd(B=0) == kda.KDA_OK
+    assert bwd(T=0, dh0=NUL) == kda.KDA_OK                 # nothing to write
+    assert lib.kda_launch_count() == n0
+
+
+def test_verify_argument_errors(lib):
+    """kda_verify_fwd: host checks, no launch."""
+    n0 = lib.kda_launch_count()
+
+    def ver(q=A, k=A, v=A, g=A, beta=A2, h0=NUL, o=A, states=A, N=3, K=8, H=2, dk=128, dv=128):
+        return lib.kda_verify_fwd(q, k, v, g, beta, h0, o, states, N, K, H, dk, dv, None)
+
+    assert ver(states=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert ver(states=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert ver(h0=MIS) == kda.KDA_ERR_INVALID_ARG
+    assert ver(o=NUL) == kda.KDA_ERR_INVALID_ARG
+    assert ver(beta=ctypes.c_void_p(0x20001)) == kda.KDA_ERR_INVALID_ARG
+    assert ver(K=-1) == kda.KDA_ERR_INVALID_ARG
+    assert ver(K=kda.VERIFY_MAX_TOKENS + 1) == kda.KDA_ERR_UNSUPPORTED
+    assert ver(dk=96) == kda.KDA_ERR_UNSUPPORTED
+    assert ver(K=0, q=NUL, states=NUL) == kda.KDA_OK
+    assert ver(N=0) == kda.KDA_OK
+    assert lib.kda_launch_count() == n0
+
+
+def test_verify_max_tokens_matches_header(lib):
+    with open(HEADER) as f:
+        m = re.search(r"#define\s+KDA_VERIFY_MAX_TOKENS\s+(\d+)", f.read())
+    assert m and int(m.group(1)) == kda.VERIFY_MAX_TOKENS
+
+
+def test_prefill_path_query(lib):
+    """kda_prefill_path launches nothing; without a GPU the SM count falls
+    back to the B200's 148."""
+    n0 = lib.kda_launch_count()
+    assert lib.kda_prefill_path(-1, 16, 2) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_prefill_path(4, 65536, 32) == 0          # 128 heads: one SM per head
+    assert lib.kda_prefill_path(1, 8192, 32) == 1           # 32 heads: clusters of four SMs
+    assert lib.kda_prefill_path(1, 1 << 20, 2) == 2         # two heads, long: segment scan
+    assert lib.kda_launch_count() == n0
+
+
 def test_selftest_limit_checked_on_host(lib):
     n0 = lib.kda_launch_count()
     assert lib.kda_selftest_bounded_wait(0, None) == kda.KDA_ERR_INVALID_ARG
@@ -185,6 +245,8 @@ def test_binding_requires_cuda_tensors(lib):
         lambda: kda.chunk_fwd_f32(xf, xf, xf, xf, bf),
         lambda: kda.decode_step(d, d, d, d, db, st),
         lambda: kda.decode_step_raw(d, d, d, d, db, st),
+        lambda: kda.verify_fwd(x, x, x, x, b),
+        lambda: kda.chunk_bwd(x, x, x, x, b, None, x),
     ]
     for call in calls:
         with pytest.raises(ValueError, match="CUDA"):
