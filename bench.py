@@ -64,6 +64,28 @@ def prefill_alg_flops(B, T, H, dk, dv, C=16):
     return B * T * H * per
 
 
+def backward_alg_bytes(B, T, H, dk, dv):
+    """Algorithmic HBM bytes of one backward: q, k, g, v, beta and dO read
+    once, dq, dk, dg, dv and dbeta written once (bf16); h0 and dhT read and
+    dh0 written (fp32)."""
+    per_token_head = (3 * dk + dv + 1 + dv) * BYTES_BF16 + (3 * dk + dv + 1) * BYTES_BF16
+    return B * T * H * per_token_head + 3 * B * H * dk * dv * 4
+
+
+def backward_alg_flops(B, T, H, dk, dv, C=32):
+    """Flops of the chunked backward as computed (32-token chunks; FMA = 2
+    flops): per chunk, the operand preparation (pair products, W, U', P W:
+    ~4 C^2 d), the forward state chain (2 C d^2), the reverse chain
+    (3 C d^2) and the chunk-local products (7 C d^2 + ~10 C^2 d)."""
+    per_chunk = 2 * (4 * C * C * dk + 2 * C * dk * dv + 3 * C * dk * dv + 7 * C * dk * dv + 10 * C * C * dk)
+    return B * H * ((T + C - 1) // C) * per_chunk
+
+
+def alu_peak_tflops(sm_mhz=1965.0, sms=148):
+    """fp32 FMA peak of the CUDA cores: SMs x 128 lanes x 2 flops x clock."""
+    return sms * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
 def decode_alg_bytes(N, H, dk, dv):
     """Per decode step: state read + written (fp32), q, k, g, v, beta read,
     o written (bf16)."""
@@ -358,6 +380,8 @@ def bench_kda(args, rank, world, local):
 
     if args.decode:
         result["decode"] = bench_decode(args, kda, dev, rank, world, hbm_gbs, peak_src)
+    if args.backward and not args.small_footprint:
+        result["backward"] = bench_backward(args, kda, dev, rank, world, hbm_gbs, peak_src)
     # the other prefill workloads of the pages' length range, each timed the
     # same way on its own inputs (each input set is far larger than L2)
     if not args.small_footprint:
@@ -366,6 +390,65 @@ def bench_kda(args, rank, world, local):
                 result[name] = bench_prefill_workload(args, kda, dev, rank, world, name,
                                                       hbm_gbs, bf16_tf, peak_src)
     return result
+
+
+def bench_backward(args, kda, dev, rank, world, hbm_gbs, peak_src):
+    """kda_chunk_bwd on the 8K workload's shape (B1 H32 T8192, the shortest
+    pre-training length), with both cotangents, timed like the prefill."""
+    import torch
+    from linear_attention_07_b200.inputs import WORKLOADS, prefill_inputs
+    w = WORKLOADS["prefill_8k"]
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    x = prefill_inputs(B, T, H, dk, dv, seed=rank_seed(w.seed + 99, rank), device=dev, h0_std=w.h0_std)
+    gen = torch.Generator(device=dev).manual_seed(rank_seed(w.seed + 98, rank))
+    dO = torch.randn((B, T, H, dv), generator=gen, device=dev).to(torch.bfloat16)
+    dhT = torch.randn((B, H, dk, dv), generator=gen, device=dev) * 0.1
+
+    def step(i):
+        kda.chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"], dO, dhT)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    steps = max(3, min(args.steps, 10))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        keep_busy(step, 0.3, torch.cuda.synchronize)
+        barrier(dev)
+        torch.cuda.synchronize()
+        n0 = kda.launch_count()
+        ev[0].record(stream)
+        for i in range(steps):
+            step(i)
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        launches = kda.launch_count() - n0
+        barrier(dev)
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), dev)
+    mean_ms = statistics.mean(per_step)
+    alg_b = backward_alg_bytes(B, T, H, dk, dv)
+    alg_f = backward_alg_flops(B, T, H, dk, dv)
+    csum = clk.summary()
+    sm_mhz = csum.get("sm_mhz") or 1965.0
+    peak_alu = alu_peak_tflops(sm_mhz)
+    ach_f = alg_f / (mean_ms / 1e3) / 1e12
+    ach_b = alg_b / (mean_ms / 1e3) / 1e9
+    out = {"metric": "KDA backward tokens/s (B1 H32 T8192 d128, bf16 in/out, fp32 arithmetic)",
+           "value": round(B * T * world * steps / (total_ms / 1e3), 1), "unit": "tokens/s",
+           "ms_per_step": round(total_ms / steps, 4), "steps": steps, "warmup": args.warmup,
+           "roofline": {"bound": "alu", "achieved": round(ach_f, 2), "peak": round(peak_alu, 1),
+                        "unit": "TFLOP/s", "frac": round(ach_f / peak_alu, 4), "traffic": None,
+                        "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x median SM clock",
+                        "alg_flops_per_launch": alg_f, "kernel": "kda_chunk_bwd (4 launches)"},
+           "hbm": {"achieved": round(ach_b, 1), "peak": hbm_gbs, "unit": "GB/s",
+                   "frac": round(ach_b / hbm_gbs, 4), "alg_bytes_per_launch": alg_b,
+                   "peak_source": peak_src + " hbm_gbs"},
+           "gpu_launches": int(launches), "clocks": csum}
+    del x, dO, dhT
+    torch.cuda.empty_cache()
+    return out
 
 
 def bench_prefill_workload(args, kda, dev, rank, world, name, hbm_gbs, bf16_tf, peak_src):
@@ -688,6 +771,8 @@ def main(argv=None):
                     type=lambda x: [y for y in x.split(",") if y],
                     help="other prefill workloads timed in the same run, reported as sub-objects "
                          "(comma-separated names; empty: none)")
+    ap.add_argument("--no-backward", dest="backward", action="store_false",
+                    help="skip the backward (kda_chunk_bwd) line")
     ap.add_argument("--small-footprint", action="store_true",
                     help="for profiler captures: one prefill input set, 16 decode steps, "
                          "no end-to-end leg and no other workloads")

@@ -243,7 +243,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                   const __nv_bfloat16* __restrict__ beta, const float* h0,
                   __nv_bfloat16* __restrict__ o, float* hT, int T, int H,
-                  int seg_len, int n_seg, uint32_t flags, float* states, int snap_every)
+                  int seg_len, int n_seg, uint32_t flags, float* states, int snap_every,
+                  uint64_t wait_ns)
 {
     using namespace pf;
     using namespace tc;
@@ -297,12 +298,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         uint32_t phase = 0;
         // one thread polls the MMA barrier; the others block on a named barrier
         auto wait_mma = [&]() {
-            if (tid == 0 && !s_abort && !mbar_wait(bar, phase & 1u, WAIT_NS)) expired();
+            if (tid == 0 && !s_abort && !mbar_wait(bar, phase & 1u, wait_ns)) expired();
             ++phase;
             __syncwarp();
             named_bar(BAR_CHAIN, NCH);
             fence_after_sync();
         };
+        uint32_t n_commit = 0;               // commits on `bar` issued by this (issuing) thread
         float S[D / 2];
         {
             const float* h0h = (h0 && !(flags & SEG_H0_EYE)) ? h0 + head_off * D * D : nullptr;
@@ -336,6 +338,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     mma_tf32_ts_w(tm + T_DX, tm + T_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
                                   id, ks > 0 ? 1u : 0u);
                 mma_commit_w(bar);
+                ++n_commit;
             }
             wait_mma();
             {   // U = U' - W S  (this half: tokens [16 hh, 16 hh + 16))
@@ -364,6 +367,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                   id3, 1u);
                 }
                 mma_commit_w(bar);
+                ++n_commit;
             }
             wait_mma();
             // B1, B2, B3 are no longer read: the prep may fill the next chunk's
@@ -422,6 +426,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
             for (int i = 0; i < D / 2; ++i) hTh[(int64_t)(64 * hh + i) * D + j] = S[i];
         }
+        // After an expired wait, the MMAs of the last commit may still run:
+        // let them finish before tensor memory is released (the issuing thread
+        // is also the waiting thread, so at most one commit is outstanding).
+        if (tid == 0 && *(volatile int*)&s_abort && n_commit > 0)
+            mbar_wait(bar, (n_commit - 1) & 1u, DRAIN_NS);
     } else {
         // ==================================================== prep warpgroups ==
         const int pt = tid - NCH;                  // 0..255
@@ -429,17 +438,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t bar = smem_u32(&s_bar[1]);
         const uint32_t rbar = smem_u32(&s_bar[2]);
         uint32_t phase = 0, rphase = 0;
+        uint32_t n_commit = 0, n_loads = 0;    // issued by pt == 0 (also the waiting thread)
         auto wait_mma = [&]() {
-            if (pt == 0 && !s_abort && !mbar_wait(bar, phase & 1u, WAIT_NS)) expired();
+            if (pt == 0 && !s_abort && !mbar_wait(bar, phase & 1u, wait_ns)) expired();
             ++phase;
             __syncwarp();
             named_bar(BAR_PREP, NPREP);
             fence_after_sync();
         };
         auto prep_sync = [&]() { named_bar(BAR_PREP, NPREP); };
-        // TMA: chunk ci's q, k, v, g rows (32 x 128 bf16 each; rows past T are zero)
+        // TMA: chunk ci's q, k, v, g rows (32 x 128 bf16 each; rows past T are zero);
+        // none after an expired wait (the raw buffer may still be in use)
         auto issue_raw = [&](int ci) {
-            if (pt == 0) {
+            if (pt == 0 && !*(volatile int*)&s_abort) {
+                ++n_loads;
                 mbar_arrive_expect_tx(rbar, 4 * RAW_T);
                 tma_load_3d(smem_u32(sm + RAW + 0 * RAW_T), &tm_q, h * D, ts + ci * C, b, rbar);
                 tma_load_3d(smem_u32(sm + RAW + 1 * RAW_T), &tm_k, h * D, ts + ci * C, b, rbar);
@@ -470,7 +482,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int tn = (ch + 1) * C + pt;
                 beta_next = (tn < Tl) ? beta[((int64_t)b * T + ts + tn) * H + h] : bzero;
             }
-            if (pt == 0 && !s_abort && !mbar_wait(rbar, rphase & 1u, WAIT_NS)) expired();
+            if (pt == 0 && !s_abort && !mbar_wait(rbar, rphase & 1u, wait_ns)) expired();
             ++rphase;
             __syncwarp();
             prep_sync();
@@ -559,6 +571,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     mma_tf32_ss_w(tm + T_DG, ad0 + step, bd0 + step, id, ks > 0 ? 1u : 0u);
                 }
                 mma_commit_w(bar);
+                ++n_commit;
             }
             if (ch + 1 < n_chunks) issue_raw(ch + 1);
 #pragma unroll
@@ -661,6 +674,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     mma_tf32_ss_w(du, av0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
                 }
                 mma_commit_w(bar);
+                ++n_commit;
             }
             // operands of the fill that do not come from the W MMA, read now
             const float* gaf = reinterpret_cast<const float*>(sm + GA);
@@ -713,6 +727,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             fence_smem_to_async();
             fence_before_sync();
             named_arrive(BAR_READY, NT);
+        }
+        // after an expired wait: the last MMAs and input load may still be in
+        // flight; let them land before tensor and shared memory are released
+        if (pt == 0 && *(volatile int*)&s_abort) {
+            if (n_commit > 0) mbar_wait(bar, (n_commit - 1) & 1u, DRAIN_NS);
+            if (n_loads > 0) mbar_wait(rbar, (n_loads - 1) & 1u, DRAIN_NS);
         }
     }
 
@@ -787,7 +807,8 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                        const __nv_bfloat16* __restrict__ beta, const float* h0,
                        __nv_bfloat16* __restrict__ o, float* hT, int T, int H,
-                       int seg_len, int n_seg, uint32_t flags, float* states, int snap_every)
+                       int seg_len, int n_seg, uint32_t flags, float* states, int snap_every,
+                       uint64_t wait_ns)
 {
     using namespace pc;
     using namespace tc;
@@ -853,6 +874,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             const uint32_t id1 = idesc_tf32(128, 2 * C, false, false);
             const uint32_t id2 = idesc_tf32(128, 64, false, false);
             const uint32_t id3 = idesc_tf32(128, 32, false, false);
+            uint32_t n_x = 0, n_k0 = 0, n_k1 = 0;   // commits on mbar, kbar0, kbar1
 #pragma unroll 1
             for (int ch = 0; ch < n_chunks; ++ch) {
                 const int slot = ch % NPREPCTA;
@@ -860,7 +882,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const uint32_t dx = (ch & 1) ? CT_DX1 : CT_DX0;
                 const uint64_t bd0 = sdesc(smem_u32(sm + sb + S_B1), PAD_LBO, SBO_K128P);
                 if (lane == 0 && !s_abort &&
-                    !mbar_wait_cluster(smem_u32(&s_bar[slot]), (uint32_t)(ch / NPREPCTA) & 1u, WAIT_NS))
+                    !mbar_wait_cluster(smem_u32(&s_bar[slot]), (uint32_t)(ch / NPREPCTA) & 1u, wait_ns))
                     expired();
                 __syncwarp();
                 named_bar(NB_ASA, NX);
@@ -880,6 +902,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                         mma_tf32_ts_w(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
                                       id1, 1u);
                     mma_commit_w(mbar);
+                    ++n_x;
                 }
                 __syncwarp();
                 named_bar(NB_U, NX);
@@ -894,6 +917,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                         mma_tf32_ts_w(tm + CT_DKU, tm + CT_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
                                       id2, ks > 0 ? 1u : 0u);
                     mma_commit_w(kbar0);
+                    ++n_k0;
 #pragma unroll
                     for (int ks = 0; ks < C / 8; ++ks)
                         mma_tf32_ts_w(tm + CT_DKU + 64, tm + CT_AU + ks * 8, b21 + (uint64_t)((ks * 2 * LBO) >> 4),
@@ -903,9 +927,19 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                         mma_tf32_ts_w(tm + dx + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * LBO) >> 4),
                                       id3, 1u);
                     mma_commit_w(kbar1);
+                    ++n_k1;
                 }
                 __syncwarp();
             }
+            // after an expired wait: the last commit of each barrier (at most
+            // one is outstanding: each is waited before the next is issued)
+            // must complete before tensor memory is released
+            if (lane == 0 && *(volatile int*)&s_abort) {
+                if (n_x > 0) mbar_wait(mbar, (n_x - 1) & 1u, DRAIN_NS);
+                if (n_k0 > 0) mbar_wait(kbar0, (n_k0 - 1) & 1u, DRAIN_NS);
+                if (n_k1 > 0) mbar_wait(kbar1, (n_k1 - 1) & 1u, DRAIN_NS);
+            }
+            __syncwarp();
         } else if (warp == NCW / 32 + 1) {
             // ------------------------------------------------------ release warp --
             // Once chunk ch - 1's last MMAs are done (and its decay applied),
@@ -917,7 +951,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 #pragma unroll 1
             for (int ch = 1; ch < n_chunks; ++ch) {
                 if (lane == 0) {
-                    if (!s_abort && !counter_wait(smem_u32(&s_odone), (uint32_t)ch, WAIT_NS)) expired();
+                    if (!s_abort && !counter_wait(smem_u32(&s_odone), (uint32_t)ch, wait_ns)) expired();
                     // After an expired wait no slot is handed back (its previous
                     // bytes may still be on their way): the preparers then give up
                     // on their own bounded waits, and at most one push per slot is
@@ -947,7 +981,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             uint32_t phase = 0;
             auto cw_bar = [&]() { named_bar(NB_CW, NCW); };
             auto wait_bar = [&](uint32_t bar, uint32_t parity) {
-                if (tid == 0 && !s_abort && !mbar_wait(bar, parity, WAIT_NS)) expired();
+                if (tid == 0 && !s_abort && !mbar_wait(bar, parity, wait_ns)) expired();
                 __syncwarp();
                 cw_bar();
                 fence_after_sync();
@@ -1048,7 +1082,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 }
                 // X of chunk ch (U' of this chunk is in the slot once its FULL phase passed)
                 if (tid == 0 && !s_abort &&
-                    !mbar_wait_cluster(smem_u32(&s_bar[slot]), (uint32_t)(ch / NPREPCTA) & 1u, WAIT_NS))
+                    !mbar_wait_cluster(smem_u32(&s_bar[slot]), (uint32_t)(ch / NPREPCTA) & 1u, wait_ns))
                     expired();
                 wait_bar(mbar, phase & 1u);
                 ++phase;
@@ -1093,7 +1127,11 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             // ------------------------------------------------------ issuer warp --
             // MMAs and input loads: the compute warps hand over at named
             // barriers and never wait on an issue.
+            uint32_t n_commit = 0, n_loads = 0;
+            // no new load after an expired wait (the raw buffer may still be read)
             auto issue_raw = [&](int ci) {
+                if (*(volatile int*)&s_abort) return;
+                ++n_loads;
                 mbar_arrive_expect_tx(rbar, 4 * RAW_T);
                 tma_load_3d(smem_u32(sm + P_RAW + 0 * RAW_T), &tm_q, h * D, ts + ci * C, b, rbar);
                 tma_load_3d(smem_u32(sm + P_RAW + 1 * RAW_T), &tm_k, h * D, ts + ci * C, b, rbar);
@@ -1116,6 +1154,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                         mma_tf32_ss_w(tm + PT_DG, ad0 + step, bd0 + step, id, ks > 0 ? 1u : 0u);
                     }
                     mma_commit_w(mbar);
+                    ++n_commit;
                 }
                 if (lane == 0 && ch + NPREPCTA < n_chunks) issue_raw(ch + NPREPCTA);
                 __syncwarp();
@@ -1134,8 +1173,15 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                         mma_tf32_ss_w(tm + PT_DU, av0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
                     }
                     mma_commit_w(mbar);
+                    ++n_commit;
                 }
             }
+            // after an expired wait: the last MMAs and input load may still be in flight
+            if (lane == 0 && *(volatile int*)&s_abort) {
+                if (n_commit > 0) mbar_wait(mbar, (n_commit - 1) & 1u, DRAIN_NS);
+                if (n_loads > 0) mbar_wait(rbar, (n_loads - 1) & 1u, DRAIN_NS);
+            }
+            __syncwarp();
         } else if (warp == NCW / 32 + 1) {
             // --------------------------------------------------------- push warp --
             // Each prepared chunk goes to its slot in the chain CTA as one bulk
@@ -1149,7 +1195,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 named_bar(NB_FILL, NX);               // the staging holds chunk ch
                 if (lane == 0) {
                     // the chain has released this slot (its previous use, chunk ch - NPREPCTA)
-                    if (ch >= NPREPCTA && !s_abort && !mbar_wait_cluster(ebar, ephase & 1u, WAIT_NS)) expired();
+                    if (ch >= NPREPCTA && !s_abort && !mbar_wait_cluster(ebar, ephase & 1u, wait_ns)) expired();
                     if (ch >= NPREPCTA) ++ephase;
                     if (!s_abort) {                   // FULL was armed by the chain
                         bulk_copy_to_rank(slot_remote, smem_u32(st), SLOT, full_remote);
@@ -1167,7 +1213,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         uint32_t phase = 0, rphase = 0;
         auto prep_sync = [&]() { named_bar(NB_CW, NCW); };
         auto wait_mma = [&]() {
-            if (pt == 0 && !s_abort && !mbar_wait(mbar, phase & 1u, WAIT_NS)) expired();
+            if (pt == 0 && !s_abort && !mbar_wait(mbar, phase & 1u, wait_ns)) expired();
             ++phase;
             __syncwarp();
             prep_sync();
@@ -1190,7 +1236,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const int tn = (ch + NPREPCTA) * C + pt;
                 beta_next = (tn < Tl) ? beta[((int64_t)b * T + ts + tn) * H + h] : bzero;
             }
-            if (pt == 0 && !s_abort && !mbar_wait(rbar, rphase & 1u, WAIT_NS)) expired();
+            if (pt == 0 && !s_abort && !mbar_wait(rbar, rphase & 1u, wait_ns)) expired();
             ++rphase;
             __syncwarp();
             prep_sync();
@@ -1460,6 +1506,21 @@ static int64_t sm_count()
 // up to SMs / 4 heads (37 on a B200); larger batches use one SM per head.
 static bool cluster_fits(int64_t heads) { return heads * (pc::NPREPCTA + 1) <= sm_count(); }
 
+// Bounded waits give up after 2 s; KDA_WAIT_LIMIT_NS (0 .. 2e9 ns) shortens
+// the limit for tests that make the prefill's own waits run out.  With 0 a
+// wait checks its phase once, without blocking, and gives up if it has not
+// completed: the first wait for an input load or for a chunk pushed by
+// another SM then gives up, since neither can land in the few hundred cycles
+// between its issue and the check.  The drain after an expired wait keeps
+// its own 20 ms limit.
+static uint64_t wait_limit_ns()
+{
+    const char* env = getenv("KDA_WAIT_LIMIT_NS");
+    if (!env || !*env) return pf::WAIT_NS;
+    const unsigned long long v = strtoull(env, nullptr, 10);
+    return v > pf::WAIT_NS ? pf::WAIT_NS : (uint64_t)v;
+}
+
 // One launch of either variant over B * n_seg segment-sequences of length
 // seg_len (n_seg = 1, seg_len = T: the plain prefill).
 static cudaError_t launch_pass(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -1473,13 +1534,13 @@ static cudaError_t launch_pass(const CUtensorMap& mq, const CUtensorMap& mk, con
         auto kern = pro ? prefill_cluster_kernel<true> : prefill_cluster_kernel<false>;
         kern<<<grid, pc::NTH, pc::SMEM_BYTES, stream>>>(
             mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags,
-            states, snap_every);
+            states, snap_every, wait_limit_ns());
     } else {
         dim3 grid(H, B * n_seg);
         auto kern = pro ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
         kern<<<grid, pf::NT, pf::SMEM_BYTES, stream>>>(
             mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags,
-            states, snap_every);
+            states, snap_every, wait_limit_ns());
     }
     return cudaGetLastError();
 }

@@ -155,7 +155,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // returns false.  No suspend-time hint is given: with a long hint the waiting
 // thread wakes measurably later (a few hundred cycles) after the phase
 // completes.  Returns true on success, false on timeout.
+// Non-blocking check of phase `parity` (mbarrier.test_wait).
+__device__ __forceinline__ uint32_t mbar_test_wait(uint32_t saddr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok) : "r"(saddr), "r"(parity) : "memory");
+    return ok;
+}
+// A limit of 0 checks once without blocking (tests that make waits run out).
 __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, uint64_t limit_ns) {
+    if (limit_ns == 0) return mbar_test_wait(saddr, parity);
     if (mbar_try_wait(saddr, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(saddr, parity)) {
@@ -178,6 +190,7 @@ __device__ __forceinline__ uint32_t counter_read(uint32_t saddr) {
 // Wait until the counter reaches `target`; false once limit_ns has passed.
 __device__ __forceinline__ bool counter_wait(uint32_t saddr, uint32_t target, uint64_t limit_ns) {
     if (counter_read(saddr) >= target) return true;
+    if (limit_ns == 0) return false;
     const uint64_t t0 = globaltimer_ns();
     while (counter_read(saddr) < target) {
         if (globaltimer_ns() - t0 > limit_ns) return false;
@@ -238,7 +251,17 @@ __device__ __forceinline__ uint32_t mbar_try_wait_cluster(uint32_t saddr, uint32
         : "=r"(ok) : "r"(saddr), "r"(parity) : "memory");
     return ok;
 }
+__device__ __forceinline__ uint32_t mbar_test_wait_cluster(uint32_t saddr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok) : "r"(saddr), "r"(parity) : "memory");
+    return ok;
+}
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t saddr, uint32_t parity, uint64_t limit_ns) {
+    if (limit_ns == 0) return mbar_test_wait_cluster(saddr, parity);
     if (mbar_try_wait_cluster(saddr, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait_cluster(saddr, parity)) {
