@@ -773,6 +773,8 @@ def main(argv=None):
                          "(comma-separated names; empty: none)")
     ap.add_argument("--no-backward", dest="backward", action="store_false",
                     help="skip the backward (kda_chunk_bwd) line")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the backward (for profiler captures); prints its line alone")
     ap.add_argument("--small-footprint", action="store_true",
                     help="for profiler captures: one prefill input set, 16 decode steps, "
                          "no end-to-end leg and no other workloads")
@@ -799,6 +801,16 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     try:
+        if args.backward_only:
+            import linear_attention_07_b200 as kda
+            dev = torch.device("cuda", local)
+            torch.cuda.set_device(dev)
+            kda.load_library()
+            hbm_gbs, _, peak_src = load_peaks()
+            res = bench_backward(args, kda, dev, rank, world, hbm_gbs, peak_src)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return 0
         res = bench_kda(args, rank, world, local)
         if rank == 0 and args.cpu_base:
             res["cpu_baseline"] = cpu_baseline(args)
