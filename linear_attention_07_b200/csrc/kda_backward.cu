@@ -186,48 +186,42 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         if (r < TILE) s4[r * LD + c] = kk * __expf(sG[(TILE - 1) * LD + c] - Gr);   // Kc (<= 1)
     }
     __syncthreads();
-    // Araw (strict lower) and Praw (lower incl): one warp per pair, lanes over channels
+    // Araw (strict lower) and Praw (lower incl) as block products: pairs inside
+    // one tile from Ka / Qa against Kf (the full 32 x 32 product is finite:
+    // the entries of mixed tiles, whose factors do not belong together, are
+    // dropped), pairs across the tiles (rows of tile 1, columns of tile 0)
+    // from Ka / Qa against Kc
     {
-        const int w = tid >> 5, lane = tid & 31;
-        for (int p = w; p < C * (C + 1) / 2; p += NT / 32) {
-            int r = 0, base = 0;
-            while (base + r + 1 <= p) { base += r + 1; ++r; }
-            const int i = p - base;                               // i <= r
-            const float* R = (r / TILE == i / TILE) ? s3 : s4;
-            float sa = 0.f, sp = 0.f;
-#pragma unroll
-            for (int j = 0; j < D / 32; ++j) {
-                const int c = lane + 32 * j;
-                const float rv = R[i * LD + c];
-                sa = fmaf(s1[r * LD + c], rv, sa);
-                sp = fmaf(s2[r * LD + c], rv, sp);
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                sa += __shfl_xor_sync(0xffffffffu, sa, off);
-                sp += __shfl_xor_sync(0xffffffffu, sp, off);
-            }
-            if (lane == 0) {
-                sA[r * L32 + i] = i < r ? sa : 0.f;
-                sP[r * L32 + i] = sp;
-                if (i < r) {
-                    sA[i * L32 + r] = 0.f;
-                    sP[i * L32 + r] = 0.f;
-                }
-            }
-        }
-        if (tid < C) sA[tid * L32 + tid] = 0.f;
+        auto same = [&](float* dst, const float* L, bool strict) {
+            tgemm<C, C, D, 4, 1>([&](int m, int kk) { return L[m * LD + kk]; },
+                                 [&](int kk, int n) { return s3[n * LD + kk]; },
+                                 [&](int m, int n, float x) {
+                                     if (m / TILE == n / TILE) dst[m * L32 + n] = (n < m || (!strict && n == m)) ? x : 0.f;
+                                     else if (n > m) dst[m * L32 + n] = 0.f;
+                                 });
+        };
+        auto cross = [&](float* dst, const float* L) {
+            tgemm<TILE, TILE, D, 1, 1>([&](int m, int kk) { return L[(TILE + m) * LD + kk]; },
+                                       [&](int kk, int n) { return s4[n * LD + kk]; },
+                                       [&](int m, int n, float x) { dst[(TILE + m) * L32 + n] = x; });
+        };
+        same(sA, s1, true);
+        same(sP, s2, false);
+        cross(sA, s1);
+        cross(sP, s2);
     }
     __syncthreads();
-    // X = (I + diag(beta) Araw)^-1 by forward substitution, one column per thread
+    // X = (I + diag(beta) Araw)^-1 by forward substitution, one column per
+    // thread (four partial sums per row keep the chain short)
     if (tid < C) {
         const int j = tid;
         float x[C];
 #pragma unroll
         for (int r = 0; r < C; ++r) {
-            float s = 0.f;
+            float s4v[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < r; ++i) s = fmaf(sA[r * L32 + i], x[i], s);
+            for (int i = 0; i < r; ++i) s4v[i & 3] = fmaf(sA[r * L32 + i], x[i], s4v[i & 3]);
+            const float s = (s4v[0] + s4v[1]) + (s4v[2] + s4v[3]);
             x[r] = (r == j) ? 1.f : (r > j ? -sB[r] * s : 0.f);
         }
 #pragma unroll
@@ -445,10 +439,15 @@ bwd_chain_kernel(const float* __restrict__ rec_all, const __nv_bfloat16* __restr
 }
 
 // ---------------------------------------------------------- local grads --
+// One CTA per chunk.  The state-sized products stream S0 and dS through
+// shared memory twice: by rows (the K dimension of U = Tm V - W S0 and
+// dU = P^T dO + Kb dS, accumulated over the rows), then by columns (the K
+// dimension of dQt = dO S0^T, dKb = U dS^T and dW = -dU S0^T).  Every block
+// product gives each thread a 4 x 4 tile of a 32 x 128 result.
 
-constexpr int LOC_BIG = 9;     // K, Q, V, dO, G, W, dKb, dQt, dW
-constexpr size_t LOC_SMEM = (size_t)(LOC_BIG * C * LD + 2 * D * LJ + 2 * C * LJ + 8 * C * L32 + 2 * C + 2 * D) *
-                            sizeof(float);
+constexpr int LOC_BIG = 11;    // K, Q, V, dO, G, W, U, dU, dKb, dQt, dW
+constexpr int BLK = D * LJ > JB * LD ? D * LJ : JB * LD;    // one S0 or dS block (either shape)
+constexpr size_t LOC_SMEM = (size_t)(LOC_BIG * C * LD + 2 * BLK + 6 * C * L32 + 2 * C + 2 * D) * sizeof(float);
 
 __device__ __forceinline__ __nv_bfloat16 to_bf(float x) { return __float2bfloat16_rn(x); }
 
@@ -463,27 +462,25 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 {
     extern __shared__ __align__(16) float sm[];
     float* bK = sm;
-    float* bQ = bK + C * LD;       // Kb during the column blocks, then Q
+    float* bQ = bK + C * LD;       // Kb during the state products, then Q
     float* bV = bQ + C * LD;       // V, then dGam
-    float* bDO = bV + C * LD;      // dO, then dKt (from W), then Kf
+    float* bDO = bV + C * LD;      // dO, then dKt (from dW), then Kf
     float* bG = bDO + C * LD;      // Gam
     float* bW = bG + C * LD;       // W, then Kt, then Ka
-    float* bDKB = bW + C * LD;     // dKb -> dk
+    float* bU = bW + C * LD;       // U
+    float* bDU = bU + C * LD;      // dU
+    float* bDKB = bDU + C * LD;    // dKb -> dk
     float* bDQT = bDKB + C * LD;   // dQt (direct) -> dq
     float* bDW = bDQT + C * LD;    // dW, then Qa
-    float* bS0 = bDW + C * LD;     // [D][LJ] start-state block, then Kc
-    float* bDS = bS0 + D * LJ;     // [D][LJ] end-gradient block
-    float* bU = bDS + D * LJ;      // [C][LJ]
-    float* bDU = bU + C * LJ;      // [C][LJ]
-    float* sA = bDU + C * LJ;      // Araw
+    float* bS0 = bDW + C * LD;     // a block of S0 (rows: [JB][LD], columns: [D][LJ]), then Kc
+    float* bDS = bS0 + BLK;        // the same block of dS
+    float* sA = bDS + BLK;         // Araw
     float* sP = sA + C * L32;      // Praw (lower incl)
-    float* sX = sP + C * L32;
-    float* sT = sX + C * L32;      // Tm
-    float* sdP = sT + C * L32;     // dO U^T (masked to lower incl after the blocks)
-    float* sdUV = sdP + C * L32;   // dU V^T
+    float* sX = sP + C * L32;      // (I + A)^-1; Tm = X diag(beta) is formed on the fly
+    float* sdP = sX + C * L32;     // dO U^T (masked to lower incl)
+    float* sdUV = sdP + C * L32;   // dU V^T, then dX X^T
     float* sdT = sdUV + C * L32;   // dTm, then dX, then dA (unscaled), then dAr
-    float* sY = sdT + C * L32;     // dX X^T
-    float* sB = sY + C * L32;      // beta [C]
+    float* sB = sdT + C * L32;     // beta [C]
     float* sDB = sB + C;           // dbeta [C]
     float* sRS = sDB + C;          // sum_j dS_ij S0_ij [D]
     float* sKS = sRS + D;          // sum_r dKb_rc Kb_rc [D]
@@ -498,6 +495,7 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     const float* rec = rec_all + (bh * n_chunks + c_idx) * R_FLOATS;
     const float* S0 = S0_all + (bh * n_chunks + c_idx) * D * D;
     const float* dS = dS_all + (bh * n_chunks + c_idx) * D * D;
+    auto Tm = [&](int r, int i) { return sX[r * L32 + i] * sB[i]; };
 
     // ---- inputs, the prep record and the chunk's decay
     load_rows(bK, k, row0, rs, Tl);
@@ -520,24 +518,47 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         sA[r * L32 + i] = rec[R_A + e];
         sP[r * L32 + i] = rec[R_P + e];
         sX[r * L32 + i] = rec[R_X + e];
-        sdP[r * L32 + i] = 0.f;
-        sdUV[r * L32 + i] = 0.f;
     }
     if (tid < D) sRS[tid] = 0.f;
     __syncthreads();
     running_sum(bG);
-    for (int e = tid; e < C * C; e += NT) {
-        const int r = e / C, i = e % C;
-        sT[r * L32 + i] = sX[r * L32 + i] * sB[i];
-    }
     __syncthreads();
     for (int e = tid; e < C * D; e += NT) {                       // Kb = K exp(Gam_C - Gam)
         const int r = e / D, c = e % D;
         bQ[r * LD + c] = bK[r * LD + c] * __expf(bG[(C - 1) * LD + c] - bG[r * LD + c]);
     }
+    // U = Tm V and dU = P^T dO, before the state terms
+    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return Tm(m, kk); },
+                         [&](int kk, int n) { return bV[kk * LD + n]; },
+                         [&](int m, int n, float x) { bU[m * LD + n] = x; });
+    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return sP[kk * L32 + m]; },
+                         [&](int kk, int n) { return bDO[kk * LD + n]; },
+                         [&](int m, int n, float x) { bDU[m * LD + n] = x; });
     __syncthreads();
 
-    // ---- the state-sized products, JB state columns at a time
+    // ---- pass 1: rows [kb, kb + JB) of S0 and dS: U -= W S0, dU += Kb dS
+#pragma unroll 1
+    for (int kb = 0; kb < D; kb += JB) {
+        for (int e = tid; e < JB * (D / 4); e += NT) {
+            const int i = e / (D / 4), c4 = (e % (D / 4)) * 4;
+            const float4 s0 = *reinterpret_cast<const float4*>(S0 + (int64_t)(kb + i) * D + c4);
+            const float4 ds = *reinterpret_cast<const float4*>(dS + (int64_t)(kb + i) * D + c4);
+            float* p0 = bS0 + i * LD + c4;
+            float* p1 = bDS + i * LD + c4;
+            p0[0] = s0.x; p0[1] = s0.y; p0[2] = s0.z; p0[3] = s0.w;
+            p1[0] = ds.x; p1[1] = ds.y; p1[2] = ds.z; p1[3] = ds.w;
+        }
+        __syncthreads();
+        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bW[m * LD + kb + kk]; },
+                              [&](int kk, int n) { return bS0[kk * LD + n]; },
+                              [&](int m, int n, float x) { bU[m * LD + n] -= x; });
+        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bQ[m * LD + kb + kk]; },
+                              [&](int kk, int n) { return bDS[kk * LD + n]; },
+                              [&](int m, int n, float x) { bDU[m * LD + n] += x; });
+        __syncthreads();
+    }
+
+    // ---- pass 2: columns [jb, jb + JB) of S0 and dS: dQt, dKb, dW and sum(dS S0)
 #pragma unroll 1
     for (int jb = 0; jb < D; jb += JB) {
         for (int e = tid; e < D * (JB / 4); e += NT) {
@@ -550,15 +571,15 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
             p1[0] = ds.x; p1[1] = ds.y; p1[2] = ds.z; p1[3] = ds.w;
         }
         __syncthreads();
-        // U = Tm V - W S0 and dU = P^T dO + Kb dS on this block (K = 32 + 128)
-        tgemm<C, JB, C + D, 2, 1>(
-            [&](int m, int kk) { return kk < C ? sT[m * L32 + kk] : -bW[m * LD + kk - C]; },
-            [&](int kk, int n) { return kk < C ? bV[kk * LD + jb + n] : bS0[(kk - C) * LJ + n]; },
-            [&](int m, int n, float x) { bU[m * LJ + n] = x; });
-        tgemm<C, JB, C + D, 2, 1>(
-            [&](int m, int kk) { return kk < C ? sP[kk * L32 + m] : bQ[m * LD + kk - C]; },
-            [&](int kk, int n) { return kk < C ? bDO[kk * LD + jb + n] : bDS[(kk - C) * LJ + n]; },
-            [&](int m, int n, float x) { bDU[m * LJ + n] = x; });
+        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bDO[m * LD + jb + kk]; },
+                              [&](int kk, int n) { return bS0[n * LJ + kk]; },
+                              [&](int m, int n, float x) { bDQT[m * LD + n] += x; });
+        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bU[m * LD + jb + kk]; },
+                              [&](int kk, int n) { return bDS[n * LJ + kk]; },
+                              [&](int m, int n, float x) { bDKB[m * LD + n] += x; });
+        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bDU[m * LD + jb + kk]; },
+                              [&](int kk, int n) { return bS0[n * LJ + kk]; },
+                              [&](int m, int n, float x) { bDW[m * LD + n] -= x; });
         if (tid < D) {
             float acc = sRS[tid];
 #pragma unroll
@@ -566,30 +587,21 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
             sRS[tid] = acc;
         }
         __syncthreads();
-        // accumulate over the block's columns j
-        tgemm<C, C, JB, 4, 1>([&](int m, int kk) { return bDO[m * LD + jb + kk]; },
-                              [&](int kk, int n) { return bU[n * LJ + kk]; },
-                              [&](int m, int n, float x) { sdP[m * L32 + n] += x; });
-        tgemm<C, C, JB, 4, 1>([&](int m, int kk) { return bDU[m * LJ + kk]; },
-                              [&](int kk, int n) { return bV[n * LD + jb + kk]; },
-                              [&](int m, int n, float x) { sdUV[m * L32 + n] += x; });
-        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bDO[m * LD + jb + kk]; },
-                              [&](int kk, int n) { return bS0[n * LJ + kk]; },
-                              [&](int m, int n, float x) { bDQT[m * LD + n] += x; });
-        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bU[m * LJ + kk]; },
-                              [&](int kk, int n) { return bDS[n * LJ + kk]; },
-                              [&](int m, int n, float x) { bDKB[m * LD + n] += x; });
-        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bDU[m * LJ + kk]; },
-                              [&](int kk, int n) { return bS0[n * LJ + kk]; },
-                              [&](int m, int n, float x) { bDW[m * LD + n] -= x; });
-        // dV = Tm^T dU on this block, straight to global memory
-        tgemm<C, JB, C, 2, 1>([&](int m, int kk) { return sT[kk * L32 + m]; },
-                              [&](int kk, int n) { return bDU[kk * LJ + n]; },
-                              [&](int m, int n, float x) {
-                                  if (m < Tl) dv[row0 + (int64_t)m * rs + jb + n] = to_bf(x);
-                              });
-        __syncthreads();
     }
+
+    // ---- products of the complete U and dU: dO U^T, dU V^T, dV = Tm^T dU
+    tgemm<C, C, D, 4, 1>([&](int m, int kk) { return bDO[m * LD + kk]; },
+                         [&](int kk, int n) { return bU[n * LD + kk]; },
+                         [&](int m, int n, float x) { sdP[m * L32 + n] = n <= m ? x : 0.f; });
+    tgemm<C, C, D, 4, 1>([&](int m, int kk) { return bDU[m * LD + kk]; },
+                         [&](int kk, int n) { return bV[n * LD + kk]; },
+                         [&](int m, int n, float x) { sdUV[m * L32 + n] = x; });
+    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return Tm(kk, m); },
+                         [&](int kk, int n) { return bDU[kk * LD + n]; },
+                         [&](int m, int n, float x) {
+                             if (m < Tl) dv[row0 + (int64_t)m * rs + n] = to_bf(x);
+                         });
+    __syncthreads();
 
     // ---- Q back in place of Kb; dGam from the direct terms; dq, dk partials
     load_rows(bQ, q, row0, rs, Tl);
@@ -618,7 +630,7 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     tgemm<C, C, D, 4, 1>([&](int m, int kk) { return bDW[m * LD + kk]; },
                          [&](int kk, int n) { return bW[n * LD + kk]; },
                          [&](int m, int n, float x) { sdT[m * L32 + n] = x + sdUV[m * L32 + n]; });
-    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return sT[kk * L32 + m]; },
+    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return Tm(kk, m); },
                          [&](int kk, int n) { return bDW[kk * LD + n]; },
                          [&](int m, int n, float x) { bDO[m * LD + n] = x; });
     __syncthreads();
@@ -638,16 +650,15 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     for (int e = tid; e < C * C; e += NT) {
         const int r = e / C, i = e % C;
         sdT[r * L32 + i] *= sB[i];
-        if (i > r) sdP[r * L32 + i] = 0.f;            // P is lower triangular incl. the diagonal
     }
     __syncthreads();
-    // Y = dX X^T;  dA = -(X^T Y), strictly lower
+    // Y = dX X^T (in sdUV);  dA = -(X^T Y), strictly lower
     tgemm<C, C, C, 4, 1>([&](int m, int kk) { return sdT[m * L32 + kk]; },
                          [&](int kk, int n) { return sX[n * L32 + kk]; },
-                         [&](int m, int n, float x) { sY[m * L32 + n] = x; });
+                         [&](int m, int n, float x) { sdUV[m * L32 + n] = x; });
     __syncthreads();
     tgemm<C, C, C, 4, 1>([&](int m, int kk) { return sX[kk * L32 + m]; },
-                         [&](int kk, int n) { return sY[kk * L32 + n]; },
+                         [&](int kk, int n) { return sdUV[kk * L32 + n]; },
                          [&](int m, int n, float x) { sdT[m * L32 + n] = n < m ? -x : 0.f; });
     __syncthreads();
     // dbeta (rows: sum_i dA_ri Araw_ri), then dAr = diag(beta) dA
