@@ -22,6 +22,20 @@ int current_sm_count()
     return n;
 }
 
+static DeviceFlags g_pool_done;
+
+void keep_pool_memory()
+{
+    once_per_device(g_pool_done, [](int dev) {
+        cudaMemPool_t pool;
+        if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+            uint64_t keep = UINT64_MAX;
+            cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        }
+        return cudaSuccess;   // a pool that keeps nothing only costs speed
+    });
+}
+
 cudaError_t decode_step_launch(const void* q, const void* k, const void* v,
                                const void* g, const void* beta, float* state,
                                void* o, int64_t NH, int dk, int dv, bool raw,

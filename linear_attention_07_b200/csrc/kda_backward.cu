@@ -22,16 +22,17 @@
 // tile boundary (both factors <= 1) -- the bound of the transcript's
 // log-decay-bound turn.
 //
-// Four launches, all fp32 arithmetic on CUDA cores:
-//   1. bwd_prep_kernel     (one CTA per chunk): Araw, Praw, X, W, U' = Tm V,
-//                           Z = Qt - P W, Kb, gC -> workspace;
-//   2. bwd_chain_kernel<0> (one CTA per (b, h, 32 state columns)): the forward
-//                           state chain S <- Diag(gC) S + Kb^T (U' - W S),
-//                           writing every chunk's start state;
-//   3. bwd_chain_kernel<1> : the reverse chain dS <- Diag(gC) dS - W^T (Kb dS)
-//                           + Z^T dO, writing every chunk's end gradient and
-//                           dh0 (state columns are independent in both chains);
-//   4. bwd_local_kernel    (one CTA per chunk): dq, dk, dv, dg, dbeta.
+// Three launches, all fp32 arithmetic on CUDA cores:
+//   1. bwd_prep_kernel   (one CTA per chunk): Araw, Praw, X, W, U' = Tm V,
+//                         Z = Qt - P W, Kb, gC -> workspace;
+//   2. bwd_chains_kernel (one CTA per (b, h, 32 state columns), two halves
+//                         side by side): the forward state chain
+//                         S <- Diag(gC) S + Kb^T (U' - W S), writing every
+//                         chunk's start state, and the reverse chain
+//                         dS <- Diag(gC) dS - W^T (Kb dS) + Z^T dO, writing every
+//                         chunk's end gradient and dh0 (state columns are
+//                         independent in both chains);
+//   3. bwd_local_kernel  (one CTA per chunk): dq, dk, dv, dg, dbeta.
 // The start states come from an fp32 chain rather than the tf32 forward
 // kernel: dg sums terms that nearly cancel, and state errors at the tf32
 // level (about 1e-3) move it by about 1e-2 of its scale.
@@ -267,16 +268,25 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 }
 
 // --------------------------------------------------------------- chains --
-// Per (b, h, NS state columns): the forward chain (REV = false) writes the
-// start state of every chunk to S_all[b][h][c]; the reverse chain (REV =
-// true) writes the gradient at the end of every chunk to S_all[b][h][c] and
-// the start-state gradient to out_last (dh0).  The chunk operands of the
-// next chunk are prefetched with cp.async while this one is processed.
+// Per (b, h, NS state columns), both chains in one CTA of 512 threads: the
+// forward chain (threads 0-255) writes the start state of every chunk to
+// S0_all[b][h][c]; the reverse chain (threads 256-511) writes the gradient at
+// the end of every chunk to dS_all[b][h][c] and the start-state gradient to
+// dh0.  The reverse chain needs only the per-chunk operands and dO, not the
+// forward's states, so the two run side by side, each half with its own
+// shared memory and named barrier.  Each operand buffer is refilled for the
+// next chunk (cp.async) as soon as the step that reads it is done: step 1's
+// operand after step 1, step 2's after step 2.
 
 constexpr int CLD = D + 4;        // operand rows: 528 B, 16-byte aligned
 constexpr int XLD = NS + 4;       // state / Y rows: 144 B
-constexpr int OPS = 3 * C * CLD + C * XLD + D;     // W, Kb, Z, (U' or dO) slice, gC: one buffer
-constexpr size_t CHAIN_SMEM = (size_t)(2 * OPS + D * XLD + C * XLD) * sizeof(float);
+// one chain's shared memory: step-1 operand [C][CLD] (+ U' slice [C][XLD]
+// forward), step-2 operands (Kb, or W and Z) [C][CLD] each (+ dO slice and gC),
+// the state slice [D][XLD] and Y [C][XLD]
+constexpr int FWD_FLOATS = 2 * C * CLD + 2 * C * XLD + D + D * XLD + C * XLD;
+constexpr int REV_FLOATS = 3 * C * CLD + C * XLD + D + D * XLD + C * XLD;
+constexpr size_t CHAIN_SMEM = (size_t)(FWD_FLOATS + REV_FLOATS) * sizeof(float);
+constexpr int NT_CHAIN = 2 * NT;
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src)
 {
@@ -285,53 +295,59 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src)
 }
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void half_sync(uint32_t id) { asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(NT) : "memory"); }
 
+// One chain over this CTA's state columns [j0, j0 + NS), run by NT threads
+// (tid = 0 .. NT - 1) that synchronise on named barrier `bar`.
 template <bool REV>
-__global__ void __launch_bounds__(NT, 1)
-bwd_chain_kernel(const float* __restrict__ rec_all, const __nv_bfloat16* __restrict__ dO,
-                 const float* __restrict__ S_init, float* __restrict__ S_all, float* __restrict__ out_last,
-                 int T, int H, int n_chunks)
+__device__ __forceinline__ void chain_run(float* sm, int tid, uint32_t bar, const float* __restrict__ rec_h,
+                                          const __nv_bfloat16* __restrict__ dO, const float* S_init,
+                                          float* __restrict__ S_all_h, float* out_last, int j0,
+                                          int64_t bh, int b, int h, int T, int H, int n_chunks)
 {
-    extern __shared__ __align__(16) float sm[];
-    float* sXs = sm + 2 * OPS;               // state slice [D][XLD]
-    float* sY = sXs + D * XLD;               // [C][XLD]
-    const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int j0 = s * NS;
-    const int tid = threadIdx.x;
-    const int64_t bh = (int64_t)b * H + h;
-    const float* rec_h = rec_all + bh * n_chunks * R_FLOATS;
+    float* o1 = sm;                                       // step 1: W (forward) or Kb (reverse)
+    float* oU = o1 + C * CLD;                             // forward: U' slice [C][XLD]
+    float* o2 = REV ? oU : oU + C * XLD;                  // step 2: Kb (forward) or W (reverse)
+    float* oZ = o2 + C * CLD;                             // reverse: Z
+    float* oS = REV ? oZ + C * CLD : o2 + C * CLD;        // reverse: dO slice (bf16 rows); forward: unused
+    float* oG = REV ? oS + C * XLD : oS + C * XLD;        // gC [D]
+    float* sXs = oG + D;                                  // state slice [D][XLD]
+    float* sY = sXs + D * XLD;                            // [C][XLD]
 
-    // prefetch the operands of chunk c into buffer `buf`
-    auto prefetch = [&](int c, int buf) {
-        float* o = sm + buf * OPS;
-        const float* r = rec_h + (int64_t)c * R_FLOATS;
+    auto fill_rows = [&](float* dst, const float* src) {  // [C][D] fp32 record rows -> [C][CLD]
         for (int e = tid; e < C * (D / 4); e += NT) {
             const int row = e / (D / 4), c4 = (e % (D / 4)) * 4;
-            cp_async16(o + 0 * C * CLD + row * CLD + c4, r + R_W + row * D + c4);
-            cp_async16(o + 1 * C * CLD + row * CLD + c4, r + R_KB + row * D + c4);
-            if (REV) cp_async16(o + 2 * C * CLD + row * CLD + c4, r + R_Z + row * D + c4);
+            cp_async16(dst + row * CLD + c4, src + row * D + c4);
         }
-        float* sl = o + 3 * C * CLD;
-        if (!REV) {
+    };
+    // step-1 operands of chunk c
+    auto fetch1 = [&](int c) {
+        const float* r = rec_h + (int64_t)c * R_FLOATS;
+        fill_rows(o1, r + (REV ? R_KB : R_W));
+        if (!REV)
             for (int e = tid; e < C * (NS / 4); e += NT) {
                 const int row = e / (NS / 4), c4 = (e % (NS / 4)) * 4;
-                cp_async16(sl + row * XLD + c4, r + R_UP + row * D + j0 + c4);
+                cp_async16(oU + row * XLD + c4, r + R_UP + row * D + j0 + c4);
             }
-        } else {
-            // dO slice: bf16 [C][NS] as raw bytes in the first half of each row
+        cp_commit();
+    };
+    // step-2 operands of chunk c
+    auto fetch2 = [&](int c) {
+        const float* r = rec_h + (int64_t)c * R_FLOATS;
+        fill_rows(o2, r + (REV ? R_W : R_KB));
+        if (REV) {
+            fill_rows(oZ, r + R_Z);
             const int t0 = c * C;
             for (int e = tid; e < C * (NS / 8); e += NT) {
                 const int row = e / (NS / 8), c8 = (e % (NS / 8)) * 8;
+                __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(oS + row * XLD) + c8;
                 if (t0 + row < T)
-                    cp_async16(reinterpret_cast<__nv_bfloat16*>(sl + row * XLD) + c8,
-                               dO + (((int64_t)b * T + t0 + row) * H + h) * D + j0 + c8);
+                    cp_async16(d, dO + (((int64_t)b * T + t0 + row) * H + h) * D + j0 + c8);
                 else
-                    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(sl + row * XLD) + c8) =
-                        make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4*>(d) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
-        for (int e = tid; e < D / 4; e += NT)
-            cp_async16(o + 3 * C * CLD + C * XLD + 4 * e, r + R_GC + 4 * e);
+        for (int e = tid; e < D / 4; e += NT) cp_async16(oG + 4 * e, r + R_GC + 4 * e);
         cp_commit();
     };
 
@@ -348,47 +364,45 @@ bwd_chain_kernel(const float* __restrict__ rec_all, const __nv_bfloat16* __restr
     }
     const int first = REV ? n_chunks - 1 : 0;
     const int step = REV ? -1 : 1;
-    if (n_chunks > 0) prefetch(first, 0);
+    if (n_chunks > 0) {
+        fetch1(first);
+        fetch2(first);
+    }
 #pragma unroll 1
     for (int n = 0; n < n_chunks; ++n) {
         const int c = first + step * n;
-        const int buf = n & 1;
+        const bool more = n + 1 < n_chunks;
         // the state at this chunk boundary
-        float* dst = S_all + (bh * n_chunks + c) * D * D;
+        float* dst = S_all_h + (int64_t)c * D * D;
 #pragma unroll
         for (int m = 0; m < 4; ++m)
             *reinterpret_cast<float4*>(dst + (int64_t)(ig + 32 * m) * D + j0 + 4 * cg) =
                 make_float4(xr[m][0], xr[m][1], xr[m][2], xr[m][3]);
-        if (n + 1 < n_chunks) prefetch(c + step, buf ^ 1); else cp_commit();
-        cp_wait_1();
-        __syncthreads();                     // chunk c's operands, the state in shared memory
-        const float* oW = sm + buf * OPS;
-        const float* oK = oW + C * CLD;
-        const float* oZ = oK + C * CLD;
-        const float* oS = oW + 3 * C * CLD;
-        const float* oG = oS + C * XLD;
-        {   // step 1: Y = U'_s - W X (forward) or Y = Kb X (reverse); thread (r, cg)
+        cp_wait_1();                         // step-1 operands of chunk c (step 2's may be in flight)
+        half_sync(bar);
+        {   // step 1: Y = U'_s - W X (forward) or Y = -(Kb X) (reverse); thread (r, cg)
             const int r = tid / (NS / 4);
-            const float* A1 = REV ? oK : oW;
             float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
             for (int i = 0; i < D; ++i) {
-                const float a = A1[r * CLD + i];
+                const float a = o1[r * CLD + i];
                 const float4 x = *reinterpret_cast<const float4*>(sXs + i * XLD + 4 * cg);
                 y.x = fmaf(a, x.x, y.x); y.y = fmaf(a, x.y, y.y);
                 y.z = fmaf(a, x.z, y.z); y.w = fmaf(a, x.w, y.w);
             }
             if (!REV) {
-                const float4 u = *reinterpret_cast<const float4*>(oS + r * XLD + 4 * cg);
+                const float4 u = *reinterpret_cast<const float4*>(oU + r * XLD + 4 * cg);
                 y = make_float4(u.x - y.x, u.y - y.y, u.z - y.z, u.w - y.w);
             } else {
-                y = make_float4(-y.x, -y.y, -y.z, -y.w);      // -(Kb dS): enters as -W^T (Kb dS)
+                y = make_float4(-y.x, -y.y, -y.z, -y.w);      // enters as -W^T (Kb dS)
             }
             *reinterpret_cast<float4*>(sY + r * XLD + 4 * cg) = y;
         }
-        __syncthreads();
+        half_sync(bar);                      // Y complete; the step-1 buffer is free
+        if (more) fetch1(c + step); else cp_commit();
+        cp_wait_1();                         // step-2 operands of chunk c
+        half_sync(bar);
         {   // step 2: X = Diag(gC) X + Kb^T Y (forward) or X = Diag(gC) X + W^T Y + Z^T dO (reverse)
-            const float* B1 = REV ? oW : oK;
             float acc[4][4];
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
@@ -401,7 +415,7 @@ bwd_chain_kernel(const float* __restrict__ rec_all, const __nv_bfloat16* __restr
                 const float4 y = *reinterpret_cast<const float4*>(sY + r * XLD + 4 * cg);
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
-                    const float bb = B1[r * CLD + ig + 32 * m];
+                    const float bb = o2[r * CLD + ig + 32 * m];
                     acc[m][0] = fmaf(bb, y.x, acc[m][0]); acc[m][1] = fmaf(bb, y.y, acc[m][1]);
                     acc[m][2] = fmaf(bb, y.z, acc[m][2]); acc[m][3] = fmaf(bb, y.w, acc[m][3]);
                 }
@@ -428,7 +442,8 @@ bwd_chain_kernel(const float* __restrict__ rec_all, const __nv_bfloat16* __restr
                     make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
             }
         }
-        __syncthreads();                     // state written; buffer `buf` free for the prefetch after next
+        half_sync(bar);                      // state written; the step-2 buffers are free
+        if (more) fetch2(c + step); else cp_commit();
     }
     if (out_last) {
 #pragma unroll
@@ -436,6 +451,23 @@ bwd_chain_kernel(const float* __restrict__ rec_all, const __nv_bfloat16* __restr
             *reinterpret_cast<float4*>(out_last + bh * D * D + (int64_t)(ig + 32 * m) * D + j0 + 4 * cg) =
                 make_float4(xr[m][0], xr[m][1], xr[m][2], xr[m][3]);
     }
+}
+
+__global__ void __launch_bounds__(NT_CHAIN, 1)
+bwd_chains_kernel(const float* __restrict__ rec_all, const __nv_bfloat16* __restrict__ dO,
+                  const float* h0, const float* dhT, float* __restrict__ S0_all, float* __restrict__ dS_all,
+                  float* dh0, int T, int H, int n_chunks)
+{
+    extern __shared__ __align__(16) float sm[];
+    const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int64_t bh = (int64_t)b * H + h;
+    const float* rec_h = rec_all + bh * n_chunks * R_FLOATS;
+    if (threadIdx.x < NT)
+        chain_run<false>(sm, threadIdx.x, 1, rec_h, dO, h0, S0_all + bh * n_chunks * D * D, nullptr,
+                         s * NS, bh, b, h, T, H, n_chunks);
+    else
+        chain_run<true>(sm + FWD_FLOATS, threadIdx.x - NT, 2, rec_h, dO, dhT, dS_all + bh * n_chunks * D * D,
+                        dh0, s * NS, bh, b, h, T, H, n_chunks);
 }
 
 // ---------------------------------------------------------- local grads --
@@ -805,8 +837,7 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     cudaError_t e = once_per_device(g_bwd_attr_done, [](int) {
         const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
         cudaError_t r = cudaFuncSetAttribute(bwd_prep_kernel, a, (int)PREP_SMEM);
-        if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_chain_kernel<false>, a, (int)CHAIN_SMEM);
-        if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_chain_kernel<true>, a, (int)CHAIN_SMEM);
+        if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_chains_kernel, a, (int)CHAIN_SMEM);
         if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_local_kernel, a, (int)LOC_SMEM);
         return r;
     });
@@ -821,6 +852,7 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     const size_t units = (size_t)B * H * n_chunks;
     const size_t bytes = units * ((size_t)R_FLOATS * sizeof(float) + 2 * state_bytes);
     float* ws = nullptr;
+    keep_pool_memory();
     e = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
     if (e != cudaSuccess) return e;
     float* rec = ws;
@@ -837,11 +869,8 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     bwd_prep_kernel<<<grid_c, NT, PREP_SMEM, stream>>>(bq, bk, bv, bg, bb, rec, T, H, n_chunks);
     e = cudaGetLastError();
     if (e == cudaSuccess) {
-        bwd_chain_kernel<false><<<grid_s, NT, CHAIN_SMEM, stream>>>(rec, bdo, h0, S0_all, nullptr, T, H, n_chunks);
-        e = cudaGetLastError();
-    }
-    if (e == cudaSuccess) {
-        bwd_chain_kernel<true><<<grid_s, NT, CHAIN_SMEM, stream>>>(rec, bdo, dhT, dS_all, dh0, T, H, n_chunks);
+        bwd_chains_kernel<<<grid_s, NT_CHAIN, CHAIN_SMEM, stream>>>(rec, bdo, h0, dhT, S0_all, dS_all, dh0, T, H,
+                                                                      n_chunks);
         e = cudaGetLastError();
     }
     if (e == cudaSuccess) {
@@ -852,7 +881,7 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     }
     const cudaError_t ef = cudaFreeAsync(ws, stream);
     if (e == cudaSuccess) e = ef;
-    note_launches(4);
+    note_launches(3);
     return e;
 }
 

@@ -39,6 +39,11 @@ cudaError_t once_per_device(DeviceFlags& done, F&& setup)
 // query fails.
 int current_sm_count();
 
+// Keep freed stream-ordered workspace in the current device's default pool
+// between calls (release threshold: never), once per device, so that a call
+// does not map its workspace anew every time.
+void keep_pool_memory();
+
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 

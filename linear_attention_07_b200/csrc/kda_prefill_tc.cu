@@ -1699,16 +1699,7 @@ static cudaError_t launch_segmented(const CUtensorMap& mq, const CUtensorMap& mk
         if (e != cudaSuccess) return e;
         ws = static_cast<float*>(p);
     } else {
-        // keep freed workspace in this device's pool between calls
-        static DeviceFlags pool_done;
-        once_per_device(pool_done, [](int dev) {
-            cudaMemPool_t pool;
-            if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
-                uint64_t keep = UINT64_MAX;
-                cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-            }
-            return cudaSuccess;   // a pool that keeps nothing only costs speed
-        });
+        keep_pool_memory();
         e = cudaMallocAsync(reinterpret_cast<void**>(&ws), bytes, stream);
         if (e != cudaSuccess) return e;
     }
