@@ -234,10 +234,10 @@ int kda_decode_step_raw(const void* q_raw, const void* k_raw, const void* v, con
  *   dq, dk, dg : bf16 [B][T][H][dk]     dv : bf16 [B][T][H][dv]
  *   dbeta      : bf16 [B][T][H]         dh0 : fp32 [B][H][dk][dv], or NULL
  *   Supported: d_k == d_v == 128.  T == 0: dh0 receives dhT (or zeros).
- * Four launches on `stream`, fp32 arithmetic throughout (the gradient of the
- * decay sums terms that nearly cancel, and tf32 state products would move
- * it by about 1e-2 of its scale): per-chunk operands, the forward state
- * chain, the reverse state chain, the chunk-local gradients.  Stream-ordered
+ * Three launches on `stream`, fp32 arithmetic throughout (the gradient of
+ * the decay sums terms that nearly cancel, and tf32 state products would
+ * move it by about 1e-2 of its scale): per-chunk operands, the forward and
+ * reverse state chains side by side, the chunk-local gradients.  Stream-ordered
  * workspace of 209,408 bytes per 32-token chunk and head (about 6.5 KB per
  * token and head; KDA_ERR_NO_MEMORY if it cannot be had).  Outputs must not
  * overlap inputs or one another.

@@ -351,12 +351,13 @@ __device__ __forceinline__ void chain_run(float* sm, int tid, uint32_t bar, cons
         cp_commit();
     };
 
-    // state slice: thread (ig, cg) owns rows ig + 32 m, columns 4 cg .. 4 cg + 3
+    // state slice: thread (ig, cg) owns rows 4 ig .. 4 ig + 3, columns 4 cg .. 4 cg + 3
+    // (float4 reads of its step-2 operand rows)
     const int ig = tid / (NS / 4), cg = tid % (NS / 4);
     float xr[4][4];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
-        const int i = ig + 32 * m;
+        const int i = 4 * ig + m;
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
         if (S_init) x = *reinterpret_cast<const float4*>(S_init + bh * D * D + (int64_t)i * D + j0 + 4 * cg);
         xr[m][0] = x.x; xr[m][1] = x.y; xr[m][2] = x.z; xr[m][3] = x.w;
@@ -376,19 +377,23 @@ __device__ __forceinline__ void chain_run(float* sm, int tid, uint32_t bar, cons
         float* dst = S_all_h + (int64_t)c * D * D;
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-            *reinterpret_cast<float4*>(dst + (int64_t)(ig + 32 * m) * D + j0 + 4 * cg) =
+            *reinterpret_cast<float4*>(dst + (int64_t)(4 * ig + m) * D + j0 + 4 * cg) =
                 make_float4(xr[m][0], xr[m][1], xr[m][2], xr[m][3]);
         cp_wait_1();                         // step-1 operands of chunk c (step 2's may be in flight)
         half_sync(bar);
         {   // step 1: Y = U'_s - W X (forward) or Y = -(Kb X) (reverse); thread (r, cg)
             const int r = tid / (NS / 4);
             float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-            for (int i = 0; i < D; ++i) {
-                const float a = o1[r * CLD + i];
-                const float4 x = *reinterpret_cast<const float4*>(sXs + i * XLD + 4 * cg);
-                y.x = fmaf(a, x.x, y.x); y.y = fmaf(a, x.y, y.y);
-                y.z = fmaf(a, x.z, y.z); y.w = fmaf(a, x.w, y.w);
+#pragma unroll 2
+            for (int i = 0; i < D; i += 4) {
+                const float4 a4 = *reinterpret_cast<const float4*>(o1 + r * CLD + i);
+                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 x = *reinterpret_cast<const float4*>(sXs + (i + u) * XLD + 4 * cg);
+                    y.x = fmaf(av[u], x.x, y.x); y.y = fmaf(av[u], x.y, y.y);
+                    y.z = fmaf(av[u], x.z, y.z); y.w = fmaf(av[u], x.w, y.w);
+                }
             }
             if (!REV) {
                 const float4 u = *reinterpret_cast<const float4*>(oU + r * XLD + 4 * cg);
@@ -404,20 +409,23 @@ __device__ __forceinline__ void chain_run(float* sm, int tid, uint32_t bar, cons
         half_sync(bar);
         {   // step 2: X = Diag(gC) X + Kb^T Y (forward) or X = Diag(gC) X + W^T Y + Z^T dO (reverse)
             float acc[4][4];
+            {
+                const float4 g4 = *reinterpret_cast<const float4*>(oG + 4 * ig);
+                const float gcv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float gcv = oG[ig + 32 * m];
+                for (int m = 0; m < 4; ++m)
 #pragma unroll
-                for (int u = 0; u < 4; ++u) acc[m][u] = gcv * xr[m][u];
+                    for (int u = 0; u < 4; ++u) acc[m][u] = gcv[m] * xr[m][u];
             }
 #pragma unroll 4
             for (int r = 0; r < C; ++r) {
                 const float4 y = *reinterpret_cast<const float4*>(sY + r * XLD + 4 * cg);
+                const float4 b4 = *reinterpret_cast<const float4*>(o2 + r * CLD + 4 * ig);
+                const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
-                    const float bb = o2[r * CLD + ig + 32 * m];
-                    acc[m][0] = fmaf(bb, y.x, acc[m][0]); acc[m][1] = fmaf(bb, y.y, acc[m][1]);
-                    acc[m][2] = fmaf(bb, y.z, acc[m][2]); acc[m][3] = fmaf(bb, y.w, acc[m][3]);
+                    acc[m][0] = fmaf(bb[m], y.x, acc[m][0]); acc[m][1] = fmaf(bb[m], y.y, acc[m][1]);
+                    acc[m][2] = fmaf(bb[m], y.z, acc[m][2]); acc[m][3] = fmaf(bb[m], y.w, acc[m][3]);
                 }
             }
             if (REV) {
@@ -426,11 +434,12 @@ __device__ __forceinline__ void chain_run(float* sm, int tid, uint32_t bar, cons
                 for (int r = 0; r < C; ++r) {
                     const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(dOs + r * 2 * XLD + 4 * cg);
                     const float2 d01 = __bfloat1622float2(d2[0]), d23 = __bfloat1622float2(d2[1]);
+                    const float4 z4 = *reinterpret_cast<const float4*>(oZ + r * CLD + 4 * ig);
+                    const float z[4] = {z4.x, z4.y, z4.z, z4.w};
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
-                        const float z = oZ[r * CLD + ig + 32 * m];
-                        acc[m][0] = fmaf(z, d01.x, acc[m][0]); acc[m][1] = fmaf(z, d01.y, acc[m][1]);
-                        acc[m][2] = fmaf(z, d23.x, acc[m][2]); acc[m][3] = fmaf(z, d23.y, acc[m][3]);
+                        acc[m][0] = fmaf(z[m], d01.x, acc[m][0]); acc[m][1] = fmaf(z[m], d01.y, acc[m][1]);
+                        acc[m][2] = fmaf(z[m], d23.x, acc[m][2]); acc[m][3] = fmaf(z[m], d23.y, acc[m][3]);
                     }
                 }
             }
@@ -438,7 +447,7 @@ __device__ __forceinline__ void chain_run(float* sm, int tid, uint32_t bar, cons
             for (int m = 0; m < 4; ++m) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) xr[m][u] = acc[m][u];
-                *reinterpret_cast<float4*>(sXs + (ig + 32 * m) * XLD + 4 * cg) =
+                *reinterpret_cast<float4*>(sXs + (4 * ig + m) * XLD + 4 * cg) =
                     make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
             }
         }
@@ -448,7 +457,7 @@ __device__ __forceinline__ void chain_run(float* sm, int tid, uint32_t bar, cons
     if (out_last) {
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-            *reinterpret_cast<float4*>(out_last + bh * D * D + (int64_t)(ig + 32 * m) * D + j0 + 4 * cg) =
+            *reinterpret_cast<float4*>(out_last + bh * D * D + (int64_t)(4 * ig + m) * D + j0 + 4 * cg) =
                 make_float4(xr[m][0], xr[m][1], xr[m][2], xr[m][3]);
     }
 }
@@ -568,19 +577,44 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
                          [&](int m, int n, float x) { bDU[m * LD + n] = x; });
     __syncthreads();
 
+    // The next block of S0 and dS is read into registers while the current one
+    // is used (2 float4 of each per thread), so the global loads overlap the
+    // block products.
+    float4 pf0[2], pf1[2];
+    auto fetch_rows = [&](int kb) {              // rows [kb, kb + JB), all columns
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = tid + u * NT, i = e / (D / 4), c4 = (e % (D / 4)) * 4;
+            pf0[u] = *reinterpret_cast<const float4*>(S0 + (int64_t)(kb + i) * D + c4);
+            pf1[u] = *reinterpret_cast<const float4*>(dS + (int64_t)(kb + i) * D + c4);
+        }
+    };
+    auto fetch_cols = [&](int jb) {              // all rows, columns [jb, jb + JB)
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = tid + u * NT, i = e / (JB / 4), c4 = (e % (JB / 4)) * 4;
+            pf0[u] = *reinterpret_cast<const float4*>(S0 + (int64_t)i * D + jb + c4);
+            pf1[u] = *reinterpret_cast<const float4*>(dS + (int64_t)i * D + jb + c4);
+        }
+    };
+    auto put = [&](float* dst, int stride, int i, int c4, float4 x) {
+        float* p = dst + i * stride + c4;
+        p[0] = x.x; p[1] = x.y; p[2] = x.z; p[3] = x.w;
+    };
+    static_assert(JB * (D / 4) == 2 * NT && D * (JB / 4) == 2 * NT, "two float4 per thread per block");
+
     // ---- pass 1: rows [kb, kb + JB) of S0 and dS: U -= W S0, dU += Kb dS
+    fetch_rows(0);
 #pragma unroll 1
     for (int kb = 0; kb < D; kb += JB) {
-        for (int e = tid; e < JB * (D / 4); e += NT) {
-            const int i = e / (D / 4), c4 = (e % (D / 4)) * 4;
-            const float4 s0 = *reinterpret_cast<const float4*>(S0 + (int64_t)(kb + i) * D + c4);
-            const float4 ds = *reinterpret_cast<const float4*>(dS + (int64_t)(kb + i) * D + c4);
-            float* p0 = bS0 + i * LD + c4;
-            float* p1 = bDS + i * LD + c4;
-            p0[0] = s0.x; p0[1] = s0.y; p0[2] = s0.z; p0[3] = s0.w;
-            p1[0] = ds.x; p1[1] = ds.y; p1[2] = ds.z; p1[3] = ds.w;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = tid + u * NT, i = e / (D / 4), c4 = (e % (D / 4)) * 4;
+            put(bS0, LD, i, c4, pf0[u]);
+            put(bDS, LD, i, c4, pf1[u]);
         }
         __syncthreads();
+        if (kb + JB < D) fetch_rows(kb + JB); else fetch_cols(0);
         tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bW[m * LD + kb + kk]; },
                               [&](int kk, int n) { return bS0[kk * LD + n]; },
                               [&](int m, int n, float x) { bU[m * LD + n] -= x; });
@@ -593,16 +627,14 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     // ---- pass 2: columns [jb, jb + JB) of S0 and dS: dQt, dKb, dW and sum(dS S0)
 #pragma unroll 1
     for (int jb = 0; jb < D; jb += JB) {
-        for (int e = tid; e < D * (JB / 4); e += NT) {
-            const int i = e / (JB / 4), c4 = (e % (JB / 4)) * 4;
-            const float4 s0 = *reinterpret_cast<const float4*>(S0 + (int64_t)i * D + jb + c4);
-            const float4 ds = *reinterpret_cast<const float4*>(dS + (int64_t)i * D + jb + c4);
-            float* p0 = bS0 + i * LJ + c4;
-            float* p1 = bDS + i * LJ + c4;
-            p0[0] = s0.x; p0[1] = s0.y; p0[2] = s0.z; p0[3] = s0.w;
-            p1[0] = ds.x; p1[1] = ds.y; p1[2] = ds.z; p1[3] = ds.w;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int e = tid + u * NT, i = e / (JB / 4), c4 = (e % (JB / 4)) * 4;
+            put(bS0, LJ, i, c4, pf0[u]);
+            put(bDS, LJ, i, c4, pf1[u]);
         }
         __syncthreads();
+        if (jb + JB < D) fetch_cols(jb + JB);
         tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bDO[m * LD + jb + kk]; },
                               [&](int kk, int n) { return bS0[n * LJ + kk]; },
                               [&](int m, int n, float x) { bDQT[m * LD + n] += x; });
