@@ -57,10 +57,11 @@ __device__ __forceinline__ float bf(const __nv_bfloat16 x) { return __bfloat162f
 
 // Rows [t0, t0 + C) of one head of a [B][T][H][D] bf16 tensor into shared
 // memory (row stride LD), zero past Tl.
+template <int NTH = NT>
 __device__ __forceinline__ void load_rows(float* dst, const __nv_bfloat16* __restrict__ src, int64_t row0,
                                           int64_t row_stride, int n_valid)
 {
-    for (int v = threadIdx.x; v < C * (D / 8); v += NT) {
+    for (int v = threadIdx.x; v < C * (D / 8); v += NTH) {
         const int r = v / (D / 8), c8 = (v % (D / 8)) * 8;
         float f[8];
         if (r < n_valid) {
@@ -99,17 +100,17 @@ __device__ __forceinline__ float tile_ref(const float* G, int r, int c)
     return r >= TILE ? G[(TILE - 1) * LD + c] : 0.f;
 }
 
-// Block GEMM on shared-memory operands, fp32 FMA, all NT threads:
+// Block GEMM on shared-memory operands, fp32 FMA, all NTH threads:
 // out(m, n, sum_k a(m, k) b(k, n)) for an M x N result.  Thread (tm, tn)
 // computes rows tm * TM .. + TM - 1 and columns tn + NC j: consecutive
 // threads read consecutive columns of a row-major b (or one column each of
 // a transposed one; odd row strides keep both conflict-free) and share the
 // a values (broadcast).
-template <int M, int N, int K, int TM, int TN, typename FA, typename FB, typename FO>
+template <int M, int N, int K, int TM, int TN, int NTH = NT, typename FA, typename FB, typename FO>
 __device__ __forceinline__ void tgemm(FA a, FB b, FO out)
 {
     constexpr int NC = N / TN, NR = M / TM;
-    static_assert(NC * NR == NT && NC * TN == N && NR * TM == M, "tile shape");
+    static_assert(NC * NR == NTH && NC * TN == N && NR * TM == M, "tile shape");
     const int t = threadIdx.x, tn = t % NC, tm = t / NC;
     float acc[TM][TN];
 #pragma unroll
@@ -489,10 +490,11 @@ bwd_chains_kernel(const float* __restrict__ rec_all, const __nv_bfloat16* __rest
 constexpr int LOC_BIG = 11;    // K, Q, V, dO, G, W, U, dU, dKb, dQt, dW
 constexpr int BLK = D * LJ > JB * LD ? D * LJ : JB * LD;    // one S0 or dS block (either shape)
 constexpr size_t LOC_SMEM = (size_t)(LOC_BIG * C * LD + 2 * BLK + 6 * C * L32 + 2 * C + 2 * D) * sizeof(float);
+constexpr int NL = 2 * NT;     // threads of the local kernel: 16 warps hide the shared-memory latency
 
 __device__ __forceinline__ __nv_bfloat16 to_bf(float x) { return __float2bfloat16_rn(x); }
 
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NL, 1)
 bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                  const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ g,
                  const __nv_bfloat16* __restrict__ beta, const __nv_bfloat16* __restrict__ dO,
@@ -539,22 +541,22 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     auto Tm = [&](int r, int i) { return sX[r * L32 + i] * sB[i]; };
 
     // ---- inputs, the prep record and the chunk's decay
-    load_rows(bK, k, row0, rs, Tl);
-    load_rows(bV, v, row0, rs, Tl);
-    load_rows(bDO, dO, row0, rs, Tl);
-    load_rows(bG, g, row0, rs, Tl);
+    load_rows<NL>(bK, k, row0, rs, Tl);
+    load_rows<NL>(bV, v, row0, rs, Tl);
+    load_rows<NL>(bDO, dO, row0, rs, Tl);
+    load_rows<NL>(bG, g, row0, rs, Tl);
     if (tid < C) {
         sB[tid] = tid < Tl ? bf(beta[((int64_t)b * T + t0 + tid) * H + h]) : 0.f;
         sDB[tid] = 0.f;
     }
-    for (int e = tid; e < C * D; e += NT) {
+    for (int e = tid; e < C * D; e += NL) {
         const int r = e / D, c = e % D;
         bW[r * LD + c] = rec[R_W + e];
         bDKB[r * LD + c] = 0.f;
         bDQT[r * LD + c] = 0.f;
         bDW[r * LD + c] = 0.f;
     }
-    for (int e = tid; e < C * C; e += NT) {
+    for (int e = tid; e < C * C; e += NL) {
         const int r = e / C, i = e % C;
         sA[r * L32 + i] = rec[R_A + e];
         sP[r * L32 + i] = rec[R_P + e];
@@ -564,15 +566,15 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     __syncthreads();
     running_sum(bG);
     __syncthreads();
-    for (int e = tid; e < C * D; e += NT) {                       // Kb = K exp(Gam_C - Gam)
+    for (int e = tid; e < C * D; e += NL) {                       // Kb = K exp(Gam_C - Gam)
         const int r = e / D, c = e % D;
         bQ[r * LD + c] = bK[r * LD + c] * __expf(bG[(C - 1) * LD + c] - bG[r * LD + c]);
     }
     // U = Tm V and dU = P^T dO, before the state terms
-    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return Tm(m, kk); },
+    tgemm<C, D, C, 2, 4, NL>([&](int m, int kk) { return Tm(m, kk); },
                          [&](int kk, int n) { return bV[kk * LD + n]; },
                          [&](int m, int n, float x) { bU[m * LD + n] = x; });
-    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return sP[kk * L32 + m]; },
+    tgemm<C, D, C, 2, 4, NL>([&](int m, int kk) { return sP[kk * L32 + m]; },
                          [&](int kk, int n) { return bDO[kk * LD + n]; },
                          [&](int m, int n, float x) { bDU[m * LD + n] = x; });
     __syncthreads();
@@ -580,19 +582,21 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     // The next block of S0 and dS is read into registers while the current one
     // is used (2 float4 of each per thread), so the global loads overlap the
     // block products.
-    float4 pf0[2], pf1[2];
+    constexpr int PF = (JB * (D / 4)) / NL;      // float4 of each matrix per thread and block
+    static_assert(JB * (D / 4) == PF * NL && D * (JB / 4) == PF * NL && PF >= 1, "block split");
+    float4 pf0[PF], pf1[PF];
     auto fetch_rows = [&](int kb) {              // rows [kb, kb + JB), all columns
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = tid + u * NT, i = e / (D / 4), c4 = (e % (D / 4)) * 4;
+        for (int u = 0; u < PF; ++u) {
+            const int e = tid + u * NL, i = e / (D / 4), c4 = (e % (D / 4)) * 4;
             pf0[u] = *reinterpret_cast<const float4*>(S0 + (int64_t)(kb + i) * D + c4);
             pf1[u] = *reinterpret_cast<const float4*>(dS + (int64_t)(kb + i) * D + c4);
         }
     };
     auto fetch_cols = [&](int jb) {              // all rows, columns [jb, jb + JB)
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = tid + u * NT, i = e / (JB / 4), c4 = (e % (JB / 4)) * 4;
+        for (int u = 0; u < PF; ++u) {
+            const int e = tid + u * NL, i = e / (JB / 4), c4 = (e % (JB / 4)) * 4;
             pf0[u] = *reinterpret_cast<const float4*>(S0 + (int64_t)i * D + jb + c4);
             pf1[u] = *reinterpret_cast<const float4*>(dS + (int64_t)i * D + jb + c4);
         }
@@ -601,24 +605,23 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         float* p = dst + i * stride + c4;
         p[0] = x.x; p[1] = x.y; p[2] = x.z; p[3] = x.w;
     };
-    static_assert(JB * (D / 4) == 2 * NT && D * (JB / 4) == 2 * NT, "two float4 per thread per block");
 
     // ---- pass 1: rows [kb, kb + JB) of S0 and dS: U -= W S0, dU += Kb dS
     fetch_rows(0);
 #pragma unroll 1
     for (int kb = 0; kb < D; kb += JB) {
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = tid + u * NT, i = e / (D / 4), c4 = (e % (D / 4)) * 4;
+        for (int u = 0; u < PF; ++u) {
+            const int e = tid + u * NL, i = e / (D / 4), c4 = (e % (D / 4)) * 4;
             put(bS0, LD, i, c4, pf0[u]);
             put(bDS, LD, i, c4, pf1[u]);
         }
         __syncthreads();
         if (kb + JB < D) fetch_rows(kb + JB); else fetch_cols(0);
-        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bW[m * LD + kb + kk]; },
+        tgemm<C, D, JB, 2, 4, NL>([&](int m, int kk) { return bW[m * LD + kb + kk]; },
                               [&](int kk, int n) { return bS0[kk * LD + n]; },
                               [&](int m, int n, float x) { bU[m * LD + n] -= x; });
-        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bQ[m * LD + kb + kk]; },
+        tgemm<C, D, JB, 2, 4, NL>([&](int m, int kk) { return bQ[m * LD + kb + kk]; },
                               [&](int kk, int n) { return bDS[kk * LD + n]; },
                               [&](int m, int n, float x) { bDU[m * LD + n] += x; });
         __syncthreads();
@@ -628,20 +631,20 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 #pragma unroll 1
     for (int jb = 0; jb < D; jb += JB) {
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int e = tid + u * NT, i = e / (JB / 4), c4 = (e % (JB / 4)) * 4;
+        for (int u = 0; u < PF; ++u) {
+            const int e = tid + u * NL, i = e / (JB / 4), c4 = (e % (JB / 4)) * 4;
             put(bS0, LJ, i, c4, pf0[u]);
             put(bDS, LJ, i, c4, pf1[u]);
         }
         __syncthreads();
         if (jb + JB < D) fetch_cols(jb + JB);
-        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bDO[m * LD + jb + kk]; },
+        tgemm<C, D, JB, 2, 4, NL>([&](int m, int kk) { return bDO[m * LD + jb + kk]; },
                               [&](int kk, int n) { return bS0[n * LJ + kk]; },
                               [&](int m, int n, float x) { bDQT[m * LD + n] += x; });
-        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bU[m * LD + jb + kk]; },
+        tgemm<C, D, JB, 2, 4, NL>([&](int m, int kk) { return bU[m * LD + jb + kk]; },
                               [&](int kk, int n) { return bDS[n * LJ + kk]; },
                               [&](int m, int n, float x) { bDKB[m * LD + n] += x; });
-        tgemm<C, D, JB, 4, 4>([&](int m, int kk) { return bDU[m * LD + jb + kk]; },
+        tgemm<C, D, JB, 2, 4, NL>([&](int m, int kk) { return bDU[m * LD + jb + kk]; },
                               [&](int kk, int n) { return bS0[n * LJ + kk]; },
                               [&](int m, int n, float x) { bDW[m * LD + n] -= x; });
         if (tid < D) {
@@ -654,13 +657,13 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     }
 
     // ---- products of the complete U and dU: dO U^T, dU V^T, dV = Tm^T dU
-    tgemm<C, C, D, 4, 1>([&](int m, int kk) { return bDO[m * LD + kk]; },
+    tgemm<C, C, D, 2, 1, NL>([&](int m, int kk) { return bDO[m * LD + kk]; },
                          [&](int kk, int n) { return bU[n * LD + kk]; },
                          [&](int m, int n, float x) { sdP[m * L32 + n] = n <= m ? x : 0.f; });
-    tgemm<C, C, D, 4, 1>([&](int m, int kk) { return bDU[m * LD + kk]; },
+    tgemm<C, C, D, 2, 1, NL>([&](int m, int kk) { return bDU[m * LD + kk]; },
                          [&](int kk, int n) { return bV[n * LD + kk]; },
                          [&](int m, int n, float x) { sdUV[m * L32 + n] = x; });
-    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return Tm(kk, m); },
+    tgemm<C, D, C, 2, 4, NL>([&](int m, int kk) { return Tm(kk, m); },
                          [&](int kk, int n) { return bDU[kk * LD + n]; },
                          [&](int m, int n, float x) {
                              if (m < Tl) dv[row0 + (int64_t)m * rs + n] = to_bf(x);
@@ -668,7 +671,7 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     __syncthreads();
 
     // ---- Q back in place of Kb; dGam from the direct terms; dq, dk partials
-    load_rows(bQ, q, row0, rs, Tl);
+    load_rows<NL>(bQ, q, row0, rs, Tl);
     if (tid < D) {                                   // sum_r dKb_rc Kb_rc, before dKb is rescaled
         const int c = tid;
         const float gl = bG[(C - 1) * LD + c];
@@ -678,7 +681,7 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         sKS[c] = acc;
     }
     __syncthreads();
-    for (int e = tid; e < C * D; e += NT) {
+    for (int e = tid; e < C * D; e += NL) {
         const int r = e / D, c = e % D;
         const float Gr = bG[r * LD + c];
         const float gam = __expf(Gr), kbf = __expf(bG[(C - 1) * LD + c] - Gr);
@@ -691,14 +694,14 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     }
     __syncthreads();
     // dTm = dW Kt^T + dU V^T;  dKt = Tm^T dW -> bDO
-    tgemm<C, C, D, 4, 1>([&](int m, int kk) { return bDW[m * LD + kk]; },
+    tgemm<C, C, D, 2, 1, NL>([&](int m, int kk) { return bDW[m * LD + kk]; },
                          [&](int kk, int n) { return bW[n * LD + kk]; },
                          [&](int m, int n, float x) { sdT[m * L32 + n] = x + sdUV[m * L32 + n]; });
-    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return Tm(kk, m); },
+    tgemm<C, D, C, 2, 4, NL>([&](int m, int kk) { return Tm(kk, m); },
                          [&](int kk, int n) { return bDW[kk * LD + n]; },
                          [&](int m, int n, float x) { bDO[m * LD + n] = x; });
     __syncthreads();
-    for (int e = tid; e < C * D; e += NT) {
+    for (int e = tid; e < C * D; e += NL) {
         const int r = e / D, c = e % D;
         const float dkt = bDO[r * LD + c];
         bDKB[r * LD + c] += dkt * __expf(bG[r * LD + c]);
@@ -711,17 +714,17 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         sDB[tid] = acc;
     }
     __syncthreads();
-    for (int e = tid; e < C * C; e += NT) {
+    for (int e = tid; e < C * C; e += NL) {
         const int r = e / C, i = e % C;
         sdT[r * L32 + i] *= sB[i];
     }
     __syncthreads();
     // Y = dX X^T (in sdUV);  dA = -(X^T Y), strictly lower
-    tgemm<C, C, C, 4, 1>([&](int m, int kk) { return sdT[m * L32 + kk]; },
+    tgemm<C, C, C, 2, 1, NL>([&](int m, int kk) { return sdT[m * L32 + kk]; },
                          [&](int kk, int n) { return sX[n * L32 + kk]; },
                          [&](int m, int n, float x) { sdUV[m * L32 + n] = x; });
     __syncthreads();
-    tgemm<C, C, C, 4, 1>([&](int m, int kk) { return sX[kk * L32 + m]; },
+    tgemm<C, C, C, 2, 1, NL>([&](int m, int kk) { return sX[kk * L32 + m]; },
                          [&](int kk, int n) { return sdUV[kk * L32 + n]; },
                          [&](int m, int n, float x) { sdT[m * L32 + n] = n < m ? -x : 0.f; });
     __syncthreads();
@@ -732,12 +735,12 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         sDB[tid] = acc;
     }
     __syncthreads();
-    for (int e = tid; e < C * C; e += NT) {
+    for (int e = tid; e < C * C; e += NL) {
         const int r = e / C, i = e % C;
         sdT[r * L32 + i] *= sB[r];
     }
     // tile-relative operands: Ka -> bW, Qa -> bDW, Kf -> bDO, Kc -> bS0 (tile 0 rows)
-    for (int e = tid; e < C * D; e += NT) {
+    for (int e = tid; e < C * D; e += NL) {
         const int r = e / D, c = e % D;
         const float Gr = bG[r * LD + c], ref = tile_ref(bG, r, c);
         const float kk = bK[r * LD + c], a = __expf(Gr - ref);
@@ -747,14 +750,15 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         if (r < TILE) bS0[r * LD + c] = kk * __expf(bG[(TILE - 1) * LD + c] - Gr);
     }
     __syncthreads();
-    // pair-product gradients: thread rows r0 .. r0 + 3 (one tile), channels lane + 32 j
+    // pair-product gradients: thread rows r0 .. r0 + RW - 1 (one tile), channels lane + 32 j
     {
-        const int r0 = 4 * (tid >> 5), lane = tid & 31;
+        constexpr int RW = C / (NL / 32);        // rows per warp
+        const int r0 = RW * (tid >> 5), lane = tid & 31;
         const int tau = r0 / TILE;
         const int i0 = tau * TILE;
-        float rk[4][4], rq[4][4], ck_s[4][4], ck_x[4][4];
+        float rk[RW][4], rq[RW][4], ck_s[RW][4], ck_x[RW][4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < RW; ++u)
 #pragma unroll
             for (int j = 0; j < 4; ++j) rk[u][j] = rq[u][j] = ck_s[u][j] = ck_x[u][j] = 0.f;
         // same tile: row role over columns i, column role over rows rr, both in [i0, i0 + 16)
@@ -770,7 +774,7 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
                 qa[j] = bDW[i * LD + c];
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < RW; ++u) {
                 const float dar = sdT[(r0 + u) * L32 + i], dpr = sdP[(r0 + u) * L32 + i];   // (row r, col i)
                 const float dac = sdT[i * L32 + r0 + u], dpc = sdP[i * L32 + r0 + u];       // (row i, col r)
 #pragma unroll
@@ -788,7 +792,7 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 #pragma unroll
                 for (int j = 0; j < 4; ++j) kc[j] = bS0[i * LD + lane + 32 * j];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < RW; ++u) {
                     const float dar = sdT[(r0 + u) * L32 + i], dpr = sdP[(r0 + u) * L32 + i];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
@@ -807,7 +811,7 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
                     qa[j] = bDW[rr * LD + lane + 32 * j];
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < RW; ++u) {
                     const float dac = sdT[rr * L32 + r0 + u], dpc = sdP[rr * L32 + r0 + u];
 #pragma unroll
                     for (int j = 0; j < 4; ++j) ck_x[u][j] = fmaf(dac, ka[j], fmaf(dpc, qa[j], ck_x[u][j]));
@@ -815,7 +819,7 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < RW; ++u) {
             const int r = r0 + u;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -845,7 +849,7 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         }
     }
     __syncthreads();
-    for (int e = tid; e < C * D; e += NT) {
+    for (int e = tid; e < C * D; e += NL) {
         const int r = e / D, c = e % D;
         if (r < Tl) {
             const int64_t o = row0 + (int64_t)r * rs + c;
@@ -906,7 +910,7 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
         e = cudaGetLastError();
     }
     if (e == cudaSuccess) {
-        bwd_local_kernel<<<grid_c, NT, LOC_SMEM, stream>>>(
+        bwd_local_kernel<<<grid_c, NL, LOC_SMEM, stream>>>(
             bq, bk, bv, bg, bb, bdo, rec, S0_all, dS_all, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk,
             (__nv_bfloat16*)dv, (__nv_bfloat16*)dg, (__nv_bfloat16*)dbeta, T, H, n_chunks);
         e = cudaGetLastError();
