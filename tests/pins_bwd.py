@@ -340,3 +340,152 @@ ALL_PINS = {
     "batch_layout_bwd": (batch_layout_bwd, 1e-14),
     "chunked_bwd_form": (chunked_bwd_form, 1e-9),
 }
+
+
+# -- 9. the GPU backward's scheme: 16-token tile references, row/column roles --
+def _tile_factors(Gam, tile):
+    """Row factor a_r = exp(Gam_r - Gam_ref(r)) (<= 1), same-tile column factor
+    b_i = exp(Gam_ref(i) - Gam_i) (<= e^{5 tile}), cross column factor
+    c_i = exp(Gam_{tile-1} - Gam_i) for the first tile (<= 1); ref(r) is Gam
+    just before r's tile."""
+    n = Gam.shape[0]
+    ref = np.zeros_like(Gam)
+    for r in range(n):
+        t0 = (r // tile) * tile
+        if t0 > 0:
+            ref[r] = Gam[t0 - 1]
+    a = np.exp(Gam - ref)
+    b = np.exp(ref - Gam)
+    c = np.exp(Gam[min(tile, n) - 1][None, :] - Gam)
+    return a, b, c
+
+
+def _pairs(L, R, a, b, c, tile, incl):
+    """G[r, i] = sum_ch L[r] R[i] exp(Gam_r - Gam_i) for i < r (or i <= r)."""
+    n = L.shape[0]
+    G = np.zeros((n, n), L.dtype)
+    for r in range(n):
+        for i in range(r + 1 if incl else r):
+            f = b[i] if i // tile == r // tile else c[i]
+            G[r, i] = np.sum(L[r] * a[r] * R[i] * f)
+    return G
+
+
+def _row_role(dG, R, a, b, c, tile):
+    """out[r] = a_r * sum_i dG[r, i] R[i] f_i  (= sum_i dG[r, i] R[i] exp(Gam_r - Gam_i))."""
+    n = dG.shape[0]
+    out = np.zeros_like(R)
+    for r in range(n):
+        for i in range(n):
+            if dG[r, i] != 0:
+                out[r] += dG[r, i] * R[i] * (b[i] if i // tile == r // tile else c[i])
+        out[r] *= a[r]
+    return out
+
+
+def _col_role(dG, L, a, b, c, tile):
+    """out[i] = sum_r dG[r, i] L[r] exp(Gam_r - Gam_i)."""
+    n = dG.shape[0]
+    out = np.zeros_like(L)
+    for i in range(n):
+        same = np.zeros(L.shape[1], L.dtype)
+        cross = np.zeros(L.shape[1], L.dtype)
+        for r in range(n):
+            if dG[r, i] != 0:
+                if r // tile == i // tile:
+                    same += dG[r, i] * L[r] * a[r]
+                else:
+                    cross += dG[r, i] * L[r] * a[r]
+        out[i] = same * b[i] + cross * c[i]
+    return out
+
+
+def tiled_chunk_bwd(q, k, v, g, beta, h0, dO, dhT, C=32, tile=16, dtype=np.float64):
+    """One head, in the order of the GPU backward: per-chunk operands (pair
+    products with tile references, X = (I + A)^-1, W, U', Z = Qt - P W, Kb),
+    the forward state chain, the reverse state chain, then the chunk-local
+    gradients, whose decayed pair terms split into row and column roles
+    (dk += row(dAr, K) + col(dAr, K) + col(dP, Q), dq += row(dP, K), and
+    dGam += k row(dAr, K) + q row(dP, K) - k col(...)).  No factor 1/gam
+    relative to the chunk start is ever formed.  Returns (dq, dk, dv, dg,
+    dbeta, dh0)."""
+    T = q.shape[0]
+    n_ch = (T + C - 1) // C
+    pad = n_ch * C - T
+    P = lambda x: np.concatenate([x, np.zeros((pad,) + x.shape[1:])]).astype(dtype)
+    q, k, v, g, beta, dO = (P(x) for x in (q, k, v, g, beta, dO))
+    recs = []
+    for ch in range(n_ch):
+        sl = slice(ch * C, (ch + 1) * C)
+        Q, K, V, G, Bt = q[sl], k[sl], v[sl], g[sl], beta[sl]
+        Gam = np.cumsum(G, axis=0)
+        a, b, c = _tile_factors(Gam, tile)
+        Kt, Qt, Kb = K * np.exp(Gam), Q * np.exp(Gam), K * np.exp(Gam[-1][None, :] - Gam)
+        Araw = _pairs(K, K, a, b, c, tile, incl=False)
+        Praw = _pairs(Q, K, a, b, c, tile, incl=True)
+        X = np.linalg.inv(np.eye(C, dtype=dtype) + Araw * Bt[:, None])
+        Tm = X * Bt[None, :]
+        W = Tm @ Kt
+        recs.append(dict(Gam=Gam, a=a, b=b, c=c, Kt=Kt, Qt=Qt, Kb=Kb, Araw=Araw, P=Praw, X=X, Tm=Tm, W=W,
+                         Up=Tm @ V, Z=Qt - Praw @ W, gC=np.exp(Gam[-1])))
+    S = h0.astype(dtype)
+    S0 = []
+    for r in recs:                                    # forward chain
+        S0.append(S)
+        S = r["gC"][:, None] * S + r["Kb"].T @ (r["Up"] - r["W"] @ S)
+    dS = dhT.astype(dtype)
+    dS_end = [None] * n_ch
+    for ch in reversed(range(n_ch)):                  # reverse chain
+        r = recs[ch]
+        dS_end[ch] = dS
+        dS = r["gC"][:, None] * dS - r["W"].T @ (r["Kb"] @ dS) + r["Z"].T @ dO[ch * C:(ch + 1) * C]
+    dh0 = dS
+    dq, dk, dv, dg, db = (np.zeros_like(x) for x in (q, k, v, g, beta))
+    for ch, r in enumerate(recs):                     # chunk-local gradients
+        sl = slice(ch * C, (ch + 1) * C)
+        Q, K, V, dOc, Bt = q[sl], k[sl], v[sl], dO[sl], beta[sl]
+        a, b, c, X, Tm = r["a"], r["b"], r["c"], r["X"], r["Tm"]
+        U = Tm @ V - r["W"] @ S0[ch]
+        dU = r["P"].T @ dOc + r["Kb"] @ dS_end[ch]
+        dP = np.tril(dOc @ U.T)
+        dQt = dOc @ S0[ch].T
+        dKb = U @ dS_end[ch].T
+        dW = -dU @ S0[ch].T
+        dTm = dW @ r["Kt"].T + dU @ V.T
+        dKt = Tm.T @ dW
+        dB = (dTm * X).sum(axis=0)
+        dA = -(X.T @ (dTm * Bt[None, :]) @ X.T) * np.tril(np.ones((C, C)), -1)
+        dB = dB + (dA * r["Araw"]).sum(axis=1)
+        dAr = dA * Bt[:, None]
+        rowK = _row_role(dAr, K, a, b, c, tile)
+        rowQ = _row_role(dP, K, a, b, c, tile)
+        colK = _col_role(dAr, K, a, b, c, tile) + _col_role(dP, Q, a, b, c, tile)
+        gam, kbf = np.exp(r["Gam"]), np.exp(r["Gam"][-1][None, :] - r["Gam"])
+        dk[sl] = dKt * gam + rowK + colK + dKb * kbf
+        dq[sl] = dQt * gam + rowQ
+        dv[sl] = Tm.T @ dU
+        db[sl] = dB
+        dGam = dKt * r["Kt"] + dQt * r["Qt"] - dKb * r["Kb"] + K * rowK + Q * rowQ - K * colK
+        dGam[-1] += (dKb * r["Kb"]).sum(axis=0) + (dS_end[ch] * S0[ch]).sum(axis=1) * r["gC"]
+        dg[sl] = np.cumsum(dGam[::-1], axis=0)[::-1]
+    cut = lambda x: x[:T]
+    return cut(dq), cut(dk), cut(dv), cut(dg), cut(db), dh0
+
+
+def tiled_scheme_form(orc, seed=29, lengths=(1, 16, 31, 33, 70)):
+    """The GPU backward's scheme against the oracle (fp64, decays down to the
+    -5 floor so every tile reference matters)."""
+    rng = np.random.default_rng(seed)
+    dk, dv = 12, 9
+    err = 0.0
+    for T in lengths:
+        q, k, v, g, beta, h0 = _rand_problem(rng, T, dk, dv, n=1)
+        g = -5.0 * rng.uniform(0.0, 1.0, g.shape)
+        dO, dhT = _cotangents(rng, 1, T, dv, dk)
+        got = tiled_chunk_bwd(q[0], k[0], v[0], g[0], beta[0], h0[0], dO[0], dhT[0])
+        want = orc.heads_bwd(q, k, v, g, beta, h0, dO, dhT)
+        err = max(err, _grad_rel(got, [w[0] for w in want]))
+    return err
+
+
+ALL_PINS["tiled_scheme_form"] = (tiled_scheme_form, 1e-10)

@@ -95,3 +95,24 @@ def test_prologue_chain_rule_special_cases(oracle_mod):
     assert np.max(np.abs((dq_raw * r).sum(axis=-1))) < 1e-14
     assert np.allclose(dz[0, 0, 0], -5.0 * 0.25, rtol=0, atol=1e-15)
     assert np.max(np.abs(dz[1, 2, 0])) < 1e-30 and np.max(np.abs(dz[2, 3, 1])) < 1e-30
+
+
+def test_tiled_scheme_is_finite_in_fp32_at_the_floor(oracle_mod):
+    """g = -5 on every channel over 64 tokens: a factor 1/gamma relative to
+    the chunk start would reach e^155 (inf in fp32); the GPU backward's tile
+    references keep every factor at or below e^80, so its scheme run in fp32
+    stays finite and close to the fp64 oracle."""
+    from pins import _rand_problem
+    rng = np.random.default_rng(31)
+    T, dk, dv = 64, 16, 8
+    q, k, v, g, beta, h0 = _rand_problem(rng, T, dk, dv, n=1)
+    g = np.full_like(g, -5.0)
+    dO = rng.standard_normal((1, T, dv))
+    dhT = rng.standard_normal((1, dk, dv))
+    got = pins_bwd.tiled_chunk_bwd(q[0], k[0], v[0], g[0], beta[0], h0[0], dO[0], dhT[0], dtype=np.float32)
+    want = oracle_mod.heads_bwd(q, k, v, g, beta, h0, dO, dhT)
+    for x, w in zip(got, want):
+        assert np.all(np.isfinite(x))
+        w = w[0]
+        scale = np.sqrt(np.mean(w * w)) + np.abs(w)
+        assert np.max(np.abs(x - w) / np.where(scale > 0, scale, 1.0)) <= 1e-3   # dg: fp32 rounding of a cancelling sum
