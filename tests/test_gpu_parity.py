@@ -403,3 +403,19 @@ def test_bounded_wait_expiry_is_reported_and_context_survives():
     o, hT = run_prefill(x)
     check_prefill(x, o, hT, TOL_BF16)
     assert kda.device_status() == kda.KDA_OK
+
+
+# ------------------------------------------------------- several devices ---
+
+@pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs two visible GPUs")
+def test_prefill_on_two_devices_in_one_process():
+    """Kernel attributes are set per device: a prefill on cuda:0 and then on
+    cuda:1 (no peer access) both launch and both match the oracle."""
+    x = prefill_inputs(1, 100, 2, 128, 128, seed=61, h0_std=0.1)
+    o_ref, hT_ref = oracle.fwd(x["q"], x["k"], x["v"], x["g"], x["beta"], x["h0"])
+    for dev in (torch.device("cuda", 0), torch.device("cuda", 1)):
+        d = {k: (None if t is None else t.to(dev)) for k, t in x.items()}
+        o, hT = kda.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["h0"])
+        torch.cuda.synchronize(dev)
+        check_out(o, o_ref, TOL_BF16)
+        assert err_state(hT, hT_ref) <= TOL_BF16
