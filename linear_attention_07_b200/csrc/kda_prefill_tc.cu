@@ -1045,20 +1045,16 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             // o of chunk cp (X buffer cp & 1, complete since chunk cp's last
             // MMA wait), written from registers: lanes hold adjacent dv
             // columns, so each warp store covers 64 contiguous bytes of a row
-            // in two halves of 8 tokens: the first while the second half of the
-            // next chunk's first product runs, the second while its state
-            // increment runs (the X buffer of chunk cp is next written by chunk
-            // cp + 2's first product, after both)
-            auto emit_output = [&](int cp, int part) {
+            auto emit_output = [&](int cp) {
                 const uint32_t dx = (cp & 1) ? CT_DX1 : CT_DX0;
-                float ov[8];
-                tmem_ld8(tm + lane_base + dx + C + 16 * hh + 8 * part, ov);
+                float ov[16];
+                tmem_ld16(tm + lane_base + dx + C + 16 * hh, ov);
                 wait_ld();
-                const int tt = cp * C + 16 * hh + 8 * part;   // token of ov[0] within the segment
+                const int tt = cp * C + 16 * hh;              // token of ov[0] within the segment
                 __nv_bfloat16* op = o + ((int64_t)b * T + ts + tt) * (int64_t)H * D + (int64_t)h * D + j;
                 if (!(flags & SEG_NO_O)) {
 #pragma unroll
-                    for (int r = 0; r < 8; ++r)
+                    for (int r = 0; r < 16; ++r)
                         if (tt + r < Tl) op[(int64_t)r * H * D] = __float2bfloat16_rn(ov[r]);
                 }
             };
@@ -1082,7 +1078,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     fence_before_sync();
                     named_arrive(NB_ASB, NX);
                     snapshot(ts / C + ch - 1);                  // S after chunk ch - 1
-                    emit_output(ch - 1, 0);
+                    emit_output(ch - 1);
                 }
                 // X of chunk ch (U' of this chunk is in the slot once its FULL phase passed)
                 if (tid == 0 && !s_abort &&
@@ -1103,7 +1099,6 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 fence_before_sync();
                 named_arrive(NB_U, NX);
                 decay(sb);                            // while Kb^T U and P U run
-                if (ch > 0) emit_output(ch - 1, 1);
                 wait_bar(kbar0, (uint32_t)ch & 1u);   // Kb^T U, first d_k half, of chunk ch
             }
             if (n_chunks > 0) {
@@ -1111,8 +1106,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 wait_bar(kbar1, (uint32_t)(n_chunks - 1) & 1u);
                 state_half(1);
                 snapshot(ts / C + n_chunks - 1);
-                emit_output(n_chunks - 1, 0);
-                emit_output(n_chunks - 1, 1);
+                emit_output(n_chunks - 1);
             }
             if (hT && !s_abort) {
                 float* hTh = hT + head_off * D * D;
