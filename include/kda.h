@@ -248,6 +248,21 @@ int kda_chunk_bwd(const void* q, const void* k, const void* v, const void* g, co
                   int B, int T, int H, int d_k, int d_v, kda_stream_t stream);
 
 /*
+ * kda_chunk_bwd_raw -- gradients of a kda_chunk_fwd_raw call: as
+ * kda_chunk_bwd, with q_raw, k_raw and the gate pre-activation z in the
+ * places of q, k and g, and dq_raw, dk_raw, dz returned for them.  The
+ * prologue runs inside the kernels as in the raw forward (q, k normalised in
+ * fp32, a zero vector staying zero with a zero gradient; g = -5 sigmoid(z),
+ * g = 0 past the end), and its chain rule (dr = (dx - x (x . dx)) / |r|,
+ * dz = -5 sigmoid(z) (1 - sigmoid(z)) dg) is applied to the outputs, so no
+ * normalised tensor is written.  Layouts, workspace, errors as kda_chunk_bwd.
+ */
+int kda_chunk_bwd_raw(const void* q_raw, const void* k_raw, const void* v, const void* z, const void* beta,
+                      const float* h0, const void* dO, const float* dhT,
+                      void* dq_raw, void* dk_raw, void* dv, void* dz, void* dbeta, float* dh0,
+                      int B, int T, int H, int d_k, int d_v, kda_stream_t stream);
+
+/*
  * kda_verify_fwd -- K consecutive tokens of each of N requests from a start
  * state, keeping the state after EVERY token (speculative decoding: verify
  * K drafted tokens, then continue from the state after the last accepted

@@ -35,7 +35,7 @@ KDA_ERR_NO_MEMORY = -5
 
 EXPORTED = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_states", "kda_chunk_fwd_f32",
             "kda_chunk_transition", "kda_state_chain", "kda_chunk_fwd_raw", "kda_decode_step",
-            "kda_decode_step_raw", "kda_verify_fwd", "kda_chunk_bwd",
+            "kda_decode_step_raw", "kda_verify_fwd", "kda_chunk_bwd", "kda_chunk_bwd_raw",
             "kda_device_status", "kda_selftest_bounded_wait",
             "kda_status_string", "kda_launch_count", "kda_prefill_path", "kda_version")
 
@@ -88,6 +88,8 @@ def load_library(path: str = LIB_PATH):
     lib.kda_chunk_bwd.argtypes = [vp, vp, vp, vp, vp, fp, vp, fp, vp, vp, vp, vp, vp, fp,
                                   i, i, i, i, i, vp]
     lib.kda_chunk_bwd.restype = i
+    lib.kda_chunk_bwd_raw.argtypes = lib.kda_chunk_bwd.argtypes
+    lib.kda_chunk_bwd_raw.restype = i
     lib.kda_verify_fwd.argtypes = [vp, vp, vp, vp, vp, fp, vp, fp, i, i, i, i, i, vp]
     lib.kda_verify_fwd.restype = i
     lib.kda_device_status.argtypes = [vp]
@@ -379,12 +381,7 @@ def verify_fwd(q, k, v, g, beta, h0=None, *, o=None, states=None):
     return o, states
 
 
-def chunk_bwd(q, k, v, g, beta, h0, dO, dhT=None, *, want_dh0=True):
-    """Gradients of chunk_fwd (kda_chunk_bwd): with L = sum(dO * o) +
-    sum(dhT * hT), returns (dq, dk, dv, dg, dbeta, dh0); dq, dk, dg, dv,
-    dbeta bf16 in the input layouts, dh0 [B, H, dk, dv] fp32 (None if
-    want_dh0 is False).  dO: [B, T, H, dv] bf16; dhT: [B, H, dk, dv] fp32 or
-    None; h0 as for chunk_fwd."""
+def _bwd(fn_name, q, k, v, g, beta, h0, dO, dhT, want_dh0):
     import torch
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -401,9 +398,24 @@ def chunk_bwd(q, k, v, g, beta, h0, dO, dhT=None, *, want_dh0=True):
     gb = torch.empty((B, T, H), dtype=torch.bfloat16, device=dev)
     gh = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_dh0 else None
     with torch.cuda.device(dev):
-        st = load_library().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
-                                          _ptr(dO), _ptr(dhT), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gg),
-                                          _ptr(gb), _ptr(gh), B, T, H, dk, dv, _stream(dev))
+        st = getattr(load_library(), fn_name)(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(h0),
+                                              _ptr(dO), _ptr(dhT), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gg),
+                                              _ptr(gb), _ptr(gh), B, T, H, dk, dv, _stream(dev))
     if st != KDA_OK:
-        raise KdaError("kda_chunk_bwd", st)
+        raise KdaError(fn_name, st)
     return gq, gk, gv, gg, gb, gh
+
+
+def chunk_bwd(q, k, v, g, beta, h0, dO, dhT=None, *, want_dh0=True):
+    """Gradients of chunk_fwd (kda_chunk_bwd): with L = sum(dO * o) +
+    sum(dhT * hT), returns (dq, dk, dv, dg, dbeta, dh0); dq, dk, dg, dv,
+    dbeta bf16 in the input layouts, dh0 [B, H, dk, dv] fp32 (None if
+    want_dh0 is False).  dO: [B, T, H, dv] bf16; dhT: [B, H, dk, dv] fp32 or
+    None; h0 as for chunk_fwd."""
+    return _bwd("kda_chunk_bwd", q, k, v, g, beta, h0, dO, dhT, want_dh0)
+
+
+def chunk_bwd_raw(q_raw, k_raw, v, z, beta, h0, dO, dhT=None, *, want_dh0=True):
+    """Gradients of chunk_fwd_raw (kda_chunk_bwd_raw): (dq_raw, dk_raw, dv,
+    dz, dbeta, dh0), the prologue and its chain rule inside the kernels."""
+    return _bwd("kda_chunk_bwd_raw", q_raw, k_raw, v, z, beta, h0, dO, dhT, want_dh0)

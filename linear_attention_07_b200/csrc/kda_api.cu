@@ -47,7 +47,8 @@ cudaError_t verify_launch(const void* q, const void* k, const void* v, const voi
 
 cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const void* g, const void* beta,
                              const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv,
-                             void* dg, void* dbeta, float* dh0, int B, int T, int H, cudaStream_t stream);
+                             void* dg, void* dbeta, float* dh0, int B, int T, int H, bool raw,
+                             cudaStream_t stream);
 
 cudaError_t prefill_tc_launch(const void* q, const void* k, const void* v, const void* g,
                               const void* beta, const float* h0, void* o, float* hT,
@@ -228,10 +229,10 @@ int kda_decode_step_raw(const void* q_raw, const void* k_raw, const void* v, con
     return decode_step_any(q_raw, k_raw, v, z, beta, state, o, N, H, dk, dv, true, stream);
 }
 
-int kda_chunk_bwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
-                  const float* h0, const void* dO, const float* dhT,
-                  void* dq, void* dk, void* dv, void* dg, void* dbeta, float* dh0,
-                  int B, int T, int H, int d_k, int d_v, kda_stream_t stream)
+static int chunk_bwd_any(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                         const float* h0, const void* dO, const float* dhT,
+                         void* dq, void* dk, void* dv, void* dg, void* dbeta, float* dh0,
+                         int B, int T, int H, int d_k, int d_v, bool raw, kda_stream_t stream)
 {
     int st = check_prefill(q, k, v, g, beta, h0, dO, dhT, B, T, H, d_k, d_v);
     if (st != KDA_OK) return st;
@@ -245,8 +246,26 @@ int kda_chunk_bwd(const void* q, const void* k, const void* v, const void* g, co
     }
     if ((int64_t)B * H == 0) return KDA_OK;
     if (T == 0 && dh0 == nullptr) return KDA_OK;
-    return status_of(chunk_bwd_launch(q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, B, T, H,
+    return status_of(chunk_bwd_launch(q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, B, T, H, raw,
                                       (cudaStream_t)stream));
+}
+
+int kda_chunk_bwd(const void* q, const void* k, const void* v, const void* g, const void* beta,
+                  const float* h0, const void* dO, const float* dhT,
+                  void* dq, void* dk, void* dv, void* dg, void* dbeta, float* dh0,
+                  int B, int T, int H, int d_k, int d_v, kda_stream_t stream)
+{
+    return chunk_bwd_any(q, k, v, g, beta, h0, dO, dhT, dq, dk, dv, dg, dbeta, dh0, B, T, H, d_k, d_v, false,
+                         stream);
+}
+
+int kda_chunk_bwd_raw(const void* q_raw, const void* k_raw, const void* v, const void* z, const void* beta,
+                      const float* h0, const void* dO, const float* dhT,
+                      void* dq_raw, void* dk_raw, void* dv, void* dz, void* dbeta, float* dh0,
+                      int B, int T, int H, int d_k, int d_v, kda_stream_t stream)
+{
+    return chunk_bwd_any(q_raw, k_raw, v, z, beta, h0, dO, dhT, dq_raw, dk_raw, dv, dz, dbeta, dh0, B, T, H,
+                         d_k, d_v, true, stream);
 }
 
 int kda_verify_fwd(const void* q, const void* k, const void* v, const void* g,

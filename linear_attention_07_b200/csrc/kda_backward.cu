@@ -94,6 +94,44 @@ __device__ __forceinline__ void running_sum(float* G)
     }
 }
 
+// The fused prologue on a chunk's rows in shared memory (row stride LD), as
+// the raw forward applies it: q and k scaled to unit norm over the channels
+// (rsqrt of the sum of squares; a zero row stays zero), the gate
+// pre-activation z turned into g = -5 sigmoid(z) (g = 0 past the end of the
+// sequence).  Any of the pointers may be null; the inverse norms are kept
+// for the chain rule.
+template <int NTH>
+__device__ __forceinline__ void prologue_rows(float* sQ, float* invQ, float* sK, float* invK, float* sG, int n_valid)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int r = warp; r < C; r += NTH / 32) {
+        float sq = 0.f, sk = 0.f;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+            const int c = lane + 32 * j;
+            if (sQ) sq = fmaf(sQ[r * LD + c], sQ[r * LD + c], sq);
+            if (sK) sk = fmaf(sK[r * LD + c], sK[r * LD + c], sk);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+        }
+        const float iq = sq > 0.f ? rsqrtf(sq) : 0.f, ik = sk > 0.f ? rsqrtf(sk) : 0.f;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+            const int c = lane + 32 * j;
+            if (sQ) sQ[r * LD + c] *= iq;
+            if (sK) sK[r * LD + c] *= ik;
+            if (sG) sG[r * LD + c] = r < n_valid ? -5.f / (1.f + __expf(-sG[r * LD + c])) : 0.f;
+        }
+        if (lane == 0) {
+            if (invQ) invQ[r] = iq;
+            if (invK) invK[r] = ik;
+        }
+    }
+}
+
 // Reference of the tile-relative factors of row r: Gam before its tile.
 __device__ __forceinline__ float tile_ref(const float* G, int r, int c)
 {
@@ -140,6 +178,7 @@ __device__ __forceinline__ void tgemm(FA a, FB b, FO out)
 constexpr int PREP_BIG = 8;                                  // K, Q, V, G, four scratch
 constexpr size_t PREP_SMEM = (size_t)(PREP_BIG * C * LD + 4 * C * L32 + C) * sizeof(float);
 
+template <bool RAW>    // RAW: q, k unnormalised and g the gate pre-activation (the fused prologue)
 __global__ void __launch_bounds__(NT, 1)
 bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                 const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ g,
@@ -174,6 +213,10 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     load_rows(sG, g, row0, rs, Tl);
     if (tid < C) sB[tid] = tid < Tl ? bf(beta[((int64_t)b * T + t0 + tid) * H + h]) : 0.f;
     __syncthreads();
+    if constexpr (RAW) {
+        prologue_rows<NT>(sQ, nullptr, sK, nullptr, sG, Tl);
+        __syncthreads();
+    }
     running_sum(sG);
     __syncthreads();
     // tile-relative operands of the pair products
@@ -489,11 +532,12 @@ bwd_chains_kernel(const float* __restrict__ rec_all, const __nv_bfloat16* __rest
 
 constexpr int LOC_BIG = 11;    // K, Q, V, dO, G, W, U, dU, dKb, dQt, dW
 constexpr int BLK = D * LJ > JB * LD ? D * LJ : JB * LD;    // one S0 or dS block (either shape)
-constexpr size_t LOC_SMEM = (size_t)(LOC_BIG * C * LD + 2 * BLK + 6 * C * L32 + 2 * C + 2 * D) * sizeof(float);
+constexpr size_t LOC_SMEM = (size_t)(LOC_BIG * C * LD + 2 * BLK + 6 * C * L32 + 4 * C + 2 * D) * sizeof(float);
 constexpr int NL = 2 * NT;     // threads of the local kernel: 16 warps hide the shared-memory latency
 
 __device__ __forceinline__ __nv_bfloat16 to_bf(float x) { return __float2bfloat16_rn(x); }
 
+template <bool RAW>    // RAW: the fused prologue, and its chain rule on dq, dk, dg
 __global__ void __launch_bounds__(NL, 1)
 bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                  const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ g,
@@ -527,6 +571,8 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     float* sDB = sB + C;           // dbeta [C]
     float* sRS = sDB + C;          // sum_j dS_ij S0_ij [D]
     float* sKS = sRS + D;          // sum_r dKb_rc Kb_rc [D]
+    float* sIQ = sKS + D;          // RAW: 1 / |q_raw| per token [C]
+    float* sIK = sIQ + C;          // RAW: 1 / |k_raw| per token [C]
 
     const int c_idx = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = c_idx * C;
@@ -564,6 +610,10 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     }
     if (tid < D) sRS[tid] = 0.f;
     __syncthreads();
+    if constexpr (RAW) {
+        prologue_rows<NL>(nullptr, nullptr, bK, sIK, bG, Tl);
+        __syncthreads();
+    }
     running_sum(bG);
     __syncthreads();
     for (int e = tid; e < C * D; e += NL) {                       // Kb = K exp(Gam_C - Gam)
@@ -672,6 +722,10 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
 
     // ---- Q back in place of Kb; dGam from the direct terms; dq, dk partials
     load_rows<NL>(bQ, q, row0, rs, Tl);
+    if constexpr (RAW) {
+        __syncthreads();
+        prologue_rows<NL>(bQ, sIQ, nullptr, nullptr, nullptr, Tl);
+    }
     if (tid < D) {                                   // sum_r dKb_rc Kb_rc, before dKb is rescaled
         const int c = tid;
         const float gl = bG[(C - 1) * LD + c];
@@ -849,6 +903,35 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         }
     }
     __syncthreads();
+    if constexpr (RAW) {
+        // the prologue's chain rule: for x = r / |r|, dr = (dx - x (x . dx)) / |r|
+        // (zero where r = 0); for g = -5 sigmoid(z), dz = dg g (1 + g / 5),
+        // with g the difference of the running sums
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int r = warp; r < C; r += NL / 32) {
+            float dotq = 0.f, dotk = 0.f;
+#pragma unroll
+            for (int j = 0; j < D / 32; ++j) {
+                const int c = lane + 32 * j;
+                dotq = fmaf(bQ[r * LD + c], bDQT[r * LD + c], dotq);
+                dotk = fmaf(bK[r * LD + c], bDKB[r * LD + c], dotk);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                dotq += __shfl_xor_sync(0xffffffffu, dotq, off);
+                dotk += __shfl_xor_sync(0xffffffffu, dotk, off);
+            }
+#pragma unroll
+            for (int j = 0; j < D / 32; ++j) {
+                const int c = lane + 32 * j;
+                bDQT[r * LD + c] = (bDQT[r * LD + c] - bQ[r * LD + c] * dotq) * sIQ[r];
+                bDKB[r * LD + c] = (bDKB[r * LD + c] - bK[r * LD + c] * dotk) * sIK[r];
+                const float gr = bG[r * LD + c] - (r > 0 ? bG[(r - 1) * LD + c] : 0.f);
+                bV[r * LD + c] *= gr * (1.f + 0.2f * gr);
+            }
+        }
+        __syncthreads();
+    }
     for (int e = tid; e < C * D; e += NL) {
         const int r = e / D, c = e % D;
         if (r < Tl) {
@@ -867,14 +950,16 @@ static DeviceFlags g_bwd_attr_done;
 
 cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const void* g, const void* beta,
                              const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv,
-                             void* dg, void* dbeta, float* dh0, int B, int T, int H, cudaStream_t stream)
+                             void* dg, void* dbeta, float* dh0, int B, int T, int H, bool raw, cudaStream_t stream)
 {
     using namespace bw;
     cudaError_t e = once_per_device(g_bwd_attr_done, [](int) {
         const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
-        cudaError_t r = cudaFuncSetAttribute(bwd_prep_kernel, a, (int)PREP_SMEM);
+        cudaError_t r = cudaFuncSetAttribute(bwd_prep_kernel<false>, a, (int)PREP_SMEM);
+        if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_prep_kernel<true>, a, (int)PREP_SMEM);
         if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_chains_kernel, a, (int)CHAIN_SMEM);
-        if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_local_kernel, a, (int)LOC_SMEM);
+        if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_local_kernel<false>, a, (int)LOC_SMEM);
+        if (r == cudaSuccess) r = cudaFuncSetAttribute(bwd_local_kernel<true>, a, (int)LOC_SMEM);
         return r;
     });
     if (e != cudaSuccess) return e;
@@ -902,7 +987,8 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     const __nv_bfloat16* bg = (const __nv_bfloat16*)g;
     const __nv_bfloat16* bb = (const __nv_bfloat16*)beta;
     const __nv_bfloat16* bdo = (const __nv_bfloat16*)dO;
-    bwd_prep_kernel<<<grid_c, NT, PREP_SMEM, stream>>>(bq, bk, bv, bg, bb, rec, T, H, n_chunks);
+    (raw ? bwd_prep_kernel<true> : bwd_prep_kernel<false>)<<<grid_c, NT, PREP_SMEM, stream>>>(
+        bq, bk, bv, bg, bb, rec, T, H, n_chunks);
     e = cudaGetLastError();
     if (e == cudaSuccess) {
         bwd_chains_kernel<<<grid_s, NT_CHAIN, CHAIN_SMEM, stream>>>(rec, bdo, h0, dhT, S0_all, dS_all, dh0, T, H,
@@ -910,7 +996,7 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
         e = cudaGetLastError();
     }
     if (e == cudaSuccess) {
-        bwd_local_kernel<<<grid_c, NL, LOC_SMEM, stream>>>(
+        (raw ? bwd_local_kernel<true> : bwd_local_kernel<false>)<<<grid_c, NL, LOC_SMEM, stream>>>(
             bq, bk, bv, bg, bb, bdo, rec, S0_all, dS_all, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk,
             (__nv_bfloat16*)dv, (__nv_bfloat16*)dg, (__nv_bfloat16*)dbeta, T, H, n_chunks);
         e = cudaGetLastError();

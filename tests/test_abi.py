@@ -175,6 +175,10 @@ def test_backward_argument_errors(lib):
     assert bwd(d_k=64, d_v=64) == kda.KDA_ERR_UNSUPPORTED
     assert bwd(B=0) == kda.KDA_OK
     assert bwd(T=0, dh0=NUL) == kda.KDA_OK                 # nothing to write
+    raw = lib.kda_chunk_bwd_raw
+    assert raw(A, A, A, A, A2, NUL, NUL, NUL, A, A, A, A, A2, A, 1, 64, 2, 128, 128, None) == kda.KDA_ERR_INVALID_ARG
+    assert raw(A, A, A, A, A2, NUL, A, NUL, A, A, A, A, A2, A, 1, 64, 2, 64, 64, None) == kda.KDA_ERR_UNSUPPORTED
+    assert raw(A, A, A, A, A2, NUL, A, NUL, A, A, A, A, A2, A, 0, 64, 2, 128, 128, None) == kda.KDA_OK
     assert lib.kda_launch_count() == n0
 
 
@@ -247,6 +251,7 @@ def test_binding_requires_cuda_tensors(lib):
         lambda: kda.decode_step_raw(d, d, d, d, db, st),
         lambda: kda.verify_fwd(x, x, x, x, b),
         lambda: kda.chunk_bwd(x, x, x, x, b, None, x),
+        lambda: kda.chunk_bwd_raw(x, x, x, x, b, None, x),
     ]
     for call in calls:
         with pytest.raises(ValueError, match="CUDA"):

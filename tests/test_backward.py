@@ -122,3 +122,25 @@ def test_bwd_matches_split_identity():
     torch.cuda.synchronize()
     joined = [torch.cat([u, w], 1) for u, w in zip(g1[:5], g2[:5])] + [g1[5]]
     check_grads(x, dO, dhT, joined, dh0_tol=2e-3)
+
+
+@pytest.mark.parametrize("B,H,T", [(1, 2, 77), (2, 3, 300)])
+def test_bwd_through_fused_prologue(B, H, T):
+    """kda_chunk_bwd_raw against the oracle's backward through the prologue
+    (q, k normalised, g = -5 sigmoid(z); zero q/k rows; ragged lengths)."""
+    from linear_attention_07_b200.inputs import raw_inputs
+    x = raw_inputs((B, T, H, 128), (B, T, H, 128), (B, T, H), seed=4800 + T, zero_rows=2)
+    gen = torch.Generator().manual_seed(4801 + T)
+    h0 = torch.randn((B, H, 128, 128), generator=gen) * 0.1
+    dO = torch.randn((B, T, H, 128), generator=gen).to(torch.bfloat16)
+    dhT = torch.randn((B, H, 128, 128), generator=gen) * 0.1
+    d = {k: t.to(DEV) for k, t in x.items()}
+    got = kda.chunk_bwd_raw(d["q"], d["k"], d["v"], d["z"], d["beta"], h0.to(DEV), dO.to(DEV), dhT.to(DEV))
+    torch.cuda.synchronize()
+    assert kda.device_status() == kda.KDA_OK
+    want = oracle.bwd_raw(x["q"], x["k"], x["v"], x["z"], x["beta"], h0, dO, dhT)
+    for name, gval, wval in zip(("dq_raw", "dk_raw", "dv", "dz", "dbeta"), got[:5], want[:5]):
+        assert torch.isfinite(gval).all(), name
+        check_out(gval, wval, TOL_BF16, what=name)
+    assert err_state(got[5], want[5]) <= 1e-3
+    assert not got[0][:, :2].float().abs().max() > 0, "zero q rows must have a zero gradient"
