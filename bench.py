@@ -441,7 +441,7 @@ def bench_backward(args, kda, dev, rank, world, hbm_gbs, peak_src):
            "roofline": {"bound": "alu", "achieved": round(ach_f, 2), "peak": round(peak_alu, 1),
                         "unit": "TFLOP/s", "frac": round(ach_f / peak_alu, 4), "traffic": None,
                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x median SM clock",
-                        "alg_flops_per_launch": alg_f, "kernel": "kda_chunk_bwd (4 launches)"},
+                        "alg_flops_per_launch": alg_f, "kernel": "kda_chunk_bwd (3 launches)"},
            "hbm": {"achieved": round(ach_b, 1), "peak": hbm_gbs, "unit": "GB/s",
                    "frac": round(ach_b / hbm_gbs, 4), "alg_bytes_per_launch": alg_b,
                    "peak_source": peak_src + " hbm_gbs"},
