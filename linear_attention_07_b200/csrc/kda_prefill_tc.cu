@@ -746,15 +746,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
 // ============================================================================
 // Cluster variant for few heads (B * H small next to the SM count): each head
-// gets a cluster of four CTAs on four SMs.  Rank 0 runs the chain; ranks 1-3
-// prepare the chunks ch with ch % 3 == rank - 1, each in its own SM, and push
-// every prepared chunk (the chain's operands and U') into slot ch % 3 of rank
-// 0's shared memory with a single bulk copy (shared::cta -> shared::cluster,
-// no multicast).  FULL[slot] (rank 0) counts the copy's bytes and is armed by
-// rank 0 itself when it hands the slot back; EMPTY (the preparing CTA) is
-// arrived on by rank 0 once the chunk's MMAs are done and its decay applied.
-// o of a chunk is written from registers, one chunk late, while the next
-// chunk's first MMA runs.  The arithmetic is the one of prefill_tc_kernel.
+// gets a cluster of four CTAs on four SMs.  Role 0 (the CTA of cluster rank
+// CHAIN_RANK) runs the chain; roles 1-3 prepare the chunks ch with
+// ch % 3 == role - 1, each in its own SM, and push every prepared chunk (the
+// chain's operands and U') into slot ch % 3 of the chain CTA's shared memory
+// with a single bulk copy (shared::cta -> shared::cluster, no multicast).
+// FULL[slot] (chain CTA) counts the copy's bytes and is armed by the chain CTA
+// itself when it hands the slot back; EMPTY (the preparing CTA) is arrived on
+// by the chain CTA once the chunk's MMAs are done and its decay applied.  o of
+// a chunk is staged one chunk late, while the next chunk's first MMA runs,
+// and written by a tensor store.  The arithmetic is the one of
+// prefill_tc_kernel.
 namespace pc {
 using namespace pf;
 constexpr int NCW = 256;                                      // compute threads per CTA (both roles)
@@ -764,7 +766,13 @@ constexpr int NTH = NCW + 64;                                 // plus an issuer 
 constexpr uint32_t NB_ASA = 1, NB_ASB = 2, NB_U = 3, NB_CW = 4;                 // chain CTA
 constexpr uint32_t NB_G = 5, NB_TB = 6, NB_STFREE = 7, NB_FILL = 8;              // preparing CTAs
 constexpr int NPREPCTA = 3;                                   // preparing CTAs per cluster (= slots)
-// slot / staging layout (identical in rank 0's slots and a preparer's staging)
+// Cluster rank of the chain CTA; the preparing CTAs follow it cyclically.
+// A cluster of four occupies two TPCs (ranks 0-1 and 2-3).  With the chain on
+// rank 0 the slots of some clusters streamed in too slowly (up to 20 % longer
+// per chunk, depending on where the cluster was placed); with the chain on
+// the second TPC every cluster kept pace (measured on the 8K workload).
+constexpr uint32_t CHAIN_RANK = 2;
+// slot / staging layout (identical in role 0's slots and a preparer's staging)
 constexpr uint32_t S_B1 = 0;                                   // [W | Qt]: N 64 x K 128 (padded)
 constexpr uint32_t S_B2 = S_B1 + 8 * SBO_K128P;                // Kb: N 128 x K 32
 constexpr uint32_t S_B3 = S_B2 + (D / 8) * SBO_K32;            // P: N 32 x K 32 (dense: vector stores)
@@ -772,10 +780,11 @@ constexpr uint32_t S_GAM = S_B3 + (C / 8) * SBO_K32;           // gamma_C, 128 f
 constexpr uint32_t S_UP = S_GAM + D * 4;                       // U' [32 tokens][128] fp32
 constexpr uint32_t SLOT = S_UP + C * D * 4;                    // bytes per chunk
 static_assert(SLOT % 16 == 0, "bulk copy size");
-// rank 0 (chain): NPREPCTA slots
+// role 0 (chain): NPREPCTA slots
 constexpr uint32_t C_SLOT0 = 0;
-constexpr uint32_t C_BYTES = NPREPCTA * SLOT;
-// ranks 1-3 (preparation)
+constexpr uint32_t C_OST = NPREPCTA * SLOT;                    // o staging of one chunk (32 x 128 bf16)
+constexpr uint32_t C_BYTES = C_OST + C * D * 2;
+// roles 1-3 (preparation)
 constexpr uint32_t P_RAW = 0;
 constexpr uint32_t P_BETA = P_RAW + 4 * RAW_T;
 constexpr uint32_t P_GEX = P_BETA + C * 4;
@@ -794,9 +803,10 @@ constexpr uint32_t P_NRM = P_YMS + TILE * (TILE + 1) * 4;    // prologue: per-wa
 constexpr uint32_t P_BYTES = P_NRM + NRM_BYTES;
 constexpr uint32_t SMEM_BYTES = P_BYTES > C_BYTES ? P_BYTES : C_BYTES;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(C_OST % 128 == 0, "tensor store source alignment");
 static_assert(P_ST % 16 == 0 && P_GA % 16 == 0 && P_GB % 16 == 0 && P_WA % 16 == 0 && P_VA % 16 == 0 &&
               P_TB % 16 == 0 && SLOT % 16 == 0, "alignment");
-// tensor memory: rank 0 uses 416 columns (512 allocated), ranks 1-3 use 128
+// tensor memory: role 0 uses 416 columns (512 allocated), roles 1-3 use 128
 constexpr uint32_t CT_AS = 0, CT_AU = 128, CT_DX0 = 160, CT_DKU = 224, CT_DX1 = 352;
 constexpr uint32_t PT_DG = 0, PT_DW = 64, PT_DU = 96;
 }  // namespace pc
@@ -805,6 +815,7 @@ template <bool PRO>       // PRO: the fused prologue (launch flag PROLOGUE)
 __global__ void __cluster_dims__(pc::NPREPCTA + 1, 1, 1) __launch_bounds__(pc::NTH, 1)
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                       const __grid_constant__ CUtensorMap tm_o,
                        const __nv_bfloat16* __restrict__ beta, const float* h0,
                        __nv_bfloat16* __restrict__ o, float* hT, int T, int H,
                        int seg_len, int n_seg, uint32_t flags, float* states, int snap_every,
@@ -814,13 +825,16 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     using namespace tc;
     extern __shared__ __align__(1024) unsigned char sm[];
     __shared__ uint32_t s_taddr;
-    __shared__ __align__(8) uint64_t s_bar[6];   // rank 0: FULL[0..2], X, KU0, KU1; ranks 1-3: EMPTY, MMA, input loads
+    __shared__ __align__(8) uint64_t s_bar[7];   // role 0: FULL[0..2], X, KU0, KU1, o staged; roles 1-3: EMPTY, MMA, input loads
     __shared__ int s_abort;
-    __shared__ uint32_t s_odone;                 // rank 0: chunks whose slot is consumed
-    __shared__ int s_last_armed[NPREPCTA];       // rank 0: last chunk whose bytes FULL[slot] expects
+    __shared__ uint32_t s_odone;                 // role 0: chunks whose slot is consumed
+    __shared__ uint32_t s_full;                  // role 0: chunks whose slot has landed (FULL observed)
+    __shared__ uint32_t s_ofree;                 // role 0: chunks whose o store has read the staging
+    __shared__ int s_last_armed[NPREPCTA];       // role 0: last chunk whose bytes FULL[slot] expects
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint32_t rank = cluster_ctarank();
+    // role: 0 = chain, 1..3 = preparing CTA (the cluster rank shifted by CHAIN_RANK)
+    const uint32_t role = (cluster_ctarank() + 4u - CHAIN_RANK) & 3u;
     // grid.y = B * n_seg: sequence b, segment [ts, ts + Tl) of it (n_seg = 1: the whole sequence)
     const int h = blockIdx.x / (NPREPCTA + 1), bb = blockIdx.y;
     const int b = bb / n_seg;
@@ -828,7 +842,8 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const int Tl = max(0, min(seg_len, T - ts));
     const int64_t head_off = (int64_t)bb * H + h;          // h0 / hT: [B * n_seg][H][D][D]
     const int n_chunks = (Tl + C - 1) / C;
-    const uint32_t ncols = rank == 0 ? 512u : 128u;
+    const uint32_t ncols = role == 0 ? 512u : 128u;
+    const bool store_o = o != nullptr && !(flags & SEG_NO_O);    // o rows go out by tensor stores
 
     if (warp == 0) {
         tmem_alloc(smem_u32(&s_taddr), ncols);
@@ -836,13 +851,16 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     }
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
+        mbar_init(smem_u32(&s_bar[6]), NCW / 32);    // one arrive per compute warp
         fence_mbar_init();
         s_abort = 0;
         s_odone = 0;
-        // rank 0: FULL[s] expects the bytes of chunk s's push; later uses are
+        s_full = 0;
+        s_ofree = 0;
+        // role 0: FULL[s] expects the bytes of chunk s's push; later uses are
         // armed when the slot is released (the push itself carries no arrive)
         for (int i = 0; i < NPREPCTA; ++i) s_last_armed[i] = -1;
-        if (rank == 0)
+        if (role == 0)
             for (int i = 0; i < NPREPCTA && i < n_chunks; ++i) {
                 mbar_arrive_expect_tx(smem_u32(&s_bar[i]), SLOT);
                 s_last_armed[i] = i;
@@ -860,7 +878,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         atomicExch(&g_prefill_status, (int)KDA_ERR_TIMEOUT);
     };
 
-    if (rank == 0) {
+    if (role == 0) {
         // ========================================================= chain CTA ==
         const uint32_t mbar = smem_u32(&s_bar[3]);   // X of each chunk
         const uint32_t kbar0 = smem_u32(&s_bar[4]);  // Kb^T U, d_k columns [0, 64)
@@ -942,14 +960,40 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             __syncwarp();
         } else if (warp == NCW / 32 + 1) {
             // ------------------------------------------------------ release warp --
-            // Once chunk ch - 1's last MMAs are done (and its decay applied),
-            // nothing reads its slot any more: hand it back to its preparer.
-            // A remote arrive is slow, so it stays off the issuer's and the
-            // compute warps' path.  Completion comes from a counter that the
-            // compute warps advance in order; a counter cannot be misread by a
-            // reader that lags.
+            // Chunk ch: observe its slot's FULL phase (a cluster-scope acquire,
+            // which costs a few hundred cycles) and publish that with a CTA
+            // counter, so the compute warps, which read U' from the slot, pay
+            // only a CTA-scope acquire on their path.  Then, once chunk ch - 1's
+            // last MMAs are done (and its decay applied), nothing reads its slot
+            // any more: hand it back to its preparer.  A remote arrive is slow,
+            // so it stays off the issuer's and the compute warps' path.
+            // Completion comes from a counter that the compute warps advance in
+            // order; a counter cannot be misread by a reader that lags.
+            // o of chunk cp, once the compute warps have staged it: one tensor
+            // store (rows past T are clipped by the tensor map), then the
+            // staging is handed back as soon as the store has read it.
+            auto store_output = [&](int cp) {
+                if (lane == 0) {
+                    if (!s_abort && !mbar_wait(smem_u32(&s_bar[6]), (uint32_t)cp & 1u, wait_ns)) expired();
+                    if (!*(volatile int*)&s_abort) {
+                        tma_store_3d(&tm_o, h * D, ts + cp * C, b, smem_u32(sm + C_OST));
+                        bulk_commit();
+                    }
+                    bulk_wait_read_all();
+                    counter_publish(smem_u32(&s_ofree), (uint32_t)cp + 1u);
+                }
+                __syncwarp();
+            };
 #pragma unroll 1
-            for (int ch = 1; ch < n_chunks; ++ch) {
+            for (int ch = 0; ch < n_chunks; ++ch) {
+                if (lane == 0) {
+                    if (!s_abort &&
+                        !mbar_wait_cluster(smem_u32(&s_bar[ch % NPREPCTA]), (uint32_t)(ch / NPREPCTA) & 1u, wait_ns))
+                        expired();
+                    if (!*(volatile int*)&s_abort) counter_publish(smem_u32(&s_full), (uint32_t)ch + 1u);
+                }
+                __syncwarp();
+                if (ch == 0) continue;
                 if (lane == 0) {
                     if (!s_abort && !counter_wait(smem_u32(&s_odone), (uint32_t)ch, wait_ns)) expired();
                     // After an expired wait no slot is handed back (its previous
@@ -963,16 +1007,20 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                             mbar_arrive_expect_tx(smem_u32(&s_bar[sl]), SLOT);
                             s_last_armed[sl] = cn;
                         }
-                        mbar_arrive_remote_relaxed(map_to_rank(smem_u32(&s_bar[0]), 1u + (uint32_t)sl));
+                        mbar_arrive_remote_relaxed(map_to_rank(smem_u32(&s_bar[0]), (CHAIN_RANK + 1u + (uint32_t)sl) & 3u));
                     }
                 }
                 __syncwarp();
+                if (store_o) store_output(ch - 1);
             }
+            if (store_o && n_chunks > 0) store_output(n_chunks - 1);
+            if (lane == 0) bulk_wait_all();   // every o store has landed (also after an expired wait)
+            __syncwarp();
         } else {
             // ----------------------------------------------------- compute warps --
             // Per chunk ch: the state increment of chunk ch - 1 by d_k halves
             // (each half handed to the issuer as soon as it is in tensor
-            // memory), the output of chunk ch - 1 (staged and written by TMA
+            // memory), the output of chunk ch - 1 (staged for a tensor store
             // while X of chunk ch is computed), then U = U' - W S, and the
             // decay S <- Diag(gamma_C) S while Kb^T U and P U run.  Chunk ch's
             // slot is then consumed and goes back to its preparer.
@@ -1043,20 +1091,27 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     }
             };
             // o of chunk cp (X buffer cp & 1, complete since chunk cp's last
-            // MMA wait), written from registers: lanes hold adjacent dv
-            // columns, so each warp store covers 64 contiguous bytes of a row
-            auto emit_output = [&](int cp) {
+            // MMA wait): the tensor-memory load is issued early (its wait is
+            // the next state half's), then the rows go to the staging buffer
+            // and the release warp writes them with one tensor store, off the
+            // compute warps' path (global stores from this SM are slow while
+            // the slots stream in).
+            float ov[16];
+            auto load_output = [&](int cp) {
                 const uint32_t dx = (cp & 1) ? CT_DX1 : CT_DX0;
-                float ov[16];
                 tmem_ld16(tm + lane_base + dx + C + 16 * hh, ov);
-                wait_ld();
-                const int tt = cp * C + 16 * hh;              // token of ov[0] within the segment
-                __nv_bfloat16* op = o + ((int64_t)b * T + ts + tt) * (int64_t)H * D + (int64_t)h * D + j;
-                if (!(flags & SEG_NO_O)) {
+            };
+            auto emit_output = [&](int cp) {
+                if (!store_o) return;
+                // the store of chunk cp - 1 has read the staging
+                if (lane == 0 && !s_abort && !counter_wait(smem_u32(&s_ofree), (uint32_t)cp, wait_ns)) expired();
+                __syncwarp();
+                __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
 #pragma unroll
-                    for (int r = 0; r < 16; ++r)
-                        if (tt + r < Tl) op[(int64_t)r * H * D] = __float2bfloat16_rn(ov[r]);
-                }
+                for (int r = 0; r < 16; ++r) ost[(16 * hh + r) * D + j] = __float2bfloat16_rn(ov[r]);
+                fence_smem_to_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&s_bar[6]));
             };
             fence_before_sync();
             if (n_chunks > 0) {                       // the initial state for chunk 0
@@ -1074,15 +1129,16 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     named_arrive(NB_ASA, NX);
                     wait_bar(kbar1, (uint32_t)(ch - 1) & 1u);   // Kb^T U second half and P U of chunk ch - 1
                     if (tid == 0) counter_publish(smem_u32(&s_odone), (uint32_t)ch);
-                    state_half(1);
+                    load_output(ch - 1);
+                    state_half(1);                              // (its wait covers the o load)
                     fence_before_sync();
                     named_arrive(NB_ASB, NX);
                     snapshot(ts / C + ch - 1);                  // S after chunk ch - 1
                     emit_output(ch - 1);
                 }
-                // X of chunk ch (U' of this chunk is in the slot once its FULL phase passed)
-                if (tid == 0 && !s_abort &&
-                    !mbar_wait_cluster(smem_u32(&s_bar[slot]), (uint32_t)(ch / NPREPCTA) & 1u, wait_ns))
+                // X of chunk ch (U' of this chunk is in the slot once its FULL
+                // phase passed: the release warp publishes that as s_full)
+                if (tid == 0 && !s_abort && !counter_wait(smem_u32(&s_full), (uint32_t)ch + 1u, wait_ns))
                     expired();
                 wait_bar(mbar, phase & 1u);
                 ++phase;
@@ -1104,6 +1160,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             if (n_chunks > 0) {
                 state_half(0);
                 wait_bar(kbar1, (uint32_t)(n_chunks - 1) & 1u);
+                load_output(n_chunks - 1);
                 state_half(1);
                 snapshot(ts / C + n_chunks - 1);
                 emit_output(n_chunks - 1);
@@ -1118,7 +1175,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         }
     } else {
         // ================================================== preparing CTAs ==
-        const int par = (int)rank - 1;             // chunks ch with ch % NPREPCTA == par
+        const int par = (int)role - 1;             // chunks ch with ch % NPREPCTA == par
         const uint32_t ebar = smem_u32(&s_bar[0]);
         const uint32_t mbar = smem_u32(&s_bar[1]);
         const uint32_t rbar = smem_u32(&s_bar[2]);
@@ -1188,8 +1245,8 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             // copy, once the chain has released the slot; then the staging is
             // handed back to the compute warps.
             uint32_t ephase = 0;
-            const uint32_t full_remote = map_to_rank(smem_u32(&s_bar[par]), 0u);
-            const uint32_t slot_remote = map_to_rank(smem_u32(sm + C_SLOT0 + par * SLOT), 0u);
+            const uint32_t full_remote = map_to_rank(smem_u32(&s_bar[par]), CHAIN_RANK);
+            const uint32_t slot_remote = map_to_rank(smem_u32(sm + C_SLOT0 + par * SLOT), CHAIN_RANK);
 #pragma unroll 1
             for (int ch = par; ch < n_chunks; ch += NPREPCTA) {
                 named_bar(NB_FILL, NX);               // the staging holds chunk ch
@@ -1435,7 +1492,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     fence_before_sync();
     __syncthreads();
     cluster_sync();                    // every push that will be issued has been issued
-    if (rank == 0 && tid == 0 && *(volatile int*)&s_abort) {
+    if (role == 0 && tid == 0 && *(volatile int*)&s_abort) {
         // An expired wait let this CTA stop consuming slots: a push into a
         // slot may still be landing.  Let each slot's last expected push land
         // (or find that it was never sent) before the shared memory is given up.
@@ -1445,7 +1502,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     }
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, ncols);
-    if (rank == 0 && tid < NCW && *(volatile int*)&s_abort)
+    if (role == 0 && tid < NCW && *(volatile int*)&s_abort)
         poison_head_outputs(o ? o + ((int64_t)b * T + ts) * (int64_t)H * D + (int64_t)h * D : nullptr,
                             (int64_t)H * D, Tl, o && !(flags & SEG_NO_O),
                             hT ? hT + head_off * D * D : nullptr, tid, NCW);
@@ -1530,10 +1587,14 @@ static cudaError_t launch_pass(const CUtensorMap& mq, const CUtensorMap& mk, con
 {
     const bool pro = (flags & pf::PROLOGUE) != 0;
     if (cluster) {
+        // o as a tensor map for the cluster variant's tensor stores
+        CUtensorMap mo;
+        memset(&mo, 0, sizeof(mo));
+        if (o && !(flags & pf::SEG_NO_O) && T > 0 && !make_map(&mo, o, B, T, H)) return cudaErrorInvalidValue;
         dim3 grid((pc::NPREPCTA + 1) * H, B * n_seg);
         auto kern = pro ? prefill_cluster_kernel<true> : prefill_cluster_kernel<false>;
         kern<<<grid, pc::NTH, pc::SMEM_BYTES, stream>>>(
-            mq, mk, mv, mg, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags,
+            mq, mk, mv, mg, mo, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags,
             states, snap_every, wait_limit_ns());
     } else {
         dim3 grid(H, B * n_seg);

@@ -279,6 +279,18 @@ __device__ __forceinline__ void bulk_copy_to_rank(uint32_t dst_cluster_saddr, ui
         :: "r"(dst_cluster_saddr), "r"(src_saddr), "r"(bytes), "r"(mbar_cluster_saddr) : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Tiled 3-D tensor store from shared memory (a bulk group; commit it).
+__device__ __forceinline__ void tma_store_3d(const void* tmap, int x, int y, int z, uint32_t src_saddr) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];"
+        :: "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(src_saddr) : "memory");
+}
+// Wait until every committed bulk group has completed, writes included.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Plain arrive (release, CTA scope) on a local mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint32_t saddr) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(saddr) : "memory");
+}
 // Wait until the source buffers of all committed bulk copies may be reused.
 __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
