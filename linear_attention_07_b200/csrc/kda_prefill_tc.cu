@@ -296,12 +296,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int hh = warp >> 2;
         const uint32_t bar = smem_u32(&s_bar[0]);
         uint32_t phase = 0;
-        // one thread polls the MMA barrier; the others block on a named barrier
+        // every thread waits on the MMA barrier itself (cheaper than a
+        // hand-over through a named barrier)
         auto wait_mma = [&]() {
-            if (tid == 0 && !s_abort && !mbar_wait(bar, phase & 1u, wait_ns)) expired();
+            if (!s_abort && !mbar_wait(bar, phase & 1u, wait_ns)) expired();
             ++phase;
-            __syncwarp();
-            named_bar(BAR_CHAIN, NCH);
             fence_after_sync();
         };
         uint32_t n_commit = 0;               // commits on `bar` issued by this (issuing) thread
@@ -440,10 +439,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         uint32_t phase = 0, rphase = 0;
         uint32_t n_commit = 0, n_loads = 0;    // issued by pt == 0 (also the waiting thread)
         auto wait_mma = [&]() {
-            if (pt == 0 && !s_abort && !mbar_wait(bar, phase & 1u, wait_ns)) expired();
+            if (!s_abort && !mbar_wait(bar, phase & 1u, wait_ns)) expired();
             ++phase;
-            __syncwarp();
-            named_bar(BAR_PREP, NPREP);
             fence_after_sync();
         };
         auto prep_sync = [&]() { named_bar(BAR_PREP, NPREP); };
@@ -763,7 +760,8 @@ constexpr int NCW = 256;                                      // compute threads
 constexpr int NX = NCW + 32;                                  // compute warps + one helper warp (hand-overs)
 constexpr int NTH = NCW + 64;                                 // plus an issuer warp and a remote-traffic warp
 // named barriers (0 is __syncthreads): issuer hand-overs and compute-warp syncs
-constexpr uint32_t NB_ASA = 1, NB_ASB = 2, NB_U = 3, NB_CW = 4;                 // chain CTA
+constexpr uint32_t NB_ASA = 1, NB_ASB = 2, NB_U = 3;                           // chain CTA
+constexpr uint32_t NB_CW = 4;                                                  // compute-warp syncs
 constexpr uint32_t NB_G = 5, NB_TB = 6, NB_STFREE = 7, NB_FILL = 8;              // preparing CTAs
 constexpr int NPREPCTA = 3;                                   // preparing CTAs per cluster (= slots)
 // Cluster rank of the chain CTA; the preparing CTAs follow it cyclically.
@@ -1027,11 +1025,11 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             const int j = 32 * sp + lane;                // dv row = TMEM lane
             const int hh = warp >> 2;                     // d_k columns [32 hh, +32) and [64 + 32 hh, +32)
             uint32_t phase = 0;
-            auto cw_bar = [&]() { named_bar(NB_CW, NCW); };
+            // Every thread waits on the MMA barrier itself: a hand-over from one
+            // polling thread through a named barrier costs a few hundred
+            // cycles per wait on this path.
             auto wait_bar = [&](uint32_t bar, uint32_t parity) {
-                if (tid == 0 && !s_abort && !mbar_wait(bar, parity, wait_ns)) expired();
-                __syncwarp();
-                cw_bar();
+                if (!s_abort && !mbar_wait(bar, parity, wait_ns)) expired();
                 fence_after_sync();
             };
             // S[32 q + i] holds d_k column 64 q + 32 hh + i of this thread's dv row
@@ -1138,8 +1136,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 }
                 // X of chunk ch (U' of this chunk is in the slot once its FULL
                 // phase passed: the release warp publishes that as s_full)
-                if (tid == 0 && !s_abort && !counter_wait(smem_u32(&s_full), (uint32_t)ch + 1u, wait_ns))
-                    expired();
+                if (!s_abort && !counter_wait(smem_u32(&s_full), (uint32_t)ch + 1u, wait_ns)) expired();
                 wait_bar(mbar, phase & 1u);
                 ++phase;
                 {   // U = U' - W S  (this thread: tokens [16 hh, 16 hh + 16))
