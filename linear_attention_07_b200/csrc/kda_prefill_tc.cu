@@ -94,11 +94,13 @@ constexpr uint32_t YMS = TMS + C * LD * 4;                     // A_10 X_00 (16 
 constexpr uint32_t OST = YMS + TILE * (TILE + 1) * 4;           // o staging, 32 x 128 bf16
 constexpr uint32_t NRM = OST + C * D * 2;                      // prologue: per-warp squared norms
 constexpr uint32_t NRM_BYTES = 2 * 4 * 2 * TILE * 4;           // [tile][warp][q, k][token]
-constexpr uint32_t SMEM_BYTES = NRM + NRM_BYTES;
+constexpr int LDT = C + 4;                                     // transposed-A row stride (16-byte rows)
+constexpr uint32_t ATM = NRM + NRM_BYTES;                      // A^T of the diagonal blocks (32 x 36 fp32)
+constexpr uint32_t SMEM_BYTES = ATM + C * LDT * 4;
 
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 static_assert(OST % 16 == 0 && GA % 16 == 0 && GB % 16 == 0 && WA % 16 == 0 && VA % 16 == 0 && TB % 16 == 0 &&
-              B1 % 16 == 0 && B2 % 16 == 0 && B3 % 16 == 0, "descriptor alignment");
+              B1 % 16 == 0 && B2 % 16 == 0 && B3 % 16 == 0 && ATM % 16 == 0, "descriptor alignment");
 
 // tensor memory columns (512 allocated)
 constexpr uint32_t T_AS = 0;     // S^T (tf32), 128
@@ -578,53 +580,82 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             fence_smem_to_async();
             wait_mma();
 
-            // ---- A and P (32 x 32) into scratch; row m of D_G is lane (m % 16) + 32 (m / 16)
-            if (pw < 3) {
-                // sp 0: rows Kh_0 (cols Kt_0, Qt_0); sp 1: rows Kh_1 (cols Kt_1, Qt_1);
-                // sp 2: rows Kb_0 (cols Kt_1, Qt_1): the block between the tiles
-                const int colK = (sp == 0) ? 0 : TILE;
-                float gk[16], gq[16];
-                tmem_ld16(tm + lane_base + T_DG + colK, gk);
-                tmem_ld16(tm + lane_base + T_DG + C + colK, gq);
-                wait_ld();
-                if (lane < TILE) {
-                    const int i = (sp == 1 ? TILE : 0) + lane;           // column of A / P
-                    const int rbase = (sp == 0) ? 0 : TILE;              // rows covered
+            // ---- A and P (32 x 32) from the Gram (row m of D_G is lane
+            // (m % 16) + 32 (m / 16)).  Sub-partition 0 holds the rows Kh_0
+            // (columns Kt_0, Qt_0), 1 the rows Kh_1 (Kt_1, Qt_1), 2 the rows
+            // Kb_0 (Kt_1, Qt_1: the blocks between the tiles).  Warps 0-2
+            // take the A columns, warps 4-6 the P columns.  The warp that
+            // holds a diagonal block of A also solves it, X = (I + A_tt)^-1,
+            // column i per lane, right-looking, from A_tt^T in shared memory
+            // (one 16-float column per step, read as four vectors).
+            {
+                const int spx = pw & 3;
+                if (spx < 3) {
+                    const bool is_p = pw >= 4;
+                    const int colK = (spx == 0) ? 0 : TILE;
+                    float gv[16];
+                    tmem_ld16(tm + lane_base + T_DG + (is_p ? C : 0) + colK, gv);
+                    wait_ld();
+                    const int i = (spx == 1 ? TILE : 0) + lane;           // column of A / P
+                    const int rbase = (spx == 0) ? 0 : TILE;              // rows covered
+                    float* atm = reinterpret_cast<float*>(sm + ATM);
+                    if (lane < TILE) {
+                        if (is_p) {
 #pragma unroll
-                    for (int r = 0; r < TILE; ++r) {
-                        const int rg = rbase + r;
-                        am[rg * LD + i] = (rg > i) ? bt[rg] * gk[r] : 0.f;
-                        pm[rg * LD + i] = (rg >= i) ? gq[r] : 0.f;
-                    }
-                    if (sp == 1) {                                        // upper-right block is zero
+                            for (int r = 0; r < TILE; ++r) {
+                                const int rg = rbase + r;
+                                pm[rg * LD + i] = (rg >= i) ? gv[r] : 0.f;
+                            }
+                            if (spx == 1) {                               // P_01 = 0
 #pragma unroll
-                        for (int r = 0; r < TILE; ++r) {
-                            am[r * LD + i] = 0.f;
-                            pm[r * LD + i] = 0.f;
+                                for (int r = 0; r < TILE; ++r) pm[r * LD + i] = 0.f;
+                            }
+                        } else if (spx == 2) {                            // A_10, all below the diagonal
+#pragma unroll
+                            for (int r = 0; r < TILE; ++r) am[(TILE + r) * LD + i] = bt[TILE + r] * gv[r];
+                        } else {                                          // column i of A_tt into row i of A^T
+#pragma unroll
+                            for (int r = 0; r < TILE; r += 4) {
+                                float e4[4];
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    const int rg = rbase + r + u;
+                                    e4[u] = (rg > i) ? bt[rg] * gv[r + u] : 0.f;
+                                }
+                                *reinterpret_cast<float4*>(atm + i * LDT + rbase + r) =
+                                    make_float4(e4[0], e4[1], e4[2], e4[3]);
+                            }
                         }
                     }
-                }
-            }
-            prep_sync();
-            // ---- diagonal blocks: X = (I + A_tt)^-1, column by column (right-looking)
-            if (pw < 2 && lane < TILE) {
-                const int off = pw * TILE;
-                const int i = lane;
-                float x[TILE];
+                    if (!is_p && spx < 2) {
+                        __syncwarp();
+                        if (lane < TILE) {
+                            const int off = spx * TILE;
+                            float x[TILE];
 #pragma unroll
-                for (int r = 0; r < TILE; ++r) x[r] = (r == i) ? 1.f : 0.f;
+                            for (int r = 0; r < TILE; ++r) x[r] = (r == lane) ? 1.f : 0.f;
 #pragma unroll
-                for (int s2 = 0; s2 < TILE; ++s2) {
+                            for (int s2 = 0; s2 < TILE; ++s2) {
+                                const float4* col = reinterpret_cast<const float4*>(atm + (off + s2) * LDT + off);
+                                float a16[TILE];
 #pragma unroll
-                    for (int r = s2 + 1; r < TILE; ++r)
-                        x[r] = fmaf(-am[(off + r) * LD + off + s2], x[s2], x[r]);
-                }
-                const float bi = bt[off + i];
+                                for (int q4 = 0; q4 < TILE / 4; ++q4) {
+                                    const float4 v4 = col[q4];
+                                    a16[4 * q4] = v4.x; a16[4 * q4 + 1] = v4.y;
+                                    a16[4 * q4 + 2] = v4.z; a16[4 * q4 + 3] = v4.w;
+                                }
 #pragma unroll
-                for (int r = 0; r < TILE; ++r) {
-                    xm[(off + r) * LD + off + i] = x[r];
-                    tmx[(off + r) * LD + off + i] = x[r] * bi;            // T_tt = X_tt diag(b)
-                    if (pw == 1) tmx[r * LD + off + i] = 0.f;            // T_01 = 0
+                                for (int r = s2 + 1; r < TILE; ++r) x[r] = fmaf(-a16[r], x[s2], x[r]);
+                            }
+                            const float bi = bt[off + lane];
+#pragma unroll
+                            for (int r = 0; r < TILE; ++r) {
+                                xm[(off + r) * LD + off + lane] = x[r];
+                                tmx[(off + r) * LD + off + lane] = x[r] * bi;     // T_tt = X_tt diag(b)
+                                if (spx == 1) tmx[r * LD + off + lane] = 0.f;     // T_01 = 0
+                            }
+                        }
+                    }
                 }
             }
             prep_sync();
