@@ -59,6 +59,7 @@ cudaError_t prefill_transition_launch(const void* q, const void* k, const void* 
 cudaError_t state_chain_launch(const float* M, const float* N, const float* h0, float* S_start, float* hT,
                                int B, int P, int H, cudaStream_t stream);
 int prefill_device_status(cudaStream_t stream);
+int bwd_device_status(cudaStream_t stream);
 int prefill_path_of(int B, int T, int H);
 cudaError_t bounded_wait_selftest_launch(uint64_t limit_ns, cudaStream_t stream);
 
@@ -299,7 +300,10 @@ const char* kda_status_string(int status)
 
 int kda_device_status(kda_stream_t stream)
 {
-    return prefill_device_status((cudaStream_t)stream);
+    const int a = prefill_device_status((cudaStream_t)stream);
+    const int b = bwd_device_status((cudaStream_t)stream);
+    if (a == KDA_ERR_CUDA || b == KDA_ERR_CUDA) return KDA_ERR_CUDA;
+    return a != KDA_OK ? a : b;
 }
 
 int kda_selftest_bounded_wait(uint64_t limit_ns, kda_stream_t stream)

@@ -37,9 +37,13 @@
 // kernel: dg sums terms that nearly cancel, and state errors at the tf32
 // level (about 1e-3) move it by about 1e-2 of its scale.
 #include "kda_common.cuh"
+#include "kda_tc.cuh"
 
 namespace kda {
 namespace bw {
+
+__device__ int g_bwd_status;     // set to KDA_ERR_TIMEOUT by a wait that expired
+constexpr uint64_t DRAIN_NS = 20000000ull;   // after an expired wait: 20 ms for the MMAs in flight
 
 constexpr int D = 128, C = 32, TILE = 16, NT = 256;
 constexpr int LD = D + 1;        // odd row stride: conflict-free row and column walks
@@ -545,9 +549,14 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
                  const float* __restrict__ rec_all, const float* __restrict__ S0_all,
                  const float* __restrict__ dS_all,
                  __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
-                 __nv_bfloat16* __restrict__ dg, __nv_bfloat16* __restrict__ dbeta, int T, int H, int n_chunks)
+                 __nv_bfloat16* __restrict__ dg, __nv_bfloat16* __restrict__ dbeta, int T, int H, int n_chunks,
+                 uint64_t wait_ns)
 {
+    using namespace tc;
     extern __shared__ __align__(16) float sm[];
+    __shared__ uint32_t s_taddr;
+    __shared__ __align__(8) uint64_t s_mbar;
+    __shared__ int s_abort;
     float* bK = sm;
     float* bQ = bK + C * LD;       // Kb during the state products, then Q
     float* bV = bQ + C * LD;       // V, then dGam
@@ -586,6 +595,20 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     const float* dS = dS_all + (bh * n_chunks + c_idx) * D * D;
     auto Tm = [&](int r, int i) { return sX[r * L32 + i] * sB[i]; };
 
+    // tensor memory (the whole of it: one CTA per SM) and the MMA barrier
+    if (tid < 32) {
+        tmem_alloc(smem_u32(&s_taddr), 512);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(smem_u32(&s_mbar), 1);
+        fence_mbar_init();
+        s_abort = 0;
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+
     // ---- inputs, the prep record and the chunk's decay
     load_rows<NL>(bK, k, row0, rs, Tl);
     load_rows<NL>(bV, v, row0, rs, Tl);
@@ -598,9 +621,6 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     for (int e = tid; e < C * D; e += NL) {
         const int r = e / D, c = e % D;
         bW[r * LD + c] = rec[R_W + e];
-        bDKB[r * LD + c] = 0.f;
-        bDQT[r * LD + c] = 0.f;
-        bDW[r * LD + c] = 0.f;
     }
     for (int e = tid; e < C * C; e += NL) {
         const int r = e / C, i = e % C;
@@ -608,7 +628,6 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         sP[r * L32 + i] = rec[R_P + e];
         sX[r * L32 + i] = rec[R_X + e];
     }
-    if (tid < D) sRS[tid] = 0.f;
     __syncthreads();
     if constexpr (RAW) {
         prologue_rows<NL>(nullptr, nullptr, bK, sIK, bG, Tl);
@@ -629,82 +648,149 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
                          [&](int m, int n, float x) { bDU[m * LD + n] = x; });
     __syncthreads();
 
-    // The next block of S0 and dS is read into registers while the current one
-    // is used (2 float4 of each per thread), so the global loads overlap the
-    // block products.
-    constexpr int PF = (JB * (D / 4)) / NL;      // float4 of each matrix per thread and block
-    static_assert(JB * (D / 4) == PF * NL && D * (JB / 4) == PF * NL && PF >= 1, "block split");
-    float4 pf0[PF], pf1[PF];
-    auto fetch_rows = [&](int kb) {              // rows [kb, kb + JB), all columns
-#pragma unroll
-        for (int u = 0; u < PF; ++u) {
-            const int e = tid + u * NL, i = e / (D / 4), c4 = (e % (D / 4)) * 4;
-            pf0[u] = *reinterpret_cast<const float4*>(S0 + (int64_t)(kb + i) * D + c4);
-            pf1[u] = *reinterpret_cast<const float4*>(dS + (int64_t)(kb + i) * D + c4);
+    // ---- the five state-sized products on the tensor cores (tf32 operands,
+    // fp32 sums), each as the transposed product with the 128-wide state
+    // dimension as the MMA's M and the 32 tokens as N:
+    //   phase A: (W S0)^T = S0^T W^T and (Kb dS)^T = dS^T Kb^T, A = S0^T, dS^T
+    //            in tensor memory (lane = d_v row), B = W, Kb;
+    //   phase B: dQt^T = S0 dO^T, dKb^T = dS U^T, (dU S0^T)^T = S0 dU^T,
+    //            A = S0, dS in tensor memory (lane = d_k row), B = dO, U, dU.
+    // B operands are K-major without swizzle, dense: element (n, k) at byte
+    // (n / 8) * 4096 + (k / 4) * 128 + (n % 8) * 16 + (k % 4) * 4 (16 KB each),
+    // in the space of dKb, dQt and dW, which are written only after phase B.
+    // Tensor memory: A at columns 0-255 (phase A: S0^T, dS^T; phase B: S0, dS);
+    // results at 256 (W S0), 288 (Kb dS), 320 (dQt), 352 (dKb), 384 (dU S0^T).
+    const uint32_t tm = s_taddr;
+    const int wp = tid >> 5, lane = tid & 31;
+    const int spw = wp & 3, cg = wp >> 2;                 // sub-partition, column group 0..3
+    const uint32_t lane_base = (uint32_t)(32 * spw) << 16;
+    const int mrow = 32 * spw + lane;                      // tensor-memory lane of this thread
+    float* bop = bDKB;                                     // B operands: 3 x 16 KB over dKb, dQt, dW
+    const uint32_t idn = idesc_tf32(128, C, false, false);
+    const uint32_t mbar = smem_u32(&s_mbar);
+    uint32_t n_commit = 0;                                 // commits on s_mbar (issued by warp 0)
+    auto expired = [&]() {
+        s_abort = 1;
+        atomicExch(&g_bwd_status, (int)KDA_ERR_TIMEOUT);
+    };
+    // a [C][LD] fp32 matrix into a B operand, rounded to tf32 (lanes: n % 8,
+    // then k / 4, so a warp stores 512 contiguous bytes)
+    auto put_b = [&](float* dst, const float* src) {
+        for (int e = tid; e < C * (D / 4); e += NL) {
+            const int n8 = e & 7, k4 = (e >> 3) & 31, ng = e >> 8;
+            const float* x = src + (8 * ng + n8) * LD + 4 * k4;
+            *reinterpret_cast<float4*>(reinterpret_cast<char*>(dst) + ng * 4096 + k4 * 128 + n8 * 16) =
+                make_float4(to_tf32(x[0]), to_tf32(x[1]), to_tf32(x[2]), to_tf32(x[3]));
         }
     };
-    auto fetch_cols = [&](int jb) {              // all rows, columns [jb, jb + JB)
+    auto issue = [&](uint32_t d_col, uint32_t a_col, const float* b) {
+        const uint64_t b0 = sdesc(smem_u32(b), 128, 4096);
 #pragma unroll
-        for (int u = 0; u < PF; ++u) {
-            const int e = tid + u * NL, i = e / (JB / 4), c4 = (e % (JB / 4)) * 4;
-            pf0[u] = *reinterpret_cast<const float4*>(S0 + (int64_t)i * D + jb + c4);
-            pf1[u] = *reinterpret_cast<const float4*>(dS + (int64_t)i * D + jb + c4);
-        }
+        for (int ks = 0; ks < D / 8; ++ks)
+            mma_tf32_ts_w(tm + d_col, tm + a_col + ks * 8, b0 + (uint64_t)(ks * 16), idn, ks > 0 ? 1u : 0u);
     };
-    auto put = [&](float* dst, int stride, int i, int c4, float4 x) {
-        float* p = dst + i * stride + c4;
-        p[0] = x.x; p[1] = x.y; p[2] = x.z; p[3] = x.w;
+    auto wait_mma = [&](uint32_t parity) {
+        if (!s_abort && !mbar_wait(mbar, parity, wait_ns)) expired();
+        fence_after_sync();
     };
 
-    // ---- pass 1: rows [kb, kb + JB) of S0 and dS: U -= W S0, dU += Kb dS
-    fetch_rows(0);
-#pragma unroll 1
-    for (int kb = 0; kb < D; kb += JB) {
+    // phase A
+    put_b(bop, bW);
+    put_b(bop + C * D, bQ);                                // Kb
+    {
+        float t32[32];
 #pragma unroll
-        for (int u = 0; u < PF; ++u) {
-            const int e = tid + u * NL, i = e / (D / 4), c4 = (e % (D / 4)) * 4;
-            put(bS0, LD, i, c4, pf0[u]);
-            put(bDS, LD, i, c4, pf1[u]);
-        }
-        __syncthreads();
-        if (kb + JB < D) fetch_rows(kb + JB); else fetch_cols(0);
-        tgemm<C, D, JB, 2, 4, NL>([&](int m, int kk) { return bW[m * LD + kb + kk]; },
-                              [&](int kk, int n) { return bS0[kk * LD + n]; },
-                              [&](int m, int n, float x) { bU[m * LD + n] -= x; });
-        tgemm<C, D, JB, 2, 4, NL>([&](int m, int kk) { return bQ[m * LD + kb + kk]; },
-                              [&](int kk, int n) { return bDS[kk * LD + n]; },
-                              [&](int m, int n, float x) { bDU[m * LD + n] += x; });
-        __syncthreads();
+        for (int i = 0; i < 32; ++i) t32[i] = to_tf32(S0[(int64_t)(32 * cg + i) * D + mrow]);
+        tmem_st32(tm + lane_base + 32 * cg, t32);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) t32[i] = to_tf32(dS[(int64_t)(32 * cg + i) * D + mrow]);
+        tmem_st32(tm + lane_base + 128 + 32 * cg, t32);
+        wait_st();
     }
+    fence_smem_to_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (wp == 0) {
+        issue(256, 0, bop);
+        issue(288, 128, bop + C * D);
+        mma_commit_w(mbar);
+        ++n_commit;
+    }
+    wait_mma(0);
+    {   // U -= W S0, dU += Kb dS (this thread: d_v row mrow, tokens [8 cg, 8 cg + 8))
+        float v8[8];
+        tmem_ld8(tm + lane_base + 256 + 8 * cg, v8);
+        wait_ld();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) bU[(8 * cg + u) * LD + mrow] -= v8[u];
+        tmem_ld8(tm + lane_base + 288 + 8 * cg, v8);
+        wait_ld();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) bDU[(8 * cg + u) * LD + mrow] += v8[u];
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
 
-    // ---- pass 2: columns [jb, jb + JB) of S0 and dS: dQt, dKb, dW and sum(dS S0)
-#pragma unroll 1
-    for (int jb = 0; jb < D; jb += JB) {
+    // phase B
+    put_b(bop, bDO);
+    put_b(bop + C * D, bU);
+    put_b(bop + 2 * C * D, bDU);
+    {
+        // S0 and dS rows (this thread: d_k row mrow, d_v columns [32 cg, 32 cg + 32)),
+        // and this slice of sum_j dS_ij S0_ij
+        const float4* s4 = reinterpret_cast<const float4*>(S0 + (int64_t)mrow * D + 32 * cg);
+        const float4* d4 = reinterpret_cast<const float4*>(dS + (int64_t)mrow * D + 32 * cg);
+        float rsum = 0.f;
 #pragma unroll
-        for (int u = 0; u < PF; ++u) {
-            const int e = tid + u * NL, i = e / (JB / 4), c4 = (e % (JB / 4)) * 4;
-            put(bS0, LJ, i, c4, pf0[u]);
-            put(bDS, LJ, i, c4, pf1[u]);
-        }
-        __syncthreads();
-        if (jb + JB < D) fetch_cols(jb + JB);
-        tgemm<C, D, JB, 2, 4, NL>([&](int m, int kk) { return bDO[m * LD + jb + kk]; },
-                              [&](int kk, int n) { return bS0[n * LJ + kk]; },
-                              [&](int m, int n, float x) { bDQT[m * LD + n] += x; });
-        tgemm<C, D, JB, 2, 4, NL>([&](int m, int kk) { return bU[m * LD + jb + kk]; },
-                              [&](int kk, int n) { return bDS[n * LJ + kk]; },
-                              [&](int m, int n, float x) { bDKB[m * LD + n] += x; });
-        tgemm<C, D, JB, 2, 4, NL>([&](int m, int kk) { return bDU[m * LD + jb + kk]; },
-                              [&](int kk, int n) { return bS0[n * LJ + kk]; },
-                              [&](int m, int n, float x) { bDW[m * LD + n] -= x; });
-        if (tid < D) {
-            float acc = sRS[tid];
+        for (int hf = 0; hf < 2; ++hf) {
+            float t16[16], d16[16];
 #pragma unroll
-            for (int j = 0; j < JB; ++j) acc = fmaf(bDS[tid * LJ + j], bS0[tid * LJ + j], acc);
-            sRS[tid] = acc;
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 a4 = s4[4 * hf + q4], b4 = d4[4 * hf + q4];
+                rsum = fmaf(a4.x, b4.x, fmaf(a4.y, b4.y, fmaf(a4.z, b4.z, fmaf(a4.w, b4.w, rsum))));
+                t16[4 * q4] = to_tf32(a4.x); t16[4 * q4 + 1] = to_tf32(a4.y);
+                t16[4 * q4 + 2] = to_tf32(a4.z); t16[4 * q4 + 3] = to_tf32(a4.w);
+                d16[4 * q4] = to_tf32(b4.x); d16[4 * q4 + 1] = to_tf32(b4.y);
+                d16[4 * q4 + 2] = to_tf32(b4.z); d16[4 * q4 + 3] = to_tf32(b4.w);
+            }
+            tmem_st16(tm + lane_base + 32 * cg + 16 * hf, t16);
+            tmem_st16(tm + lane_base + 128 + 32 * cg + 16 * hf, d16);
         }
-        __syncthreads();
+        wait_st();
+        bDS[cg * D + mrow] = rsum;                         // partial sums, added below
     }
+    fence_smem_to_async();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (wp == 0 && !__any_sync(0xffffffffu, *(volatile int*)&s_abort != 0)) {
+        issue(320, 0, bop);                                // dQt^T = S0 dO^T
+        issue(352, 128, bop + C * D);                      // dKb^T = dS U^T
+        issue(384, 0, bop + 2 * C * D);                    // (dU S0^T)^T = S0 dU^T
+        mma_commit_w(mbar);
+        ++n_commit;
+    }
+    wait_mma(1);
+    {   // this thread: d_k row mrow, tokens [8 cg, 8 cg + 8)
+        float v8[8];
+        tmem_ld8(tm + lane_base + 320 + 8 * cg, v8);
+        wait_ld();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) bDQT[(8 * cg + u) * LD + mrow] = v8[u];
+        tmem_ld8(tm + lane_base + 352 + 8 * cg, v8);
+        wait_ld();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) bDKB[(8 * cg + u) * LD + mrow] = v8[u];
+        tmem_ld8(tm + lane_base + 384 + 8 * cg, v8);
+        wait_ld();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) bDW[(8 * cg + u) * LD + mrow] = -v8[u];
+    }
+    if (tid < D) sRS[tid] = bDS[tid] + bDS[D + tid] + bDS[2 * D + tid] + bDS[3 * D + tid];
+    fence_before_sync();
+    __syncthreads();
 
     // ---- products of the complete U and dU: dO U^T, dU V^T, dV = Tm^T dU
     tgemm<C, C, D, 2, 1, NL>([&](int m, int kk) { return bDO[m * LD + kk]; },
@@ -942,6 +1028,29 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
         }
     }
     if (tid < Tl) dbeta[((int64_t)b * T + t0 + tid) * H + h] = to_bf(sDB[tid]);
+
+    // After an expired wait the MMAs of the last commit may still run: let
+    // them finish before tensor memory is released, and mark the chunk's
+    // gradients as invalid (NaN) so a partial result never passes for one.
+    const bool aborted = *(volatile int*)&s_abort != 0;
+    if (tid == 0 && aborted && n_commit > 0) mbar_wait(mbar, (n_commit - 1) & 1u, DRAIN_NS);
+    fence_before_sync();
+    __syncthreads();
+    if (tid < 32) tmem_dealloc(tm, 512);
+    if (aborted) {
+        const __nv_bfloat16 nan = __float2bfloat16_rn(__int_as_float(0x7fc00000));
+        for (int e = tid; e < C * D; e += NL) {
+            const int r = e / D, c = e % D;
+            if (r < Tl) {
+                const int64_t o = row0 + (int64_t)r * rs + c;
+                dq[o] = nan;
+                dk[o] = nan;
+                dg[o] = nan;
+                dv[o] = nan;
+            }
+        }
+        if (tid < Tl) dbeta[((int64_t)b * T + t0 + tid) * H + h] = nan;
+    }
 }
 
 }  // namespace bw
@@ -998,13 +1107,28 @@ cudaError_t chunk_bwd_launch(const void* q, const void* k, const void* v, const 
     if (e == cudaSuccess) {
         (raw ? bwd_local_kernel<true> : bwd_local_kernel<false>)<<<grid_c, NL, LOC_SMEM, stream>>>(
             bq, bk, bv, bg, bb, bdo, rec, S0_all, dS_all, (__nv_bfloat16*)dq, (__nv_bfloat16*)dk,
-            (__nv_bfloat16*)dv, (__nv_bfloat16*)dg, (__nv_bfloat16*)dbeta, T, H, n_chunks);
+            (__nv_bfloat16*)dv, (__nv_bfloat16*)dg, (__nv_bfloat16*)dbeta, T, H, n_chunks,
+            bounded_wait_limit_ns());
         e = cudaGetLastError();
     }
     const cudaError_t ef = cudaFreeAsync(ws, stream);
     if (e == cudaSuccess) e = ef;
     note_launches(3);
     return e;
+}
+
+// Reads and clears the timeout flag of the backward kernels (blocking).
+int bwd_device_status(cudaStream_t stream)
+{
+    int st = 0, zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&st, bw::g_bwd_status, sizeof(int), 0,
+                                  cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (cudaMemcpyToSymbolAsync(bw::g_bwd_status, &zero, sizeof(int), 0,
+                                cudaMemcpyHostToDevice, stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
+    return st;
 }
 
 }  // namespace kda

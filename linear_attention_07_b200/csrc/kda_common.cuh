@@ -43,6 +43,9 @@ int current_sm_count();
 // between calls (release threshold: never), once per device, so that a call
 // does not map its workspace anew every time.
 void keep_pool_memory();
+// Limit of every bounded device-side wait: 2 s, or KDA_WAIT_LIMIT_NS
+// (0 .. 2e9 ns) for tests that make the waits run out.
+uint64_t bounded_wait_limit_ns();
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }

@@ -1598,13 +1598,14 @@ static bool cluster_fits(int64_t heads) { return heads * (pc::NPREPCTA + 1) <= s
 // another SM then gives up, since neither can land in the few hundred cycles
 // between its issue and the check.  The drain after an expired wait keeps
 // its own 20 ms limit.
-static uint64_t wait_limit_ns()
+uint64_t bounded_wait_limit_ns()
 {
     const char* env = getenv("KDA_WAIT_LIMIT_NS");
     if (!env || !*env) return pf::WAIT_NS;
     const unsigned long long v = strtoull(env, nullptr, 10);
     return v > pf::WAIT_NS ? pf::WAIT_NS : (uint64_t)v;
 }
+static uint64_t wait_limit_ns() { return bounded_wait_limit_ns(); }
 
 // One launch of either variant over B * n_seg segment-sequences of length
 // seg_len (n_seg = 1, seg_len = T: the plain prefill).
