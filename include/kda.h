@@ -234,10 +234,14 @@ int kda_decode_step_raw(const void* q_raw, const void* k_raw, const void* v, con
  *   dq, dk, dg : bf16 [B][T][H][dk]     dv : bf16 [B][T][H][dv]
  *   dbeta      : bf16 [B][T][H]         dh0 : fp32 [B][H][dk][dv], or NULL
  *   Supported: d_k == d_v == 128.  T == 0: dh0 receives dhT (or zeros).
- * Three launches on `stream`, fp32 arithmetic throughout (the gradient of
- * the decay sums terms that nearly cancel, and tf32 state products would
- * move it by about 1e-2 of its scale): per-chunk operands, the forward and
- * reverse state chains side by side, the chunk-local gradients.  Stream-ordered
+ * Three launches on `stream`: per-chunk operands and the forward and reverse
+ * state chains in fp32 (the gradient of the decay sums terms that nearly
+ * cancel, and chunk-start states at tf32 precision would move it by about
+ * 1e-2 of its scale), then the chunk-local gradients, whose five
+ * state-sized products (W S0, Kb dS, dO S0^T, U dS^T, dU S0^T) run as tf32
+ * tensor-core MMAs from the fp32 states and the rest in fp32.  The local
+ * kernel's waits for its MMAs are bounded as the prefill's (a chunk whose
+ * wait expired gets NaN gradients; kda_device_status reports it).  Stream-ordered
  * workspace of 209,408 bytes per 32-token chunk and head (about 6.5 KB per
  * token and head; KDA_ERR_NO_MEMORY if it cannot be had).  Outputs must not
  * overlap inputs or one another.
@@ -293,10 +297,12 @@ int kda_verify_fwd(const void* q, const void* k, const void* v, const void* g,
 /*
  * kda_device_status -- KDA_OK, or KDA_ERR_TIMEOUT if a kernel of this
  * library gave up on a bounded device-side wait since the last call (every
- * wait between the roles of a prefill kernel gives up after 2 s).  The
- * kernel then returns early and fills the o rows and hT of the affected
- * heads with NaN (intermediate states, if asked for, are undefined), so a
- * partial result never passes for a real one.  Reads and clears the flag;
+ * wait between the roles of a prefill kernel, and the backward's waits for
+ * its tensor-core products, give up after 2 s).  The kernel then winds down
+ * and fills the o rows and hT of the affected heads (backward: the dq, dk,
+ * dv, dg and dbeta rows of the affected chunk) with NaN (intermediate
+ * states, if asked for, are undefined), so a partial result never passes
+ * for a real one.  Reads and clears the flag;
  * synchronises `stream`.  KDA_ERR_CUDA if a CUDA call fails.
  */
 int kda_device_status(kda_stream_t stream);
