@@ -330,9 +330,10 @@ constexpr int CLD = D + 4;        // operand rows: 528 B, 16-byte aligned
 constexpr int XLD = NS + 4;       // state / Y rows: 144 B
 // one chain's shared memory: step-1 operand [C][CLD] (+ U' slice [C][XLD]
 // forward), step-2 operands (Kb, or W and Z) [C][CLD] each (+ dO slice and gC),
-// the state slice [D][XLD] and Y [C][XLD]
-constexpr int FWD_FLOATS = 2 * C * CLD + 2 * C * XLD + D + D * XLD + C * XLD;
-constexpr int REV_FLOATS = 3 * C * CLD + C * XLD + D + D * XLD + C * XLD;
+// the state slice [D][XLD], Y [C][XLD] and step 1's partial sums over four K
+// slices [4][C][XLD]
+constexpr int FWD_FLOATS = 2 * C * CLD + 2 * C * XLD + D + D * XLD + C * XLD + 4 * C * XLD;
+constexpr int REV_FLOATS = 3 * C * CLD + C * XLD + D + D * XLD + C * XLD + 4 * C * XLD;
 constexpr size_t CHAIN_SMEM = (size_t)(FWD_FLOATS + REV_FLOATS) * sizeof(float);
 constexpr int NT_CHAIN = 2 * NT;
 
@@ -340,6 +341,11 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
                  :: "r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src) : "memory");
+}
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned start) into L2.
+__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
@@ -361,6 +367,7 @@ __device__ __forceinline__ void chain_run(float* sm, int tid, uint32_t bar, cons
     float* oG = REV ? oS + C * XLD : oS + C * XLD;        // gC [D]
     float* sXs = oG + D;                                  // state slice [D][XLD]
     float* sY = sXs + D * XLD;                            // [C][XLD]
+    float* sYp = sY + C * XLD;                            // step-1 partial sums, 4 K slices [4][C][XLD]
 
     auto fill_rows = [&](float* dst, const float* src) {  // [C][D] fp32 record rows -> [C][CLD]
         for (int e = tid; e < C * (D / 4); e += NT) {
@@ -429,19 +436,39 @@ __device__ __forceinline__ void chain_run(float* sm, int tid, uint32_t bar, cons
                 make_float4(xr[m][0], xr[m][1], xr[m][2], xr[m][3]);
         cp_wait_1();                         // step-1 operands of chunk c (step 2's may be in flight)
         half_sync(bar);
-        {   // step 1: Y = U'_s - W X (forward) or Y = -(Kb X) (reverse); thread (r, cg)
-            const int r = tid / (NS / 4);
-            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 2
-            for (int i = 0; i < D; i += 4) {
-                const float4 a4 = *reinterpret_cast<const float4*>(o1 + r * CLD + i);
-                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+        {   // step 1, partial sums: thread (rows 4 r4 .. + 3, columns 4 cq .. + 3,
+            // K slice [32 ks, 32 ks + 32)); a 4 x 4 register tile per slice
+            // reads one float4 of X and four scalars of the operand per k
+            const int cq = tid & 7, r4 = (tid >> 3) & 7, ks = tid >> 6;
+            float acc[4][4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float4 x = *reinterpret_cast<const float4*>(sXs + (i + u) * XLD + 4 * cg);
-                    y.x = fmaf(av[u], x.x, y.x); y.y = fmaf(av[u], x.y, y.y);
-                    y.z = fmaf(av[u], x.z, y.z); y.w = fmaf(av[u], x.w, y.w);
+            for (int m = 0; m < 4; ++m)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[m][u] = 0.f;
+#pragma unroll 4
+            for (int kk = 0; kk < 32; ++kk) {
+                const int i = 32 * ks + kk;
+                const float4 x = *reinterpret_cast<const float4*>(sXs + i * XLD + 4 * cq);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const float w = o1[(4 * r4 + m) * CLD + i];
+                    acc[m][0] = fmaf(w, x.x, acc[m][0]); acc[m][1] = fmaf(w, x.y, acc[m][1]);
+                    acc[m][2] = fmaf(w, x.z, acc[m][2]); acc[m][3] = fmaf(w, x.w, acc[m][3]);
                 }
+            }
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                *reinterpret_cast<float4*>(sYp + (ks * C + 4 * r4 + m) * XLD + 4 * cq) =
+                    make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
+        }
+        half_sync(bar);                      // partial sums complete; the step-1 buffer is free
+        {   // Y = U'_s - W X (forward) or Y = -(Kb X) (reverse); thread (r, cg)
+            const int r = tid / (NS / 4);
+            float4 y = *reinterpret_cast<const float4*>(sYp + r * XLD + 4 * cg);
+#pragma unroll
+            for (int k2 = 1; k2 < 4; ++k2) {
+                const float4 p = *reinterpret_cast<const float4*>(sYp + (k2 * C + r) * XLD + 4 * cg);
+                y = make_float4(y.x + p.x, y.y + p.y, y.z + p.z, y.w + p.w);
             }
             if (!REV) {
                 const float4 u = *reinterpret_cast<const float4*>(oU + r * XLD + 4 * cg);
@@ -451,7 +478,7 @@ __device__ __forceinline__ void chain_run(float* sm, int tid, uint32_t bar, cons
             }
             *reinterpret_cast<float4*>(sY + r * XLD + 4 * cg) = y;
         }
-        half_sync(bar);                      // Y complete; the step-1 buffer is free
+        half_sync(bar);                      // Y complete
         if (more) fetch1(c + step); else cp_commit();
         cp_wait_1();                         // step-2 operands of chunk c
         half_sync(bar);
@@ -609,6 +636,11 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     __syncthreads();
     fence_after_sync();
 
+    if (tid == 0) {                        // the chunk's states and record, on their way to L2
+        l2_prefetch(S0, D * D * 4);
+        l2_prefetch(dS, D * D * 4);
+        l2_prefetch(rec, R_FLOATS * 4);
+    }
     // ---- inputs, the prep record and the chunk's decay
     load_rows<NL>(bK, k, row0, rs, Tl);
     load_rows<NL>(bV, v, row0, rs, Tl);
