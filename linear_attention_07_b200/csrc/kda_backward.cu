@@ -179,29 +179,28 @@ __device__ __forceinline__ void tgemm(FA a, FB b, FO out)
 
 // ---------------------------------------------------------------- prep --
 
-constexpr int PREP_BIG = 8;                                  // K, Q, V, G, four scratch
-constexpr size_t PREP_SMEM = (size_t)(PREP_BIG * C * LD + 4 * C * L32 + C) * sizeof(float);
+// Six [C][LD] arrays (buffers reused as their contents die) and three
+// [C][L32] ones: 111,872 bytes, so two CTAs share an SM and overlap their
+// serial phases (the triangular solve runs on one warp).
+constexpr size_t PREP_SMEM = (size_t)(6 * C * LD + 3 * C * L32 + C) * sizeof(float);
 
 template <bool RAW>    // RAW: q, k unnormalised and g the gate pre-activation (the fused prologue)
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT, 2)
 bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                 const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ g,
                 const __nv_bfloat16* __restrict__ beta, float* __restrict__ rec_all, int T, int H, int n_chunks)
 {
     extern __shared__ __align__(16) float sm[];
-    float* sK = sm;
-    float* sQ = sK + C * LD;
-    float* sV = sQ + C * LD;
-    float* sG = sV + C * LD;
-    float* s1 = sG + C * LD;
-    float* s2 = s1 + C * LD;
-    float* s3 = s2 + C * LD;
-    float* s4 = s3 + C * LD;
-    float* sA = s4 + C * LD;       // Araw
+    float* sK = sm;                // K, then V (from the pair products on)
+    float* sQ = sK + C * LD;       // Q, then Kc in rows 0-15 (cross-tile pairs)
+    float* sG = sQ + C * LD;       // G, the running sum of g
+    float* s1 = sG + C * LD;       // Ka, then Kt
+    float* s2 = s1 + C * LD;       // Qa, then U'
+    float* s3 = s2 + C * LD;       // Kf, then W
+    float* sA = s3 + C * LD;       // Araw
     float* sP = sA + C * L32;      // Praw (lower incl)
-    float* sX = sP + C * L32;      // (I + A)^-1
-    float* sT = sX + C * L32;      // Tm
-    float* sB = sT + C * L32;      // beta
+    float* sX = sP + C * L32;      // (I + A)^-1; Tm = X diag(beta) is formed on the fly
+    float* sB = sX + C * L32;      // beta
 
     const int c_idx = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int t0 = c_idx * C;
@@ -210,10 +209,10 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     const int64_t rs = (int64_t)H * D;
     const int64_t row0 = ((int64_t)b * T + t0) * rs + (int64_t)h * D;
     float* rec = rec_all + (((int64_t)b * H + h) * n_chunks + c_idx) * R_FLOATS;
+    auto Tm = [&](int r, int i) { return sX[r * L32 + i] * sB[i]; };
 
     load_rows(sK, k, row0, rs, Tl);
     load_rows(sQ, q, row0, rs, Tl);
-    load_rows(sV, v, row0, rs, Tl);
     load_rows(sG, g, row0, rs, Tl);
     if (tid < C) sB[tid] = tid < Tl ? bf(beta[((int64_t)b * T + t0 + tid) * H + h]) : 0.f;
     __syncthreads();
@@ -223,16 +222,29 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     }
     running_sum(sG);
     __syncthreads();
-    // tile-relative operands of the pair products
+    // tile-relative operands of the pair products; Kb and gC go straight to the
+    // record.  Each (r, c) is read and written by one thread, so Kc may take
+    // the place of Q in rows 0-15.
     for (int e = tid; e < C * D; e += NT) {
         const int r = e / D, c = e % D;
         const float Gr = sG[r * LD + c], ref = tile_ref(sG, r, c);
-        const float kk = sK[r * LD + c];
+        const float kk = sK[r * LD + c], qq = sQ[r * LD + c];
         const float a = __expf(Gr - ref);
         s1[r * LD + c] = kk * a;                                  // Ka
-        s2[r * LD + c] = sQ[r * LD + c] * a;                      // Qa
+        s2[r * LD + c] = qq * a;                                  // Qa
         s3[r * LD + c] = kk * __expf(ref - Gr);                   // Kf (<= e^80)
-        if (r < TILE) s4[r * LD + c] = kk * __expf(sG[(TILE - 1) * LD + c] - Gr);   // Kc (<= 1)
+        rec[R_KB + e] = kk * __expf(sG[(C - 1) * LD + c] - Gr);   // Kb
+        if (r < TILE) sQ[r * LD + c] = kk * __expf(sG[(TILE - 1) * LD + c] - Gr);   // Kc (<= 1)
+    }
+    if (tid < D) rec[R_GC + tid] = __expf(sG[(C - 1) * LD + tid]);
+    // V, read from global memory now and stored where K was once the pair
+    // products are done
+    constexpr int VPT = C * (D / 8) / NT;                     // 16-byte vectors per thread
+    uint4 vr[VPT];
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+        const int e = tid + u * NT, r = e / (D / 8), c8 = (e % (D / 8)) * 8;
+        vr[u] = r < Tl ? *reinterpret_cast<const uint4*>(v + row0 + (int64_t)r * rs + c8) : make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
     // Araw (strict lower) and Praw (lower incl) as block products: pairs inside
@@ -251,7 +263,7 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         };
         auto cross = [&](float* dst, const float* L) {
             tgemm<TILE, TILE, D, 1, 1>([&](int m, int kk) { return L[(TILE + m) * LD + kk]; },
-                                       [&](int kk, int n) { return s4[n * LD + kk]; },
+                                       [&](int kk, int n) { return sQ[n * LD + kk]; },
                                        [&](int m, int n, float x) { dst[(TILE + m) * L32 + n] = x; });
         };
         same(sA, s1, true);
@@ -259,9 +271,25 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         cross(sA, s1);
         cross(sP, s2);
     }
+#pragma unroll
+    for (int u = 0; u < VPT; ++u) {
+        const int e = tid + u * NT, r = e / (D / 8), c8 = (e % (D / 8)) * 8;
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&vr[u]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 x = __bfloat1622float2(p2[j]);
+            sK[r * LD + c8 + 2 * j] = x.x;
+            sK[r * LD + c8 + 2 * j + 1] = x.y;
+        }
+    }
     __syncthreads();
-    // X = (I + diag(beta) Araw)^-1 by forward substitution, one column per
-    // thread (four partial sums per row keep the chain short)
+    // Kt = K gam = Ka exp(ref) in place (Ka is no longer read); X = (I +
+    // diag(beta) Araw)^-1 by forward substitution, one column per thread (four
+    // partial sums per row keep the chain short)
+    for (int e = tid; e < C * D; e += NT) {
+        const int r = e / D, c = e % D;
+        s1[r * LD + c] *= __expf(tile_ref(sG, r, c));
+    }
     if (tid < C) {
         const int j = tid;
         float x[C];
@@ -274,39 +302,31 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
             x[r] = (r == j) ? 1.f : (r > j ? -sB[r] * s : 0.f);
         }
 #pragma unroll
-        for (int r = 0; r < C; ++r) {
-            sX[r * L32 + j] = x[r];
-            sT[r * L32 + j] = x[r] * sB[j];
-        }
+        for (int r = 0; r < C; ++r) sX[r * L32 + j] = x[r];
     }
     __syncthreads();
-    // Kt = K gam into s3 (Kf no longer needed)
-    for (int e = tid; e < C * D; e += NT) {
-        const int r = e / D, c = e % D;
-        s3[r * LD + c] = sK[r * LD + c] * __expf(sG[r * LD + c]);
-    }
+    // W = Tm Kt -> s3 (Kf is no longer read)
+    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return Tm(m, kk); },
+                         [&](int kk, int n) { return s1[kk * LD + n]; },
+                         [&](int m, int n, float x) { s3[m * LD + n] = x; });
     __syncthreads();
-    // W = Tm Kt -> s1;  U' = Tm V -> s2
-    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return sT[m * L32 + kk]; },
+    // Z = Qt - P W -> record, with Qt = Q gam = Qa exp(ref)
+    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return sP[m * L32 + kk]; },
                          [&](int kk, int n) { return s3[kk * LD + n]; },
-                         [&](int m, int n, float x) { s1[m * LD + n] = x; });
-    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return sT[m * L32 + kk]; },
-                         [&](int kk, int n) { return sV[kk * LD + n]; },
+                         [&](int m, int n, float x) {
+                             rec[R_Z + m * D + n] = s2[m * LD + n] * __expf(tile_ref(sG, m, n)) - x;
+                         });
+    __syncthreads();
+    // U' = Tm V -> s2 (Qa is no longer read)
+    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return Tm(m, kk); },
+                         [&](int kk, int n) { return sK[kk * LD + n]; },
                          [&](int m, int n, float x) { s2[m * LD + n] = x; });
     __syncthreads();
-    // Z = Qt - P W -> global
-    tgemm<C, D, C, 4, 4>([&](int m, int kk) { return sP[m * L32 + kk]; },
-                         [&](int kk, int n) { return s1[kk * LD + n]; },
-                         [&](int m, int n, float x) {
-                             rec[R_Z + m * D + n] = sQ[m * LD + n] * __expf(sG[m * LD + n]) - x;
-                         });
     for (int e = tid; e < C * D; e += NT) {
         const int r = e / D, c = e % D;
-        rec[R_KB + e] = sK[r * LD + c] * __expf(sG[(C - 1) * LD + c] - sG[r * LD + c]);
-        rec[R_W + e] = s1[r * LD + c];
+        rec[R_W + e] = s3[r * LD + c];
         rec[R_UP + e] = s2[r * LD + c];
     }
-    if (tid < D) rec[R_GC + tid] = __expf(sG[(C - 1) * LD + tid]);
     for (int e = tid; e < C * C; e += NT) {
         const int r = e / C, i = e % C;
         rec[R_A + e] = sA[r * L32 + i];
