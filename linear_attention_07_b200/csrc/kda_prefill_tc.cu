@@ -448,13 +448,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         auto prep_sync = [&]() { named_bar(BAR_PREP, NPREP); };
         // TMA: chunk ci's q, k, v, g rows (32 x 128 bf16 each; rows past T are zero);
         // none after an expired wait (the raw buffer may still be in use)
+        // (with v = 0, the transition pass of the segment scan, v is not loaded)
+        const bool load_v = !(flags & SEG_V_ZERO);
         auto issue_raw = [&](int ci) {
             if (pt == 0 && !*(volatile int*)&s_abort) {
                 ++n_loads;
-                mbar_arrive_expect_tx(rbar, 4 * RAW_T);
+                mbar_arrive_expect_tx(rbar, (load_v ? 4 : 3) * RAW_T);
                 tma_load_3d(smem_u32(sm + RAW + 0 * RAW_T), &tm_q, h * D, ts + ci * C, b, rbar);
                 tma_load_3d(smem_u32(sm + RAW + 1 * RAW_T), &tm_k, h * D, ts + ci * C, b, rbar);
-                tma_load_3d(smem_u32(sm + RAW + 2 * RAW_T), &tm_v, h * D, ts + ci * C, b, rbar);
+                if (load_v) tma_load_3d(smem_u32(sm + RAW + 2 * RAW_T), &tm_v, h * D, ts + ci * C, b, rbar);
                 tma_load_3d(smem_u32(sm + RAW + 3 * RAW_T), &tm_g, h * D, ts + ci * C, b, rbar);
             }
         };
@@ -1214,13 +1216,15 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             // barriers and never wait on an issue.
             uint32_t n_commit = 0, n_loads = 0;
             // no new load after an expired wait (the raw buffer may still be read)
+            // (with v = 0, the transition pass of the segment scan, v is not loaded)
+            const bool load_v = !(flags & SEG_V_ZERO);
             auto issue_raw = [&](int ci) {
                 if (*(volatile int*)&s_abort) return;
                 ++n_loads;
-                mbar_arrive_expect_tx(rbar, 4 * RAW_T);
+                mbar_arrive_expect_tx(rbar, (load_v ? 4 : 3) * RAW_T);
                 tma_load_3d(smem_u32(sm + P_RAW + 0 * RAW_T), &tm_q, h * D, ts + ci * C, b, rbar);
                 tma_load_3d(smem_u32(sm + P_RAW + 1 * RAW_T), &tm_k, h * D, ts + ci * C, b, rbar);
-                tma_load_3d(smem_u32(sm + P_RAW + 2 * RAW_T), &tm_v, h * D, ts + ci * C, b, rbar);
+                if (load_v) tma_load_3d(smem_u32(sm + P_RAW + 2 * RAW_T), &tm_v, h * D, ts + ci * C, b, rbar);
                 tma_load_3d(smem_u32(sm + P_RAW + 3 * RAW_T), &tm_g, h * D, ts + ci * C, b, rbar);
             };
             if (lane == 0 && par < n_chunks) issue_raw(par);
