@@ -177,6 +177,51 @@ __device__ __forceinline__ void tgemm(FA a, FB b, FO out)
         for (int j = 0; j < TN; ++j) out(tm * TM + i, tn + NC * j, acc[i][j]);
 }
 
+// Block GEMM for a small output and a long K: a TM x TN register tile per
+// thread over one of KS slices of K, the KS slices of a tile in KS
+// consecutive lanes and summed with shuffles (every lane then writes TM TN /
+// KS of the tile's outputs).  A slice takes four consecutive k out of every
+// 4 KS, so the lanes of a slice group read k values four apart: with odd
+// row strides the transposed reads of b fall on distinct banks.
+template <int M, int N, int K, int TM, int TN, int KS, int NTH, typename FA, typename FB, typename FO>
+__device__ __forceinline__ void tgemm_ks(FA a, FB b, FO out)
+{
+    constexpr int NC = N / TN, NR = M / TM;
+    static_assert(NC * NR * KS == NTH && NC * TN == N && NR * TM == M, "tile shape");
+    static_assert(K % (4 * KS) == 0 && (KS & (KS - 1)) == 0 && KS <= 32 && (TM * TN) % KS == 0, "K slices");
+    const int t = threadIdx.x, ks = t % KS, tile = t / KS, tn = tile % NC, tm = tile / NC;
+    float acc[TM][TN];
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+#pragma unroll 2
+    for (int q = 0; q < K / (4 * KS); ++q) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int k = q * 4 * KS + 4 * ks + r;
+            float av[TM], bv[TN];
+#pragma unroll
+            for (int i = 0; i < TM; ++i) av[i] = a(tm * TM + i, k);
+#pragma unroll
+            for (int j = 0; j < TN; ++j) bv[j] = b(k, tn + NC * j);
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+#pragma unroll
+                for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+    }
+#pragma unroll
+    for (int off = 1; off < KS; off <<= 1)
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < TN; ++j) acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], off);
+#pragma unroll
+    for (int e = 0; e < TM * TN; ++e)
+        if (e % KS == ks) out(tm * TM + e / TN, tn + NC * (e % TN), acc[e / TN][e % TN]);
+}
+
 // ---------------------------------------------------------------- prep --
 
 // Six [C][LD] arrays (buffers reused as their contents die) and three
@@ -254,7 +299,7 @@ bwd_prep_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     // from Ka / Qa against Kc
     {
         auto same = [&](float* dst, const float* L, bool strict) {
-            tgemm<C, C, D, 4, 1>([&](int m, int kk) { return L[m * LD + kk]; },
+            tgemm_ks<C, C, D, 4, 4, 4, NT>([&](int m, int kk) { return L[m * LD + kk]; },
                                  [&](int kk, int n) { return s3[n * LD + kk]; },
                                  [&](int m, int n, float x) {
                                      if (m / TILE == n / TILE) dst[m * L32 + n] = (n < m || (!strict && n == m)) ? x : 0.f;
@@ -845,10 +890,10 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     __syncthreads();
 
     // ---- products of the complete U and dU: dO U^T, dU V^T, dV = Tm^T dU
-    tgemm<C, C, D, 2, 1, NL>([&](int m, int kk) { return bDO[m * LD + kk]; },
+    tgemm_ks<C, C, D, 4, 4, 8, NL>([&](int m, int kk) { return bDO[m * LD + kk]; },
                          [&](int kk, int n) { return bU[n * LD + kk]; },
                          [&](int m, int n, float x) { sdP[m * L32 + n] = n <= m ? x : 0.f; });
-    tgemm<C, C, D, 2, 1, NL>([&](int m, int kk) { return bDU[m * LD + kk]; },
+    tgemm_ks<C, C, D, 4, 4, 8, NL>([&](int m, int kk) { return bDU[m * LD + kk]; },
                          [&](int kk, int n) { return bV[n * LD + kk]; },
                          [&](int m, int n, float x) { sdUV[m * L32 + n] = x; });
     tgemm<C, D, C, 2, 4, NL>([&](int m, int kk) { return Tm(kk, m); },
@@ -886,7 +931,7 @@ bwd_local_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __res
     }
     __syncthreads();
     // dTm = dW Kt^T + dU V^T;  dKt = Tm^T dW -> bDO
-    tgemm<C, C, D, 2, 1, NL>([&](int m, int kk) { return bDW[m * LD + kk]; },
+    tgemm_ks<C, C, D, 4, 4, 8, NL>([&](int m, int kk) { return bDW[m * LD + kk]; },
                          [&](int kk, int n) { return bW[n * LD + kk]; },
                          [&](int m, int n, float x) { sdT[m * L32 + n] = x + sdUV[m * L32 + n]; });
     tgemm<C, D, C, 2, 4, NL>([&](int m, int kk) { return Tm(kk, m); },
