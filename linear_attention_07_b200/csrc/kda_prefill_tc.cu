@@ -803,11 +803,14 @@ constexpr int NPREPCTA = 3;                                   // preparing CTAs 
 // per chunk, depending on where the cluster was placed); with the chain on
 // the second TPC every cluster kept pace (measured on the 8K workload).
 constexpr uint32_t CHAIN_RANK = 2;
-// slot / staging layout (identical in role 0's slots and a preparer's staging)
+// slot / staging layout (identical in role 0's slots and a preparer's staging);
+// the chain's operands are fp16, K-major (core matrices of 8 rows x 8 elements)
+constexpr uint32_t H_SBO_K128P = (D / 8) * PAD_LBO;            // 2304: K = 128, padded
+constexpr uint32_t H_SBO_K32 = (C / 8) * LBO;                  // 512: K = 32, dense
 constexpr uint32_t S_B1 = 0;                                   // [W | Qt]: N 64 x K 128 (padded)
-constexpr uint32_t S_B2 = S_B1 + 8 * SBO_K128P;                // Kb: N 128 x K 32
-constexpr uint32_t S_B3 = S_B2 + (D / 8) * SBO_K32;            // P: N 32 x K 32 (dense: vector stores)
-constexpr uint32_t S_GAM = S_B3 + (C / 8) * SBO_K32;           // gamma_C, 128 fp32
+constexpr uint32_t S_B2 = S_B1 + 8 * H_SBO_K128P;              // Kb: N 128 x K 32
+constexpr uint32_t S_B3 = S_B2 + (D / 8) * H_SBO_K32;          // P: N 32 x K 32 (dense: vector stores)
+constexpr uint32_t S_GAM = S_B3 + (C / 8) * H_SBO_K32;         // gamma_C, 128 fp32
 constexpr uint32_t S_UP = S_GAM + D * 4;                       // U' [32 tokens][128] fp32
 constexpr uint32_t SLOT = S_UP + C * D * 4;                    // bytes per chunk
 static_assert(SLOT % 16 == 0, "bulk copy size");
@@ -920,16 +923,18 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             // the compute warps have written that half of the tf32 state), then,
             // once U is in tensor memory, Kb^T U by d_k halves (one commit each,
             // so the next state update starts on the first half) and P U.
-            const uint32_t id1 = idesc_tf32(128, 2 * C, false, false);
-            const uint32_t id2 = idesc_tf32(128, 64, false, false);
-            const uint32_t id3 = idesc_tf32(128, 32, false, false);
+            // fp16 operands (kind::f16, K = 16 per MMA): the state S^T and U^T
+            // in tensor memory as packed pairs, [W | Qt], Kb and P in the slot
+            const uint32_t id1 = idesc_f16(128, 2 * C);
+            const uint32_t id2 = idesc_f16(128, 64);
+            const uint32_t id3 = idesc_f16(128, 32);
             uint32_t n_x = 0, n_k0 = 0, n_k1 = 0;   // commits on mbar, kbar0, kbar1
 #pragma unroll 1
             for (int ch = 0; ch < n_chunks; ++ch) {
                 const int slot = ch % NPREPCTA;
                 const uint32_t sb = C_SLOT0 + slot * SLOT;
                 const uint32_t dx = (ch & 1) ? CT_DX1 : CT_DX0;
-                const uint64_t bd0 = sdesc(smem_u32(sm + sb + S_B1), PAD_LBO, SBO_K128P);
+                const uint64_t bd0 = sdesc(smem_u32(sm + sb + S_B1), PAD_LBO, H_SBO_K128P);
                 if (lane == 0 && !s_abort &&
                     !mbar_wait_cluster(smem_u32(&s_bar[slot]), (uint32_t)(ch / NPREPCTA) & 1u, wait_ns))
                     expired();
@@ -938,18 +943,18 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 fence_after_sync();
                 if (!warp_flag(s_abort)) {
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks)
-                        mma_tf32_ts_w(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
-                                      id1, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < D / 32; ++ks)
+                        mma_f16_ts_w(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                     id1, ks > 0 ? 1u : 0u);
                 }
                 __syncwarp();
                 named_bar(NB_ASB, NX);
                 fence_after_sync();
                 if (!warp_flag(s_abort)) {
 #pragma unroll
-                    for (int ks = D / 16; ks < D / 8; ++ks)
-                        mma_tf32_ts_w(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
-                                      id1, 1u);
+                    for (int ks = D / 32; ks < D / 16; ++ks)
+                        mma_f16_ts_w(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                     id1, 1u);
                     mma_commit_w(mbar);
                     ++n_x;
                 }
@@ -958,23 +963,23 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 fence_after_sync();
                 if (!warp_flag(s_abort)) {
                     // Kb rows [64, 128) start 8 core-matrix rows of SBO_K32 further
-                    const uint64_t b20 = sdesc(smem_u32(sm + sb + S_B2), LBO, SBO_K32);
-                    const uint64_t b21 = sdesc(smem_u32(sm + sb + S_B2 + 8 * SBO_K32), LBO, SBO_K32);
-                    const uint64_t b30 = sdesc(smem_u32(sm + sb + S_B3), LBO, SBO_K32);
+                    const uint64_t b20 = sdesc(smem_u32(sm + sb + S_B2), LBO, H_SBO_K32);
+                    const uint64_t b21 = sdesc(smem_u32(sm + sb + S_B2 + 8 * H_SBO_K32), LBO, H_SBO_K32);
+                    const uint64_t b30 = sdesc(smem_u32(sm + sb + S_B3), LBO, H_SBO_K32);
 #pragma unroll
-                    for (int ks = 0; ks < C / 8; ++ks)
-                        mma_tf32_ts_w(tm + CT_DKU, tm + CT_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
-                                      id2, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        mma_f16_ts_w(tm + CT_DKU, tm + CT_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                     id2, ks > 0 ? 1u : 0u);
                     mma_commit_w(kbar0);
                     ++n_k0;
 #pragma unroll
-                    for (int ks = 0; ks < C / 8; ++ks)
-                        mma_tf32_ts_w(tm + CT_DKU + 64, tm + CT_AU + ks * 8, b21 + (uint64_t)((ks * 2 * LBO) >> 4),
-                                      id2, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        mma_f16_ts_w(tm + CT_DKU + 64, tm + CT_AU + ks * 8, b21 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                     id2, ks > 0 ? 1u : 0u);
 #pragma unroll
-                    for (int ks = 0; ks < C / 8; ++ks)
-                        mma_tf32_ts_w(tm + dx + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * LBO) >> 4),
-                                      id3, 1u);
+                    for (int ks = 0; ks < C / 16; ++ks)
+                        mma_f16_ts_w(tm + dx + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                     id3, 1u);
                     mma_commit_w(kbar1);
                     ++n_k1;
                 }
@@ -1065,8 +1070,18 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 if (!s_abort && !mbar_wait(bar, parity, wait_ns)) expired();
                 fence_after_sync();
             };
-            // S[32 q + i] holds d_k column 64 q + 32 hh + i of this thread's dv row
+            // S[32 q + i] holds d_k column 64 q + 32 hh + i of this thread's dv row.
+            // The MMA copy of S^T is fp16, two d_k columns per tensor-memory
+            // column: d_k columns [64 q + 32 hh, +32) are packed columns
+            // [32 q + 16 hh, +16) of CT_AS.
             float S[D / 2];
+            auto put_state = [&](int q2) {
+                float hp[16];
+#pragma unroll
+                for (int w = 0; w < 16; ++w) hp[w] = pack_f16x2(S[32 * q2 + 2 * w], S[32 * q2 + 2 * w + 1]);
+                tmem_st16(tm + lane_base + CT_AS + 32 * q2 + 16 * hh, hp);
+                wait_st();
+            };
             {
                 const float* h0h = (h0 && !(flags & SEG_H0_EYE)) ? h0 + head_off * D * D : nullptr;
 #pragma unroll
@@ -1077,12 +1092,8 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                         S[32 * q2 + i] = (flags & SEG_H0_EYE) ? (row == j ? 1.f : 0.f)
                                                               : (h0h ? h0h[(int64_t)row * D + j] : 0.f);
                     }
-                    float t32[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) t32[i] = to_tf32(S[32 * q2 + i]);
-                    tmem_st32(tm + lane_base + CT_AS + 64 * q2 + 32 * hh, t32);
+                    put_state(q2);
                 }
-                wait_st();
             }
             // S <- S + Kb^T U on d_k half q2 (the decay is already applied)
             auto state_half = [&](int q2) {
@@ -1090,12 +1101,8 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 tmem_ld32(tm + lane_base + CT_DKU + 64 * q2 + 32 * hh, d);
                 wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    S[32 * q2 + i] += d[i];
-                    d[i] = to_tf32(S[32 * q2 + i]);
-                }
-                tmem_st32(tm + lane_base + CT_AS + 64 * q2 + 32 * hh, d);
-                wait_st();
+                for (int i = 0; i < 32; ++i) S[32 * q2 + i] += d[i];
+                put_state(q2);
             };
             // the fp32 state after chunk gc of the sequence, when it ends a snapshot block
             auto snapshot = [&](int gc) {
@@ -1172,14 +1179,16 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 if (!s_abort && !counter_wait(smem_u32(&s_full), (uint32_t)ch + 1u, wait_ns)) expired();
                 wait_bar(mbar, phase & 1u);
                 ++phase;
-                {   // U = U' - W S  (this thread: tokens [16 hh, 16 hh + 16))
+                {   // U = U' - W S  (this thread: tokens [16 hh, 16 hh + 16)),
+                    // fp16 pairs into packed columns [8 hh, 8 hh + 8) of CT_AU
                     const float* up = reinterpret_cast<const float*>(sm + sb + S_UP);
-                    float x[16];
+                    float x[16], hp[8];
                     tmem_ld16(tm + lane_base + dx + 16 * hh, x);
                     wait_ld();
 #pragma unroll
-                    for (int r = 0; r < 16; ++r) x[r] = to_tf32(up[(16 * hh + r) * D + j] - x[r]);
-                    tmem_st16(tm + lane_base + CT_AU + 16 * hh, x);
+                    for (int r = 0; r < 16; r += 2)
+                        hp[r >> 1] = pack_f16x2(up[(16 * hh + r) * D + j] - x[r], up[(16 * hh + r + 1) * D + j] - x[r + 1]);
+                    tmem_st8(tm + lane_base + CT_AU + 8 * hh, hp);
                     wait_st();
                 }
                 fence_before_sync();
@@ -1479,15 +1488,18 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 #pragma unroll
             for (int rr = 0; rr < TILE; ++rr) {
                 const int r = tau * TILE + rr;
-                qf[rr] = to_tf32(gbf[off_kmajor(C + r, c, PAD_LBO, SBO_K128P) >> 2] * fq);
+                qf[rr] = gbf[off_kmajor(C + r, c, PAD_LBO, SBO_K128P) >> 2] * fq;
                 const int row = tau ? (TILE + rr) : (C + rr);
-                kf[rr] = to_tf32(gaf[off_kmajor(row, c, PAD_LBO, SBO_K128P) >> 2] * fk);
+                kf[rr] = gaf[off_kmajor(row, c, PAD_LBO, SBO_K128P) >> 2] * fk;
             }
-            float pf4[4];
-            {
-                const int r = pt & 31, i = (pt >> 5) * 4;     // lane = row: no bank conflicts
-#pragma unroll
-                for (int u = 0; u < 4; ++u) pf4[u] = to_tf32(pm[r * LD + i + u]);
+            // P as fp16, eight K-adjacent entries per thread (threads 0-127;
+            // lane = row: no bank conflicts)
+            uint4 pf8 = make_uint4(0u, 0u, 0u, 0u);
+            if (pt < 4 * C) {
+                const int r = pt & 31, i = (pt >> 5) * 8;
+                const float* row = pm + r * LD + i;
+                pf8 = make_uint4(__float_as_uint(pack_f16x2(row[0], row[1])), __float_as_uint(pack_f16x2(row[2], row[3])),
+                                 __float_as_uint(pack_f16x2(row[4], row[5])), __float_as_uint(pack_f16x2(row[6], row[7])));
             }
             // the previous chunk's bulk copy has finished reading the staging
             wait_mma();
@@ -1497,21 +1509,28 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 tmem_ld16(tm + lane_base + PT_DW + 16 * tau, w);
                 tmem_ld16(tm + lane_base + PT_DU + 16 * tau, upv);
                 wait_ld();
+                // [W | Qt] (fp16, element (token, d_k channel c)) and U' (fp32)
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
-                    st_f32(st, S_B1 + off_kmajor(16 * tau + r, c, PAD_LBO, SBO_K128P), to_tf32(w[r]));
+                    *reinterpret_cast<uint16_t*>(st + S_B1 + off16_kmajor(16 * tau + r, c, PAD_LBO, H_SBO_K128P)) =
+                        to_f16_bits(w[r]);
                     reinterpret_cast<float*>(st + S_UP)[(16 * tau + r) * D + c] = upv[r];
                 }
 #pragma unroll
                 for (int rr = 0; rr < TILE; ++rr)
-                    st_f32(st, S_B1 + off_kmajor(C + tau * TILE + rr, c, PAD_LBO, SBO_K128P), qf[rr]);
+                    *reinterpret_cast<uint16_t*>(st + S_B1 + off16_kmajor(C + tau * TILE + rr, c, PAD_LBO, H_SBO_K128P)) =
+                        to_f16_bits(qf[rr]);
+                // Kb (fp16, element (d_k channel c, token)): 8 tokens per vector
 #pragma unroll
-                for (int rr = 0; rr < TILE; rr += 4)
-                    st_f32x4(st, S_B2 + off_kmajor(c, tau * TILE + rr, LBO, SBO_K32),
-                             kf[rr], kf[rr + 1], kf[rr + 2], kf[rr + 3]);
-                {
-                    const int r = pt & 31, i = (pt >> 5) * 4;
-                    st_f32x4(st, S_B3 + off_kmajor(r, i, LBO, SBO_K32), pf4[0], pf4[1], pf4[2], pf4[3]);
+                for (int rr = 0; rr < TILE; rr += 8)
+                    *reinterpret_cast<uint4*>(st + S_B2 + off16_kmajor(c, tau * TILE + rr, LBO, H_SBO_K32)) =
+                        make_uint4(__float_as_uint(pack_f16x2(kf[rr], kf[rr + 1])),
+                                   __float_as_uint(pack_f16x2(kf[rr + 2], kf[rr + 3])),
+                                   __float_as_uint(pack_f16x2(kf[rr + 4], kf[rr + 5])),
+                                   __float_as_uint(pack_f16x2(kf[rr + 6], kf[rr + 7])));
+                if (pt < 4 * C) {
+                    const int r = pt & 31, i = (pt >> 5) * 8;
+                    *reinterpret_cast<uint4*>(st + S_B3 + off16_kmajor(r, i, LBO, H_SBO_K32)) = pf8;
                 }
                 if (tau == 0) reinterpret_cast<float*>(st + S_GAM)[c] = gam_c;
             }

@@ -1,23 +1,30 @@
-// sm_100a building blocks: tcgen05 MMA (kind::tf32), tensor memory, shared
-// memory matrix descriptors and mbarriers, as inline PTX.
+// sm_100a building blocks: tcgen05 MMA (kind::tf32 and kind::f16), tensor
+// memory, shared memory matrix descriptors and mbarriers, as inline PTX.
 //
-// Shared-memory operand layouts (no swizzle, 32-bit elements).  A "core
-// matrix" is 8 rows x 16 bytes stored contiguously (128 B).
+// Shared-memory operand layouts (no swizzle).  A "core matrix" is 8 rows x
+// 16 bytes stored contiguously (128 B): 4 elements of 32 bits or 8 of 16 bits
+// along K.  For 32-bit elements:
 //   K-major  (K contiguous):  element (mn, k) at
 //       (mn / 8) * SBO + (k / 4) * LBO + (mn % 8) * 16 + (k % 4) * 4
 //   MN-major (MN contiguous): element (mn, k) at
 //       (mn / 4) * SBO + (k / 8) * LBO + (k % 8) * 16 + (mn % 4) * 4
+// and for 16-bit elements, K-major:
+//       (mn / 8) * SBO + (k / 8) * LBO + (mn % 8) * 16 + (k % 8) * 2
 // LBO is the byte distance between core matrices adjacent along K, SBO the
 // distance between core matrices adjacent along M/N.  One tf32 MMA consumes
-// K = 8: two K-adjacent core matrices (K-major) or one (MN-major), so the
-// descriptor start advances by 2*LBO (K-major) or LBO (MN-major) per step.
+// K = 8 and one f16 MMA K = 16: in both cases two K-adjacent core matrices
+// (K-major) or one (MN-major, tf32), so the descriptor start advances by
+// 2*LBO (K-major) or LBO (MN-major) per step.
 //
 // Tensor memory: 128 lanes x 512 columns of 32 bits.  An M = 128
 // accumulator puts row m in lane m; an M = 64 accumulator puts row m in
-// lane (m % 16) + 32 * (m / 16).  Warp w may only access lanes
+// lane (m % 16) + 32 * (m / 16).  A 16-bit A operand held in tensor memory
+// packs two K-adjacent elements per column (the even k in the low half), so
+// an f16 MMA reads 8 columns.  Warp w may only access lanes
 // [32 (w % 4), 32 (w % 4) + 32).
 #pragma once
 #include <stdint.h>
+#include <cuda_fp16.h>
 
 namespace kda {
 namespace tc {
@@ -48,6 +55,19 @@ __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn_major,
          | ((b_mn_major ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17)
          | ((uint32_t)(M >> 4) << 24);
+}
+
+// Instruction descriptor for kind::f16 with fp16 A and B (format code 0 for
+// both) and fp32 accumulation; K-major operands.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+    return (1u << 4)                              // D format: f32
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
+}
+
+// Byte offset of 16-bit element (mn, k) in the no-swizzle K-major layout.
+__host__ __device__ constexpr uint32_t off16_kmajor(int mn, int k, uint32_t lbo, uint32_t sbo) {
+    return (uint32_t)(mn / 8) * sbo + (uint32_t)(k / 8) * lbo + (uint32_t)(mn % 8) * 16u + (uint32_t)(k % 8) * 2u;
 }
 
 // Byte offsets inside the no-swizzle canonical layouts (32-bit elements).
@@ -85,6 +105,16 @@ __device__ __forceinline__ void mma_tf32_ts_w(uint32_t d_tmem, uint32_t a_tmem, 
         "elect.sync _|p, 0xffffffff;\n\t"
         "setp.ne.b32 q, %4, 0;\n\t"
         "@p tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, q;\n\t}\n"
+        :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_f16_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "setp.ne.b32 q, %4, 0;\n\t"
+        "@p tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, q;\n\t}\n"
         :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
@@ -340,6 +370,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+        :: "r"(taddr),
+           "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+           "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+           "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -372,6 +412,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
            "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
            "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
         : "memory");
+}
+
+// Two fp32 values rounded to fp16 (nearest, ties to even) and packed into one
+// 32-bit word, lo in the low half; returned as the word's bit pattern in a
+// float register (the tensor-memory stores take 32-bit words).
+__device__ __forceinline__ float pack_f16x2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return __uint_as_float(*reinterpret_cast<const uint32_t*>(&h));
+}
+__device__ __forceinline__ uint16_t to_f16_bits(float x) {
+    return __half_as_ushort(__float2half_rn(x));
 }
 
 // Round an fp32 value to tf32 (nearest, ties away from zero): add half of the
