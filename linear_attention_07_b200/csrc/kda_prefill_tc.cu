@@ -38,11 +38,14 @@
 //   * the segment scan for very few heads on long sequences: every sequence
 //     cut into segments run in parallel by either kernel, joined through
 //     their transitions (description above launch_segmented).
-// Every MMA is tf32 (kind::tf32) with fp32 accumulation, issued by a whole
-// converged warp with elect.sync.  Operands are rounded to tf32 once, to
-// nearest (ties away from zero), by an integer add-and-mask: bf16 operands
-// would leave errors of a few percent of rms(o) on these products (the q.k
-// diagonal times a large u); tf32 leaves a few tenths of a percent.
+// Every MMA accumulates in fp32 and is issued by a whole converged warp with
+// elect.sync.  The products that take the decay-scaled keys (the Gram and WY
+// products, factors up to e^80) are tf32 (kind::tf32); operands are rounded to
+// tf32 once, to nearest (ties away from zero), by an integer add-and-mask:
+// bf16 operands would leave errors of a few percent of rms(o) on these
+// products (the q.k diagonal times a large u); tf32 leaves a few tenths of a
+// percent.  The cluster kernel's chain products take fp16 instead (same
+// significand; see there).
 // Shared-memory operands use the no-swizzle K-major layout; when the thread
 // that produces a value owns the K index, the K-direction core-matrix stride
 // is padded to 144 B so that a warp's scalar stores hit distinct banks.
@@ -784,9 +787,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // FULL[slot] (chain CTA) counts the copy's bytes and is armed by the chain CTA
 // itself when it hands the slot back; EMPTY (the preparing CTA) is arrived on
 // by the chain CTA once the chunk's MMAs are done and its decay applied.  o of
-// a chunk is staged one chunk late, while the next chunk's first MMA runs,
-// and written by a tensor store.  The arithmetic is the one of
-// prefill_tc_kernel.
+// a chunk is staged one chunk late, while the next chunk's first MMA runs, in
+// one of two buffers, and written by a tensor store.  The arithmetic is the
+// one of prefill_tc_kernel, except that the chain's three products
+// (S^T [W | Qt]^T, Kb^T U, P U) take fp16 operands (kind::f16, K = 16 per
+// MMA): fp16 keeps tf32's 10-bit significand, and these operands are bounded
+// (|Qt|, |Kb|, |P| <= 1 for unit-norm q and k; S, W and U of the order of h0
+// and v), far inside fp16's range (65504).  Half as many MMAs per chunk, and
+// half the slot bytes for those operands.
 namespace pc {
 using namespace pf;
 constexpr int NCW = 256;                                      // compute threads per CTA (both roles)
@@ -816,8 +824,9 @@ constexpr uint32_t SLOT = S_UP + C * D * 4;                    // bytes per chun
 static_assert(SLOT % 16 == 0, "bulk copy size");
 // role 0 (chain): NPREPCTA slots
 constexpr uint32_t C_SLOT0 = 0;
-constexpr uint32_t C_OST = NPREPCTA * SLOT;                    // o staging of one chunk (32 x 128 bf16)
-constexpr uint32_t C_BYTES = C_OST + C * D * 2;
+constexpr uint32_t C_OST = NPREPCTA * SLOT;                    // o staging, two chunks (2 x 32 x 128 bf16)
+constexpr uint32_t OST_BYTES = C * D * 2;
+constexpr uint32_t C_BYTES = C_OST + 2 * OST_BYTES;
 // roles 1-3 (preparation)
 constexpr uint32_t P_RAW = 0;
 constexpr uint32_t P_BETA = P_RAW + 4 * RAW_T;
@@ -837,7 +846,7 @@ constexpr uint32_t P_NRM = P_YMS + TILE * (TILE + 1) * 4;    // prologue: per-wa
 constexpr uint32_t P_BYTES = P_NRM + NRM_BYTES;
 constexpr uint32_t SMEM_BYTES = P_BYTES > C_BYTES ? P_BYTES : C_BYTES;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(C_OST % 128 == 0, "tensor store source alignment");
+static_assert(C_OST % 128 == 0 && OST_BYTES % 128 == 0, "tensor store source alignment");
 static_assert(P_ST % 16 == 0 && P_GA % 16 == 0 && P_GB % 16 == 0 && P_WA % 16 == 0 && P_VA % 16 == 0 &&
               P_TB % 16 == 0 && SLOT % 16 == 0, "alignment");
 // tensor memory: role 0 uses 416 columns (512 allocated), roles 1-3 use 128
@@ -859,7 +868,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     using namespace tc;
     extern __shared__ __align__(1024) unsigned char sm[];
     __shared__ uint32_t s_taddr;
-    __shared__ __align__(8) uint64_t s_bar[7];   // role 0: FULL[0..2], X, KU0, KU1, o staged; roles 1-3: EMPTY, MMA, input loads
+    __shared__ __align__(8) uint64_t s_bar[8];   // role 0: FULL[0..2], X, KU0, KU1, o staged[0..1]; roles 1-3: EMPTY, MMA, input loads
     __shared__ int s_abort;
     __shared__ uint32_t s_odone;                 // role 0: chunks whose slot is consumed
     __shared__ uint32_t s_full;                  // role 0: chunks whose slot has landed (FULL observed)
@@ -886,6 +895,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     if (tid == 0) {
         for (int i = 0; i < 6; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
         mbar_init(smem_u32(&s_bar[6]), NCW / 32);    // one arrive per compute warp
+        mbar_init(smem_u32(&s_bar[7]), NCW / 32);
         fence_mbar_init();
         s_abort = 0;
         s_odone = 0;
@@ -999,20 +1009,24 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             // Chunk ch: observe its slot's FULL phase (a cluster-scope acquire,
             // which costs a few hundred cycles) and publish that with a CTA
             // counter, so the compute warps, which read U' from the slot, pay
-            // only a CTA-scope acquire on their path.  Then, once chunk ch - 1's
-            // last MMAs are done (and its decay applied), nothing reads its slot
-            // any more: hand it back to its preparer.  A remote arrive is slow,
-            // so it stays off the issuer's and the compute warps' path.
-            // Completion comes from a counter that the compute warps advance in
-            // order; a counter cannot be misread by a reader that lags.
-            // o of chunk cp, once the compute warps have staged it: one tensor
-            // store (rows past T are clipped by the tensor map), then the
-            // staging is handed back as soon as the store has read it.
+            // only a CTA-scope acquire on their path (publishing it from the
+            // issuer, which waits on FULL too, put the release on the MMA path
+            // and was slower).  Then, once chunk ch - 1's last MMAs are done (and
+            // its decay applied), nothing reads its slot any more: hand it back
+            // to its preparer.  A remote arrive is slow, so it stays off the
+            // issuer's and the compute warps' path.  Completion comes from a
+            // counter that the compute warps advance in order; a counter cannot
+            // be misread by a reader that lags.
+            // o of chunk cp, once the compute warps have staged it in buffer
+            // cp & 1: one tensor store (rows past T are clipped by the tensor
+            // map), then the buffer is handed back as soon as the store has
+            // read it (the compute warps refill it two chunks later).
             auto store_output = [&](int cp) {
                 if (lane == 0) {
-                    if (!s_abort && !mbar_wait(smem_u32(&s_bar[6]), (uint32_t)cp & 1u, wait_ns)) expired();
+                    const uint32_t ob = (uint32_t)cp & 1u;
+                    if (!s_abort && !mbar_wait(smem_u32(&s_bar[6 + ob]), ((uint32_t)cp >> 1) & 1u, wait_ns)) expired();
                     if (!*(volatile int*)&s_abort) {
-                        tma_store_3d(&tm_o, h * D, ts + cp * C, b, smem_u32(sm + C_OST));
+                        tma_store_3d(&tm_o, h * D, ts + cp * C, b, smem_u32(sm + C_OST + ob * OST_BYTES));
                         bulk_commit();
                     }
                     bulk_wait_read_all();
@@ -1141,15 +1155,17 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             };
             auto emit_output = [&](int cp) {
                 if (!store_o) return;
-                // the store of chunk cp - 1 has read the staging
-                if (lane == 0 && !s_abort && !counter_wait(smem_u32(&s_ofree), (uint32_t)cp, wait_ns)) expired();
+                // the store of chunk cp - 2 has read buffer cp & 1
+                if (lane == 0 && cp >= 2 && !s_abort && !counter_wait(smem_u32(&s_ofree), (uint32_t)cp - 1u, wait_ns))
+                    expired();
                 __syncwarp();
-                __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + C_OST);
+                const uint32_t ob = (uint32_t)cp & 1u;
+                __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + C_OST + ob * OST_BYTES);
 #pragma unroll
                 for (int r = 0; r < 16; ++r) ost[(16 * hh + r) * D + j] = __float2bfloat16_rn(ov[r]);
                 fence_smem_to_async();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&s_bar[6]));
+                if (lane == 0) mbar_arrive(smem_u32(&s_bar[6 + ob]));
             };
             fence_before_sync();
             if (n_chunks > 0) {                       // the initial state for chunk 0
