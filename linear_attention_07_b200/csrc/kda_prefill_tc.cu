@@ -794,7 +794,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // MMA): fp16 keeps tf32's 10-bit significand, and these operands are bounded
 // (|Qt|, |Kb|, |P| <= 1 for unit-norm q and k; S, W and U of the order of h0
 // and v), far inside fp16's range (65504).  Half as many MMAs per chunk, and
-// half the slot bytes for those operands.
+// half the slot bytes for those operands.  fp16's range is the price: entries
+// below 2^-14 lose significand bits (2^-24 absolute), so a state whose scale
+// is itself tiny would lose relative accuracy.  The transition pass of the
+// segment scan (state from I, v = 0, decaying towards zero, whose relative
+// accuracy is tested) therefore runs the same kernel with tf32 operands.
 namespace pc {
 using namespace pf;
 constexpr int NCW = 256;                                      // compute threads per CTA (both roles)
@@ -811,23 +815,9 @@ constexpr int NPREPCTA = 3;                                   // preparing CTAs 
 // per chunk, depending on where the cluster was placed); with the chain on
 // the second TPC every cluster kept pace (measured on the 8K workload).
 constexpr uint32_t CHAIN_RANK = 2;
-// slot / staging layout (identical in role 0's slots and a preparer's staging);
-// the chain's operands are fp16, K-major (core matrices of 8 rows x 8 elements)
-constexpr uint32_t H_SBO_K128P = (D / 8) * PAD_LBO;            // 2304: K = 128, padded
-constexpr uint32_t H_SBO_K32 = (C / 8) * LBO;                  // 512: K = 32, dense
-constexpr uint32_t S_B1 = 0;                                   // [W | Qt]: N 64 x K 128 (padded)
-constexpr uint32_t S_B2 = S_B1 + 8 * H_SBO_K128P;              // Kb: N 128 x K 32
-constexpr uint32_t S_B3 = S_B2 + (D / 8) * H_SBO_K32;          // P: N 32 x K 32 (dense: vector stores)
-constexpr uint32_t S_GAM = S_B3 + (C / 8) * H_SBO_K32;         // gamma_C, 128 fp32
-constexpr uint32_t S_UP = S_GAM + D * 4;                       // U' [32 tokens][128] fp32
-constexpr uint32_t SLOT = S_UP + C * D * 4;                    // bytes per chunk
-static_assert(SLOT % 16 == 0, "bulk copy size");
-// role 0 (chain): NPREPCTA slots
+constexpr uint32_t OST_BYTES = C * D * 2;                      // o staging of one chunk (32 x 128 bf16)
 constexpr uint32_t C_SLOT0 = 0;
-constexpr uint32_t C_OST = NPREPCTA * SLOT;                    // o staging, two chunks (2 x 32 x 128 bf16)
-constexpr uint32_t OST_BYTES = C * D * 2;
-constexpr uint32_t C_BYTES = C_OST + 2 * OST_BYTES;
-// roles 1-3 (preparation)
+// roles 1-3 (preparation): the fixed part of the layout
 constexpr uint32_t P_RAW = 0;
 constexpr uint32_t P_BETA = P_RAW + 4 * RAW_T;
 constexpr uint32_t P_GEX = P_BETA + C * 4;
@@ -837,24 +827,49 @@ constexpr uint32_t P_WA = P_GB + 8 * SBO_K128P;
 constexpr uint32_t P_VA = P_WA + (D / 8) * SBO_K32;
 constexpr uint32_t P_TB = P_VA + (D / 8) * SBO_K32;
 constexpr uint32_t P_ST = P_TB + (C / 8) * SBO_K32P;           // staging of one slot
-constexpr uint32_t P_AMS = P_ST + SLOT;
-constexpr uint32_t P_PMS = P_AMS + C * LD * 4;
-constexpr uint32_t P_XMS = P_PMS + C * LD * 4;
-constexpr uint32_t P_TMS = P_XMS + C * LD * 4;
-constexpr uint32_t P_YMS = P_TMS + C * LD * 4;
-constexpr uint32_t P_NRM = P_YMS + TILE * (TILE + 1) * 4;    // prologue: per-warp squared norms
-constexpr uint32_t P_BYTES = P_NRM + NRM_BYTES;
-constexpr uint32_t SMEM_BYTES = P_BYTES > C_BYTES ? P_BYTES : C_BYTES;
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(C_OST % 128 == 0 && OST_BYTES % 128 == 0, "tensor store source alignment");
 static_assert(P_ST % 16 == 0 && P_GA % 16 == 0 && P_GB % 16 == 0 && P_WA % 16 == 0 && P_VA % 16 == 0 &&
-              P_TB % 16 == 0 && SLOT % 16 == 0, "alignment");
+              P_TB % 16 == 0, "alignment");
+// The operands of the chain's three products, fp16 (H) or tf32, K-major:
+// the slot layout (identical in role 0's slots and a preparer's staging) and
+// everything that depends on its size.  fp16 is the default; the transition
+// pass of the segment scan (state from I, v = 0) takes tf32, because its
+// states shrink towards fp16's subnormal range while their relative accuracy
+// is still wanted.
+template <bool H> struct Chain {
+    static constexpr int KSTEP = H ? 16 : 8;                             // K per MMA
+    static constexpr uint32_t SBO_B1 = H ? (D / 8) * PAD_LBO : SBO_K128P;  // [W | Qt], K = 128, padded
+    static constexpr uint32_t SBO_B23 = H ? (C / 8) * LBO : SBO_K32;       // Kb, P: K = 32, dense
+    static constexpr uint32_t S_B1 = 0;                                  // [W | Qt]: N 64 x K 128
+    static constexpr uint32_t S_B2 = S_B1 + 8 * SBO_B1;                  // Kb: N 128 x K 32
+    static constexpr uint32_t S_B3 = S_B2 + (D / 8) * SBO_B23;           // P: N 32 x K 32
+    static constexpr uint32_t S_GAM = S_B3 + (C / 8) * SBO_B23;          // gamma_C, 128 fp32
+    static constexpr uint32_t S_UP = S_GAM + D * 4;                      // U' [32 tokens][128] fp32
+    static constexpr uint32_t SLOT = S_UP + C * D * 4;                   // bytes per chunk
+    // role 0: NPREPCTA slots, then NOST o staging buffers (two fit next to
+    // fp16 slots, one next to tf32 slots)
+    static constexpr int NOST = H ? 2 : 1;
+    static constexpr uint32_t C_OST = NPREPCTA * SLOT;
+    static constexpr uint32_t C_BYTES = C_OST + NOST * OST_BYTES;
+    // roles 1-3: the staging of one slot, then the solve's scratch
+    static constexpr uint32_t P_AMS = P_ST + SLOT;
+    static constexpr uint32_t P_PMS = P_AMS + C * LD * 4;
+    static constexpr uint32_t P_XMS = P_PMS + C * LD * 4;
+    static constexpr uint32_t P_TMS = P_XMS + C * LD * 4;
+    static constexpr uint32_t P_YMS = P_TMS + C * LD * 4;
+    static constexpr uint32_t P_NRM = P_YMS + TILE * (TILE + 1) * 4;   // prologue: per-warp squared norms
+    static constexpr uint32_t P_BYTES = P_NRM + NRM_BYTES;
+    static constexpr uint32_t SMEM_BYTES = P_BYTES > C_BYTES ? P_BYTES : C_BYTES;
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+    static_assert(SLOT % 16 == 0, "bulk copy size");
+    static_assert(C_OST % 128 == 0 && OST_BYTES % 128 == 0, "tensor store source alignment");
+};
 // tensor memory: role 0 uses 416 columns (512 allocated), roles 1-3 use 128
 constexpr uint32_t CT_AS = 0, CT_AU = 128, CT_DX0 = 160, CT_DKU = 224, CT_DX1 = 352;
 constexpr uint32_t PT_DG = 0, PT_DW = 64, PT_DU = 96;
 }  // namespace pc
 
-template <bool PRO>       // PRO: the fused prologue (launch flag PROLOGUE)
+// PRO: the fused prologue (launch flag PROLOGUE); F16: fp16 chain operands
+template <bool PRO, bool F16>
 __global__ void __cluster_dims__(pc::NPREPCTA + 1, 1, 1) __launch_bounds__(pc::NTH, 1)
 prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -866,6 +881,21 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 {
     using namespace pc;
     using namespace tc;
+    using CH = Chain<F16>;
+    constexpr uint32_t S_B1 = CH::S_B1, S_B2 = CH::S_B2, S_B3 = CH::S_B3, S_GAM = CH::S_GAM, S_UP = CH::S_UP;
+    constexpr uint32_t SLOT = CH::SLOT, C_OST = CH::C_OST;
+    constexpr int NOST = CH::NOST;
+    constexpr uint32_t P_AMS = CH::P_AMS, P_PMS = CH::P_PMS, P_XMS = CH::P_XMS, P_TMS = CH::P_TMS,
+                       P_YMS = CH::P_YMS, P_NRM = CH::P_NRM;
+    // the chain's MMAs: kind::f16 or kind::tf32 by the operand type
+    auto mma_chain = [](uint32_t d, uint32_t a_tmem, uint64_t b_desc, uint32_t id, uint32_t acc) {
+        if constexpr (F16) mma_f16_ts_w(d, a_tmem, b_desc, id, acc);
+        else mma_tf32_ts_w(d, a_tmem, b_desc, id, acc);
+    };
+    auto idesc_chain = [](int M, int N) -> uint32_t {
+        if constexpr (F16) return idesc_f16(M, N);
+        else return idesc_tf32(M, N, false, false);
+    };
     extern __shared__ __align__(1024) unsigned char sm[];
     __shared__ uint32_t s_taddr;
     __shared__ __align__(8) uint64_t s_bar[8];   // role 0: FULL[0..2], X, KU0, KU1, o staged[0..1]; roles 1-3: EMPTY, MMA, input loads
@@ -933,18 +963,20 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             // the compute warps have written that half of the tf32 state), then,
             // once U is in tensor memory, Kb^T U by d_k halves (one commit each,
             // so the next state update starts on the first half) and P U.
-            // fp16 operands (kind::f16, K = 16 per MMA): the state S^T and U^T
-            // in tensor memory as packed pairs, [W | Qt], Kb and P in the slot
-            const uint32_t id1 = idesc_f16(128, 2 * C);
-            const uint32_t id2 = idesc_f16(128, 64);
-            const uint32_t id3 = idesc_f16(128, 32);
+            // With fp16 operands (kind::f16, K = 16 per MMA) the state S^T and
+            // U^T sit in tensor memory as packed pairs; either way an MMA reads
+            // 8 tensor-memory columns of A and two K-adjacent core matrices of B.
+            const uint32_t id1 = idesc_chain(128, 2 * C);
+            const uint32_t id2 = idesc_chain(128, 64);
+            const uint32_t id3 = idesc_chain(128, 32);
+            constexpr int NKX = D / CH::KSTEP, NKU = C / CH::KSTEP;   // K steps of X and of Kb^T U, P U
             uint32_t n_x = 0, n_k0 = 0, n_k1 = 0;   // commits on mbar, kbar0, kbar1
 #pragma unroll 1
             for (int ch = 0; ch < n_chunks; ++ch) {
                 const int slot = ch % NPREPCTA;
                 const uint32_t sb = C_SLOT0 + slot * SLOT;
                 const uint32_t dx = (ch & 1) ? CT_DX1 : CT_DX0;
-                const uint64_t bd0 = sdesc(smem_u32(sm + sb + S_B1), PAD_LBO, H_SBO_K128P);
+                const uint64_t bd0 = sdesc(smem_u32(sm + sb + S_B1), PAD_LBO, CH::SBO_B1);
                 if (lane == 0 && !s_abort &&
                     !mbar_wait_cluster(smem_u32(&s_bar[slot]), (uint32_t)(ch / NPREPCTA) & 1u, wait_ns))
                     expired();
@@ -953,18 +985,18 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 fence_after_sync();
                 if (!warp_flag(s_abort)) {
 #pragma unroll
-                    for (int ks = 0; ks < D / 32; ++ks)
-                        mma_f16_ts_w(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
-                                     id1, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < NKX / 2; ++ks)
+                        mma_chain(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                  id1, ks > 0 ? 1u : 0u);
                 }
                 __syncwarp();
                 named_bar(NB_ASB, NX);
                 fence_after_sync();
                 if (!warp_flag(s_abort)) {
 #pragma unroll
-                    for (int ks = D / 32; ks < D / 16; ++ks)
-                        mma_f16_ts_w(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
-                                     id1, 1u);
+                    for (int ks = NKX / 2; ks < NKX; ++ks)
+                        mma_chain(tm + dx, tm + CT_AS + ks * 8, bd0 + (uint64_t)((ks * 2 * PAD_LBO) >> 4),
+                                  id1, 1u);
                     mma_commit_w(mbar);
                     ++n_x;
                 }
@@ -973,23 +1005,23 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 fence_after_sync();
                 if (!warp_flag(s_abort)) {
                     // Kb rows [64, 128) start 8 core-matrix rows of SBO_K32 further
-                    const uint64_t b20 = sdesc(smem_u32(sm + sb + S_B2), LBO, H_SBO_K32);
-                    const uint64_t b21 = sdesc(smem_u32(sm + sb + S_B2 + 8 * H_SBO_K32), LBO, H_SBO_K32);
-                    const uint64_t b30 = sdesc(smem_u32(sm + sb + S_B3), LBO, H_SBO_K32);
+                    const uint64_t b20 = sdesc(smem_u32(sm + sb + S_B2), LBO, CH::SBO_B23);
+                    const uint64_t b21 = sdesc(smem_u32(sm + sb + S_B2 + 8 * CH::SBO_B23), LBO, CH::SBO_B23);
+                    const uint64_t b30 = sdesc(smem_u32(sm + sb + S_B3), LBO, CH::SBO_B23);
 #pragma unroll
-                    for (int ks = 0; ks < C / 16; ++ks)
-                        mma_f16_ts_w(tm + CT_DKU, tm + CT_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
-                                     id2, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < NKU; ++ks)
+                        mma_chain(tm + CT_DKU, tm + CT_AU + ks * 8, b20 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                  id2, ks > 0 ? 1u : 0u);
                     mma_commit_w(kbar0);
                     ++n_k0;
 #pragma unroll
-                    for (int ks = 0; ks < C / 16; ++ks)
-                        mma_f16_ts_w(tm + CT_DKU + 64, tm + CT_AU + ks * 8, b21 + (uint64_t)((ks * 2 * LBO) >> 4),
-                                     id2, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < NKU; ++ks)
+                        mma_chain(tm + CT_DKU + 64, tm + CT_AU + ks * 8, b21 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                  id2, ks > 0 ? 1u : 0u);
 #pragma unroll
-                    for (int ks = 0; ks < C / 16; ++ks)
-                        mma_f16_ts_w(tm + dx + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * LBO) >> 4),
-                                     id3, 1u);
+                    for (int ks = 0; ks < NKU; ++ks)
+                        mma_chain(tm + dx + C, tm + CT_AU + ks * 8, b30 + (uint64_t)((ks * 2 * LBO) >> 4),
+                                  id3, 1u);
                     mma_commit_w(kbar1);
                     ++n_k1;
                 }
@@ -1018,13 +1050,13 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             // counter that the compute warps advance in order; a counter cannot
             // be misread by a reader that lags.
             // o of chunk cp, once the compute warps have staged it in buffer
-            // cp & 1: one tensor store (rows past T are clipped by the tensor
+            // cp % NOST: one tensor store (rows past T are clipped by the tensor
             // map), then the buffer is handed back as soon as the store has
-            // read it (the compute warps refill it two chunks later).
+            // read it (the compute warps refill it NOST chunks later).
             auto store_output = [&](int cp) {
                 if (lane == 0) {
-                    const uint32_t ob = (uint32_t)cp & 1u;
-                    if (!s_abort && !mbar_wait(smem_u32(&s_bar[6 + ob]), ((uint32_t)cp >> 1) & 1u, wait_ns)) expired();
+                    const uint32_t ob = (uint32_t)cp % NOST;
+                    if (!s_abort && !mbar_wait(smem_u32(&s_bar[6 + ob]), ((uint32_t)cp / NOST) & 1u, wait_ns)) expired();
                     if (!*(volatile int*)&s_abort) {
                         tma_store_3d(&tm_o, h * D, ts + cp * C, b, smem_u32(sm + C_OST + ob * OST_BYTES));
                         bulk_commit();
@@ -1085,15 +1117,22 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 fence_after_sync();
             };
             // S[32 q + i] holds d_k column 64 q + 32 hh + i of this thread's dv row.
-            // The MMA copy of S^T is fp16, two d_k columns per tensor-memory
-            // column: d_k columns [64 q + 32 hh, +32) are packed columns
-            // [32 q + 16 hh, +16) of CT_AS.
+            // The MMA copy of S^T: fp16 with two d_k columns per tensor-memory
+            // column (d_k columns [64 q + 32 hh, +32) in packed columns
+            // [32 q + 16 hh, +16) of CT_AS), or tf32 with one.
             float S[D / 2];
             auto put_state = [&](int q2) {
-                float hp[16];
+                if constexpr (F16) {
+                    float hp[16];
 #pragma unroll
-                for (int w = 0; w < 16; ++w) hp[w] = pack_f16x2(S[32 * q2 + 2 * w], S[32 * q2 + 2 * w + 1]);
-                tmem_st16(tm + lane_base + CT_AS + 32 * q2 + 16 * hh, hp);
+                    for (int w = 0; w < 16; ++w) hp[w] = pack_f16x2(S[32 * q2 + 2 * w], S[32 * q2 + 2 * w + 1]);
+                    tmem_st16(tm + lane_base + CT_AS + 32 * q2 + 16 * hh, hp);
+                } else {
+                    float t32[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) t32[i] = to_tf32(S[32 * q2 + i]);
+                    tmem_st32(tm + lane_base + CT_AS + 64 * q2 + 32 * hh, t32);
+                }
                 wait_st();
             };
             {
@@ -1155,11 +1194,12 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             };
             auto emit_output = [&](int cp) {
                 if (!store_o) return;
-                // the store of chunk cp - 2 has read buffer cp & 1
-                if (lane == 0 && cp >= 2 && !s_abort && !counter_wait(smem_u32(&s_ofree), (uint32_t)cp - 1u, wait_ns))
+                // the store of chunk cp - NOST has read buffer cp % NOST
+                if (lane == 0 && cp >= NOST && !s_abort &&
+                    !counter_wait(smem_u32(&s_ofree), (uint32_t)(cp - NOST + 1), wait_ns))
                     expired();
                 __syncwarp();
-                const uint32_t ob = (uint32_t)cp & 1u;
+                const uint32_t ob = (uint32_t)cp % NOST;
                 __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + C_OST + ob * OST_BYTES);
 #pragma unroll
                 for (int r = 0; r < 16; ++r) ost[(16 * hh + r) * D + j] = __float2bfloat16_rn(ov[r]);
@@ -1195,16 +1235,25 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 if (!s_abort && !counter_wait(smem_u32(&s_full), (uint32_t)ch + 1u, wait_ns)) expired();
                 wait_bar(mbar, phase & 1u);
                 ++phase;
-                {   // U = U' - W S  (this thread: tokens [16 hh, 16 hh + 16)),
-                    // fp16 pairs into packed columns [8 hh, 8 hh + 8) of CT_AU
+                {   // U = U' - W S  (this thread: tokens [16 hh, 16 hh + 16)): fp16
+                    // pairs into packed columns [8 hh, 8 hh + 8) of CT_AU, or tf32
+                    // into columns [16 hh, 16 hh + 16)
                     const float* up = reinterpret_cast<const float*>(sm + sb + S_UP);
-                    float x[16], hp[8];
+                    float x[16];
                     tmem_ld16(tm + lane_base + dx + 16 * hh, x);
                     wait_ld();
+                    if constexpr (F16) {
+                        float hp[8];
 #pragma unroll
-                    for (int r = 0; r < 16; r += 2)
-                        hp[r >> 1] = pack_f16x2(up[(16 * hh + r) * D + j] - x[r], up[(16 * hh + r + 1) * D + j] - x[r + 1]);
-                    tmem_st8(tm + lane_base + CT_AU + 8 * hh, hp);
+                        for (int r = 0; r < 16; r += 2)
+                            hp[r >> 1] = pack_f16x2(up[(16 * hh + r) * D + j] - x[r],
+                                                    up[(16 * hh + r + 1) * D + j] - x[r + 1]);
+                        tmem_st8(tm + lane_base + CT_AU + 8 * hh, hp);
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < 16; ++r) x[r] = to_tf32(up[(16 * hh + r) * D + j] - x[r]);
+                        tmem_st16(tm + lane_base + CT_AU + 16 * hh, x);
+                    }
                     wait_st();
                 }
                 fence_before_sync();
@@ -1508,14 +1557,21 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const int row = tau ? (TILE + rr) : (C + rr);
                 kf[rr] = gaf[off_kmajor(row, c, PAD_LBO, SBO_K128P) >> 2] * fk;
             }
-            // P as fp16, eight K-adjacent entries per thread (threads 0-127;
-            // lane = row: no bank conflicts)
-            uint4 pf8 = make_uint4(0u, 0u, 0u, 0u);
-            if (pt < 4 * C) {
-                const int r = pt & 31, i = (pt >> 5) * 8;
+            // P, element (n = r, k = i) (lane = row: no bank conflicts): fp16,
+            // eight K-adjacent entries per thread (threads 0-127), or tf32, four
+            uint4 pf4 = make_uint4(0u, 0u, 0u, 0u);
+            if constexpr (F16) {
+                if (pt < 4 * C) {
+                    const int r = pt & 31, i = (pt >> 5) * 8;
+                    const float* row = pm + r * LD + i;
+                    pf4 = make_uint4(__float_as_uint(pack_f16x2(row[0], row[1])), __float_as_uint(pack_f16x2(row[2], row[3])),
+                                     __float_as_uint(pack_f16x2(row[4], row[5])), __float_as_uint(pack_f16x2(row[6], row[7])));
+                }
+            } else {
+                const int r = pt & 31, i = (pt >> 5) * 4;
                 const float* row = pm + r * LD + i;
-                pf8 = make_uint4(__float_as_uint(pack_f16x2(row[0], row[1])), __float_as_uint(pack_f16x2(row[2], row[3])),
-                                 __float_as_uint(pack_f16x2(row[4], row[5])), __float_as_uint(pack_f16x2(row[6], row[7])));
+                pf4 = make_uint4(__float_as_uint(to_tf32(row[0])), __float_as_uint(to_tf32(row[1])),
+                                 __float_as_uint(to_tf32(row[2])), __float_as_uint(to_tf32(row[3])));
             }
             // the previous chunk's bulk copy has finished reading the staging
             wait_mma();
@@ -1525,28 +1581,44 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 tmem_ld16(tm + lane_base + PT_DW + 16 * tau, w);
                 tmem_ld16(tm + lane_base + PT_DU + 16 * tau, upv);
                 wait_ld();
-                // [W | Qt] (fp16, element (token, d_k channel c)) and U' (fp32)
+                // [W | Qt] (element (token, d_k channel c)) and U' (fp32)
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
-                    *reinterpret_cast<uint16_t*>(st + S_B1 + off16_kmajor(16 * tau + r, c, PAD_LBO, H_SBO_K128P)) =
-                        to_f16_bits(w[r]);
+                    if constexpr (F16)
+                        *reinterpret_cast<uint16_t*>(st + S_B1 + off16_kmajor(16 * tau + r, c, PAD_LBO, CH::SBO_B1)) =
+                            to_f16_bits(w[r]);
+                    else
+                        st_f32(st, S_B1 + off_kmajor(16 * tau + r, c, PAD_LBO, CH::SBO_B1), to_tf32(w[r]));
                     reinterpret_cast<float*>(st + S_UP)[(16 * tau + r) * D + c] = upv[r];
                 }
 #pragma unroll
-                for (int rr = 0; rr < TILE; ++rr)
-                    *reinterpret_cast<uint16_t*>(st + S_B1 + off16_kmajor(C + tau * TILE + rr, c, PAD_LBO, H_SBO_K128P)) =
-                        to_f16_bits(qf[rr]);
-                // Kb (fp16, element (d_k channel c, token)): 8 tokens per vector
+                for (int rr = 0; rr < TILE; ++rr) {
+                    if constexpr (F16)
+                        *reinterpret_cast<uint16_t*>(st + S_B1 + off16_kmajor(C + tau * TILE + rr, c, PAD_LBO, CH::SBO_B1)) =
+                            to_f16_bits(qf[rr]);
+                    else
+                        st_f32(st, S_B1 + off_kmajor(C + tau * TILE + rr, c, PAD_LBO, CH::SBO_B1), to_tf32(qf[rr]));
+                }
+                // Kb (element (d_k channel c, token)): 8 (fp16) or 4 (tf32) tokens per vector
+                if constexpr (F16) {
 #pragma unroll
-                for (int rr = 0; rr < TILE; rr += 8)
-                    *reinterpret_cast<uint4*>(st + S_B2 + off16_kmajor(c, tau * TILE + rr, LBO, H_SBO_K32)) =
-                        make_uint4(__float_as_uint(pack_f16x2(kf[rr], kf[rr + 1])),
-                                   __float_as_uint(pack_f16x2(kf[rr + 2], kf[rr + 3])),
-                                   __float_as_uint(pack_f16x2(kf[rr + 4], kf[rr + 5])),
-                                   __float_as_uint(pack_f16x2(kf[rr + 6], kf[rr + 7])));
-                if (pt < 4 * C) {
-                    const int r = pt & 31, i = (pt >> 5) * 8;
-                    *reinterpret_cast<uint4*>(st + S_B3 + off16_kmajor(r, i, LBO, H_SBO_K32)) = pf8;
+                    for (int rr = 0; rr < TILE; rr += 8)
+                        *reinterpret_cast<uint4*>(st + S_B2 + off16_kmajor(c, tau * TILE + rr, LBO, CH::SBO_B23)) =
+                            make_uint4(__float_as_uint(pack_f16x2(kf[rr], kf[rr + 1])),
+                                       __float_as_uint(pack_f16x2(kf[rr + 2], kf[rr + 3])),
+                                       __float_as_uint(pack_f16x2(kf[rr + 4], kf[rr + 5])),
+                                       __float_as_uint(pack_f16x2(kf[rr + 6], kf[rr + 7])));
+                    if (pt < 4 * C) {
+                        const int r = pt & 31, i = (pt >> 5) * 8;
+                        *reinterpret_cast<uint4*>(st + S_B3 + off16_kmajor(r, i, LBO, CH::SBO_B23)) = pf4;
+                    }
+                } else {
+#pragma unroll
+                    for (int rr = 0; rr < TILE; rr += 4)
+                        st_f32x4(st, S_B2 + off_kmajor(c, tau * TILE + rr, LBO, CH::SBO_B23),
+                                 to_tf32(kf[rr]), to_tf32(kf[rr + 1]), to_tf32(kf[rr + 2]), to_tf32(kf[rr + 3]));
+                    const int r = pt & 31, i = (pt >> 5) * 4;
+                    *reinterpret_cast<uint4*>(st + S_B3 + off_kmajor(r, i, LBO, CH::SBO_B23)) = pf4;
                 }
                 if (tau == 0) reinterpret_cast<float*>(st + S_GAM)[c] = gam_c;
             }
@@ -1612,8 +1684,14 @@ static cudaError_t set_prefill_attributes()
         const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
         cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<false>, a, (int)pf::SMEM_BYTES);
         if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_tc_kernel<true>, a, (int)pf::SMEM_BYTES);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_cluster_kernel<false>, a, (int)pc::SMEM_BYTES);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(prefill_cluster_kernel<true>, a, (int)pc::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_cluster_kernel<false, true>, a, (int)pc::Chain<true>::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_cluster_kernel<true, true>, a, (int)pc::Chain<true>::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_cluster_kernel<false, false>, a, (int)pc::Chain<false>::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(prefill_cluster_kernel<true, false>, a, (int)pc::Chain<false>::SMEM_BYTES);
         if (e == cudaSuccess) e = segment_combine_attribute();
         return e;
     });
@@ -1660,8 +1738,12 @@ static cudaError_t launch_pass(const CUtensorMap& mq, const CUtensorMap& mk, con
         memset(&mo, 0, sizeof(mo));
         if (o && !(flags & pf::SEG_NO_O) && T > 0 && !make_map(&mo, o, B, T, H)) return cudaErrorInvalidValue;
         dim3 grid((pc::NPREPCTA + 1) * H, B * n_seg);
-        auto kern = pro ? prefill_cluster_kernel<true> : prefill_cluster_kernel<false>;
-        kern<<<grid, pc::NTH, pc::SMEM_BYTES, stream>>>(
+        // fp16 chain operands, except for the transition pass (state from I)
+        const bool h16 = !(flags & pf::SEG_H0_EYE);
+        auto kern = h16 ? (pro ? prefill_cluster_kernel<true, true> : prefill_cluster_kernel<false, true>)
+                        : (pro ? prefill_cluster_kernel<true, false> : prefill_cluster_kernel<false, false>);
+        const uint32_t smem = h16 ? pc::Chain<true>::SMEM_BYTES : pc::Chain<false>::SMEM_BYTES;
+        kern<<<grid, pc::NTH, smem, stream>>>(
             mq, mk, mv, mg, mo, (const __nv_bfloat16*)beta, h0, (__nv_bfloat16*)o, hT, T, H, seg_len, n_seg, flags,
             states, snap_every, wait_limit_ns());
     } else {
