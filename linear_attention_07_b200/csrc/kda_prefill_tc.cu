@@ -827,6 +827,7 @@ constexpr uint32_t P_WA = P_GB + 8 * SBO_K128P;
 constexpr uint32_t P_VA = P_WA + (D / 8) * SBO_K32;
 constexpr uint32_t P_TB = P_VA + (D / 8) * SBO_K32;
 constexpr uint32_t P_ST = P_TB + (C / 8) * SBO_K32P;           // staging of one slot
+constexpr int ATM_LD = 16;     // row stride (floats) of a transposed 16 x 16 diagonal block of A (16-byte rows)
 static_assert(P_ST % 16 == 0 && P_GA % 16 == 0 && P_GB % 16 == 0 && P_WA % 16 == 0 && P_VA % 16 == 0 &&
               P_TB % 16 == 0, "alignment");
 // The operands of the chain's three products, fp16 (H) or tf32, K-major:
@@ -858,9 +859,15 @@ template <bool H> struct Chain {
     static constexpr uint32_t P_YMS = P_TMS + C * LD * 4;
     static constexpr uint32_t P_NRM = P_YMS + TILE * (TILE + 1) * 4;   // prologue: per-warp squared norms
     static constexpr uint32_t P_BYTES = P_NRM + NRM_BYTES;
+    // A^T of the two diagonal blocks, used only between the Gram MMA and the
+    // diagonal solve: it shares the bytes of YMS and NRM (YMS is written after
+    // the solve, NRM is used before the Gram MMA), which keeps the tf32
+    // layout inside the shared-memory budget
+    static constexpr uint32_t P_ATM = P_YMS;
+    static_assert(2 * TILE * ATM_LD * 4 <= TILE * (TILE + 1) * 4 + NRM_BYTES, "A^T fits YMS and NRM");
     static constexpr uint32_t SMEM_BYTES = P_BYTES > C_BYTES ? P_BYTES : C_BYTES;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-    static_assert(SLOT % 16 == 0, "bulk copy size");
+    static_assert(SLOT % 16 == 0 && P_ATM % 16 == 0, "bulk copy size, vector rows");
     static_assert(C_OST % 128 == 0 && OST_BYTES % 128 == 0, "tensor store source alignment");
 };
 // tensor memory: role 0 uses 416 columns (512 allocated), roles 1-3 use 128
@@ -886,7 +893,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     constexpr uint32_t SLOT = CH::SLOT, C_OST = CH::C_OST;
     constexpr int NOST = CH::NOST;
     constexpr uint32_t P_AMS = CH::P_AMS, P_PMS = CH::P_PMS, P_XMS = CH::P_XMS, P_TMS = CH::P_TMS,
-                       P_YMS = CH::P_YMS, P_NRM = CH::P_NRM;
+                       P_YMS = CH::P_YMS, P_NRM = CH::P_NRM, P_ATM = CH::P_ATM;
     // the chain's MMAs: kind::f16 or kind::tf32 by the operand type
     auto mma_chain = [](uint32_t d, uint32_t a_tmem, uint64_t b_desc, uint32_t id, uint32_t acc) {
         if constexpr (F16) mma_f16_ts_w(d, a_tmem, b_desc, id, acc);
@@ -1375,11 +1382,10 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         const int pw = warp;
         uint32_t phase = 0, rphase = 0;
         auto prep_sync = [&]() { named_bar(NB_CW, NCW); };
+        // every thread waits on the MMA barrier itself
         auto wait_mma = [&]() {
-            if (pt == 0 && !s_abort && !mbar_wait(mbar, phase & 1u, wait_ns)) expired();
+            if (!s_abort && !mbar_wait(mbar, phase & 1u, wait_ns)) expired();
             ++phase;
-            __syncwarp();
-            prep_sync();
             fence_after_sync();
         };
         const __nv_bfloat16 bzero = __float2bfloat16_rn(0.f);
@@ -1475,50 +1481,81 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                          to_tf32(vr[rr]), to_tf32(vr[rr + 1]), to_tf32(vr[rr + 2]), to_tf32(vr[rr + 3]));
             fence_smem_to_async();
             wait_mma();
-            // A and P into scratch (row m of D_G is lane (m % 16) + 32 (m / 16))
-            if (pw < 3) {
-                const int colK = (sp == 0) ? 0 : TILE;
-                float gk[16], gq[16];
-                tmem_ld16(tm + lane_base + PT_DG + colK, gk);
-                tmem_ld16(tm + lane_base + PT_DG + C + colK, gq);
-                wait_ld();
-                if (lane < TILE) {
-                    const int i = (sp == 1 ? TILE : 0) + lane;
-                    const int rbase = (sp == 0) ? 0 : TILE;
+            // A and P (32 x 32) from the Gram (row m of D_G is lane (m % 16) +
+            // 32 (m / 16)).  Sub-partition 0 holds the rows Kh_0 (columns Kt_0,
+            // Qt_0), 1 the rows Kh_1 (Kt_1, Qt_1), 2 the rows Kb_0 (Kt_1, Qt_1:
+            // the block between the tiles).  Warps 0-2 take the A columns,
+            // warps 4-6 the P columns.  The warp that holds a diagonal block of
+            // A also solves it, X = (I + A_tt)^-1, column i per lane, forward
+            // substitution, from A_tt^T in shared memory (one 16-float column
+            // per step, read as four vectors), with no barrier in between.
+            {
+                const int spx = pw & 3;
+                if (spx < 3) {
+                    const bool is_p = pw >= 4;
+                    const int colK = (spx == 0) ? 0 : TILE;
+                    float gv[16];
+                    tmem_ld16(tm + lane_base + PT_DG + (is_p ? C : 0) + colK, gv);
+                    wait_ld();
+                    const int i = (spx == 1 ? TILE : 0) + lane;           // column of A / P
+                    const int rbase = (spx == 0) ? 0 : TILE;              // rows covered
+                    float* atm = reinterpret_cast<float*>(sm + P_ATM) + spx * TILE * ATM_LD;
+                    if (lane < TILE) {
+                        if (is_p) {
 #pragma unroll
-                    for (int r = 0; r < TILE; ++r) {
-                        const int rg = rbase + r;
-                        am[rg * LD + i] = (rg > i) ? bt[rg] * gk[r] : 0.f;
-                        pm[rg * LD + i] = (rg >= i) ? gq[r] : 0.f;
-                    }
-                    if (sp == 1) {
+                            for (int r = 0; r < TILE; ++r) {
+                                const int rg = rbase + r;
+                                pm[rg * LD + i] = (rg >= i) ? gv[r] : 0.f;
+                            }
+                            if (spx == 1) {                               // P_01 = 0
 #pragma unroll
-                        for (int r = 0; r < TILE; ++r) {
-                            am[r * LD + i] = 0.f;
-                            pm[r * LD + i] = 0.f;
+                                for (int r = 0; r < TILE; ++r) pm[r * LD + i] = 0.f;
+                            }
+                        } else if (spx == 2) {                            // A_10, all below the diagonal
+#pragma unroll
+                            for (int r = 0; r < TILE; ++r) am[(TILE + r) * LD + i] = bt[TILE + r] * gv[r];
+                        } else {                                          // column i of A_tt into row i of A_tt^T
+#pragma unroll
+                            for (int r = 0; r < TILE; r += 4) {
+                                float e4[4];
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    const int rg = rbase + r + u;
+                                    e4[u] = (rg > i) ? bt[rg] * gv[r + u] : 0.f;
+                                }
+                                *reinterpret_cast<float4*>(atm + lane * ATM_LD + r) = make_float4(e4[0], e4[1], e4[2], e4[3]);
+                            }
                         }
                     }
-                }
-            }
-            prep_sync();
-            if (pw < 2 && lane < TILE) {
-                const int off = pw * TILE;
-                const int i = lane;
-                float x[TILE];
+                    if (!is_p && spx < 2) {
+                        __syncwarp();
+                        if (lane < TILE) {
+                            const int off = spx * TILE;
+                            float x[TILE];
 #pragma unroll
-                for (int r = 0; r < TILE; ++r) x[r] = (r == i) ? 1.f : 0.f;
+                            for (int r = 0; r < TILE; ++r) x[r] = (r == lane) ? 1.f : 0.f;
 #pragma unroll
-                for (int s2 = 0; s2 < TILE; ++s2) {
+                            for (int s2 = 0; s2 < TILE; ++s2) {
+                                const float4* col = reinterpret_cast<const float4*>(atm + s2 * ATM_LD);
+                                float a16[TILE];
 #pragma unroll
-                    for (int r = s2 + 1; r < TILE; ++r)
-                        x[r] = fmaf(-am[(off + r) * LD + off + s2], x[s2], x[r]);
-                }
-                const float bi = bt[off + i];
+                                for (int q4 = 0; q4 < TILE / 4; ++q4) {
+                                    const float4 v4 = col[q4];
+                                    a16[4 * q4] = v4.x; a16[4 * q4 + 1] = v4.y;
+                                    a16[4 * q4 + 2] = v4.z; a16[4 * q4 + 3] = v4.w;
+                                }
 #pragma unroll
-                for (int r = 0; r < TILE; ++r) {
-                    xm[(off + r) * LD + off + i] = x[r];
-                    tmx[(off + r) * LD + off + i] = x[r] * bi;
-                    if (pw == 1) tmx[r * LD + off + i] = 0.f;
+                                for (int r = s2 + 1; r < TILE; ++r) x[r] = fmaf(-a16[r], x[s2], x[r]);
+                            }
+                            const float bi = bt[off + lane];
+#pragma unroll
+                            for (int r = 0; r < TILE; ++r) {
+                                xm[(off + r) * LD + off + lane] = x[r];
+                                tmx[(off + r) * LD + off + lane] = x[r] * bi;     // T_tt = X_tt diag(b)
+                                if (spx == 1) tmx[r * LD + off + lane] = 0.f;     // T_01 = 0
+                            }
+                        }
+                    }
                 }
             }
             prep_sync();

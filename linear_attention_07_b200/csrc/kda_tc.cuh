@@ -8,13 +8,16 @@
 //       (mn / 8) * SBO + (k / 4) * LBO + (mn % 8) * 16 + (k % 4) * 4
 //   MN-major (MN contiguous): element (mn, k) at
 //       (mn / 4) * SBO + (k / 8) * LBO + (k % 8) * 16 + (mn % 4) * 4
-// and for 16-bit elements, K-major:
-//       (mn / 8) * SBO + (k / 8) * LBO + (mn % 8) * 16 + (k % 8) * 2
+// and for 16-bit elements:
+//   K-major:  (mn / 8) * SBO + (k / 8) * LBO + (mn % 8) * 16 + (k % 8) * 2
+//   MN-major: (mn / 8) * SBO + (k / 8) * LBO + (k % 8) * 16 + (mn % 8) * 2
+// (so a K-major tile of a matrix is an MN-major tile of its transpose, with
+// LBO and SBO exchanged)
 // LBO is the byte distance between core matrices adjacent along K, SBO the
 // distance between core matrices adjacent along M/N.  One tf32 MMA consumes
-// K = 8 and one f16 MMA K = 16: in both cases two K-adjacent core matrices
-// (K-major) or one (MN-major, tf32), so the descriptor start advances by
-// 2*LBO (K-major) or LBO (MN-major) per step.
+// K = 8 and one f16 MMA K = 16: two K-adjacent core matrices (K-major, and
+// MN-major f16) or one (MN-major tf32), so the descriptor start advances by
+// 2*LBO or LBO per step.
 //
 // Tensor memory: 128 lanes x 512 columns of 32 bits.  An M = 128
 // accumulator puts row m in lane m; an M = 64 accumulator puts row m in
@@ -58,9 +61,10 @@ __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn_major,
 }
 
 // Instruction descriptor for kind::f16 with fp16 A and B (format code 0 for
-// both) and fp32 accumulation; K-major operands.
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+// both) and fp32 accumulation; A K-major, B K-major or MN-major.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn_major = false) {
     return (1u << 4)                              // D format: f32
+         | ((b_mn_major ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17)
          | ((uint32_t)(M >> 4) << 24);
 }
