@@ -135,12 +135,28 @@ def load_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def tensor_fractions(alg_flops, launch_ms, bf16_tflops):
-    """Algorithmic tensor throughput of a prefill launch against the peak of
-    its own MMA type: every prefill MMA is kind::tf32, whose peak is taken as
-    half the measured bf16 peak (the nominal tf32 : bf16 ratio, 1 : 2)."""
+def prefill_state_flops(B, T, H, dk, dv):
+    """Flops of the three state-sized products (W S, Q S, K^T U: 6 dk dv per
+    token-head), the part of prefill_alg_flops the cluster kernel runs as
+    fp16 MMAs."""
+    return B * T * H * 6 * dk * dv
+
+
+def tensor_fractions(alg_flops, state_flops, launch_ms, bf16_tflops, variant=""):
+    """Algorithmic tensor throughput of a prefill launch against the peaks of
+    its MMA types.  The cluster kernel runs the three state-sized products as
+    kind::f16 (fp16 shares the bf16 peak) and the intra-chunk products as
+    kind::tf32 (half that: the nominal tf32 : bf16 ratio, 1 : 2); the one-SM
+    kernel runs every product as tf32.  tensor_frac_mma is the time these
+    flops need at their own peaks over the launch time; tensor_frac_tf32 and
+    tensor_frac_bf16 put all of them on one peak."""
     tf = alg_flops / (launch_ms / 1e3) / 1e12
+    f16 = min(float(state_flops), float(alg_flops)) if variant.startswith("cluster") else 0.0
+    t_need = ((alg_flops - f16) / (bf16_tflops / 2.0) + f16 / bf16_tflops) / 1e12
     return {"tensor_alg_tflops": round(tf, 2),
+            "tensor_frac_mma": round(t_need / (launch_ms / 1e3), 4),
+            "mma_kinds": ("state products fp16 (kind::f16), intra-chunk products tf32"
+                          if f16 > 0 else "every product tf32 (kind::tf32)"),
             "tensor_frac_tf32": round(tf / (bf16_tflops / 2.0), 4),
             "tensor_peak_tf32": round(bf16_tflops / 2.0, 1),
             "tensor_peak_note": "tf32 peak = measured bf16 peak x 1/2 (nominal tf32:bf16 ratio)",
@@ -347,7 +363,8 @@ def bench_kda(args, rank, world, local):
                 "alg_bytes_per_launch": alg_b,
                 "kernel": "kda_chunk_fwd",
                 "variant": kda.prefill_path(B, T, H)}
-    roofline.update(tensor_fractions(alg_f, launch_ms, bf16_tf))
+    roofline.update(tensor_fractions(alg_f, prefill_state_flops(B, T, H, dk, dv), launch_ms, bf16_tf,
+                                     roofline["variant"]))
 
     result = {
         "metric": METRIC,
@@ -497,7 +514,8 @@ def bench_prefill_workload(args, kda, dev, rank, world, name, hbm_gbs, bf16_tf, 
             "peak_source": peak_src + " hbm_gbs (burst copy)",
             "alg_bytes_per_launch": alg_b, "kernel": "kda_chunk_fwd",
             "variant": kda.prefill_path(B, T, H)}
-    roof.update(tensor_fractions(prefill_alg_flops(B, T, H, dk, dv), launch_ms, bf16_tf))
+    roof.update(tensor_fractions(prefill_alg_flops(B, T, H, dk, dv), prefill_state_flops(B, T, H, dk, dv),
+                                 launch_ms, bf16_tf, roof["variant"]))
     out = {"metric": "KDA prefill tokens/s (%s)" % w.note,
            "value": round(B * T * world * args.steps / (total_ms / 1e3), 1), "unit": "tokens/s",
            "ms_per_step": round(total_ms / args.steps, 4),

@@ -82,10 +82,17 @@ typedef enum {
  * o_t is written for every token; hT is S after the last token.  The work is
  * done in 16-token tiles on the tensor cores with an fp32 master state (the
  * "T11E1" transcript's log-decay-bound turn is what makes the diagonal tiles
- * dense): every MMA takes tf32 operands (each rounded once, to nearest) and
- * accumulates in fp32, which keeps o within 1e-2 of the exact recurrence
- * where bf16 operands would not.  Returns KDA_ERR_UNSUPPORTED for other
- * dk/dv.
+ * dense).  Every MMA accumulates in fp32 and rounds each operand once, to
+ * nearest: to tf32 for the products of decay-scaled keys (factors up to
+ * e^80) and, on the cluster path (few heads), to fp16 for the three
+ * state-sized products S^T W^T, S^T Qt^T and U^T Kb.  Both keep a 10-bit
+ * significand, which keeps o within 1e-2 of the exact recurrence where bf16
+ * operands would not.  fp16's range is the cluster path's input contract:
+ * h0 and v entries far below 65504 in magnitude (as unit-norm q and k
+ * imply for the other operands); state entries below 2^-14 of absolute
+ * size lose significand bits (absolute error up to 2^-24), negligible for
+ * states of the order of 1e-3 or larger.  Returns KDA_ERR_UNSUPPORTED for
+ * other dk/dv.
  *
  * Segment scan: with B*H <= 8 and T >= 4096 each sequence is cut into P
  * segments that run in parallel (P about SMs / (B*H), at least 256 tokens
@@ -147,7 +154,9 @@ int kda_chunk_fwd_states(const void* q, const void* k, const void* v, const void
  * so that running the sequence from any start state S0 ends at
  * M S0 + (the state it reaches from zero).  Computed on the tensor cores as
  * the state reached from S = I with v = 0 (every state column evolves on its
- * own), no o written.  q, k, g: bf16 [B][T][H][dk]; beta: bf16 [B][T][H];
+ * own), no o written, with tf32 operands in every product (M decays towards
+ * zero and keeps its relative accuracy there, which fp16 operands would
+ * not).  q, k, g: bf16 [B][T][H][dk]; beta: bf16 [B][T][H];
  * M: fp32 [B][H][dk][dk] (T == 0: the identity).  Supported: dk == 128.
  * With kda_state_chain this joins segments of one sequence that were run
  * independently (for example one segment per GPU).
