@@ -72,6 +72,9 @@ constexpr uint32_t LBO = 128;                // dense K-direction core-matrix st
 constexpr uint32_t SBO_K128P = (D / 4) * PAD_LBO;   // 4608: K = 128, padded
 constexpr uint32_t SBO_K32 = (C / 4) * LBO;         // 1024: K = 32, dense
 constexpr uint32_t SBO_K32P = (C / 4) * PAD_LBO;    // 1152: K = 32, padded
+// the same layouts for 16-bit elements (core matrices of 8 rows x 8 elements)
+constexpr uint32_t H_SBO_K32 = (C / 8) * LBO;        // 512: K = 32, dense
+constexpr uint32_t H_SBO_K32P = (C / 8) * PAD_LBO;   // 576: K = 32, padded
 
 // shared memory map (bytes)
 constexpr uint32_t RAW = 0;                                    // q, k, v, g rows of a chunk (bf16)
@@ -1331,16 +1334,23 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 named_bar(NB_TB, NX);                 // T, K~ f and V staged
                 fence_after_sync();
                 if (!warp_flag(s_abort)) {
-                    const uint32_t id = idesc_tf32(128, 32, false, false);
-                    const uint64_t bd0 = sdesc(smem_u32(sm + P_TB), PAD_LBO, SBO_K32P);
-                    const uint64_t aw0 = sdesc(smem_u32(sm + P_WA), LBO, SBO_K32);
-                    const uint64_t av0 = sdesc(smem_u32(sm + P_VA), LBO, SBO_K32);
+                    // W^T = Kt^T T^T and U'^T = V^T T^T: fp16 operands with the
+                    // fp16 chain (K = 16 per MMA), tf32 otherwise
+                    const uint32_t id = F16 ? idesc_f16(128, 32) : idesc_tf32(128, 32, false, false);
+                    const uint64_t bd0 = sdesc(smem_u32(sm + P_TB), PAD_LBO, F16 ? H_SBO_K32P : SBO_K32P);
+                    const uint64_t aw0 = sdesc(smem_u32(sm + P_WA), LBO, F16 ? H_SBO_K32 : SBO_K32);
+                    const uint64_t av0 = sdesc(smem_u32(sm + P_VA), LBO, F16 ? H_SBO_K32 : SBO_K32);
 #pragma unroll
-                    for (int ks = 0; ks < C / 8; ++ks) {
+                    for (int ks = 0; ks < C / CH::KSTEP; ++ks) {
                         const uint64_t bstep = (uint64_t)((ks * 2 * PAD_LBO) >> 4);
                         const uint64_t astep = (uint64_t)((ks * 2 * LBO) >> 4);
-                        mma_tf32_ss_w(tm + PT_DW, aw0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
-                        mma_tf32_ss_w(tm + PT_DU, av0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                        if constexpr (F16) {
+                            mma_f16_ss_w(tm + PT_DW, aw0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                            mma_f16_ss_w(tm + PT_DU, av0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                        } else {
+                            mma_tf32_ss_w(tm + PT_DW, aw0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                            mma_tf32_ss_w(tm + PT_DU, av0 + astep, bd0 + bstep, id, ks > 0 ? 1u : 0u);
+                        }
                     }
                     mma_commit_w(mbar);
                     ++n_commit;
@@ -1443,7 +1453,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 fq = f;
                 fk = tau ? e : oe;
                 float p = 1.f;
-                float kc[4];
+                float kc[8];
 #pragma unroll
                 for (int rr = 0; rr < TILE; ++rr) {
                     const int r = tau * TILE + rr;
@@ -1452,9 +1462,20 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     const float qt = qr[rr] * p;
                     st_f32(sm, P_GB + off_kmajor(r, c, PAD_LBO, SBO_K128P), to_tf32(kt));
                     st_f32(sm, P_GB + off_kmajor(C + r, c, PAD_LBO, SBO_K128P), qt);   // full fp32: see below
-                    kc[rr & 3] = to_tf32(kt * f);
-                    if ((rr & 3) == 3)
-                        st_f32x4(sm, P_WA + off_kmajor(c, r - 3, LBO, SBO_K32), kc[0], kc[1], kc[2], kc[3]);
+                    // Kt (chunk-relative) for W: fp16, 8 tokens per vector, or tf32, 4
+                    if constexpr (F16) {
+                        kc[rr & 7] = kt * f;
+                        if ((rr & 7) == 7)
+                            *reinterpret_cast<uint4*>(sm + P_WA + off16_kmajor(c, r - 7, LBO, H_SBO_K32)) =
+                                make_uint4(__float_as_uint(pack_f16x2(kc[0], kc[1])),
+                                           __float_as_uint(pack_f16x2(kc[2], kc[3])),
+                                           __float_as_uint(pack_f16x2(kc[4], kc[5])),
+                                           __float_as_uint(pack_f16x2(kc[6], kc[7])));
+                    } else {
+                        kc[rr & 3] = to_tf32(kt * f);
+                        if ((rr & 3) == 3)
+                            st_f32x4(sm, P_WA + off_kmajor(c, r - 3, LBO, SBO_K32), kc[0], kc[1], kc[2], kc[3]);
+                    }
                 }
                 const float inv = 1.f / e;
                 float sgm = 1.f;
@@ -1475,10 +1496,20 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             fence_smem_to_async();
             fence_before_sync();
             named_arrive(NB_G, NX);
+            if constexpr (F16) {
 #pragma unroll
-            for (int rr = 0; rr < TILE; rr += 4)
-                st_f32x4(sm, P_VA + off_kmajor(c, tau * TILE + rr, LBO, SBO_K32),
-                         to_tf32(vr[rr]), to_tf32(vr[rr + 1]), to_tf32(vr[rr + 2]), to_tf32(vr[rr + 3]));
+                for (int rr = 0; rr < TILE; rr += 8)
+                    *reinterpret_cast<uint4*>(sm + P_VA + off16_kmajor(c, tau * TILE + rr, LBO, H_SBO_K32)) =
+                        make_uint4(__float_as_uint(pack_f16x2(vr[rr], vr[rr + 1])),
+                                   __float_as_uint(pack_f16x2(vr[rr + 2], vr[rr + 3])),
+                                   __float_as_uint(pack_f16x2(vr[rr + 4], vr[rr + 5])),
+                                   __float_as_uint(pack_f16x2(vr[rr + 6], vr[rr + 7])));
+            } else {
+#pragma unroll
+                for (int rr = 0; rr < TILE; rr += 4)
+                    st_f32x4(sm, P_VA + off_kmajor(c, tau * TILE + rr, LBO, SBO_K32),
+                             to_tf32(vr[rr]), to_tf32(vr[rr + 1]), to_tf32(vr[rr + 2]), to_tf32(vr[rr + 3]));
+            }
             fence_smem_to_async();
             wait_mma();
             // A and P (32 x 32) from the Gram (row m of D_G is lane (m % 16) +
@@ -1575,11 +1606,15 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 tmx[(TILE + r) * LD + i] = -z * bt[i];
             }
             prep_sync();
-            {
+            {   // T into the B operand of the WY products: element (n = r, k = i)
                 const int r = pt >> 3, i = (pt & 7) * 4;
                 const float* row = tmx + r * LD + i;
-                st_f32x4(sm, P_TB + off_kmajor(r, i, PAD_LBO, SBO_K32P),
-                         to_tf32(row[0]), to_tf32(row[1]), to_tf32(row[2]), to_tf32(row[3]));
+                if constexpr (F16)
+                    *reinterpret_cast<uint2*>(sm + P_TB + off16_kmajor(r, i, PAD_LBO, H_SBO_K32P)) =
+                        make_uint2(__float_as_uint(pack_f16x2(row[0], row[1])), __float_as_uint(pack_f16x2(row[2], row[3])));
+                else
+                    st_f32x4(sm, P_TB + off_kmajor(r, i, PAD_LBO, SBO_K32P),
+                             to_tf32(row[0]), to_tf32(row[1]), to_tf32(row[2]), to_tf32(row[3]));
             }
             fence_smem_to_async();
             fence_before_sync();
