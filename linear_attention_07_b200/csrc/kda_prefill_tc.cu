@@ -1421,6 +1421,9 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             prep_sync();
             float gam_c, fq, fk;
             float vr[TILE];
+            // fp16 instantiation: the chunk-relative Qt and Kb of this thread's
+            // channel and tile, as fp16 pairs, kept in registers for the fill
+            uint32_t qh[TILE / 2], kh[TILE / 2];
             {
                 const __nv_bfloat16* __restrict__ rq = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW + 0 * RAW_T);
                 const __nv_bfloat16* __restrict__ rk = reinterpret_cast<const __nv_bfloat16*>(sm + P_RAW + 1 * RAW_T);
@@ -1454,6 +1457,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 fk = tau ? e : oe;
                 float p = 1.f;
                 float kc[8];
+                float qprev = 0.f;
 #pragma unroll
                 for (int rr = 0; rr < TILE; ++rr) {
                     const int r = tau * TILE + rr;
@@ -1462,6 +1466,10 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     const float qt = qr[rr] * p;
                     st_f32(sm, P_GB + off_kmajor(r, c, PAD_LBO, SBO_K128P), to_tf32(kt));
                     st_f32(sm, P_GB + off_kmajor(C + r, c, PAD_LBO, SBO_K128P), qt);   // full fp32: see below
+                    if constexpr (F16) {
+                        if (rr & 1) qh[rr >> 1] = __float_as_uint(pack_f16x2(qprev, qt * fq));
+                        else qprev = qt * fq;
+                    }
                     // Kt (chunk-relative) for W: fp16, 8 tokens per vector, or tf32, 4
                     if constexpr (F16) {
                         kc[rr & 7] = kt * f;
@@ -1479,17 +1487,24 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 }
                 const float inv = 1.f / e;
                 float sgm = 1.f;
+                float knext = 0.f;
 #pragma unroll
                 for (int rr = TILE - 1; rr >= 0; --rr) {
                     const int r = tau * TILE + rr;
                     const float kb = kr[rr] * sgm;
                     // Qt (above), Kh and Kb_0 stay in full fp32: the operand fill
                     // rescales them into the chunk-relative Qt and Kb and rounds
-                    // to tf32 once (rounding here too would round those twice);
+                    // them once (rounding here too would round those twice);
                     // the Gram MMA reads the rows as tf32 (low mantissa bits
-                    // ignored).
+                    // ignored).  The fp16 instantiation forms the chunk-relative
+                    // values here, from the same fp32 numbers the fill would read.
                     st_f32(sm, P_GA + off_kmajor(r, c, PAD_LBO, SBO_K128P), kb * inv);
                     if (tau == 0) st_f32(sm, P_GA + off_kmajor(C + rr, c, PAD_LBO, SBO_K128P), kb);
+                    if constexpr (F16) {
+                        const float kf = tau ? (kb * inv) * fk : kb * fk;
+                        if (rr & 1) knext = kf;
+                        else kh[rr >> 1] = __float_as_uint(pack_f16x2(kf, knext));
+                    }
                     sgm *= a[rr];
                 }
             }
@@ -1619,15 +1634,17 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             fence_smem_to_async();
             fence_before_sync();
             named_arrive(NB_TB, NX);
-            const float* gaf = reinterpret_cast<const float*>(sm + P_GA);
-            const float* gbf = reinterpret_cast<const float*>(sm + P_GB);
             float qf[TILE], kf[TILE];
+            if constexpr (!F16) {
+                const float* gaf = reinterpret_cast<const float*>(sm + P_GA);
+                const float* gbf = reinterpret_cast<const float*>(sm + P_GB);
 #pragma unroll
-            for (int rr = 0; rr < TILE; ++rr) {
-                const int r = tau * TILE + rr;
-                qf[rr] = gbf[off_kmajor(C + r, c, PAD_LBO, SBO_K128P) >> 2] * fq;
-                const int row = tau ? (TILE + rr) : (C + rr);
-                kf[rr] = gaf[off_kmajor(row, c, PAD_LBO, SBO_K128P) >> 2] * fk;
+                for (int rr = 0; rr < TILE; ++rr) {
+                    const int r = tau * TILE + rr;
+                    qf[rr] = gbf[off_kmajor(C + r, c, PAD_LBO, SBO_K128P) >> 2] * fq;
+                    const int row = tau ? (TILE + rr) : (C + rr);
+                    kf[rr] = gaf[off_kmajor(row, c, PAD_LBO, SBO_K128P) >> 2] * fk;
+                }
             }
             // P, element (n = r, k = i) (lane = row: no bank conflicts): fp16,
             // eight K-adjacent entries per thread (threads 0-127), or tf32, four
@@ -1667,7 +1684,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 for (int rr = 0; rr < TILE; ++rr) {
                     if constexpr (F16)
                         *reinterpret_cast<uint16_t*>(st + S_B1 + off16_kmajor(C + tau * TILE + rr, c, PAD_LBO, CH::SBO_B1)) =
-                            to_f16_bits(qf[rr]);
+                            (uint16_t)((rr & 1) ? (qh[rr >> 1] >> 16) : (qh[rr >> 1] & 0xffffu));
                     else
                         st_f32(st, S_B1 + off_kmajor(C + tau * TILE + rr, c, PAD_LBO, CH::SBO_B1), to_tf32(qf[rr]));
                 }
@@ -1676,10 +1693,7 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 #pragma unroll
                     for (int rr = 0; rr < TILE; rr += 8)
                         *reinterpret_cast<uint4*>(st + S_B2 + off16_kmajor(c, tau * TILE + rr, LBO, CH::SBO_B23)) =
-                            make_uint4(__float_as_uint(pack_f16x2(kf[rr], kf[rr + 1])),
-                                       __float_as_uint(pack_f16x2(kf[rr + 2], kf[rr + 3])),
-                                       __float_as_uint(pack_f16x2(kf[rr + 4], kf[rr + 5])),
-                                       __float_as_uint(pack_f16x2(kf[rr + 6], kf[rr + 7])));
+                            make_uint4(kh[rr / 2], kh[rr / 2 + 1], kh[rr / 2 + 2], kh[rr / 2 + 3]);
                     if (pt < 4 * C) {
                         const int r = pt & 31, i = (pt >> 5) * 8;
                         *reinterpret_cast<uint4*>(st + S_B3 + off16_kmajor(r, i, LBO, CH::SBO_B23)) = pf4;
