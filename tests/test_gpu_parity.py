@@ -152,6 +152,22 @@ def test_bf16_both_prefill_variants(monkeypatch, variant, T):
     assert kda.device_status() == kda.KDA_OK
 
 
+@pytest.mark.parametrize("variant", ["fused", "cluster"])
+@pytest.mark.parametrize("scale", [1e-3, 30.0])
+def test_bf16_input_scale(monkeypatch, variant, scale):
+    """v and h0 scaled down (states of order 1e-3, still normal fp16 numbers)
+    and up (|U| and |S| of order 100): the cluster kernel's fp16 state
+    products keep the stated error at both ends of the documented range,
+    like the all-tf32 one-SM kernel."""
+    monkeypatch.setenv("KDA_PREFILL_VARIANT", variant)
+    x = prefill_inputs(1, 300, 3, 128, 128, seed=620, h0_std=0.1)
+    x["v"] = (x["v"].float() * scale).to(torch.bfloat16)
+    x["h0"] = x["h0"] * scale
+    o, hT = run_prefill(x)
+    check_prefill(x, o, hT, TOL_BF16)
+    assert kda.device_status() == kda.KDA_OK
+
+
 # ------------------------------------------------------ segment scan ---
 
 @pytest.mark.parametrize("B,H,T,pin", [(1, 1, 5000, 0.0), (1, 2, 4096, 0.1), (2, 1, 6173, 0.0)])
