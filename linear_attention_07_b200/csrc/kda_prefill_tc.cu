@@ -39,13 +39,14 @@
 //     cut into segments run in parallel by either kernel, joined through
 //     their transitions (description above launch_segmented).
 // Every MMA accumulates in fp32 and is issued by a whole converged warp with
-// elect.sync.  The products that take the decay-scaled keys (the Gram and WY
-// products, factors up to e^80) are tf32 (kind::tf32); operands are rounded to
-// tf32 once, to nearest (ties away from zero), by an integer add-and-mask:
-// bf16 operands would leave errors of a few percent of rms(o) on these
-// products (the q.k diagonal times a large u); tf32 leaves a few tenths of a
-// percent.  The cluster kernel's chain products take fp16 instead (same
-// significand; see there).
+// elect.sync.  The Gram product takes the decay-scaled keys (factors up to
+// e^80) and is tf32 (kind::tf32) in both kernels, and so is every product of
+// the one-SM kernel; operands are rounded to tf32 once, to nearest (ties away
+// from zero), by an integer add-and-mask: bf16 operands would leave errors of
+// a few percent of rms(o) on these products (the q.k diagonal times a large
+// u); a 10-bit significand leaves a few tenths of a percent.  The cluster
+// kernel's chain and WY products take fp16 instead (the same significand;
+// see there).
 // Shared-memory operands use the no-swizzle K-major layout; when the thread
 // that produces a value owns the K index, the K-direction core-matrix stride
 // is padded to 144 B so that a warp's scalar stores hit distinct banks.
@@ -791,10 +792,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // itself when it hands the slot back; EMPTY (the preparing CTA) is arrived on
 // by the chain CTA once the chunk's MMAs are done and its decay applied.  o of
 // a chunk is staged one chunk late, while the next chunk's first MMA runs, in
-// one of two buffers, and written by a tensor store.  The arithmetic is the
+// one of two buffers (one in the tf32 instantiation), and written by a tensor
+// store.  The arithmetic is the
 // one of prefill_tc_kernel, except that the chain's three products
-// (S^T [W | Qt]^T, Kb^T U, P U) take fp16 operands (kind::f16, K = 16 per
-// MMA): fp16 keeps tf32's 10-bit significand, and these operands are bounded
+// (S^T [W | Qt]^T, Kb^T U, P U) and the preparers' WY products (T Kt, T V)
+// take fp16 operands (kind::f16, K = 16 per MMA): fp16 keeps tf32's 10-bit
+// significand, and these operands are bounded
 // (|Qt|, |Kb|, |P| <= 1 for unit-norm q and k; S, W and U of the order of h0
 // and v), far inside fp16's range (65504).  Half as many MMAs per chunk, and
 // half the slot bytes for those operands.  fp16's range is the price: entries
