@@ -186,3 +186,23 @@ def test_a_missing_wait_is_caught(monkeypatch):
     assert res["mode"].startswith("pipelined")
     with pytest.raises(AssertionError, match="unordered"):
         _verify(sim, 5, 6)
+
+
+def test_tensor_fraction_uses_each_products_own_peak():
+    """tensor_frac_mma: the state products on the fp16 peak for the cluster
+    kernel and everything on the tf32 peak (half of it) otherwise; the
+    one-peak fractions stay as they were."""
+    B, T, H, d = 1, 8192, 32, 128
+    alg = bench.prefill_alg_flops(B, T, H, d, d)
+    state = bench.prefill_state_flops(B, T, H, d, d)
+    assert state == B * T * H * 6 * d * d and 0 < state < alg
+    peak, ms = 1600.0, 0.5
+    one_sm = bench.tensor_fractions(alg, state, ms, peak, "one SM per head")
+    cluster = bench.tensor_fractions(alg, state, ms, peak, "cluster of four SMs per head")
+    sec = ms / 1e3
+    assert one_sm["tensor_frac_mma"] == pytest.approx(alg / (peak / 2 * 1e12) / sec, rel=1e-3)
+    assert one_sm["tensor_frac_mma"] == one_sm["tensor_frac_tf32"]
+    want = ((alg - state) / (peak / 2 * 1e12) + state / (peak * 1e12)) / sec
+    assert cluster["tensor_frac_mma"] == pytest.approx(want, rel=1e-3)
+    assert cluster["tensor_frac_bf16"] < cluster["tensor_frac_mma"] < cluster["tensor_frac_tf32"]
+    assert "fp16" in cluster["mma_kinds"] and "fp16" not in one_sm["mma_kinds"]
