@@ -1246,25 +1246,27 @@ prefill_cluster_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 // X of chunk ch (U' of this chunk is in the slot once its FULL
                 // phase passed: the release warp publishes that as s_full)
                 if (!s_abort && !counter_wait(smem_u32(&s_full), (uint32_t)ch + 1u, wait_ns)) expired();
-                wait_bar(mbar, phase & 1u);
-                ++phase;
                 {   // U = U' - W S  (this thread: tokens [16 hh, 16 hh + 16)): fp16
                     // pairs into packed columns [8 hh, 8 hh + 8) of CT_AU, or tf32
-                    // into columns [16 hh, 16 hh + 16)
+                    // into columns [16 hh, 16 hh + 16).  U' is read before the
+                    // wait for X, off the path from X to U.
                     const float* up = reinterpret_cast<const float*>(sm + sb + S_UP);
+                    float upr[16];
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) upr[r] = up[(16 * hh + r) * D + j];
+                    wait_bar(mbar, phase & 1u);
+                    ++phase;
                     float x[16];
                     tmem_ld16(tm + lane_base + dx + 16 * hh, x);
                     wait_ld();
                     if constexpr (F16) {
                         float hp[8];
 #pragma unroll
-                        for (int r = 0; r < 16; r += 2)
-                            hp[r >> 1] = pack_f16x2(up[(16 * hh + r) * D + j] - x[r],
-                                                    up[(16 * hh + r + 1) * D + j] - x[r + 1]);
+                        for (int r = 0; r < 16; r += 2) hp[r >> 1] = pack_f16x2(upr[r] - x[r], upr[r + 1] - x[r + 1]);
                         tmem_st8(tm + lane_base + CT_AU + 8 * hh, hp);
                     } else {
 #pragma unroll
-                        for (int r = 0; r < 16; ++r) x[r] = to_tf32(up[(16 * hh + r) * D + j] - x[r]);
+                        for (int r = 0; r < 16; ++r) x[r] = to_tf32(upr[r] - x[r]);
                         tmem_st16(tm + lane_base + CT_AU + 16 * hh, x);
                     }
                     wait_st();
