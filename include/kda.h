@@ -85,9 +85,10 @@ typedef enum {
  * dense).  Every MMA accumulates in fp32 and rounds each operand once, to
  * nearest: to tf32 for the products of decay-scaled keys (factors up to
  * e^80) and, on the cluster path (few heads), to fp16 for the three
- * state-sized products S^T W^T, S^T Qt^T and U^T Kb.  Both keep a 10-bit
- * significand, which keeps o within 1e-2 of the exact recurrence where bf16
- * operands would not.  fp16's range is the cluster path's input contract:
+ * state-sized products S^T W^T, S^T Qt^T and U^T Kb, for P U and for the
+ * WY products T Kt and T V (tf32 for all of them on the one-SM path).  Both
+ * keep a 10-bit significand, which keeps o within 1e-2 of the exact
+ * recurrence where bf16 operands would not.  fp16's range is the cluster path's input contract:
  * h0 and v entries far below 65504 in magnitude (as unit-norm q and k
  * imply for the other operands); state entries below 2^-14 of absolute
  * size lose significand bits (absolute error up to 2^-24), negligible for
